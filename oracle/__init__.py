@@ -1,0 +1,164 @@
+"""fp64 CPU oracle of the Mamba-3 SSM layer scan -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s cpu-baseline /
+reference leg may import this package.  The product package
+``selective_state_space_m3_b200`` never imports it, and the two share no code.
+
+The arithmetic lives in ``m3_oracle.c`` (plain C, double precision, the literal
+token-by-token recurrence); this module only compiles it with gcc and marshals
+float64 numpy arrays through ctypes.
+
+Passages followed (page titles and sections):
+  * "Mamba-3" summary (b-lab.team), section 1 "Exponential-Trapezoidal
+    Discretization": h_t = a_t h_{t-1} + b_t B_{t-1} x_{t-1} + g_t B_t x_t with
+    a_t = exp(dt A), b_t = (1-lam) dt exp(dt A), g_t = lam dt.
+  * same page, section 2 "Complex-Valued State Space Model": Proposition 2
+    (block-diagonal R(dt theta[i]) rotations, y = C^T h) and Proposition 3
+    (the rotation moved onto B and C as a cumulative phase, oracle_rope_bc).
+  * same page, section 3 "MIMO": B, C in R^{N x R}, x in R^{P x R}.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "m3_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_BUILD, "libm3oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_int) for k in
+                ("batch", "seqlen", "nheads", "ngroups", "headdim", "dstate", "rank")]
+
+
+def build(force: bool = False) -> str:
+    """Compile m3_oracle.c into oracle/_build/libm3oracle.so (gcc, -O2, OpenMP)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-std=c99",
+                        "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _bind(lib):
+    P = ctypes.POINTER(ctypes.c_double)
+    D = ctypes.POINTER(_Dims)
+    lib.oracle_scan.argtypes = [D] + [P] * 14
+    lib.oracle_scan.restype = ctypes.c_int
+    lib.oracle_step.argtypes = [D] + [P] * 11
+    lib.oracle_step.restype = ctypes.c_int
+    lib.oracle_rope_bc.argtypes = [D] + [P] * 7
+    lib.oracle_rope_bc.restype = ctypes.c_int
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = _bind(ctypes.CDLL(build()))
+    return _lib
+
+
+def compile_variant(source_text: str, tag: str):
+    """Compile a modified copy of the oracle source (tests plant mistakes in
+    it to show that the pins catch them) and return a ctypes handle usable as
+    the ``lib=`` argument of scan/step/rope_bc."""
+    os.makedirs(_BUILD, exist_ok=True)
+    src = os.path.join(_BUILD, f"variant_{tag}_{os.getpid()}.c")
+    so = src[:-2] + ".so"
+    with open(src, "w") as f:
+        f.write(source_text)
+    subprocess.run(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-std=c99",
+                    "-o", so, src, "-lm"], check=True)
+    return _bind(ctypes.CDLL(so))
+
+
+def source_text() -> str:
+    with open(_SRC) as f:
+        return f.read()
+
+
+def _p(a):
+    if a is None:
+        return None
+    assert a.dtype == np.float64 and a.flags["C_CONTIGUOUS"], "oracle takes C-contiguous float64"
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _f64(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float64)
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def scan(x, B, C, dt, A, lam, theta, init_h=None, init_pB=None, init_pX=None, lib=None):
+    """Full-sequence oracle.
+
+    x [b,t,h,r,p]; B, C [b,t,g,r,n]; dt, lam [b,t,h]; A [h]; theta [b,t,g,n/2];
+    optional carry init_h [b,h,n,p], init_pB [b,h,r,n], init_pX [b,h,r,p].
+    Returns (y [b,t,h,r,p], h [b,h,n,p], prev_B [b,h,r,n], prev_x [b,h,r,p]).
+    """
+    x, B, C, dt, A, lam, theta = map(_f64, (x, B, C, dt, A, lam, theta))
+    init_h, init_pB, init_pX = map(_f64, (init_h, init_pB, init_pX))
+    b, L, H, R, P = x.shape
+    G, N = B.shape[2], B.shape[4]
+    d = _Dims(b, L, H, G, P, N, R)
+    y = np.zeros((b, L, H, R, P))
+    hL = np.zeros((b, H, N, P))
+    pB = np.zeros((b, H, R, N))
+    pX = np.zeros((b, H, R, P))
+    rc = (lib or _load()).oracle_scan(ctypes.byref(d), _p(x), _p(B), _p(C), _p(dt), _p(A), _p(lam),
+                             _p(theta), _p(init_h), _p(init_pB), _p(init_pX),
+                             _p(y), _p(hL), _p(pB), _p(pX))
+    if rc != 0:
+        raise ValueError("oracle_scan rejected its arguments")
+    return y, hL, pB, pX
+
+
+def step(h, prev_B, prev_x, x, B, C, dt, A, lam, theta, lib=None):
+    """One decode token.  h [b,h,n,p], prev_B [b,h,r,n], prev_x [b,h,r,p];
+    x [b,h,r,p]; B, C [b,g,r,n]; dt, lam [b,h]; A [h]; theta [b,g,n/2].
+    Returns (y [b,h,r,p], h', prev_B', prev_x') as new arrays."""
+    h, prev_B, prev_x = (np.array(a, dtype=np.float64, order="C", copy=True)
+                         for a in (h, prev_B, prev_x))
+    x, B, C, dt, A, lam, theta = map(_f64, (x, B, C, dt, A, lam, theta))
+    b, H, R, P = x.shape
+    G, N = B.shape[1], B.shape[3]
+    d = _Dims(b, 1, H, G, P, N, R)
+    y = np.zeros((b, H, R, P))
+    rc = (lib or _load()).oracle_step(ctypes.byref(d), _p(h), _p(prev_B), _p(prev_x), _p(x), _p(B),
+                             _p(C), _p(dt), _p(A), _p(lam), _p(theta), _p(y))
+    if rc != 0:
+        raise ValueError("oracle_step rejected its arguments")
+    return y, h, prev_B, prev_x
+
+
+def rope_bc(B, C, dt, theta, nheads, lib=None):
+    """Cumulative phase and rotated B, C per head.
+    Returns (B_rot [b,t,h,r,n], C_rot [b,t,h,r,n], phase [b,t,h,n/2])."""
+    B, C, dt, theta = map(_f64, (B, C, dt, theta))
+    b, L, G, R, N = B.shape
+    d = _Dims(b, L, nheads, G, 1, N, R)
+    Bo = np.zeros((b, L, nheads, R, N))
+    Co = np.zeros((b, L, nheads, R, N))
+    ph = np.zeros((b, L, nheads, N // 2))
+    rc = (lib or _load()).oracle_rope_bc(ctypes.byref(d), _p(B), _p(C), _p(dt), _p(theta),
+                                _p(Bo), _p(Co), _p(ph))
+    if rc != 0:
+        raise ValueError("oracle_rope_bc rejected its arguments")
+    return Bo, Co, ph

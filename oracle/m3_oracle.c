@@ -1,0 +1,236 @@
+/*
+ * m3_oracle.c -- plain, slow, fp64 CPU oracle of the Mamba-3 SSM layer scan.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and
+ * bench.py's cpu_baseline / reference leg may load this library.  The product
+ * path (selective_state_space_m3_b200) never links, imports or calls it, and
+ * this file shares no code, header, table or constant with the CUDA sources.
+ *
+ * What it computes (all in double precision, token by token, no chunking,
+ * no reordering beyond the loops written below):
+ *
+ *   For every batch b and head h (group g = h / (H/G)):
+ *     alpha_t = exp(dt_t * A_h)
+ *     beta_t  = (1 - lambda_t) * dt_t * exp(dt_t * A_h)
+ *     gamma_t = lambda_t * dt_t
+ *       -- "Mamba-3" summary (b-lab.team), section 1 "Exponential-Trapezoidal
+ *          Discretization": the recurrence and the definitions of alpha, beta,
+ *          gamma.
+ *     R_t = blockdiag_i R(dt_t * theta_t[i]),  R(phi) = [[cos,-sin],[sin,cos]]
+ *       -- same page, section 2 "Complex-Valued State Space Model"
+ *          (Proposition 2), the 2x2 rotation blocks.
+ *     h_t = R_t (alpha_t h_{t-1} + beta_t B_{t-1} X_{t-1}^T) + gamma_t B_t X_t^T
+ *     y_t = C_t^T h_t                          (R x P per head: MIMO, section 3)
+ *
+ *   Reading (the pages never print the trapezoid and the rotation together):
+ *   the rotation R_t multiplies the whole t-1 -> t transition, i.e. both the
+ *   carried state and the beta term, because beta carries exp(dt A), which
+ *   for the complex SSM is exp(dt (A + i theta)).  This is the reading under
+ *   which Proposition 3 (data-dependent RoPE on B and C) holds with every B_s
+ *   rotated by its own cumulative phase.
+ *
+ * Layouts (row-major, innermost last):
+ *   x      [b][t][h][r][p]        y      [b][t][h][r][p]
+ *   B, C   [b][t][g][r][n]        theta  [b][t][g][N/2]
+ *   dt,lam [b][t][h]              A      [h]
+ *   carry: h [b][h][n][p], prev_B [b][h][r][n], prev_x [b][h][r][p]
+ *   Rotary pair i occupies state rows (2i, 2i+1).
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    int batch, seqlen, nheads, ngroups, headdim, dstate, rank;
+} oracle_dims;
+
+static int dims_ok(const oracle_dims* d)
+{
+    if (!d) return 0;
+    if (d->batch < 0 || d->seqlen < 0 || d->nheads <= 0 || d->ngroups <= 0) return 0;
+    if (d->headdim <= 0 || d->dstate <= 0 || d->rank <= 0) return 0;
+    if (d->dstate % 2 != 0) return 0;
+    if (d->nheads % d->ngroups != 0) return 0;
+    return 1;
+}
+
+/* One token of the recurrence for one (b, h), in the original frame.
+ * H: N*P state, PB: R*N previous B (stored [r][n]), PX: R*P previous x.
+ * xt: R*P, Bt/Ct: R*N, th: N/2, yt: R*P (output). */
+static void step_bh(int N, int P, int R,
+                    double* H, double* PB, double* PX,
+                    const double* xt, const double* Bt, const double* Ct,
+                    double d, double a, double lam, const double* th,
+                    double* yt)
+{
+    const double alpha = exp(d * a);
+    const double beta = (1.0 - lam) * d * exp(d * a);
+    const double gamma = lam * d;
+
+    /* carried part: alpha h + beta * B_{t-1} X_{t-1}^T */
+    for (int n = 0; n < N; ++n)
+        for (int p = 0; p < P; ++p) {
+            double bx = 0.0;
+            for (int r = 0; r < R; ++r) bx += PB[r * N + n] * PX[r * P + p];
+            H[n * P + p] = alpha * H[n * P + p] + beta * bx;
+        }
+
+    /* rotation R_t on every pair (2i, 2i+1), every column p */
+    for (int i = 0; i < N / 2; ++i) {
+        const double phi = d * th[i];
+        const double c = cos(phi), s = sin(phi);
+        for (int p = 0; p < P; ++p) {
+            const double u0 = H[(2 * i) * P + p];
+            const double u1 = H[(2 * i + 1) * P + p];
+            H[(2 * i) * P + p] = c * u0 - s * u1;
+            H[(2 * i + 1) * P + p] = s * u0 + c * u1;
+        }
+    }
+
+    /* current input: + gamma * B_t X_t^T */
+    for (int n = 0; n < N; ++n)
+        for (int p = 0; p < P; ++p) {
+            double bx = 0.0;
+            for (int r = 0; r < R; ++r) bx += Bt[r * N + n] * xt[r * P + p];
+            H[n * P + p] += gamma * bx;
+        }
+
+    /* readout y_t = C_t^T h_t : [r][p] */
+    for (int r = 0; r < R; ++r)
+        for (int p = 0; p < P; ++p) {
+            double acc = 0.0;
+            for (int n = 0; n < N; ++n) acc += Ct[r * N + n] * H[n * P + p];
+            yt[r * P + p] = acc;
+        }
+
+    /* the next step's beta term needs this step's (B, x) */
+    memcpy(PB, Bt, sizeof(double) * (size_t)R * N);
+    memcpy(PX, xt, sizeof(double) * (size_t)R * P);
+}
+
+/* Full sequence.  init_h / init_pB / init_pX may be NULL (zeros).
+ * y must hold batch*seqlen*H*R*P doubles.  out_h / out_pB / out_pX may be NULL.
+ * Returns 0 on success, -1 on bad arguments. */
+int oracle_scan(const oracle_dims* d,
+                const double* x, const double* B, const double* C,
+                const double* dt, const double* A, const double* lam,
+                const double* theta,
+                const double* init_h, const double* init_pB, const double* init_pX,
+                double* y, double* out_h, double* out_pB, double* out_pX)
+{
+    if (!dims_ok(d) || !x || !B || !C || !dt || !A || !lam || !theta || !y) return -1;
+    const int Bn = d->batch, L = d->seqlen, H = d->nheads, G = d->ngroups;
+    const int P = d->headdim, N = d->dstate, R = d->rank;
+    const int hpg = H / G;
+
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < Bn; ++b)
+        for (int h = 0; h < H; ++h) {
+            const int g = h / hpg;
+            double* Hs = (double*)calloc((size_t)N * P, sizeof(double));
+            double* PB = (double*)calloc((size_t)R * N, sizeof(double));
+            double* PX = (double*)calloc((size_t)R * P, sizeof(double));
+            const size_t bh = (size_t)b * H + h;
+            if (init_h) memcpy(Hs, init_h + bh * N * P, sizeof(double) * (size_t)N * P);
+            if (init_pB) memcpy(PB, init_pB + bh * R * N, sizeof(double) * (size_t)R * N);
+            if (init_pX) memcpy(PX, init_pX + bh * R * P, sizeof(double) * (size_t)R * P);
+            for (int t = 0; t < L; ++t) {
+                const size_t bt = (size_t)b * L + t;
+                const double* xt = x + ((bt * H + h) * R) * P;
+                const double* Bt = B + ((bt * G + g) * R) * N;
+                const double* Ct = C + ((bt * G + g) * R) * N;
+                const double* th = theta + (bt * G + g) * (N / 2);
+                double* yt = y + ((bt * H + h) * R) * P;
+                step_bh(N, P, R, Hs, PB, PX, xt, Bt, Ct,
+                        dt[bt * H + h], A[h], lam[bt * H + h], th, yt);
+            }
+            if (out_h) memcpy(out_h + bh * N * P, Hs, sizeof(double) * (size_t)N * P);
+            if (out_pB) memcpy(out_pB + bh * R * N, PB, sizeof(double) * (size_t)R * N);
+            if (out_pX) memcpy(out_pX + bh * R * P, PX, sizeof(double) * (size_t)R * P);
+            free(Hs); free(PB); free(PX);
+        }
+    return 0;
+}
+
+/* One decode token for every (b, h): the carry (h, prev_B, prev_x) is updated
+ * in place.  Per-token layouts: x [b][h][r][p], B/C [b][g][r][n],
+ * theta [b][g][N/2], dt/lam [b][h], y [b][h][r][p].  d->seqlen is ignored. */
+int oracle_step(const oracle_dims* d,
+                double* h_state, double* prev_B, double* prev_x,
+                const double* x, const double* B, const double* C,
+                const double* dt, const double* A, const double* lam,
+                const double* theta, double* y)
+{
+    if (!dims_ok(d) || !h_state || !prev_B || !prev_x || !x || !B || !C ||
+        !dt || !A || !lam || !theta || !y) return -1;
+    const int Bn = d->batch, H = d->nheads, G = d->ngroups;
+    const int P = d->headdim, N = d->dstate, R = d->rank;
+    const int hpg = H / G;
+
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < Bn; ++b)
+        for (int h = 0; h < H; ++h) {
+            const int g = h / hpg;
+            const size_t bh = (size_t)b * H + h;
+            const size_t bg = (size_t)b * G + g;
+            step_bh(N, P, R, h_state + bh * N * P, prev_B + bh * R * N, prev_x + bh * R * P,
+                    x + bh * R * P, B + bg * R * N, C + bg * R * N,
+                    dt[bh], A[h], lam[bh], theta + bg * (N / 2), y + bh * R * P);
+        }
+    return 0;
+}
+
+/* Cumulative phase and rotated B, C (the "RoPE trick", Proposition 3 of the
+ * same page):  Phi_t[i] = sum_{s<=t} dt_s theta_s[i]  (per head, since dt is),
+ *   (Bt_{2i}, Bt_{2i+1}) = R(Phi_t[i])^T (B_{2i}, B_{2i+1})
+ *                        = ( cos*B_{2i} + sin*B_{2i+1}, -sin*B_{2i} + cos*B_{2i+1} ).
+ * Outputs: B_rot, C_rot [b][t][h][r][n]; phase [b][t][h][N/2] (unreduced,
+ * may be NULL). */
+int oracle_rope_bc(const oracle_dims* d,
+                   const double* B, const double* C, const double* dt,
+                   const double* theta, double* B_rot, double* C_rot, double* phase)
+{
+    if (!dims_ok(d) || !B || !C || !dt || !theta || !B_rot || !C_rot) return -1;
+    const int Bn = d->batch, L = d->seqlen, H = d->nheads, G = d->ngroups;
+    const int N = d->dstate, R = d->rank, hpg = H / G;
+
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < Bn; ++b)
+        for (int h = 0; h < H; ++h) {
+            const int g = h / hpg;
+            double* Phi = (double*)calloc((size_t)N / 2, sizeof(double));
+            for (int t = 0; t < L; ++t) {
+                const size_t bt = (size_t)b * L + t;
+                const double dd = dt[bt * H + h];
+                const double* th = theta + (bt * G + g) * (N / 2);
+                for (int i = 0; i < N / 2; ++i) Phi[i] += dd * th[i];
+                if (phase)
+                    memcpy(phase + (bt * H + h) * (N / 2), Phi, sizeof(double) * (size_t)N / 2);
+                for (int r = 0; r < R; ++r) {
+                    const double* Bs = B + ((bt * G + g) * R + r) * N;
+                    const double* Cs = C + ((bt * G + g) * R + r) * N;
+                    double* Bo = B_rot + ((bt * H + h) * R + r) * N;
+                    double* Co = C_rot + ((bt * H + h) * R + r) * N;
+                    for (int i = 0; i < N / 2; ++i) {
+                        const double c = cos(Phi[i]), s = sin(Phi[i]);
+                        Bo[2 * i] = c * Bs[2 * i] + s * Bs[2 * i + 1];
+                        Bo[2 * i + 1] = -s * Bs[2 * i] + c * Bs[2 * i + 1];
+                        Co[2 * i] = c * Cs[2 * i] + s * Cs[2 * i + 1];
+                        Co[2 * i + 1] = -s * Cs[2 * i] + c * Cs[2 * i + 1];
+                    }
+                }
+            }
+            free(Phi);
+        }
+    return 0;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
