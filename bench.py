@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Throughput of the Mamba-3 SSM layer scan on B200 GPUs.
+
+Default workload: the chunked prefill (m3_scan_fwd) of the 1.5B-scale MIMO
+layer -- batch 8, 32 heads, L = 4096, P = 64, N = 128, rank 4, chunk 64,
+bfloat16 x/B/C, float32 dt/A/lambda/theta -- on synthetic seeded inputs
+(m3_synth).  One step = one m3_scan_fwd over the whole batch, final carry
+included.  The decode step (m3_step, batch 256, 32 heads, rank 4, carry from
+the prefill) is measured in the same run and reported under "decode".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs its own independent
+batch (weak scaling, no collective on the data path); the timed region is
+bracketed by a barrier and device syncs, and the max over ranks is reported.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "tokens/sec per SSM layer (chunked fwd, decode step) and % of roofline on 1 B200"
+CFG = 2                      # the 1.5B-like MIMO layer
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return dict(hbm=float(j["hbm_gbs"]), bf16=float(j["bf16_tflops"]),
+                    bf16_sus=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), src="measured")
+    return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS, bf16_sus=1400.0, src="fallback")
+
+
+# ------------------------------------------------------------ clocks (NVML) --
+class ClockSampler:
+    """Samples SM clock and clock-event reasons every 20 ms in a thread."""
+    BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks",
+            0x1: "gpu_idle"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self._stop = threading.Event()
+        self.active = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = repr(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                if self.active:
+                    mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                    bits = self.fn(self.h)
+                    util = self.nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                    self.samples.append((mhz, bits, util))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        loaded = [s for s in self.samples if s[2] > 0] or self.samples
+        reasons = set()
+        for _, bits, _ in loaded:
+            for b, name in self.BITS.items():
+                if bits & b and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median([s[0] for s in loaded]) if loaded else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons), "samples": len(loaded)}
+
+
+# ----------------------------------------------------------------- sizes --
+def algorithmic_bytes(t: dict, y, fin) -> int:
+    """Compulsory bytes of one prefill: every input read once, y and the final
+    carry written once."""
+    n = sum(v.numel() * v.element_size() for v in t.values())
+    n += y.numel() * y.element_size()
+    for v in (fin.h, fin.prev_B, fin.prev_x):
+        n += v.numel() * v.element_size()
+    return n
+
+
+def algorithmic_flops(s, tile_rows=128) -> float:
+    """Causal chunked-scan FLOPs per token-head: intra-chunk Gram + masked
+    product ((Q+1) R^2 (N+P) with Q the chunk), plus the state terms
+    (chunk output C~ S and chunk state B~^T X: 4 R N P)."""
+    Q, R, N, P = s.chunk, s.rank, s.dstate, s.headdim
+    per = (Q + 1) * R * R * (N + P) + 4 * R * N * P
+    return float(per) * s.batch * s.seqlen * s.nheads
+
+
+# ------------------------------------------------------------- reference --
+def run_reference(args, rank):
+    if rank != 0:
+        return 0
+    import numpy as np
+    import torch
+    import m3_synth
+    import oracle
+    s = m3_synth.CONFIGS[CFG]
+    # bounded sample: batch row 0, all heads, the whole sequence (about 11
+    # CPU-seconds per step at ~0.35 s per head)
+    sub = m3_synth.shrink(s, batch=1)
+    inp = m3_synth.make_scan_inputs(sub)
+    f = {k: v.to(torch.float64).numpy() for k, v in inp.items()}
+    for _ in range(args.warmup):
+        oracle.scan(**f)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.scan(**f)
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    toks = sub.batch * sub.seqlen
+    val = toks / dt
+    cores = oracle.num_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": m3_synth.CONFIG_NAMES[CFG], "global_batch": s.batch, "seq_len": s.seqlen,
+                       "sample": "batch row 0 of 8, all 32 heads, full L=4096 per step"},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": "1 of 8 batch rows (32 heads x 4096 tokens) per step"},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def cpu_baseline_sample():
+    """The oracle on a bounded sample of the same workload (batch rows 0-1,
+    all heads, full L), timed on this host's cores."""
+    import torch
+    import m3_synth
+    import oracle
+    s = m3_synth.CONFIGS[CFG]
+    sub = m3_synth.shrink(s, batch=2)
+    inp = m3_synth.make_scan_inputs(sub)
+    f = {k: v.to(torch.float64).numpy() for k, v in inp.items()}
+    t0 = time.perf_counter()
+    oracle.scan(**f)
+    dt = time.perf_counter() - t0
+    return {"value": sub.batch * sub.seqlen / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"2 of 8 batch rows (64 head-sequences x 4096 tokens), {dt:.1f} s wall"}
+
+
+# ------------------------------------------------------------------ ours --
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import m3_synth
+    import selective_state_space_m3_b200 as m3
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    pk = peaks()
+    s = m3_synth.CONFIGS[CFG]
+    s = m3_synth.shrink(s, seed=s.seed + 1000 * rank)     # each rank its own problem
+    host = m3_synth.make_scan_inputs(s)
+    dev = {k: v.cuda() for k, v in host.items()}
+    d = m3.Dims(s.batch, s.seqlen, s.nheads, s.ngroups, s.headdim, s.dstate, s.rank, s.chunk, m3.M3_BF16)
+    plan = m3.m3_scan_plan(d)
+    y = torch.empty_like(dev["x"])
+    ws = torch.zeros(m3.m3_scan_workspace_size(d), dtype=torch.uint8, device="cuda")
+    fin = m3.Carry(torch.empty(s.batch, s.nheads, s.dstate, s.headdim, device="cuda"),
+                   torch.empty(s.batch, s.nheads, s.rank, s.dstate, device="cuda", dtype=torch.bfloat16),
+                   torch.empty(s.batch, s.nheads, s.rank, s.headdim, device="cuda", dtype=torch.bfloat16))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        m3.m3_scan_fwd(d, dev["x"], dev["B"], dev["C"], dev["dt"], dev["A"], dev["lam"], dev["theta"],
+                       y, ws, final_state=fin, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert m3.m3_device_status(ws) == m3.M3_OK
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        clk.active = True
+        barrier()
+        torch.cuda.synchronize()
+        t_all0 = torch.cuda.Event(enable_timing=True)
+        t_all1 = torch.cuda.Event(enable_timing=True)
+        t_all0.record(stream)
+        for e0, e1 in ev:
+            e0.record(stream)
+            step()
+            e1.record(stream)
+        t_all1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        clk.active = False
+    assert m3.m3_device_status(ws) == m3.M3_OK
+    total_ms = max_over_ranks(t_all0.elapsed_time(t_all1))
+    per_launch_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    ms_per_step = total_ms / args.steps
+    tokens = s.batch * s.seqlen
+    value = world * tokens * args.steps / (total_ms / 1e3)
+
+    abytes = algorithmic_bytes(dev, y, fin)
+    aflops = algorithmic_flops(s)
+    achieved_gbs = abytes / (per_launch_ms / 1e3) / 1e9
+    tflops = aflops / (per_launch_ms / 1e3) / 1e12
+    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": achieved_gbs / pk["hbm"], "traffic": None,
+                "peak_source": pk["src"],
+                "kernel": "m3_scan_fwd (whole call: %d launch%s)" % (plan["launches"],
+                                                                     "" if plan["launches"] == 1 else "es"),
+                "algorithmic_bytes_per_launch": abytes,
+                "tensor_tflops": tflops, "tensor_frac_of_bf16_peak": tflops / pk["bf16"]}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": m3_synth.CONFIG_NAMES[CFG], "global_batch": s.batch * world,
+                       "seq_len": s.seqlen, "nheads": s.nheads, "headdim": s.headdim, "dstate": s.dstate,
+                       "rank": s.rank, "chunk": s.chunk,
+                       "parallelism": "replicas" if world == 1 else f"dp{world}",
+                       "l2": "inputs 3.5 GB per step >> 126 MB L2; no flush",
+                       "path": plan["path"], "segments": plan["segments"], "chunk_used": plan["chunk_used"]},
+            "roofline": roofline, "clocks": clk.summary(),
+            "gpu_launches": plan["launches"] * args.steps}
+
+    # ---- end to end: pinned host buffers in, y out, copies inside the timed region
+    if not args.no_e2e:
+        pinned = {k: v.pin_memory() for k, v in host.items()}
+        y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+        d2h = y_host.numel() * y_host.element_size()
+        ke = max(2, min(args.steps, 4))
+
+        def e2e_step():
+            for k, v in pinned.items():
+                dev[k].copy_(v, non_blocking=True)
+            step()
+            y_host.copy_(y, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms = max_over_ranks(e0.elapsed_time(e1))
+        line["e2e"] = {"value": world * tokens * ke / (ms / 1e3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke}
+
+    # ---- decode: m3_step x decode_steps in one CUDA graph, carry from the prefill
+    if not args.no_decode:
+        dec = m3_synth.DECODE
+        reps = dec.batch // s.batch
+        state = m3.Carry(fin.h.repeat(reps, 1, 1, 1).contiguous(),
+                         fin.prev_B.repeat(reps, 1, 1, 1).contiguous(),
+                         fin.prev_x.repeat(reps, 1, 1, 1).contiguous())
+        pool = 64      # distinct tokens (22 MB each; 1.4 GB >> L2), cycled
+        toks = []
+        for k in range(pool):
+            t = m3_synth.make_decode_token(m3_synth.DecodeShape(seed=dec.seed + 1000 * rank), k)
+            toks.append({n: v.cuda() for n, v in t.items()})
+        Ad = dev["A"]
+        dd = m3.Dims(dec.batch, 1, dec.nheads, dec.ngroups, dec.headdim, dec.dstate, dec.rank, 1, m3.M3_BF16)
+        yd = torch.empty_like(toks[0]["x"])
+        S = args.decode_steps
+
+        def run_steps(n, st):
+            for k in range(n):
+                t = toks[k % pool]
+                m3.m3_step(dd, state, t["x"], t["B"], t["C"], t["dt"], Ad, t["lam"], t["theta"], yd, stream=st)
+
+        run_steps(3, stream)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run_steps(S, torch.cuda.current_stream())
+        g.replay()
+        torch.cuda.synchronize()
+        reps_t = 2
+        with ClockSampler(local) as clk2:
+            clk2.active = True
+            barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps_t):
+                g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            clk2.active = False
+        ms = max_over_ranks(e0.elapsed_time(e1))
+        per_step_us = ms * 1e3 / (reps_t * S)
+        t0 = toks[0]
+        step_bytes = (2 * state.h.numel() * 4 + 2 * (state.prev_B.numel() + state.prev_x.numel()) * 2 +
+                      sum(v.numel() * v.element_size() for v in t0.values()) + yd.numel() * 2 +
+                      Ad.numel() * 4)
+        gbs = step_bytes / (per_step_us * 1e-6) / 1e9
+        line["decode"] = {"workload": m3_synth.CONFIG_NAMES[4], "tokens_per_s": world * dec.batch / (per_step_us * 1e-6),
+                          "us_per_step": per_step_us, "steps_timed": reps_t * S,
+                          "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                                       "frac": gbs / pk["hbm"], "algorithmic_bytes_per_launch": step_bytes,
+                                       "traffic": None},
+                          "gpu_launches": reps_t * S, "clocks": clk2.summary(),
+                          "inputs": f"{pool} distinct tokens cycled ({pool * 22} MB > L2)"}
+        del g
+
+    if rank == 0 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline_sample()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

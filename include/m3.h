@@ -1,0 +1,166 @@
+/*
+ * m3.h -- C ABI of the B200 (sm_100a) Mamba-3 SSM layer scan.
+ *
+ * The operation.  Per batch b and head h (group g = h / (nheads/ngroups)), a
+ * state h_t in R^{N x P} follows the exponential-trapezoidal recurrence with
+ * data-dependent rotations and MIMO rank-R inputs:
+ *
+ *   alpha_t = exp(dt_t A_h),  beta_t = (1 - lambda_t) dt_t exp(dt_t A_h),
+ *   gamma_t = lambda_t dt_t
+ *       ("Mamba-3" summary, b-lab.team, section 1 "Exponential-Trapezoidal
+ *        Discretization", the recurrence and the definitions below it)
+ *   R_t = blockdiag_i R(dt_t theta_t[i]),  R(phi) = [[cos phi, -sin phi],
+ *                                                    [sin phi,  cos phi]]
+ *       (same page, section 2 "Complex-Valued State Space Model",
+ *        Proposition 2)
+ *   h_t = R_t (alpha_t h_{t-1} + beta_t B_{t-1} X_{t-1}^T) + gamma_t B_t X_t^T
+ *   y_t = C_t^T h_t                         (R x P per head; section 3 "MIMO")
+ *
+ * The rotation applied to the beta term is this library's reading of the
+ * pages (they print the trapezoid and the rotation separately); it is the
+ * reading under which Proposition 3 -- the rotation moved onto B and C as a
+ * cumulative phase -- holds, and the prefill kernels rely on it.
+ *
+ * Layouts (C order, innermost index last; every tensor densely packed):
+ *   x, y    [batch][seqlen][nheads][rank][headdim]     io dtype
+ *   B, C    [batch][seqlen][ngroups][rank][dstate]     io dtype
+ *   dt, lambda [batch][seqlen][nheads]                 float32
+ *   A       [nheads]                                   float32
+ *   theta   [batch][seqlen][ngroups][dstate/2]         float32
+ *   carry:  h      [batch][nheads][dstate][headdim]    float32
+ *           prev_B [batch][nheads][rank][dstate]       io dtype
+ *           prev_x [batch][nheads][rank][headdim]      io dtype
+ * Rotary pair i is state rows (2i, 2i+1) (interleaved).  Heads of one group
+ * share B, C and theta; dt, lambda and A are per head.  The io dtype is
+ * float32 or bfloat16; arithmetic is float32 (tensor-core products take
+ * bfloat16 operands with float32 accumulation on the bfloat16 path).
+ *
+ * Ownership and threading.  Every pointer is a device pointer owned by the
+ * caller (except m3_scan_workspace_size's output and the dims/carry structs,
+ * which are host memory read during the call).  The library allocates no
+ * device memory, keeps no state between calls apart from cached device
+ * attributes, and never synchronises the stream except in m3_device_status.
+ * Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ * stream).  Calls on different streams are independent if they share no
+ * buffers.  Device pointers must be 16-byte aligned.
+ *
+ * Errors.  Argument, shape and alignment checks run on the host before any
+ * launch and return M3_ERR_INVALID_ARG / M3_ERR_UNSUPPORTED / M3_ERR_WORKSPACE
+ * with nothing enqueued.  A failed launch returns M3_ERR_CUDA.  Kernels that
+ * wait on on-chip barriers bound every wait; on expiry they record
+ * M3_ERR_DEVICE_TIMEOUT in the workspace's status word and return early,
+ * which m3_device_status reports.  No C++ exception crosses this boundary.
+ */
+#ifndef M3_H_
+#define M3_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum m3_status {
+    M3_OK = 0,
+    M3_ERR_INVALID_ARG = 1,     /* null pointer, bad size, misaligned pointer */
+    M3_ERR_UNSUPPORTED = 2,     /* valid but outside what the kernels handle  */
+    M3_ERR_WORKSPACE = 3,       /* workspace missing or smaller than required */
+    M3_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed       */
+    M3_ERR_DEVICE_TIMEOUT = 5   /* a kernel's bounded on-chip wait expired    */
+} m3_status;
+
+typedef enum m3_dtype { M3_F32 = 0, M3_BF16 = 1 } m3_dtype;
+
+typedef struct m3_dims {
+    int batch;      /* >= 0 (0 = nothing to do)                               */
+    int seqlen;     /* L >= 0 for m3_scan_fwd / m3_rope_bc; ignored by m3_step */
+    int nheads;     /* H >= 1                                                  */
+    int ngroups;    /* G >= 1, H % G == 0                                      */
+    int headdim;    /* P >= 1                                                  */
+    int dstate;     /* N >= 2, even (N/2 rotary pairs)                         */
+    int rank;       /* R >= 1 (1 = SISO)                                       */
+    int chunk;      /* Q >= 1: chunk length of the chunked prefill            */
+    int io_dtype;   /* m3_dtype of x, B, C, y, prev_B, prev_x                  */
+} m3_dims;
+
+/* The recurrent carry between calls: the state and the previous token's
+ * (B, x), which the next token's beta term needs.  In m3_scan_fwd's `init`
+ * any member may be NULL (read as zeros); in its `final_state` any member may
+ * be NULL (not written).  m3_step needs all three. */
+typedef struct m3_carry {
+    float* h;
+    void* prev_B;
+    void* prev_x;
+} m3_carry;
+
+/* Bytes of device workspace m3_scan_fwd needs for `dims` (0 is never
+ * returned: the first 256 bytes hold the status word).  Host-only. */
+m3_status m3_scan_workspace_size(const m3_dims* dims, size_t* bytes);
+
+/* Chunked prefill over a whole sequence.
+ * Computes y_t for t = 0..L-1 from the recurrence above, starting from
+ * `init` (h_{-1}, B_{-1}, x_{-1}; NULL = zeros), and writes the carry after
+ * the last token into `final_state` (h_{L-1}, B_{L-1}, x_{L-1}) if given.
+ * The chunked form follows the pages' state-space-duality view: inside a
+ * chunk the output is the product of the two-band masked matrix with X
+ * ("Mamba-3" summary, section 1, last paragraph: a decay mask times a
+ * two-band matrix), across chunks the state is passed on; with B and C
+ * rotated by their cumulative phase (section 2, Proposition 3) the rotation
+ * leaves the state recurrence.  `final_state` may alias `init`.
+ * `workspace` is device memory of at least m3_scan_workspace_size bytes,
+ * owned by the caller and zero-filled once before its first use (its first
+ * 256 bytes hold the status word that m3_device_status reads and clears);
+ * calls that share a workspace must not overlap on the device. */
+m3_status m3_scan_fwd(const m3_dims* dims,
+                      const void* x, const void* B, const void* C,
+                      const float* dt, const float* A, const float* lambda,
+                      const float* theta,
+                      const m3_carry* init,
+                      void* y, m3_carry* final_state,
+                      void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/* One decode token with carried state (the recurrence above for a single t).
+ * Per-token layouts drop the seqlen axis: x, y [batch][nheads][rank][headdim];
+ * B, C [batch][ngroups][rank][dstate]; dt, lambda [batch][nheads];
+ * theta [batch][ngroups][dstate/2].  `state` is read and updated in place
+ * (h, prev_B, prev_x all required).  dims->seqlen and dims->chunk are
+ * ignored.  No workspace: this kernel has no on-chip waits. */
+m3_status m3_step(const m3_dims* dims, m3_carry* state,
+                  const void* x, const void* B, const void* C,
+                  const float* dt, const float* A, const float* lambda,
+                  const float* theta, void* y, void* stream);
+
+/* Cumulative phase and rotated B, C ("Mamba-3" summary, section 2,
+ * Proposition 3, the "RoPE trick"):
+ *   Phi_t[i] = sum_{s <= t} dt_s theta_s[i]   (per head: dt is per head)
+ *   (B~_{2i}, B~_{2i+1}) = R(Phi_t[i])^T (B_{2i}, B_{2i+1}), same for C.
+ * Outputs B_rot, C_rot [batch][seqlen][nheads][rank][dstate] in the io dtype;
+ * `phase` [batch][seqlen][nheads][dstate/2] float32, reduced to [-pi, pi]
+ * (may be NULL).  dims->headdim and dims->chunk are ignored. */
+m3_status m3_rope_bc(const m3_dims* dims,
+                     const void* B, const void* C,
+                     const float* dt, const float* theta,
+                     void* B_rot, void* C_rot, float* phase,
+                     void* stream);
+
+/* How m3_scan_fwd will run `dims` (host-only, nothing launched): the number
+ * of kernel launches one call makes, the segments each (batch, head)
+ * sequence is cut into, the chunk length the kernels use, and the path
+ * (0 = SIMT float32, 1 = tcgen05 tensor cores).  Any output may be NULL. */
+m3_status m3_scan_plan(const m3_dims* dims, int* launches, int* segments,
+                       int* chunk_used, int* path);
+
+/* Waits for `stream`, then reads and clears the status word at the start of
+ * a workspace used by m3_scan_fwd: M3_OK, or M3_ERR_DEVICE_TIMEOUT if a
+ * bounded on-chip wait expired (that call's outputs are then invalid). */
+m3_status m3_device_status(void* workspace, void* stream);
+
+/* Static, never NULL. */
+const char* m3_status_string(m3_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* M3_H_ */

@@ -1,0 +1,192 @@
+"""B200 (sm_100a) Mamba-3 SSM layer scan -- Python binding of include/m3.h.
+
+The functions below carry the C ABI's names and only marshal arguments: they
+check tensor placement, dtype and contiguity, turn tensors into device
+pointers and call ``libm3.so`` through ctypes on the current torch stream.
+Every step of the scan runs in the library's CUDA kernels; there is no
+PyTorch or CPU implementation behind these calls, and importing the package
+fails if the library has not been built (``python -m
+selective_state_space_m3_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libm3.so")
+
+M3_OK, M3_ERR_INVALID_ARG, M3_ERR_UNSUPPORTED, M3_ERR_WORKSPACE, M3_ERR_CUDA, M3_ERR_DEVICE_TIMEOUT = range(6)
+M3_F32, M3_BF16 = 0, 1
+
+
+class M3Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {m3_status_string(status)} (status {status})")
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_int) for k in
+                ("batch", "seqlen", "nheads", "ngroups", "headdim", "dstate", "rank", "chunk",
+                 "io_dtype")]
+
+
+class _Carry(ctypes.Structure):
+    _fields_ = [("h", ctypes.c_void_p), ("prev_B", ctypes.c_void_p), ("prev_x", ctypes.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: the CUDA library must be built "
+                          "(python -m selective_state_space_m3_b200.build)")
+    lib = ctypes.CDLL(LIB_PATH)
+    V, S, I = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    D, C = ctypes.POINTER(_Dims), ctypes.POINTER(_Carry)
+    lib.m3_scan_workspace_size.argtypes = [D, ctypes.POINTER(S)]
+    lib.m3_scan_fwd.argtypes = [D, V, V, V, V, V, V, V, C, V, C, V, S, V]
+    lib.m3_step.argtypes = [D, C, V, V, V, V, V, V, V, V, V]
+    lib.m3_rope_bc.argtypes = [D, V, V, V, V, V, V, V, V]
+    lib.m3_device_status.argtypes = [V, V]
+    IP = ctypes.POINTER(I)
+    lib.m3_scan_plan.argtypes = [D, IP, IP, IP, IP]
+    lib.m3_scan_plan.restype = I
+    lib.m3_status_string.argtypes = [I]
+    lib.m3_status_string.restype = ctypes.c_char_p
+    for f in ("m3_scan_workspace_size", "m3_scan_fwd", "m3_step", "m3_rope_bc", "m3_device_status"):
+        getattr(lib, f).restype = I
+    return lib
+
+
+_lib = _load()
+
+# every symbol include/m3.h declares (checked by the CPU test suite)
+ABI_SYMBOLS = ("m3_scan_workspace_size", "m3_scan_fwd", "m3_step", "m3_rope_bc",
+               "m3_scan_plan", "m3_device_status", "m3_status_string")
+
+
+@dataclasses.dataclass
+class Dims:
+    batch: int
+    seqlen: int
+    nheads: int
+    ngroups: int
+    headdim: int
+    dstate: int
+    rank: int = 1
+    chunk: int = 64
+    io_dtype: int = M3_BF16
+
+    def c(self) -> _Dims:
+        return _Dims(self.batch, self.seqlen, self.nheads, self.ngroups, self.headdim,
+                     self.dstate, self.rank, self.chunk, self.io_dtype)
+
+
+@dataclasses.dataclass
+class Carry:
+    h: Optional[torch.Tensor] = None        # [b][h][n][p] float32
+    prev_B: Optional[torch.Tensor] = None   # [b][h][r][n] io dtype
+    prev_x: Optional[torch.Tensor] = None   # [b][h][r][p] io dtype
+
+    def c(self) -> _Carry:
+        return _Carry(_ptr(self.h), _ptr(self.prev_B), _ptr(self.prev_x))
+
+
+def io_dtype_of(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return M3_BF16
+    if t.dtype == torch.float32:
+        return M3_F32
+    raise TypeError(f"io tensors must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("m3 takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("m3 takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(status: int, what: str):
+    if status != M3_OK:
+        raise M3Error(status, what)
+
+
+def m3_status_string(status: int) -> str:
+    return _lib.m3_status_string(int(status)).decode()
+
+
+def m3_scan_workspace_size(dims: Dims) -> int:
+    n = ctypes.c_size_t(0)
+    d = dims.c()
+    _check(_lib.m3_scan_workspace_size(ctypes.byref(d), ctypes.byref(n)), "m3_scan_workspace_size")
+    return int(n.value)
+
+
+def m3_scan_plan(dims: Dims) -> dict:
+    """Host-only: launches per call, segments, chunk length used, path."""
+    d = dims.c()
+    out = [ctypes.c_int(0) for _ in range(4)]
+    _check(_lib.m3_scan_plan(ctypes.byref(d), *[ctypes.byref(o) for o in out]), "m3_scan_plan")
+    return dict(launches=out[0].value, segments=out[1].value, chunk_used=out[2].value,
+                path=("simt", "tcgen05")[out[3].value])
+
+
+def m3_scan_fwd(dims: Dims, x, B, C, dt, A, lam, theta, y, workspace,
+                init: Optional[Carry] = None, final_state: Optional[Carry] = None, stream=None) -> None:
+    """Chunked prefill (see include/m3.h).  All tensors on the device,
+    contiguous, in the ABI's layouts; ``y`` and ``final_state`` are written."""
+    d = dims.c()
+    ci = init.c() if init is not None else None
+    cf = final_state.c() if final_state is not None else None
+    st = _lib.m3_scan_fwd(ctypes.byref(d), _ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A), _ptr(lam),
+                          _ptr(theta), ctypes.byref(ci) if ci is not None else None, _ptr(y),
+                          ctypes.byref(cf) if cf is not None else None, _ptr(workspace),
+                          workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "m3_scan_fwd")
+
+
+def m3_step(dims: Dims, state: Carry, x, B, C, dt, A, lam, theta, y, stream=None) -> None:
+    """One decode token; ``state`` is updated in place."""
+    d = dims.c()
+    cs = state.c()
+    st = _lib.m3_step(ctypes.byref(d), ctypes.byref(cs), _ptr(x), _ptr(B), _ptr(C), _ptr(dt),
+                      _ptr(A), _ptr(lam), _ptr(theta), _ptr(y), _stream(stream))
+    _check(st, "m3_step")
+
+
+def m3_rope_bc(dims: Dims, B, C, dt, theta, B_rot, C_rot, phase=None, stream=None) -> None:
+    d = dims.c()
+    st = _lib.m3_rope_bc(ctypes.byref(d), _ptr(B), _ptr(C), _ptr(dt), _ptr(theta), _ptr(B_rot),
+                         _ptr(C_rot), _ptr(phase), _stream(stream))
+    _check(st, "m3_rope_bc")
+
+
+def m3_device_status(workspace, stream=None) -> int:
+    """Synchronises the stream; returns (and clears) the workspace status."""
+    return int(_lib.m3_device_status(_ptr(workspace), _stream(stream)))
+
+
+def raw_lib():
+    """The ctypes handle (for calls that pass raw pointers)."""
+    return _lib
+
+
+__all__ = ["Dims", "Carry", "M3Error", "m3_scan_workspace_size", "m3_scan_fwd", "m3_step",
+           "m3_rope_bc", "m3_scan_plan", "m3_device_status", "m3_status_string", "io_dtype_of", "ABI_SYMBOLS",
+           "M3_F32", "M3_BF16", "raw_lib", "LIB_PATH"]

@@ -1,0 +1,250 @@
+// m3_api.cu -- the C ABI of include/m3.h: argument checks, the launch plan,
+// the workspace layout and the dispatch to the kernels.
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "m3_common.cuh"
+#include "m3_kernels.h"
+
+namespace m3 {
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static m3_status check_dims(const m3_dims* d, bool need_seq) {
+    if (!d) return M3_ERR_INVALID_ARG;
+    if (d->batch < 0 || d->nheads < 1 || d->ngroups < 1 || d->headdim < 1 || d->dstate < 2 ||
+        d->rank < 1)
+        return M3_ERR_INVALID_ARG;
+    if (need_seq && (d->seqlen < 0 || d->chunk < 1)) return M3_ERR_INVALID_ARG;
+    if (d->dstate % 2 != 0 || d->nheads % d->ngroups != 0) return M3_ERR_INVALID_ARG;
+    if (d->io_dtype != M3_F32 && d->io_dtype != M3_BF16) return M3_ERR_INVALID_ARG;
+    // sizes whose element counts would overflow the kernels' 32-bit per-head indexing
+    if ((long long)d->dstate * d->headdim > (1LL << 24) || d->rank > 64 || d->dstate > 1024)
+        return M3_ERR_UNSUPPORTED;
+    return M3_OK;
+}
+
+static bool ptrs_ok(std::initializer_list<const void*> ps) {
+    for (const void* p : ps)
+        if (!p || !aligned16(p)) return false;
+    return true;
+}
+
+static bool opt_ptrs_ok(std::initializer_list<const void*> ps) {
+    for (const void* p : ps)
+        if (p && !aligned16(p)) return false;
+    return true;
+}
+
+static size_t io_bytes(const m3_dims& d) { return d.io_dtype == M3_BF16 ? 2 : 4; }
+
+// ---------------------------------------------------------------- plan --
+struct Plan {
+    int qs;      // chunk length the kernel uses
+    int nseg;    // segments per (b, h)
+    int cps;     // chunks per segment
+};
+
+static int env_int(const char* name, int dflt) {
+    const char* v = getenv(name);
+    if (!v || !*v) return dflt;
+    return atoi(v);
+}
+
+// SIMT path: the kernel keeps one chunk of rotated B, C, X, the masked Gram
+// and the state in shared memory, so the chunk it uses is the caller's chunk
+// when that fits, else halved until it does (the chunked result does not
+// depend on the chunk length except through rounding).
+static m3_status make_plan(const m3_dims& d, Plan* pl) {
+    const size_t kMaxSmem = 200 * 1024;
+    int qs = d.chunk;
+    if (d.seqlen > 0 && qs > d.seqlen) qs = d.seqlen;
+    while (qs > 1 && simt_smem_bytes(qs, d.rank, d.dstate, d.headdim, false) > kMaxSmem) qs = (qs + 1) / 2;
+    if (simt_smem_bytes(qs, d.rank, d.dstate, d.headdim, false) > kMaxSmem) return M3_ERR_UNSUPPORTED;
+    const long long nchunks = d.seqlen > 0 ? (d.seqlen + qs - 1) / qs : 0;
+    const long long units = (long long)d.batch * d.nheads;
+    int nseg = 1;
+    // enough independent segments to fill the GPU twice over, at >= 2 chunks each
+    if (units > 0 && nchunks >= 4) {
+        long long want = (2 * 148 + units - 1) / units;
+        long long cap = nchunks / 2;
+        nseg = (int)(want < cap ? want : cap);
+        if (nseg < 1) nseg = 1;
+    }
+    const int forced = env_int("M3_SCAN_NSEG", 0);   // tuning / test knob
+    if (forced > 0) nseg = (int)(forced < nchunks ? forced : (nchunks > 0 ? nchunks : 1));
+    int cps = nchunks > 0 ? (int)((nchunks + nseg - 1) / nseg) : 1;
+    if (nchunks > 0) nseg = (int)((nchunks + cps - 1) / cps);   // drop empty segments
+    pl->qs = qs;
+    pl->nseg = nseg;
+    pl->cps = cps;
+    return M3_OK;
+}
+
+struct WsLayout {
+    size_t sloc, decay, phase, sin, total;
+};
+
+static size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static WsLayout ws_layout(const m3_dims& d, const Plan& pl) {
+    WsLayout w;
+    size_t off = kWorkspaceHeaderBytes;
+    const size_t units = (size_t)d.batch * d.nheads * (pl.nseg > 1 ? pl.nseg : 0);
+    const size_t NP = (size_t)d.dstate * d.headdim;
+    w.sloc = off;  off = round256(off + units * NP * sizeof(float));
+    w.decay = off; off = round256(off + units * sizeof(float));
+    w.phase = off; off = round256(off + units * (d.dstate / 2) * sizeof(float));
+    w.sin = off;   off = round256(off + units * NP * sizeof(float));
+    w.total = off;
+    return w;
+}
+
+}  // namespace m3
+
+using namespace m3;
+
+extern "C" {
+
+const char* m3_status_string(m3_status s) {
+    switch (s) {
+        case M3_OK: return "ok";
+        case M3_ERR_INVALID_ARG: return "invalid argument (null, misaligned or bad size)";
+        case M3_ERR_UNSUPPORTED: return "shape not supported by the kernels";
+        case M3_ERR_WORKSPACE: return "workspace missing or too small";
+        case M3_ERR_CUDA: return "CUDA runtime error";
+        case M3_ERR_DEVICE_TIMEOUT: return "a bounded on-chip wait expired on the device";
+    }
+    return "unknown status";
+}
+
+m3_status m3_scan_workspace_size(const m3_dims* d, size_t* bytes) {
+    if (!bytes) return M3_ERR_INVALID_ARG;
+    m3_status s = check_dims(d, true);
+    if (s != M3_OK) return s;
+    Plan pl;
+    s = make_plan(*d, &pl);
+    if (s != M3_OK) return s;
+    *bytes = ws_layout(*d, pl).total;
+    return M3_OK;
+}
+
+m3_status m3_scan_plan(const m3_dims* d, int* launches, int* segments, int* chunk_used, int* path) {
+    m3_status s = check_dims(d, true);
+    if (s != M3_OK) return s;
+    Plan pl;
+    s = make_plan(*d, &pl);
+    if (s != M3_OK) return s;
+    const bool work = d->batch > 0 && d->seqlen > 0;
+    if (launches) *launches = work ? (pl.nseg > 1 ? 3 : 1) : 0;
+    if (segments) *segments = pl.nseg;
+    if (chunk_used) *chunk_used = pl.qs;
+    if (path) *path = 0;
+    return M3_OK;
+}
+
+m3_status m3_scan_fwd(const m3_dims* d, const void* x, const void* B, const void* C, const float* dt,
+                      const float* A, const float* lambda, const float* theta, const m3_carry* init,
+                      void* y, m3_carry* fin, void* workspace, size_t ws_bytes, void* stream) {
+    m3_status s = check_dims(d, true);
+    if (s != M3_OK) return s;
+    const bool work = d->batch > 0 && d->seqlen > 0;
+    if (work && !ptrs_ok({x, B, C, dt, A, lambda, theta, y})) return M3_ERR_INVALID_ARG;
+    if (init && !opt_ptrs_ok({init->h, init->prev_B, init->prev_x})) return M3_ERR_INVALID_ARG;
+    if (fin && !opt_ptrs_ok({fin->h, fin->prev_B, fin->prev_x})) return M3_ERR_INVALID_ARG;
+    Plan pl;
+    s = make_plan(*d, &pl);
+    if (s != M3_OK) return s;
+    const WsLayout w = ws_layout(*d, pl);
+    if (!workspace || !aligned16(workspace) || ws_bytes < w.total) return M3_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t NP = (size_t)d->dstate * d->headdim;
+    const size_t units = (size_t)d->batch * d->nheads;
+
+    if (!work) {
+        // no tokens: the carry passes through unchanged
+        if (fin && d->batch > 0) {
+            const size_t hb = units * NP * sizeof(float);
+            const size_t bb = units * d->rank * d->dstate * io_bytes(*d);
+            const size_t xb = units * d->rank * d->headdim * io_bytes(*d);
+            cudaError_t e = cudaSuccess;
+            if (fin->h)
+                e = (init && init->h) ? cudaMemcpyAsync(fin->h, init->h, hb, cudaMemcpyDeviceToDevice, st)
+                                      : cudaMemsetAsync(fin->h, 0, hb, st);
+            if (e == cudaSuccess && fin->prev_B)
+                e = (init && init->prev_B)
+                        ? cudaMemcpyAsync(fin->prev_B, init->prev_B, bb, cudaMemcpyDeviceToDevice, st)
+                        : cudaMemsetAsync(fin->prev_B, 0, bb, st);
+            if (e == cudaSuccess && fin->prev_x)
+                e = (init && init->prev_x)
+                        ? cudaMemcpyAsync(fin->prev_x, init->prev_x, xb, cudaMemcpyDeviceToDevice, st)
+                        : cudaMemsetAsync(fin->prev_x, 0, xb, st);
+            if (e != cudaSuccess) return M3_ERR_CUDA;
+        }
+        return M3_OK;
+    }
+
+    ScanParams q;
+    memset(&q, 0, sizeof(q));
+    q.batch = d->batch; q.seqlen = d->seqlen; q.nheads = d->nheads; q.ngroups = d->ngroups;
+    q.headdim = d->headdim; q.dstate = d->dstate; q.rank = d->rank;
+    q.qs = pl.qs; q.nseg = pl.nseg; q.cps = pl.cps;
+    q.x = x; q.B = B; q.C = C; q.dt = dt; q.A = A; q.lam = lambda; q.theta = theta;
+    if (init) { q.init_h = init->h; q.init_pB = init->prev_B; q.init_pX = init->prev_x; }
+    q.y = y;
+    if (fin) { q.fin_h = fin->h; q.fin_pB = fin->prev_B; q.fin_pX = fin->prev_x; }
+    char* ws = static_cast<char*>(workspace);
+    q.ws_sloc = reinterpret_cast<float*>(ws + w.sloc);
+    q.ws_decay = reinterpret_cast<float*>(ws + w.decay);
+    q.ws_phase = reinterpret_cast<float*>(ws + w.phase);
+    q.ws_sin = reinterpret_cast<float*>(ws + w.sin);
+    cudaError_t e = launch_scan_simt(*d, q, st);
+    return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+m3_status m3_step(const m3_dims* d, m3_carry* state, const void* x, const void* B, const void* C,
+                  const float* dt, const float* A, const float* lambda, const float* theta, void* y,
+                  void* stream) {
+    m3_status s = check_dims(d, false);
+    if (s != M3_OK) return s;
+    if (!state) return M3_ERR_INVALID_ARG;
+    if (d->batch > 0 &&
+        !ptrs_ok({state->h, state->prev_B, state->prev_x, x, B, C, dt, A, lambda, theta, y}))
+        return M3_ERR_INVALID_ARG;
+    StepParams q;
+    q.batch = d->batch; q.nheads = d->nheads; q.ngroups = d->ngroups;
+    q.headdim = d->headdim; q.dstate = d->dstate;
+    q.h = state->h; q.prev_B = state->prev_B; q.prev_x = state->prev_x;
+    q.x = x; q.B = B; q.C = C; q.dt = dt; q.A = A; q.lam = lambda; q.theta = theta; q.y = y;
+    return launch_step(*d, q, (cudaStream_t)stream);
+}
+
+m3_status m3_rope_bc(const m3_dims* d, const void* B, const void* C, const float* dt, const float* theta,
+                     void* B_rot, void* C_rot, float* phase, void* stream) {
+    m3_status s = check_dims(d, false);
+    if (s != M3_OK) return s;
+    if (d->seqlen < 0) return M3_ERR_INVALID_ARG;
+    if (d->batch > 0 && d->seqlen > 0 && !ptrs_ok({B, C, dt, theta, B_rot, C_rot}))
+        return M3_ERR_INVALID_ARG;
+    if (!opt_ptrs_ok({phase})) return M3_ERR_INVALID_ARG;
+    RopeParams q;
+    q.batch = d->batch; q.seqlen = d->seqlen; q.nheads = d->nheads; q.ngroups = d->ngroups;
+    q.dstate = d->dstate; q.rank = d->rank;
+    q.B = B; q.C = C; q.dt = dt; q.theta = theta; q.B_rot = B_rot; q.C_rot = C_rot; q.phase = phase;
+    return launch_rope(*d, q, (cudaStream_t)stream);
+}
+
+m3_status m3_device_status(void* workspace, void* stream) {
+    if (!workspace) return M3_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return M3_ERR_CUDA;
+    WorkspaceHeader hdr;
+    if (cudaMemcpy(&hdr, workspace, sizeof(hdr), cudaMemcpyDeviceToHost) != cudaSuccess) return M3_ERR_CUDA;
+    if (hdr.status != 0) {
+        if (cudaMemset(workspace, 0, sizeof(hdr)) != cudaSuccess) return M3_ERR_CUDA;
+        return (m3_status)hdr.status;
+    }
+    return M3_OK;
+}
+
+}  // extern "C"

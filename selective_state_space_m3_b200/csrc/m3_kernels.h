@@ -1,0 +1,68 @@
+// m3_kernels.h -- launch parameters and host launchers of the scan, step
+// and rope kernels (internal to the library; the public ABI is include/m3.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "../../include/m3.h"
+
+namespace m3 {
+
+struct StepParams {
+    int batch, nheads, ngroups, headdim, dstate;
+    float* h;            // [b][h][n][p] fp32, in/out
+    void* prev_B;        // [b][h][r][n] io, in/out
+    void* prev_x;        // [b][h][r][p] io, in/out
+    const void* x;       // [b][h][r][p] io
+    const void* B;       // [b][g][r][n] io
+    const void* C;       // [b][g][r][n] io
+    const float* dt;     // [b][h]
+    const float* A;      // [h]
+    const float* lam;    // [b][h]
+    const float* theta;  // [b][g][n/2]
+    void* y;             // [b][h][r][p] io
+};
+
+struct RopeParams {
+    int batch, seqlen, nheads, ngroups, dstate, rank;
+    const void* B;        // [b][t][g][r][n]
+    const void* C;
+    const float* dt;      // [b][t][h]
+    const float* theta;   // [b][t][g][n/2]
+    void* B_rot;          // [b][t][h][r][n]
+    void* C_rot;
+    float* phase;         // [b][t][h][n/2] or null
+};
+
+struct ScanParams {
+    int batch, seqlen, nheads, ngroups, headdim, dstate, rank;
+    int qs;      // chunk length the kernel uses (tokens)
+    int nseg;    // segments per (b, h)
+    int cps;     // chunks per segment
+    const void* x;
+    const void* B;
+    const void* C;
+    const float* dt;
+    const float* A;
+    const float* lam;
+    const float* theta;
+    const float* init_h;
+    const void* init_pB;
+    const void* init_pX;
+    void* y;
+    float* fin_h;
+    void* fin_pB;
+    void* fin_pX;
+    float* ws_sloc;    // [b][h][seg][N][P]
+    float* ws_decay;   // [b][h][seg]
+    float* ws_phase;   // [b][h][seg][N/2]
+    float* ws_sin;     // [b][h][seg][N][P]
+};
+
+m3_status launch_step(const m3_dims& d, const StepParams& q, cudaStream_t st);
+m3_status launch_rope(const m3_dims& d, const RopeParams& q, cudaStream_t st);
+size_t simt_smem_bytes(int qs, int R, int N, int P, bool summary);
+cudaError_t launch_scan_simt(const m3_dims& d, const ScanParams& q, cudaStream_t st);
+
+}  // namespace m3

@@ -1,0 +1,130 @@
+"""CPU checks of the C ABI (no GPU, no kernel launches).
+
+* libm3.so loads and exports every function include/m3.h declares.
+* Host-side validation returns its status before anything is enqueued: the
+  pointers passed here are never dereferenced (bad sizes, misalignment and
+  small workspaces are all rejected first).
+* The workspace-size query is host-only.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import selective_state_space_m3_b200 as m3
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "m3.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(m3_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_abi():
+    assert set(declared_functions()) == set(m3.ABI_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(m3.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", m3.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(m3_[a-z0-9_]+)$", out, flags=re.M))
+    assert set(declared_functions()) <= exported
+
+
+def test_status_strings():
+    for s in range(6):
+        assert m3.m3_status_string(s)
+    assert m3.m3_status_string(99) == "unknown status"
+
+
+LIB = m3.raw_lib()
+GOOD = 0x10000          # 16-byte aligned fake device addresses (never touched)
+BAD = 0x10008
+
+
+def dims(**kw):
+    base = dict(batch=2, seqlen=64, nheads=4, ngroups=2, headdim=16, dstate=16, rank=2, chunk=16,
+                io_dtype=m3.M3_BF16)
+    base.update(kw)
+    return m3.Dims(**base)
+
+
+def scan_status(d, ptr=GOOD, ws=GOOD, ws_bytes=1 << 30, y=GOOD, init=None, fin=None):
+    cd = d.c()
+    return LIB.m3_scan_fwd(ctypes.byref(cd), ptr, ptr, ptr, ptr, ptr, ptr, ptr,
+                           ctypes.byref(init) if init is not None else None, y,
+                           ctypes.byref(fin) if fin is not None else None, ws, ws_bytes, None)
+
+
+def test_workspace_size_is_host_only_and_positive():
+    n = m3.m3_scan_workspace_size(dims())
+    assert n >= 256 and n % 256 == 0
+    n2 = m3.m3_scan_workspace_size(dims(batch=1, nheads=1, ngroups=1, seqlen=4096))
+    assert n2 > 256          # a long single sequence is split into segments
+
+
+@pytest.mark.parametrize("bad", [
+    dict(dstate=15), dict(nheads=3, ngroups=2), dict(batch=-1), dict(seqlen=-1), dict(rank=0),
+    dict(headdim=0), dict(chunk=0), dict(io_dtype=7), dict(ngroups=0),
+])
+def test_scan_rejects_bad_dims(bad):
+    assert scan_status(dims(**bad)) == m3.M3_ERR_INVALID_ARG
+
+
+def test_scan_rejects_null_and_misaligned_pointers():
+    assert scan_status(dims(), ptr=0) == m3.M3_ERR_INVALID_ARG
+    assert scan_status(dims(), ptr=BAD) == m3.M3_ERR_INVALID_ARG
+    assert scan_status(dims(), y=BAD) == m3.M3_ERR_INVALID_ARG
+    bad_carry = m3._Carry(BAD, None, None)
+    assert scan_status(dims(), init=bad_carry) == m3.M3_ERR_INVALID_ARG
+    assert scan_status(dims(), fin=bad_carry) == m3.M3_ERR_INVALID_ARG
+
+
+def test_scan_rejects_small_or_missing_workspace():
+    need = m3.m3_scan_workspace_size(dims())
+    assert scan_status(dims(), ws_bytes=need - 1) == m3.M3_ERR_WORKSPACE
+    assert scan_status(dims(), ws=0) == m3.M3_ERR_WORKSPACE
+    assert scan_status(dims(), ws=BAD) == m3.M3_ERR_WORKSPACE
+
+
+def test_unsupported_sizes():
+    n = ctypes.c_size_t(0)
+    cd = dims(dstate=2048).c()
+    assert LIB.m3_scan_workspace_size(ctypes.byref(cd), ctypes.byref(n)) == m3.M3_ERR_UNSUPPORTED
+
+
+def test_step_rejects_bad_arguments():
+    d = dims().c()
+    good = m3._Carry(GOOD, GOOD, GOOD)
+    args = [GOOD] * 8
+    assert LIB.m3_step(ctypes.byref(d), None, *args, None) == m3.M3_ERR_INVALID_ARG
+    assert LIB.m3_step(ctypes.byref(d), ctypes.byref(m3._Carry(GOOD, None, GOOD)), *args,
+                       None) == m3.M3_ERR_INVALID_ARG
+    assert LIB.m3_step(ctypes.byref(d), ctypes.byref(m3._Carry(BAD, GOOD, GOOD)), *args,
+                       None) == m3.M3_ERR_INVALID_ARG
+    d_odd = dims(dstate=9).c()
+    assert LIB.m3_step(ctypes.byref(d_odd), ctypes.byref(good), *args, None) == m3.M3_ERR_INVALID_ARG
+    d_bad_p = dims(headdim=12).c()      # P/4 = 3: not a power of two
+    assert LIB.m3_step(ctypes.byref(d_bad_p), ctypes.byref(good), *args, None) == m3.M3_ERR_UNSUPPORTED
+
+
+def test_rope_rejects_bad_arguments():
+    d = dims().c()
+    assert LIB.m3_rope_bc(ctypes.byref(d), GOOD, 0, GOOD, GOOD, GOOD, GOOD, None,
+                          None) == m3.M3_ERR_INVALID_ARG
+    assert LIB.m3_rope_bc(ctypes.byref(d), GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, BAD,
+                          None) == m3.M3_ERR_INVALID_ARG
+
+
+def test_null_dims():
+    n = ctypes.c_size_t(0)
+    assert LIB.m3_scan_workspace_size(None, ctypes.byref(n)) == m3.M3_ERR_INVALID_ARG
+    assert LIB.m3_device_status(None, None) == m3.M3_ERR_INVALID_ARG

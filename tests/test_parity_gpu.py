@@ -1,0 +1,271 @@
+"""Parity of the CUDA path with the fp64 oracle (needs a B200).
+
+Every case draws seeded inputs from m3_synth, runs the library through its
+C ABI (the Python binding), runs the oracle on the same stored values, and
+compares element by element: relative L2 within the workload table's bound
+(1e-4 for float32 io, 2e-2 for bfloat16 io with float32 accumulation), with
+the per-element max-abs difference reported.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import m3_synth
+import oracle
+from tests._util import dims_of, empty_carry, f64, gpu_scan, max_abs, rel_l2, slice_bh, tol_for
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import selective_state_space_m3_b200 as m3
+
+
+def _oracle_full(inp, init=None):
+    args = {k: f64(v) for k, v in inp.items()}
+    kw = {}
+    if init is not None:
+        kw = dict(init_h=f64(init.h), init_pB=f64(init.prev_B), init_pX=f64(init.prev_x))
+    return oracle.scan(**args, **kw)
+
+
+def _check(name, got, want, tol):
+    r = rel_l2(got, want)
+    print(f"{name}: rel_l2={r:.3e} max_abs={max_abs(got, want):.3e}")
+    assert np.all(np.isfinite(np.asarray(got, np.float64))), name
+    assert r <= tol, f"{name}: rel_l2 {r:.3e} > {tol:.1e}"
+
+
+# ------------------------------------------------------------ small cases --
+SMALL = [
+    # shape, id  -- span several chunks and a ragged tail
+    (m3_synth.ScanShape(1, 256, 1, 1, 16, 16, 1, 32, "f32", 0.0, 0), "cfg0_full"),
+    (m3_synth.ScanShape(2, 300, 4, 2, 16, 16, 2, 32, "f32", 0.0, 11), "f32_mimo_ragged"),
+    (m3_synth.ScanShape(2, 333, 4, 2, 64, 128, 1, 64, "bf16", 0.0, 12), "bf16_siso_ragged"),
+    (m3_synth.ScanShape(1, 200, 3, 3, 64, 128, 4, 64, "bf16", 0.0, 13), "bf16_mimo_r4"),
+    (m3_synth.ScanShape(2, 260, 8, 1, 64, 128, 1, 64, "bf16", 0.0, 14), "bf16_shared_group"),
+    (m3_synth.ScanShape(1, 520, 2, 2, 64, 128, 1, 128, "bf16", -1.0, 15), "bf16_long_dt"),
+]
+
+
+@pytest.mark.parametrize("shape,name", SMALL, ids=[n for _, n in SMALL])
+def test_scan_matches_oracle(shape, name):
+    inp = m3_synth.make_scan_inputs(shape)
+    y, fin = gpu_scan(shape, inp)
+    yo, ho, pBo, pXo = _oracle_full(inp)
+    tol = tol_for(shape.dtype)
+    _check(f"{name} y", f64(y), yo, tol)
+    _check(f"{name} h", f64(fin.h), ho, tol)
+    assert np.array_equal(f64(fin.prev_B), pBo)      # exact copies of stored inputs
+    assert np.array_equal(f64(fin.prev_x), pXo)
+
+
+@pytest.mark.parametrize("nseg", [1, 2, 3, 7])
+def test_scan_segment_split_matches_oracle(nseg, monkeypatch):
+    """The multi-segment path (summary, combine, main) against the oracle."""
+    monkeypatch.setenv("M3_SCAN_NSEG", str(nseg))
+    shape = m3_synth.ScanShape(2, 290, 2, 1, 16, 16, 2, 16, "f32", 0.0, 21)
+    inp = m3_synth.make_scan_inputs(shape)
+    init = m3_synth.make_carry(2, 2, 16, 16, 2, "f32", 21)
+    init = m3.Carry(init["h"].cuda(), init["prev_B"].cuda(), init["prev_x"].cuda())
+    y, fin = gpu_scan(shape, inp, init=init)
+    yo, ho, _, _ = _oracle_full(inp, init)
+    _check(f"nseg{nseg} y", f64(y), yo, 1e-4)
+    _check(f"nseg{nseg} h", f64(fin.h), ho, 1e-4)
+
+
+def test_scan_with_initial_carry_bf16():
+    shape = m3_synth.ScanShape(2, 190, 4, 4, 64, 128, 4, 64, "bf16", 0.0, 22)
+    inp = m3_synth.make_scan_inputs(shape)
+    c = m3_synth.make_carry(2, 4, 128, 64, 4, "bf16", 22, scale=0.3)
+    init = m3.Carry(c["h"].cuda(), c["prev_B"].cuda(), c["prev_x"].cuda())
+    y, fin = gpu_scan(shape, inp, init=init)
+    yo, ho, _, _ = _oracle_full(inp, init)
+    _check("carry y", f64(y), yo, 2e-2)
+    _check("carry h", f64(fin.h), ho, 2e-2)
+
+
+def test_split_sequence_equals_single_call():
+    """scan(L1) then scan(L - L1) through the carry equals scan(L)."""
+    shape = m3_synth.ScanShape(1, 400, 2, 2, 64, 128, 2, 64, "bf16", 0.0, 23)
+    inp = m3_synth.make_scan_inputs(shape)
+    y, fin = gpu_scan(shape, inp)
+    L1 = 150
+    s1 = m3_synth.shrink(shape, seqlen=L1)
+    s2 = m3_synth.shrink(shape, seqlen=400 - L1)
+    i1 = {k: (v[:, :L1].contiguous() if k != "A" else v) for k, v in inp.items()}
+    i2 = {k: (v[:, L1:].contiguous() if k != "A" else v) for k, v in inp.items()}
+    ya, fa = gpu_scan(s1, i1)
+    yb, fb = gpu_scan(s2, i2, init=fa)
+    yo, ho, _, _ = _oracle_full(inp)
+    _check("split y", np.concatenate([f64(ya), f64(yb)], axis=1), yo, 2e-2)
+    _check("split h", f64(fb.h), ho, 2e-2)
+    _check("split vs single y", np.concatenate([f64(ya), f64(yb)], axis=1), f64(y), 2e-2)
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64, 128])
+def test_chunk_length_does_not_change_the_result(chunk):
+    shape = m3_synth.ScanShape(1, 256, 2, 2, 16, 16, 1, 32, "f32", 0.0, 24)
+    inp = m3_synth.make_scan_inputs(shape)
+    y, fin = gpu_scan(shape, inp, chunk=chunk)
+    yo, ho, _, _ = _oracle_full(inp)
+    _check(f"chunk{chunk} y", f64(y), yo, 1e-4)
+    _check(f"chunk{chunk} h", f64(fin.h), ho, 1e-4)
+
+
+def test_empty_sequence_passes_the_carry_through():
+    shape = m3_synth.ScanShape(2, 0, 2, 1, 16, 16, 1, 32, "f32", 0.0, 25)
+    d = dims_of(shape)
+    c = m3_synth.make_carry(2, 2, 16, 16, 1, "f32", 25)
+    init = m3.Carry(c["h"].cuda(), c["prev_B"].cuda(), c["prev_x"].cuda())
+    fin = empty_carry(shape)
+    ws = torch.zeros(m3.m3_scan_workspace_size(d), dtype=torch.uint8, device="cuda")
+    z = torch.empty(0, device="cuda")
+    m3.m3_scan_fwd(d, z, z, z, z, torch.zeros(2, device="cuda"), z, z, z, ws, init=init, final_state=fin)
+    torch.cuda.synchronize()
+    assert torch.equal(fin.h, init.h) and torch.equal(fin.prev_B, init.prev_B)
+    # batch 0: nothing to do, no error
+    d0 = dims_of(m3_synth.shrink(shape, batch=0, seqlen=10))
+    m3.m3_scan_fwd(d0, z, z, z, z, z, z, z, z, ws)
+
+
+def test_single_token_sequence():
+    shape = m3_synth.ScanShape(3, 1, 2, 2, 64, 128, 4, 64, "bf16", 0.0, 26)
+    inp = m3_synth.make_scan_inputs(shape)
+    y, fin = gpu_scan(shape, inp)
+    yo, ho, _, _ = _oracle_full(inp)
+    _check("L1 y", f64(y), yo, 2e-2)
+    _check("L1 h", f64(fin.h), ho, 2e-2)
+
+
+# ------------------------------------------------------------------ rope --
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_rope_bc_matches_oracle(dtype):
+    shape = m3_synth.ScanShape(2, 300, 4, 2, 16, 32, 2, 32, dtype, 0.0, 31)
+    inp = m3_synth.make_scan_inputs(shape)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    d = dims_of(shape)
+    io = dev["B"].dtype
+    Bo = torch.empty((2, 300, 4, 2, 32), device="cuda", dtype=io)
+    Co = torch.empty_like(Bo)
+    ph = torch.empty((2, 300, 4, 16), device="cuda", dtype=torch.float32)
+    m3.m3_rope_bc(d, dev["B"], dev["C"], dev["dt"], dev["theta"], Bo, Co, ph)
+    torch.cuda.synchronize()
+    Bw, Cw, Pw = oracle.rope_bc(f64(inp["B"]), f64(inp["C"]), f64(inp["dt"]), f64(inp["theta"]), nheads=4)
+    tol = 1e-5 if dtype == "f32" else 2e-2
+    _check("rope B", f64(Bo), Bw, tol)
+    _check("rope C", f64(Co), Cw, tol)
+    ang = np.angle(np.exp(1j * (f64(ph) - Pw)))
+    print(f"rope phase max angular error {np.max(np.abs(ang)):.3e}")
+    assert np.max(np.abs(ang)) < 1e-5
+    assert np.max(np.abs(f64(ph))) <= np.pi + 1e-6
+
+
+# ------------------------------------------------------------------ step --
+@pytest.mark.parametrize("dtype,R", [("f32", 1), ("f32", 2), ("bf16", 4), ("bf16", 1), ("bf16", 8)])
+def test_step_matches_oracle(dtype, R):
+    dec = m3_synth.DecodeShape(batch=3, nheads=4, ngroups=2, headdim=64 if dtype == "bf16" else 16,
+                               dstate=128 if dtype == "bf16" else 16, rank=R, steps=12, dtype=dtype, seed=40 + R)
+    c = m3_synth.make_carry(3, 4, dec.dstate, dec.headdim, R, dtype, 40 + R, scale=0.5)
+    state = m3.Carry(c["h"].cuda(), c["prev_B"].cuda(), c["prev_x"].cuda())
+    A = -torch.exp(torch.linspace(-2, 1, 4))
+    Ad = A.cuda()
+    h, pB, pX = f64(c["h"]), f64(c["prev_B"]), f64(c["prev_x"])
+    d = m3.Dims(3, 1, 4, 2, dec.headdim, dec.dstate, R, 1, m3.M3_BF16 if dtype == "bf16" else m3.M3_F32)
+    tol = 1e-5 if dtype == "f32" else 2e-2
+    for k in range(dec.steps):
+        tok = m3_synth.make_decode_token(dec, k)
+        dv = {n: v.cuda() for n, v in tok.items()}
+        y = torch.empty_like(dv["x"])
+        m3.m3_step(d, state, dv["x"], dv["B"], dv["C"], dv["dt"], Ad, dv["lam"], dv["theta"], y)
+        yo, h, pB, pX = oracle.step(h, pB, pX, f64(tok["x"]), f64(tok["B"]), f64(tok["C"]),
+                                    f64(tok["dt"]), f64(A), f64(tok["lam"]), f64(tok["theta"]))
+        torch.cuda.synchronize()
+        _check(f"step{k} y", f64(y), yo, tol)
+    _check("step h", f64(state.h), h, 1e-4 if dtype == "bf16" else 1e-5)
+    assert np.array_equal(f64(state.prev_B), pB) and np.array_equal(f64(state.prev_x), pX)
+
+
+def test_scan_then_steps_equals_longer_scan():
+    shape = m3_synth.ScanShape(2, 100, 2, 2, 64, 128, 4, 64, "bf16", 0.0, 50)
+    inp = m3_synth.make_scan_inputs(shape)
+    L0 = 90
+    s0 = m3_synth.shrink(shape, seqlen=L0)
+    i0 = {k: (v[:, :L0].contiguous() if k != "A" else v) for k, v in inp.items()}
+    _, state = gpu_scan(s0, i0)
+    d = dims_of(shape)
+    ys = []
+    for t in range(L0, 100):
+        tok = {k: inp[k][:, t].contiguous().cuda() for k in ("x", "B", "C", "dt", "lam", "theta")}
+        y = torch.empty_like(tok["x"])
+        m3.m3_step(d, state, tok["x"], tok["B"], tok["C"], tok["dt"], inp["A"].cuda(), tok["lam"],
+                   tok["theta"], y)
+        ys.append(f64(y))
+    torch.cuda.synchronize()
+    yo, ho, _, _ = _oracle_full(inp)
+    _check("scan+steps y", np.stack(ys, axis=1), yo[:, L0:], 2e-2)
+    _check("scan+steps h", f64(state.h), ho, 2e-2)
+
+
+# ----------------------------------------------- full-size, sampled outputs --
+def _sampled_full(cfg, samples):
+    shape = m3_synth.CONFIGS[cfg]
+    inp = m3_synth.make_scan_inputs(shape)
+    y, fin = gpu_scan(shape, inp)
+    tol = tol_for(shape.dtype)
+    for (b, h) in samples:
+        one = slice_bh(inp, shape, b, h)
+        yo, ho, _, _ = oracle.scan(**one)
+        _check(f"cfg{cfg} b{b} h{h} y", f64(y[b:b + 1, :, h:h + 1]), yo, tol)
+        _check(f"cfg{cfg} b{b} h{h} h", f64(fin.h[b:b + 1, h:h + 1]), ho, tol)
+
+
+def test_config0_full_size():
+    _sampled_full(0, [(0, 0)])
+
+
+def test_config1_full_size_sampled():
+    _sampled_full(1, [(0, 0), (1, 5), (3, 7)])
+
+
+def test_config2_full_size_sampled():
+    _sampled_full(2, [(0, 0), (3, 17), (7, 31)])
+
+
+def test_config3_full_size_sampled():
+    _sampled_full(3, [(0, 0), (0, 21)])
+
+
+def test_config4_decode_full_batch_sampled():
+    """Decode at the full batch (256 sequences, 32 heads, R=4) for 32 tokens,
+    from the oracle's final carry of config 2's first batch row (tiled over
+    the 256 sequences), sampled sequences compared with the oracle."""
+    dec = m3_synth.DECODE
+    c2 = m3_synth.CONFIGS[2]
+    inp2 = m3_synth.make_scan_inputs(c2)
+    one = {k: f64(v[0:1]) if k != "A" else f64(v) for k, v in inp2.items()}
+    _, h0, pB0, pX0 = oracle.scan(**one)                       # [1][32][...]
+    reps = dec.batch
+    state = m3.Carry(torch.from_numpy(np.repeat(h0, reps, 0).astype(np.float32)).cuda(),
+                     torch.from_numpy(np.repeat(pB0, reps, 0).astype(np.float32)).to(torch.bfloat16).cuda(),
+                     torch.from_numpy(np.repeat(pX0, reps, 0).astype(np.float32)).to(torch.bfloat16).cuda())
+    A = inp2["A"]
+    d = m3.Dims(dec.batch, 1, dec.nheads, dec.ngroups, dec.headdim, dec.dstate, dec.rank, 1, m3.M3_BF16)
+    sample = list(range(0, dec.batch, 32))
+    h = np.repeat(h0, len(sample), 0)
+    pB = np.repeat(pB0, len(sample), 0)
+    pX = np.repeat(pX0, len(sample), 0)
+    hstate_f32 = f64(state.h)[sample]
+    h = hstate_f32                                         # the fp32-stored carry both sides start from
+    for k in range(32):
+        tok = m3_synth.make_decode_token(dec, k)
+        dv = {n: v.cuda() for n, v in tok.items()}
+        y = torch.empty_like(dv["x"])
+        m3.m3_step(d, state, dv["x"], dv["B"], dv["C"], dv["dt"], A.cuda(), dv["lam"], dv["theta"], y)
+        sub = {n: f64(v[sample]) for n, v in tok.items()}
+        yo, h, pB, pX = oracle.step(h, pB, pX, sub["x"], sub["B"], sub["C"], sub["dt"], f64(A),
+                                    sub["lam"], sub["theta"])
+        torch.cuda.synchronize()
+        _check(f"decode t{k} y", f64(y)[sample], yo, 2e-2)
+    _check("decode h", f64(state.h)[sample], h, 2e-2)
