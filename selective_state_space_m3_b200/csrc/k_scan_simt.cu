@@ -269,6 +269,13 @@ static cudaError_t launch_simt_T(const ScanParams& q, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+// the combine step on its own (used by the tensor-core path, bf16 carry)
+cudaError_t launch_scan_combine(const ScanParams& q, cudaStream_t st) {
+    const int NHP = q.dstate / 2 * q.headdim;
+    scan_combine_kernel<__nv_bfloat16><<<dim3((NHP + 255) / 256, q.nheads, q.batch), 256, 0, st>>>(q);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_scan_simt(const m3_dims& d, const ScanParams& q, cudaStream_t st) {
     return d.io_dtype == M3_BF16 ? launch_simt_T<__nv_bfloat16>(q, st) : launch_simt_T<float>(q, st);
 }

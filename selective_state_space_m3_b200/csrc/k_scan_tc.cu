@@ -1,0 +1,710 @@
+// k_scan_tc.cu -- chunked prefill of the Mamba-3 SSM layer on the sm_100a
+// tensor cores (tcgen05 + TMEM + TMA), bfloat16 io, N = 128, P = 64.
+//
+// Same chunked algebra as the SIMT path (k_scan_simt.cu, and the header of
+// that file): with B and C rotated by their cumulative phase ("Mamba-3"
+// summary, b-lab.team, section 2, Proposition 3) the recurrence inside a
+// chunk is the two-band masked matrix of section 1, and the state is passed
+// between chunks.  Here a chunk is one 128-row tile (T = 128 / R tokens x R
+// ranks), the size of one UMMA M=128 operand; the result does not depend on
+// the chunk length except through rounding.
+//
+// Per CTA: one (batch, head, segment); the CTA walks the segment's tiles.
+// Threads: warp 0 -- one lane issues the TMA loads and the tcgen05.mma;
+//          warps 1..4 -- 128 workers; worker warp w reads TMEM lanes
+//          32*(w%4) .. +31 (a warp can only reach its own lane quarter).
+// Per tile:
+//   TMA     B, C (bf16, SWIZZLE_128B, K-major: rows (t,r), 2 atoms of 64 n)
+//           and X (rows (t,r), 64 p) into shared memory.
+//   workers dt/lambda -> a_t (block scan), gamma, c, w = e^{a_last-a}c, e^{a};
+//           cumulative phase per rotary pair (double running sum, one thread
+//           per (pair, half tile)); rotate B and C in place.
+//   MMA 1   G = C~ B~^T (128x128, K=128)      -> TMEM cols [0,128)
+//           Y_inter = C~ S_bf (128x64, K=128) -> TMEM cols [192,256)
+//   workers scale B~ rows by w; P = mask o G -> bf16 over C~'s smem.
+//   MMA 2   S_loc = (w B~)^T X (128x64, K=128) -> TMEM cols [128,192)
+//           Y_intra = P X (128x64, K=128)      -> TMEM cols [0,64)
+//   workers S = e^{a_last} S + S_loc (float32, registers, thread = state row);
+//           S_bf = bf16(S) for the next tile; y = Y_intra + e^{a_t} Y_inter.
+// Two CTAs share an SM (about 101 KB of shared memory and 256 TMEM columns
+// each), so one CTA's loads overlap the other's math.
+//
+// Every wait on an mbarrier is bounded (1 s); on expiry the kernel records
+// M3_ERR_DEVICE_TIMEOUT in the workspace status word, finishes the tile with
+// no further waiting and returns after freeing its TMEM.
+#include <cuda.h>
+
+#include "m3_common.cuh"
+#include "m3_kernels.h"
+
+namespace m3 {
+namespace tc {
+
+constexpr int kRows = 128;
+constexpr int kN = 128;
+constexpr int kP = 64;
+constexpr int kThreads = 160;
+constexpr uint64_t kWaitNs = 1000000000ull;
+
+// shared memory map (offsets from a 1024-byte aligned base)
+constexpr int OFF_B = 0;          // 32 KB: B~ (two 16 KB atoms)
+constexpr int OFF_C = 32768;      // 32 KB: C~, later P
+constexpr int OFF_X = 65536;      // 16 KB: X
+constexpr int OFF_S = 81920;      // 16 KB: S_bf (rows n, 64 p)
+constexpr int OFF_MISC = 98304;
+constexpr int MISC_BYTES = 5120;
+constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;   // + alignment slack
+
+struct Misc {
+    uint64_t bar[8];              // load, ops, g, bw, p, y, free, spare
+    uint32_t tmem_base;
+    int abort_flag;
+    int drain_flag;               // abort flag of the final drain waits (never set by others)
+    int pad[13];
+    float dt[128], lam[128];
+    float a[128], gam[128], cf[128], w[128], ea[128];
+    float scan[4];
+    float scal[4];                // [0] tile decay, [1] segment log-decay, [2..3] next dt/lambda
+    double phi[64];               // phase carry per rotary pair (reduced)
+    double half_sum[64];
+};
+static_assert(sizeof(Misc) <= MISC_BYTES, "misc region too small");
+
+enum { BAR_LOAD = 0, BAR_OPS, BAR_G, BAR_BW, BAR_P, BAR_Y, BAR_FREE };
+
+// ------------------------------------------------------------ PTX wrappers --
+__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(su32(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait.  Returns false when the CTA is aborting (this wait or an
+// earlier one expired); the caller then carries on without waiting.
+__device__ __noinline__ bool mbar_wait_flag(uint64_t* b, uint32_t parity, int* abortp, int* status, int where) {
+    if (mbar_try(b, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try(b, parity)) return true;
+        if (*(volatile int*)abortp) return false;
+        if (globaltimer_ns() - t0 > kWaitNs) {
+            *(volatile int*)abortp = 1;
+            if (status) {
+                atomicCAS(status, 0, (int)M3_ERR_DEVICE_TIMEOUT);
+                status[1] = where;
+            }
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Misc* m, int* status, int where) {
+    return mbar_wait_flag(b, parity, &m->abort_flag, status, where);
+}
+
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                            int c2, int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+        ::"r"(dst), "l"((uint64_t)map), "r"(su32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void workers_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// all 128 workers get the OR of `cond` (named barrier 1 with a reduction), so
+// they take the same branch
+__device__ __forceinline__ int workers_any(int cond) {
+    int r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.s32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, 128, p;\n\t"
+        "selp.s32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(cond)
+        : "memory");
+    return r;
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(dst)), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A[smem desc] x B[smem desc], bf16 inputs, fp32 accumulate
+__device__ __forceinline__ void umma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
+                 : "memory");
+}
+
+// 32 lanes x 32 consecutive fp32 columns; thread = lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+// Shared-memory matrix descriptor, SWIZZLE_128B (sm_100 layout: start>>4,
+// LBO>>4 at bit 16, SBO>>4 at bit 32, version 1 at bit 46, swizzle 2 at 61).
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor, kind::f16: D f32, A/B bf16, majors, N>>3, M>>4.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// byte offset of 16-byte chunk `c` (0..7) of row `row` inside a 128-row
+// SWIZZLE_128B atom (rows of 128 bytes, chunk index XOR row%8)
+__device__ __forceinline__ uint32_t sw128(int row, int c) { return (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4)); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
+    __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
+    return __bfloat1622float2(v);
+}
+
+// ------------------------------------------------------------------ kernel --
+template <int R, bool SUMMARY>
+__global__ void __launch_bounds__(kThreads, 2)
+    scan_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
+                   const __grid_constant__ CUtensorMap tmX, ScanParams q, int* status) {
+    constexpr int T = kRows / R;       // tokens per tile
+    constexpr int TH = T / 2;          // tokens per half tile (phase pass)
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    Misc* m = reinterpret_cast<Misc*>(smem + OFF_MISC);
+    const uint32_t sbase = su32(smem);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int L = q.seqlen, H = q.nheads, G = q.ngroups;
+    const int g = h / (H / G);
+    const int tok0 = seg * q.cps * T;
+    const int tok1 = min(L, (seg + 1) * q.cps * T);
+    const int ntiles = (tok1 - tok0 + T - 1) / T;
+    const size_t bh = (size_t)b * H + h;
+    const size_t bhs = bh * q.nseg + seg;
+    const float Ah = q.A[h];
+
+    // ---- setup
+    if (tid == 0) {
+        mbar_init(&m->bar[BAR_LOAD], 1);
+        mbar_init(&m->bar[BAR_OPS], 128);
+        mbar_init(&m->bar[BAR_G], 1);
+        mbar_init(&m->bar[BAR_BW], 128);
+        mbar_init(&m->bar[BAR_P], 128);
+        mbar_init(&m->bar[BAR_Y], 1);
+        mbar_init(&m->bar[BAR_FREE], 128);
+        mbar_init(&m->bar[7], 1);
+        m->abort_flag = 0;
+        m->drain_flag = 0;
+        m->scal[1] = 0.f;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_async_smem();
+    }
+    if (warp == 0) {
+        tmem_alloc(&m->tmem_base, 256);
+        tmem_relinquish();
+    }
+
+    // workers: state rows in registers (thread = state row n), S_bf, phase carry
+    const int wk = tid - 32;                  // worker index 0..127
+    const int wq = warp & 3;                  // TMEM lane quarter of this warp
+    const int row = wq * 32 + lane;           // tile row / state row owned in TMEM
+    float S[kP];
+    if (warp > 0) {
+        if (wk < 64) m->phi[wk] = 0.0;
+        const int n = row;
+        if (SUMMARY) {
+#pragma unroll
+            for (int p = 0; p < kP; ++p) S[p] = 0.f;
+        } else if (q.nseg > 1) {
+            const float4* src = reinterpret_cast<const float4*>(q.ws_sin + (bhs * kN + n) * kP);
+#pragma unroll
+            for (int c = 0; c < kP / 4; ++c) {
+                const float4 v = src[c];
+                S[4 * c] = v.x; S[4 * c + 1] = v.y; S[4 * c + 2] = v.z; S[4 * c + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int p = 0; p < kP; ++p) S[p] = q.init_h ? q.init_h[(bh * kN + n) * kP + p] : 0.f;
+            if (q.init_pB && q.init_pX) {
+                const float w0 = (1.f - q.lam[(size_t)b * L * H + h]) * q.dt[(size_t)b * L * H + h];
+                const __nv_bfloat16* pB = static_cast<const __nv_bfloat16*>(q.init_pB) + bh * R * kN;
+                const __nv_bfloat16* pX = static_cast<const __nv_bfloat16*>(q.init_pX) + bh * R * kP;
+                for (int r = 0; r < R; ++r) {
+                    const float bv = w0 * __bfloat162float(pB[r * kN + n]);
+#pragma unroll
+                    for (int p = 0; p < kP; ++p) S[p] = fmaf(bv, __bfloat162float(pX[r * kP + p]), S[p]);
+                }
+            }
+        }
+        if (!SUMMARY) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint4 v;
+                v.x = pack_bf16x2(S[8 * c + 0], S[8 * c + 1]);
+                v.y = pack_bf16x2(S[8 * c + 2], S[8 * c + 3]);
+                v.z = pack_bf16x2(S[8 * c + 4], S[8 * c + 5]);
+                v.w = pack_bf16x2(S[8 * c + 6], S[8 * c + 7]);
+                *reinterpret_cast<uint4*>(smem + OFF_S + sw128(n, c)) = v;
+            }
+            fence_async_smem();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = m->tmem_base;
+
+    const float* theta = q.theta;
+    const float* dtp = q.dt;
+    const float* lamp = q.lam;
+    __nv_bfloat16* yg = static_cast<__nv_bfloat16*>(q.y);
+
+    uint32_t pending_load = 0;   // control lane: a TMA load is in flight
+    uint32_t load_par = 0;       // its mbarrier phase
+
+    for (int k = 0; k < ntiles; ++k) {
+        const int t0 = tok0 + k * T;
+        const int qc = min(T, tok1 - t0);
+        const uint32_t par = k & 1;
+        if (warp == 0) {
+            if (*(volatile int*)&m->abort_flag) break;
+        } else if (workers_any(*(volatile int*)&m->abort_flag)) {
+            break;
+        }
+
+        if (warp == 0) {
+            if (lane == 0) {
+                // ---------------- producer + MMA issuer
+                if (k > 0) mbar_wait(&m->bar[BAR_FREE], (k - 1) & 1, m, status, 1);
+                const uint32_t bytes = SUMMARY ? (32768u + 16384u) : (65536u + 16384u);
+                mbar_expect_tx(&m->bar[BAR_LOAD], bytes);
+                tma_load_5d(sbase + OFF_B, &tmB, &m->bar[BAR_LOAD], 0, 0, g, t0, b);
+                tma_load_5d(sbase + OFF_B + 16384, &tmB, &m->bar[BAR_LOAD], 64, 0, g, t0, b);
+                if (!SUMMARY) {
+                    tma_load_5d(sbase + OFF_C, &tmC, &m->bar[BAR_LOAD], 0, 0, g, t0, b);
+                    tma_load_5d(sbase + OFF_C + 16384, &tmC, &m->bar[BAR_LOAD], 64, 0, g, t0, b);
+                }
+                tma_load_5d(sbase + OFF_X, &tmX, &m->bar[BAR_LOAD], 0, 0, h, t0, b);
+                pending_load = 1;
+                load_par = par;
+                mbar_wait(&m->bar[BAR_OPS], par, m, status, 2);
+                pending_load = 0;       // workers saw the load complete before arriving
+                tc_fence_after();
+                const uint32_t d_g = tmem, d_sl = tmem + 128, d_yx = tmem + 192;
+                if (!SUMMARY) {
+                    // G = C~ B~^T : both K-major, K = n in two 64-wide atoms
+                    constexpr uint32_t idG = idesc_bf16(128, 128, 0, 0);
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        umma(d_g, sdesc(sbase + OFF_C + off, 16, 1024), sdesc(sbase + OFF_B + off, 16, 1024), idG,
+                             kk > 0);
+                    }
+                    // Y_inter = C~ S_bf : A K-major (K = n), B MN-major (K = n rows, N = p)
+                    constexpr uint32_t idY = idesc_bf16(128, 64, 0, 1);
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t offa = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        umma(d_yx, sdesc(sbase + OFF_C + offa, 16, 1024),
+                             sdesc(sbase + OFF_S + kk * 2048, 8192, 1024), idY, kk > 0);
+                    }
+                    umma_commit(&m->bar[BAR_G]);
+                    mbar_wait(&m->bar[BAR_BW], par, m, status, 3);
+                    tc_fence_after();
+                }
+                // S_loc = (w B~)^T X : A MN-major (M = n, two 64-wide blocks 16 KB apart),
+                // B MN-major (N = p); K = tile rows, 16 rows (2 KB) per instruction
+                constexpr uint32_t idS = idesc_bf16(128, 64, 1, 1);
+                for (int kk = 0; kk < 8; ++kk)
+                    umma(d_sl, sdesc(sbase + OFF_B + kk * 2048, 16384, 1024),
+                         sdesc(sbase + OFF_X + kk * 2048, 8192, 1024), idS, kk > 0);
+                if (!SUMMARY) {
+                    mbar_wait(&m->bar[BAR_P], par, m, status, 4);
+                    tc_fence_after();
+                    // Y_intra = P X : A K-major (K = tile cols in two atoms), B MN-major
+                    constexpr uint32_t idI = idesc_bf16(128, 64, 0, 1);
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t offa = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        umma(d_g, sdesc(sbase + OFF_C + offa, 16, 1024),
+                             sdesc(sbase + OFF_X + kk * 2048, 8192, 1024), idI, kk > 0);
+                    }
+                }
+                umma_commit(&m->bar[BAR_Y]);
+            }
+            __syncwarp();
+            continue;
+        }
+
+        // ---------------------------------------------------------- workers
+        const int pi = wk & 63, half = wk >> 6;
+        float th[TH];
+#pragma unroll
+        for (int kk = 0; kk < TH; ++kk) {
+            const int t = half * TH + kk;
+            th[kk] = (t < qc) ? __ldg(theta + (((size_t)b * L + t0 + t) * G + g) * (kN / 2) + pi) : 0.f;
+        }
+        if (wk < T) {
+            const size_t o = ((size_t)b * L + t0 + wk) * H + h;
+            m->dt[wk] = (wk < qc) ? __ldg(dtp + o) : 0.f;
+            m->lam[wk] = (wk < qc) ? __ldg(lamp + o) : 1.f;
+        }
+        if (wk == 0) {
+            const int tn = t0 + qc;
+            const size_t o = ((size_t)b * L + tn) * H + h;
+            m->scal[2] = (tn < L) ? __ldg(dtp + o) : 0.f;
+            m->scal[3] = (tn < L) ? __ldg(lamp + o) : 1.f;
+        }
+        workers_sync();
+        // a_t = sum_{s<=t} dt_s A (inclusive block scan over the tile's tokens)
+        {
+            float v = (wk < qc) ? m->dt[wk] * Ah : 0.f;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
+            }
+            if (lane == 31) m->scan[warp - 1] = v;
+            workers_sync();
+            const int ww = warp - 1;
+            for (int j = 0; j < ww; ++j) v += m->scan[j];
+            if (wk < T) m->a[wk] = v;
+        }
+        workers_sync();
+        const float a_last = m->a[T - 1];
+        if (wk < T) {
+            if (wk < qc) {
+                const float d = m->dt[wk], lam = m->lam[wk];
+                const float gam = lam * d;
+                const float nxt = (wk + 1 < qc) ? (1.f - m->lam[wk + 1]) * m->dt[wk + 1]
+                                                : (1.f - m->scal[3]) * m->scal[2];
+                const float c = gam + nxt;
+                const float a = m->a[wk];
+                m->gam[wk] = gam;
+                m->cf[wk] = c;
+                m->w[wk] = expf(a_last - a) * c;
+                m->ea[wk] = expf(a);
+            } else {
+                m->gam[wk] = 0.f; m->cf[wk] = 0.f; m->w[wk] = 0.f; m->ea[wk] = 0.f;
+            }
+        }
+        // phase pass 1: this half's total
+        const double carry = m->phi[pi];
+        double acc = 0.0;
+#pragma unroll
+        for (int kk = 0; kk < TH; ++kk) acc += (double)m->dt[half * TH + kk] * (double)th[kk];
+        if (half == 0) m->half_sum[pi] = acc;
+        if (wk == 0) {
+            m->scal[0] = expf(a_last);
+            m->scal[1] += a_last;
+        }
+        mbar_wait(&m->bar[BAR_LOAD], par, m, status, 10);
+        workers_sync();
+        const double start = carry + (half ? m->half_sum[pi] : 0.0);
+        if (half == 1) m->phi[pi] = wrap_pi(start + acc);
+        // phase pass 2: rotate B (and C) rows (t, r) at pair pi, in place
+        {
+            const uint32_t atom = (uint32_t)(pi >> 5) * 16384u;
+            const int chunk = (pi & 31) >> 2;
+            const uint32_t inb = (uint32_t)(pi & 3) * 4u;
+            double ph = start;
+#pragma unroll
+            for (int kk = 0; kk < TH; ++kk) {
+                const int t = half * TH + kk;
+                ph += (double)m->dt[t] * (double)th[kk];
+                if (t < qc) {
+                    float sv, cv;
+                    __sincosf((float)wrap_pi(ph), &sv, &cv);
+                    const float wsc = SUMMARY ? m->w[t] : 1.f;
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        const int rw = t * R + r;
+                        const uint32_t off = atom + sw128(rw, chunk) + inb;
+                        uint32_t* pb = reinterpret_cast<uint32_t*>(smem + OFF_B + off);
+                        const float2 bv = unpack_bf16x2(*pb);
+                        *pb = pack_bf16x2(wsc * (cv * bv.x + sv * bv.y), wsc * (-sv * bv.x + cv * bv.y));
+                        if (!SUMMARY) {
+                            uint32_t* pc = reinterpret_cast<uint32_t*>(smem + OFF_C + off);
+                            const float2 cvv = unpack_bf16x2(*pc);
+                            *pc = pack_bf16x2(cv * cvv.x + sv * cvv.y, -sv * cvv.x + cv * cvv.y);
+                        }
+                    }
+                }
+            }
+        }
+        fence_async_smem();
+        mbar_arrive(&m->bar[BAR_OPS]);
+
+        const int tr = row / R;              // token of this thread's tile row
+        if (!SUMMARY) {
+            mbar_wait(&m->bar[BAR_G], par, m, status, 11);
+            tc_fence_after();
+            // scale row `row` of B~ by w_t (the state contribution weight)
+            {
+                const float wt = m->w[tr];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    uint4* p = reinterpret_cast<uint4*>(smem + OFF_B + (c >> 3) * 16384 + sw128(row, c & 7));
+                    uint4 v = *p;
+                    float2 f;
+                    f = unpack_bf16x2(v.x); v.x = pack_bf16x2(wt * f.x, wt * f.y);
+                    f = unpack_bf16x2(v.y); v.y = pack_bf16x2(wt * f.x, wt * f.y);
+                    f = unpack_bf16x2(v.z); v.z = pack_bf16x2(wt * f.x, wt * f.y);
+                    f = unpack_bf16x2(v.w); v.w = pack_bf16x2(wt * f.x, wt * f.y);
+                    *p = v;
+                }
+            }
+            fence_async_smem();
+            mbar_arrive(&m->bar[BAR_BW]);
+            // P = (two-band decay mask) o G, bf16, K-major over C~'s smem
+            {
+                const float a_t = m->a[tr];
+#pragma unroll 1
+                for (int cg = 0; cg < 4; ++cg) {
+                    float v[32];
+                    tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + cg * 32, v);
+#pragma unroll
+                    for (int j0 = 0; j0 < 32; j0 += R) {
+                        const int u = (cg * 32 + j0) / R;
+                        float mk = 0.f;
+                        if (u <= tr) mk = expf(a_t - m->a[u]) * (u == tr ? m->gam[u] : m->cf[u]);
+#pragma unroll
+                        for (int r = 0; r < R; ++r) v[j0 + r] *= mk;
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int cc = cg * 4 + c;      // 16-byte chunk over 128 columns
+                        uint4 o;
+                        o.x = pack_bf16x2(v[8 * c + 0], v[8 * c + 1]);
+                        o.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+                        o.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
+                        o.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
+                        *reinterpret_cast<uint4*>(smem + OFF_C + (cc >> 3) * 16384 + sw128(row, cc & 7)) = o;
+                    }
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(&m->bar[BAR_P]);
+        }
+
+        mbar_wait(&m->bar[BAR_Y], par, m, status, 12);
+        tc_fence_after();
+        // state: S = e^{a_last} S + S_loc   (thread = state row)
+        {
+            const float dec = m->scal[0];
+#pragma unroll
+            for (int cg = 0; cg < 2; ++cg) {
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + 128 + cg * 32, v);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) S[cg * 32 + j] = fmaf(dec, S[cg * 32 + j], v[j]);
+            }
+            if (!SUMMARY) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint4 v;
+                    v.x = pack_bf16x2(S[8 * c + 0], S[8 * c + 1]);
+                    v.y = pack_bf16x2(S[8 * c + 2], S[8 * c + 3]);
+                    v.z = pack_bf16x2(S[8 * c + 4], S[8 * c + 5]);
+                    v.w = pack_bf16x2(S[8 * c + 6], S[8 * c + 7]);
+                    *reinterpret_cast<uint4*>(smem + OFF_S + sw128(row, c)) = v;
+                }
+            }
+        }
+        if (!SUMMARY) {
+            // y = Y_intra + e^{a_t} Y_inter  (thread = tile row (t, r))
+            const float ea = m->ea[tr];
+#pragma unroll 1
+            for (int cg = 0; cg < 2; ++cg) {
+                float yi[32], yx[32];
+                tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + cg * 32, yi);
+                tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + 192 + cg * 32, yx);
+                if (tr < qc) {
+                    uint4* dst = reinterpret_cast<uint4*>(
+                        yg + ((((size_t)b * L + t0 + tr) * H + h) * R + (row % R)) * kP + cg * 32);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint4 o;
+                        o.x = pack_bf16x2(fmaf(ea, yx[8 * c + 0], yi[8 * c + 0]), fmaf(ea, yx[8 * c + 1], yi[8 * c + 1]));
+                        o.y = pack_bf16x2(fmaf(ea, yx[8 * c + 2], yi[8 * c + 2]), fmaf(ea, yx[8 * c + 3], yi[8 * c + 3]));
+                        o.z = pack_bf16x2(fmaf(ea, yx[8 * c + 4], yi[8 * c + 4]), fmaf(ea, yx[8 * c + 5], yi[8 * c + 5]));
+                        o.w = pack_bf16x2(fmaf(ea, yx[8 * c + 6], yi[8 * c + 6]), fmaf(ea, yx[8 * c + 7], yi[8 * c + 7]));
+                        dst[c] = o;
+                    }
+                }
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(&m->bar[BAR_FREE]);
+    }
+
+    // ---- epilogue of the segment
+    if (warp == 0 && lane == 0) {
+        // an aborted tile may still have a TMA load in flight: let it land
+        if (pending_load) mbar_wait_flag(&m->bar[BAR_LOAD], load_par, &m->drain_flag, nullptr, 0);
+        // all MMAs this thread issued are complete before TMEM is freed
+        umma_commit(&m->bar[7]);
+        mbar_wait_flag(&m->bar[7], 0, &m->drain_flag, nullptr, 0);
+    }
+    if (warp > 0) {
+        const int n = row;
+        if (SUMMARY) {
+            float4* dst = reinterpret_cast<float4*>(q.ws_sloc + (bhs * kN + n) * kP);
+#pragma unroll
+            for (int c = 0; c < kP / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
+            if (wk < 64) q.ws_phase[bhs * (kN / 2) + wk] = (float)m->phi[wk];
+            if (wk == 0) q.ws_decay[bhs] = m->scal[1];
+        } else if (seg == q.nseg - 1) {
+            if (q.fin_h) {
+                float sv, cv;
+                sincosf((float)m->phi[n >> 1], &sv, &cv);
+                float* dst = q.fin_h + (bh * kN + n) * kP;
+#pragma unroll
+                for (int p = 0; p < kP; ++p) {
+                    const float other = __shfl_xor_sync(0xffffffffu, S[p], 1);
+                    dst[p] = (n & 1) ? (sv * other + cv * S[p]) : (cv * S[p] - sv * other);
+                }
+            }
+            if (q.fin_pB && L > 0) {
+                const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(q.B) + (((size_t)b * L + L - 1) * G + g) * R * kN;
+                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(q.fin_pB) + bh * R * kN;
+                for (int e = wk; e < R * kN; e += 128) o[e] = s[e];
+            }
+            if (q.fin_pX && L > 0) {
+                const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(q.x) + (((size_t)b * L + L - 1) * H + h) * R * kP;
+                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(q.fin_pX) + bh * R * kP;
+                for (int e = wk; e < R * kP; e += 128) o[e] = s[e];
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// ------------------------------------------------------------------- host --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) != cudaSuccess ||
+            qr != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// 5-D map over [b][t][grp][r][inner] with a box of (64 inner, R, 1, T, 1)
+static bool make_map(CUtensorMap* map, const void* base, int inner, int R, int grp, int L, int batch, int T) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[5] = {(cuuint64_t)inner, (cuuint64_t)R, (cuuint64_t)grp, (cuuint64_t)L, (cuuint64_t)batch};
+    const cuuint64_t e = 2;   // bf16
+    const cuuint64_t strides[4] = {inner * e, (cuuint64_t)R * inner * e, (cuuint64_t)grp * R * inner * e,
+                                   (cuuint64_t)L * grp * R * inner * e};
+    const cuuint32_t box[5] = {64, (cuuint32_t)R, 1, (cuuint32_t)T, 1};
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace tc
+
+bool tc_eligible(const m3_dims& d) {
+    return d.io_dtype == M3_BF16 && d.dstate == tc::kN && d.headdim == tc::kP &&
+           (d.rank == 1 || d.rank == 2 || d.rank == 4 || d.rank == 8);
+}
+
+int tc_tile_tokens(int rank) { return tc::kRows / rank; }
+
+template <int R>
+static cudaError_t launch_tc_R(const ScanParams& q, int* status, cudaStream_t st) {
+    using namespace tc;
+    constexpr int T = kRows / R;
+    CUtensorMap mB, mC, mX;
+    if (!make_map(&mB, q.B, kN, R, q.ngroups, q.seqlen, q.batch, T) ||
+        !make_map(&mC, q.C, kN, R, q.ngroups, q.seqlen, q.batch, T) ||
+        !make_map(&mX, q.x, kP, R, q.nheads, q.seqlen, q.batch, T))
+        return cudaErrorInvalidValue;
+    cudaFuncSetAttribute(scan_tc_kernel<R, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaFuncSetAttribute(scan_tc_kernel<R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (q.nseg > 1) {
+        scan_tc_kernel<R, true><<<dim3(q.nseg - 1, q.nheads, q.batch), kThreads, SMEM_BYTES, st>>>(mB, mC, mX, q, status);
+        cudaError_t e = launch_scan_combine(q, st);
+        if (e != cudaSuccess) return e;
+    }
+    scan_tc_kernel<R, false><<<dim3(q.nseg, q.nheads, q.batch), kThreads, SMEM_BYTES, st>>>(mB, mC, mX, q, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scan_tc(const m3_dims& d, const ScanParams& q, int* status, cudaStream_t st) {
+    switch (d.rank) {
+        case 1: return launch_tc_R<1>(q, status, st);
+        case 2: return launch_tc_R<2>(q, status, st);
+        case 4: return launch_tc_R<4>(q, status, st);
+        case 8: return launch_tc_R<8>(q, status, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace m3

@@ -41,7 +41,8 @@ static size_t io_bytes(const m3_dims& d) { return d.io_dtype == M3_BF16 ? 2 : 4;
 
 // ---------------------------------------------------------------- plan --
 struct Plan {
-    int qs;      // chunk length the kernel uses
+    int path;    // 0 = SIMT float32, 1 = tcgen05
+    int qs;      // chunk length the kernels use (tokens)
     int nseg;    // segments per (b, h)
     int cps;     // chunks per segment
 };
@@ -52,22 +53,50 @@ static int env_int(const char* name, int dflt) {
     return atoi(v);
 }
 
-// SIMT path: the kernel keeps one chunk of rotated B, C, X, the masked Gram
-// and the state in shared memory, so the chunk it uses is the caller's chunk
-// when that fits, else halved until it does (the chunked result does not
-// depend on the chunk length except through rounding).
+static bool env_is(const char* name, const char* val) {
+    const char* v = getenv(name);
+    return v && strcmp(v, val) == 0;
+}
+
+// SM count of the current device (a cached device attribute; 148 on B200
+// and when no device can be queried)
+static int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+// Path and chunking.  tcgen05 path: a chunk is one 128-row UMMA tile
+// (128/R tokens).  SIMT path: the kernel keeps one chunk of rotated B, C, X,
+// the masked Gram and the state in shared memory, so it uses the caller's
+// chunk when that fits, else halves it until it does.  The chunked result
+// does not depend on the chunk length except through rounding.
+// Segments: a (b, h) sequence is cut into segments only when there are too
+// few sequences to give every SM work (two resident CTAs per SM).
 static m3_status make_plan(const m3_dims& d, Plan* pl) {
     const size_t kMaxSmem = 200 * 1024;
-    int qs = d.chunk;
-    if (d.seqlen > 0 && qs > d.seqlen) qs = d.seqlen;
-    while (qs > 1 && simt_smem_bytes(qs, d.rank, d.dstate, d.headdim, false) > kMaxSmem) qs = (qs + 1) / 2;
-    if (simt_smem_bytes(qs, d.rank, d.dstate, d.headdim, false) > kMaxSmem) return M3_ERR_UNSUPPORTED;
+    const bool tc = tc_eligible(d) && !env_is("M3_SCAN_PATH", "simt");
+    int qs;
+    if (tc) {
+        qs = tc_tile_tokens(d.rank);
+    } else {
+        qs = d.chunk;
+        if (d.seqlen > 0 && qs > d.seqlen) qs = d.seqlen;
+        while (qs > 1 && simt_smem_bytes(qs, d.rank, d.dstate, d.headdim, false) > kMaxSmem) qs = (qs + 1) / 2;
+        if (simt_smem_bytes(qs, d.rank, d.dstate, d.headdim, false) > kMaxSmem) return M3_ERR_UNSUPPORTED;
+    }
     const long long nchunks = d.seqlen > 0 ? (d.seqlen + qs - 1) / qs : 0;
     const long long units = (long long)d.batch * d.nheads;
+    const long long sms = sm_count();
     int nseg = 1;
-    // enough independent segments to fill the GPU twice over, at >= 2 chunks each
-    if (units > 0 && nchunks >= 4) {
-        long long want = (2 * 148 + units - 1) / units;
+    if (units > 0 && units < sms && nchunks >= 4) {
+        long long want = (2 * sms) / units;
         long long cap = nchunks / 2;
         nseg = (int)(want < cap ? want : cap);
         if (nseg < 1) nseg = 1;
@@ -76,6 +105,7 @@ static m3_status make_plan(const m3_dims& d, Plan* pl) {
     if (forced > 0) nseg = (int)(forced < nchunks ? forced : (nchunks > 0 ? nchunks : 1));
     int cps = nchunks > 0 ? (int)((nchunks + nseg - 1) / nseg) : 1;
     if (nchunks > 0) nseg = (int)((nchunks + cps - 1) / cps);   // drop empty segments
+    pl->path = tc ? 1 : 0;
     pl->qs = qs;
     pl->nseg = nseg;
     pl->cps = cps;
@@ -140,7 +170,7 @@ m3_status m3_scan_plan(const m3_dims* d, int* launches, int* segments, int* chun
     if (launches) *launches = work ? (pl.nseg > 1 ? 3 : 1) : 0;
     if (segments) *segments = pl.nseg;
     if (chunk_used) *chunk_used = pl.qs;
-    if (path) *path = 0;
+    if (path) *path = pl.path;
     return M3_OK;
 }
 
@@ -199,7 +229,8 @@ m3_status m3_scan_fwd(const m3_dims* d, const void* x, const void* B, const void
     q.ws_decay = reinterpret_cast<float*>(ws + w.decay);
     q.ws_phase = reinterpret_cast<float*>(ws + w.phase);
     q.ws_sin = reinterpret_cast<float*>(ws + w.sin);
-    cudaError_t e = launch_scan_simt(*d, q, st);
+    cudaError_t e = pl.path == 1 ? launch_scan_tc(*d, q, reinterpret_cast<int*>(workspace), st)
+                                 : launch_scan_simt(*d, q, st);
     return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }
 

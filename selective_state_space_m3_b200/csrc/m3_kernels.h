@@ -64,5 +64,11 @@ m3_status launch_step(const m3_dims& d, const StepParams& q, cudaStream_t st);
 m3_status launch_rope(const m3_dims& d, const RopeParams& q, cudaStream_t st);
 size_t simt_smem_bytes(int qs, int R, int N, int P, bool summary);
 cudaError_t launch_scan_simt(const m3_dims& d, const ScanParams& q, cudaStream_t st);
+cudaError_t launch_scan_combine(const ScanParams& q, cudaStream_t st);
+// tensor-core path (bf16, N = 128, P = 64, rank 1/2/4/8); `status` is the
+// workspace status word its bounded waits report to
+bool tc_eligible(const m3_dims& d);
+int tc_tile_tokens(int rank);
+cudaError_t launch_scan_tc(const m3_dims& d, const ScanParams& q, int* status, cudaStream_t st);
 
 }  // namespace m3

@@ -49,8 +49,13 @@ SMALL = [
 ]
 
 
+@pytest.mark.parametrize("path", ["auto", "simt"])
 @pytest.mark.parametrize("shape,name", SMALL, ids=[n for _, n in SMALL])
-def test_scan_matches_oracle(shape, name):
+def test_scan_matches_oracle(shape, name, path, monkeypatch):
+    """Every small case on the default path (tcgen05 for bf16 N=128 P=64) and
+    on the SIMT path forced."""
+    if path == "simt":
+        monkeypatch.setenv("M3_SCAN_PATH", "simt")
     inp = m3_synth.make_scan_inputs(shape)
     y, fin = gpu_scan(shape, inp)
     yo, ho, pBo, pXo = _oracle_full(inp)
@@ -63,7 +68,8 @@ def test_scan_matches_oracle(shape, name):
 
 @pytest.mark.parametrize("nseg", [1, 2, 3, 7])
 def test_scan_segment_split_matches_oracle(nseg, monkeypatch):
-    """The multi-segment path (summary, combine, main) against the oracle."""
+    """The multi-segment path (summary, combine, main) against the oracle,
+    float32 SIMT."""
     monkeypatch.setenv("M3_SCAN_NSEG", str(nseg))
     shape = m3_synth.ScanShape(2, 290, 2, 1, 16, 16, 2, 16, "f32", 0.0, 21)
     inp = m3_synth.make_scan_inputs(shape)
@@ -73,6 +79,27 @@ def test_scan_segment_split_matches_oracle(nseg, monkeypatch):
     yo, ho, _, _ = _oracle_full(inp, init)
     _check(f"nseg{nseg} y", f64(y), yo, 1e-4)
     _check(f"nseg{nseg} h", f64(fin.h), ho, 1e-4)
+
+
+@pytest.mark.parametrize("R", [1, 2, 4, 8])
+@pytest.mark.parametrize("nseg", [1, 3])
+def test_tc_segments_and_ranks(R, nseg, monkeypatch):
+    """tcgen05 path: every supported rank, one and several segments, ragged
+    tail, nonzero initial carry."""
+    monkeypatch.setenv("M3_SCAN_NSEG", str(nseg))
+    T = 128 // R
+    L = 5 * T + 7
+    shape = m3_synth.ScanShape(2, L, 2, 2, 64, 128, R, 64, "bf16", 0.0, 60 + R)
+    inp = m3_synth.make_scan_inputs(shape)
+    c = m3_synth.make_carry(2, 2, 128, 64, R, "bf16", 60 + R, scale=0.3)
+    init = m3.Carry(c["h"].cuda(), c["prev_B"].cuda(), c["prev_x"].cuda())
+    d = dims_of(shape)
+    plan = m3.m3_scan_plan(d)
+    assert plan["path"] == "tcgen05" and plan["segments"] == nseg
+    y, fin = gpu_scan(shape, inp, init=init)
+    yo, ho, _, _ = _oracle_full(inp, init)
+    _check(f"tc R{R} nseg{nseg} y", f64(y), yo, 2e-2)
+    _check(f"tc R{R} nseg{nseg} h", f64(fin.h), ho, 2e-2)
 
 
 def test_scan_with_initial_carry_bf16():
