@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the layer's batch (profiling captures of a smaller case)")
     return ap.parse_args()
 
 
@@ -230,6 +232,8 @@ def main():
     pk = peaks()
     s = m3_synth.CONFIGS[CFG]
     s = m3_synth.shrink(s, seed=s.seed + 1000 * rank)     # each rank its own problem
+    if args.batch > 0:
+        s = m3_synth.shrink(s, batch=args.batch)
     host = m3_synth.make_scan_inputs(s)
     dev = {k: v.cuda() for k, v in host.items()}
     d = m3.Dims(s.batch, s.seqlen, s.nheads, s.ngroups, s.headdim, s.dstate, s.rank, s.chunk, m3.M3_BF16)
@@ -329,10 +333,10 @@ def main():
     # ---- decode: m3_step x decode_steps in one CUDA graph, carry from the prefill
     if not args.no_decode:
         dec = m3_synth.DECODE
-        reps = dec.batch // s.batch
-        state = m3.Carry(fin.h.repeat(reps, 1, 1, 1).contiguous(),
-                         fin.prev_B.repeat(reps, 1, 1, 1).contiguous(),
-                         fin.prev_x.repeat(reps, 1, 1, 1).contiguous())
+        reps = -(-dec.batch // s.batch)
+        state = m3.Carry(fin.h.repeat(reps, 1, 1, 1)[:dec.batch].contiguous(),
+                         fin.prev_B.repeat(reps, 1, 1, 1)[:dec.batch].contiguous(),
+                         fin.prev_x.repeat(reps, 1, 1, 1)[:dec.batch].contiguous())
         pool = 64      # distinct tokens (22 MB each; 1.4 GB >> L2), cycled
         toks = []
         for k in range(pool):

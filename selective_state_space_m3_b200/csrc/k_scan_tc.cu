@@ -11,14 +11,17 @@
 //
 // Per CTA: one (batch, head, segment); the CTA walks the segment's tiles.
 // Threads: warp 0 -- one lane issues the TMA loads and the tcgen05.mma;
-//          warps 1..4 -- 128 workers; worker warp w reads TMEM lanes
-//          32*(w%4) .. +31 (a warp can only reach its own lane quarter).
+//          warps 1..8 -- 256 workers in two warpgroups; a worker warp reads
+//          TMEM lanes 32*(warp%4) .. +31 (a warp can only reach its own lane
+//          quarter), so each warpgroup covers all 128 rows and the two split
+//          the columns of row-wise work.
 // Per tile:
 //   TMA     B, C (bf16, SWIZZLE_128B, K-major: rows (t,r), 2 atoms of 64 n)
-//           and X (rows (t,r), 64 p) into shared memory.
+//           and X (rows (t,r), 64 p) into shared memory; issued as soon as
+//           the previous tile's MMAs have read those buffers.
 //   workers dt/lambda -> a_t (block scan), gamma, c, w = e^{a_last-a}c, e^{a};
 //           cumulative phase per rotary pair (double running sum, one thread
-//           per (pair, half tile)); rotate B and C in place.
+//           per (pair, quarter tile)); rotate B and C in place.
 //   MMA 1   G = C~ B~^T (128x128, K=128)      -> TMEM cols [0,128)
 //           Y_inter = C~ S_bf (128x64, K=128) -> TMEM cols [192,256)
 //   workers scale B~ rows by w; P = mask o G -> bf16 over C~'s smem.
@@ -26,8 +29,9 @@
 //           Y_intra = P X (128x64, K=128)      -> TMEM cols [0,64)
 //   workers S = e^{a_last} S + S_loc (float32, registers, thread = state row);
 //           S_bf = bf16(S) for the next tile; y = Y_intra + e^{a_t} Y_inter.
-// Two CTAs share an SM (about 101 KB of shared memory and 256 TMEM columns
-// each), so one CTA's loads overlap the other's math.
+// Two CTAs share an SM (about 105 KB of shared memory, 256 TMEM columns and
+// at most 96 registers per thread each), so one CTA's loads and MMAs overlap
+// the other's SIMT work.
 //
 // Every wait on an mbarrier is bounded (1 s); on expiry the kernel records
 // M3_ERR_DEVICE_TIMEOUT in the workspace status word, finishes the tile with
@@ -43,7 +47,8 @@ namespace tc {
 constexpr int kRows = 128;
 constexpr int kN = 128;
 constexpr int kP = 64;
-constexpr int kThreads = 160;
+constexpr int kWorkers = 256;
+constexpr int kThreads = 32 + kWorkers;
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 // shared memory map (offsets from a 1024-byte aligned base)
@@ -52,7 +57,7 @@ constexpr int OFF_C = 32768;      // 32 KB: C~, later P
 constexpr int OFF_X = 65536;      // 16 KB: X
 constexpr int OFF_S = 81920;      // 16 KB: S_bf (rows n, 64 p)
 constexpr int OFF_MISC = 98304;
-constexpr int MISC_BYTES = 5120;
+constexpr int MISC_BYTES = 7168;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;   // + alignment slack
 
 struct Misc {
@@ -62,15 +67,15 @@ struct Misc {
     int drain_flag;               // abort flag of the final drain waits (never set by others)
     int pad[13];
     float dt[128], lam[128];
-    float a[128], gam[128], cf[128], w[128], ea[128];
-    float scan[4];
+    float a[128], a2[128], gam[128], cf[128], w[128], ea[128];
+    float scan[8];
     float scal[4];                // [0] tile decay, [1] segment log-decay, [2..3] next dt/lambda
     double phi[64];               // phase carry per rotary pair (reduced)
-    double half_sum[64];
+    double qsum[4][64];           // per-quarter phase totals of the current tile
 };
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region too small");
 
-enum { BAR_LOAD = 0, BAR_OPS, BAR_G, BAR_BW, BAR_P, BAR_Y, BAR_FREE };
+enum { BAR_LOAD = 0, BAR_OPS, BAR_G, BAR_BW, BAR_P, BAR_Y, BAR_DRAIN };
 
 // ------------------------------------------------------------ PTX wrappers --
 __device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -130,15 +135,15 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void workers_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-// all 128 workers get the OR of `cond` (named barrier 1 with a reduction), so
+__device__ __forceinline__ void workers_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// all 256 workers get the OR of `cond` (named barrier 1 with a reduction), so
 // they take the same branch
 __device__ __forceinline__ int workers_any(int cond) {
     int r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.s32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, 1, 128, p;\n\t"
+        "bar.red.or.pred q, 1, 256, p;\n\t"
         "selp.s32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
         : "r"(cond)
@@ -189,6 +194,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 }
 
+// 32 lanes x 16 consecutive fp32 columns; thread = lane
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+}
+
 // Shared-memory matrix descriptor, SWIZZLE_128B (sm_100 layout: start>>4,
 // LBO>>4 at bit 16, SBO>>4 at bit 32, version 1 at bit 46, swizzle 2 at 61).
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -210,17 +230,54 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
-    __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
-    return __bfloat1622float2(v);
+    // bf16 -> f32 is a 16-bit shift of the bit pattern
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+__device__ __forceinline__ uint32_t pack2(float2 v) { return pack_bf16x2(v.x, v.y); }
+// (x, y) -> (c x + s y, c y - s x): the transposed 2x2 rotation R(phi)^T
+__device__ __forceinline__ float2 rot_t(float2 v, float2 cc, float2 sn) {
+    // cc = (c, c), sn = (s, -s)
+    return __ffma2_rn(cc, v, __fmul2_rn(sn, make_float2(v.y, v.x)));
+}
+__device__ __forceinline__ uint4 scale_chunk(uint4 v, float2 w) {
+    v.x = pack2(__fmul2_rn(w, unpack_bf16x2(v.x)));
+    v.y = pack2(__fmul2_rn(w, unpack_bf16x2(v.y)));
+    v.z = pack2(__fmul2_rn(w, unpack_bf16x2(v.z)));
+    v.w = pack2(__fmul2_rn(w, unpack_bf16x2(v.w)));
+    return v;
+}
+// 8 consecutive floats -> one 16-byte chunk of bf16
+__device__ __forceinline__ uint4 pack_chunk(const float* f) {
+    uint4 o;
+    o.x = pack_bf16x2(f[0], f[1]);
+    o.y = pack_bf16x2(f[2], f[3]);
+    o.z = pack_bf16x2(f[4], f[5]);
+    o.w = pack_bf16x2(f[6], f[7]);
+    return o;
+}
+// reduce a float angle to [-pi, pi] (two-constant additive reduction:
+// 2*pi split into a float head and tail so k*2pi is formed exactly enough)
+__device__ __forceinline__ float wrap_pi_f(float x) {
+    constexpr float kInv2Pi = 0.15915494309189535f;
+    constexpr float k2PiHi = 6.28318548202514648f;      // float(2 pi)
+    constexpr float k2PiLo = -1.7484555314695172e-7f;   // 2 pi - float(2 pi)
+    const float k = rintf(x * kInv2Pi);
+    return fmaf(-k, k2PiLo, fmaf(-k, k2PiHi, x));
 }
 
 // ------------------------------------------------------------------ kernel --
+// Worker w (0..255) belongs to warpgroup wg = w / 128 and warp-in-group
+// wq = warp % 4, which is the TMEM lane quarter the warp may read.  "Row"
+// work (one tile row or state row per thread) is split between the two
+// warpgroups by columns; token work (coefficients, phases, rotation) is
+// split by (rotary pair, token quarter).
 template <int R, bool SUMMARY>
 __global__ void __launch_bounds__(kThreads, 2)
     scan_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
                    const __grid_constant__ CUtensorMap tmX, ScanParams q, int* status) {
     constexpr int T = kRows / R;       // tokens per tile
-    constexpr int TH = T / 2;          // tokens per half tile (phase pass)
+    constexpr int TQ = T / 4;          // tokens per quarter tile (phase pass)
+    constexpr float kLog2e = 1.4426950408889634f;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     Misc* m = reinterpret_cast<Misc*>(smem + OFF_MISC);
@@ -240,13 +297,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ---- setup
     if (tid == 0) {
         mbar_init(&m->bar[BAR_LOAD], 1);
-        mbar_init(&m->bar[BAR_OPS], 128);
+        mbar_init(&m->bar[BAR_OPS], kWorkers);
         mbar_init(&m->bar[BAR_G], 1);
-        mbar_init(&m->bar[BAR_BW], 128);
-        mbar_init(&m->bar[BAR_P], 128);
+        mbar_init(&m->bar[BAR_BW], kWorkers);
+        mbar_init(&m->bar[BAR_P], kWorkers);
         mbar_init(&m->bar[BAR_Y], 1);
-        mbar_init(&m->bar[BAR_FREE], 128);
-        mbar_init(&m->bar[7], 1);
+        mbar_init(&m->bar[BAR_DRAIN], 1);
         m->abort_flag = 0;
         m->drain_flag = 0;
         m->scal[1] = 0.f;
@@ -258,27 +314,28 @@ __global__ void __launch_bounds__(kThreads, 2)
         tmem_relinquish();
     }
 
-    // workers: state rows in registers (thread = state row n), S_bf, phase carry
-    const int wk = tid - 32;                  // worker index 0..127
+    const int wk = tid - 32;                  // worker index 0..255
+    const int wg = wk >> 7;                   // warpgroup: column half of row work
     const int wq = warp & 3;                  // TMEM lane quarter of this warp
     const int row = wq * 32 + lane;           // tile row / state row owned in TMEM
-    float S[kP];
+    const int c0 = wg * (kP / 2);             // this warpgroup's state / y columns
+    float S[kP / 2];                          // state row `row`, columns c0 .. c0+31
     if (warp > 0) {
         if (wk < 64) m->phi[wk] = 0.0;
         const int n = row;
         if (SUMMARY) {
 #pragma unroll
-            for (int p = 0; p < kP; ++p) S[p] = 0.f;
+            for (int p = 0; p < kP / 2; ++p) S[p] = 0.f;
         } else if (q.nseg > 1) {
-            const float4* src = reinterpret_cast<const float4*>(q.ws_sin + (bhs * kN + n) * kP);
+            const float4* src = reinterpret_cast<const float4*>(q.ws_sin + (bhs * kN + n) * kP + c0);
 #pragma unroll
-            for (int c = 0; c < kP / 4; ++c) {
+            for (int c = 0; c < kP / 8; ++c) {
                 const float4 v = src[c];
                 S[4 * c] = v.x; S[4 * c + 1] = v.y; S[4 * c + 2] = v.z; S[4 * c + 3] = v.w;
             }
         } else {
 #pragma unroll
-            for (int p = 0; p < kP; ++p) S[p] = q.init_h ? q.init_h[(bh * kN + n) * kP + p] : 0.f;
+            for (int p = 0; p < kP / 2; ++p) S[p] = q.init_h ? q.init_h[(bh * kN + n) * kP + c0 + p] : 0.f;
             if (q.init_pB && q.init_pX) {
                 const float w0 = (1.f - q.lam[(size_t)b * L * H + h]) * q.dt[(size_t)b * L * H + h];
                 const __nv_bfloat16* pB = static_cast<const __nv_bfloat16*>(q.init_pB) + bh * R * kN;
@@ -286,19 +343,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int r = 0; r < R; ++r) {
                     const float bv = w0 * __bfloat162float(pB[r * kN + n]);
 #pragma unroll
-                    for (int p = 0; p < kP; ++p) S[p] = fmaf(bv, __bfloat162float(pX[r * kP + p]), S[p]);
+                    for (int p = 0; p < kP / 2; ++p) S[p] = fmaf(bv, __bfloat162float(pX[r * kP + c0 + p]), S[p]);
                 }
             }
         }
         if (!SUMMARY) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 uint4 v;
                 v.x = pack_bf16x2(S[8 * c + 0], S[8 * c + 1]);
                 v.y = pack_bf16x2(S[8 * c + 2], S[8 * c + 3]);
                 v.z = pack_bf16x2(S[8 * c + 4], S[8 * c + 5]);
                 v.w = pack_bf16x2(S[8 * c + 6], S[8 * c + 7]);
-                *reinterpret_cast<uint4*>(smem + OFF_S + sw128(n, c)) = v;
+                *reinterpret_cast<uint4*>(smem + OFF_S + sw128(n, 4 * wg + c)) = v;
             }
             fence_async_smem();
         }
@@ -307,6 +364,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = m->tmem_base;
+    const uint32_t tlane = tmem + ((uint32_t)(wq * 32) << 16);   // this warp's lane quarter
 
     const float* theta = q.theta;
     const float* dtp = q.dt;
@@ -329,7 +387,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (warp == 0) {
             if (lane == 0) {
                 // ---------------- producer + MMA issuer
-                if (k > 0) mbar_wait(&m->bar[BAR_FREE], (k - 1) & 1, m, status, 1);
+                // The previous tile's MMAs are the last readers of B, C, X: once
+                // they complete, the next tile's loads can land while the
+                // workers still run that tile's epilogue.
+                if (k > 0) mbar_wait(&m->bar[BAR_Y], (k - 1) & 1, m, status, 1);
                 const uint32_t bytes = SUMMARY ? (32768u + 16384u) : (65536u + 16384u);
                 mbar_expect_tx(&m->bar[BAR_LOAD], bytes);
                 tma_load_5d(sbase + OFF_B, &tmB, &m->bar[BAR_LOAD], 0, 0, g, t0, b);
@@ -388,11 +449,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
 
         // ---------------------------------------------------------- workers
-        const int pi = wk & 63, half = wk >> 6;
-        float th[TH];
+        // token work mapping: rotary pair pi, token quarter qt
+        const int pi = wk & 63, qt = wk >> 6;
+        float th[TQ];
 #pragma unroll
-        for (int kk = 0; kk < TH; ++kk) {
-            const int t = half * TH + kk;
+        for (int kk = 0; kk < TQ; ++kk) {
+            const int t = qt * TQ + kk;
             th[kk] = (t < qc) ? __ldg(theta + (((size_t)b * L + t0 + t) * G + g) * (kN / 2) + pi) : 0.f;
         }
         if (wk < T) {
@@ -433,51 +495,58 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const float a = m->a[wk];
                 m->gam[wk] = gam;
                 m->cf[wk] = c;
-                m->w[wk] = expf(a_last - a) * c;
-                m->ea[wk] = expf(a);
+                m->w[wk] = exp2f((a_last - a) * kLog2e) * c;
+                m->ea[wk] = exp2f(a * kLog2e);
+                m->a2[wk] = a * kLog2e;
             } else {
                 m->gam[wk] = 0.f; m->cf[wk] = 0.f; m->w[wk] = 0.f; m->ea[wk] = 0.f;
+                m->a2[wk] = a_last * kLog2e;
             }
         }
-        // phase pass 1: this half's total
+        // phase pass 1: this quarter's total
         const double carry = m->phi[pi];
         double acc = 0.0;
 #pragma unroll
-        for (int kk = 0; kk < TH; ++kk) acc += (double)m->dt[half * TH + kk] * (double)th[kk];
-        if (half == 0) m->half_sum[pi] = acc;
+        for (int kk = 0; kk < TQ; ++kk) acc += (double)(m->dt[qt * TQ + kk] * th[kk]);
+        m->qsum[qt][pi] = acc;
         if (wk == 0) {
-            m->scal[0] = expf(a_last);
+            m->scal[0] = exp2f(a_last * kLog2e);
             m->scal[1] += a_last;
         }
         mbar_wait(&m->bar[BAR_LOAD], par, m, status, 10);
         workers_sync();
-        const double start = carry + (half ? m->half_sum[pi] : 0.0);
-        if (half == 1) m->phi[pi] = wrap_pi(start + acc);
-        // phase pass 2: rotate B (and C) rows (t, r) at pair pi, in place
+        double start = carry;
+        for (int j = 0; j < qt; ++j) start += m->qsum[j][pi];
+        if (qt == 3) m->phi[pi] = wrap_pi(start + acc);
+        // phase pass 2: rotate B (and C) rows (t, r) at pair pi, in place.
+        // The start phase is exact (double, reduced); inside the quarter the
+        // running phase is float, reduced every token.
         {
             const uint32_t atom = (uint32_t)(pi >> 5) * 16384u;
             const int chunk = (pi & 31) >> 2;
             const uint32_t inb = (uint32_t)(pi & 3) * 4u;
-            double ph = start;
+            float ph = (float)wrap_pi(start);
 #pragma unroll
-            for (int kk = 0; kk < TH; ++kk) {
-                const int t = half * TH + kk;
-                ph += (double)m->dt[t] * (double)th[kk];
+            for (int kk = 0; kk < TQ; ++kk) {
+                const int t = qt * TQ + kk;
+                ph = wrap_pi_f(fmaf(m->dt[t], th[kk], ph));
                 if (t < qc) {
                     float sv, cv;
-                    __sincosf((float)wrap_pi(ph), &sv, &cv);
-                    const float wsc = SUMMARY ? m->w[t] : 1.f;
+                    __sincosf(ph, &sv, &cv);
+                    float2 cc = make_float2(cv, cv), sn = make_float2(sv, -sv);
+                    if (SUMMARY) {
+                        const float wsc = m->w[t];
+                        cc = make_float2(wsc * cv, wsc * cv);
+                        sn = make_float2(wsc * sv, -wsc * sv);
+                    }
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
-                        const int rw = t * R + r;
-                        const uint32_t off = atom + sw128(rw, chunk) + inb;
+                        const uint32_t off = atom + sw128(t * R + r, chunk) + inb;
                         uint32_t* pb = reinterpret_cast<uint32_t*>(smem + OFF_B + off);
-                        const float2 bv = unpack_bf16x2(*pb);
-                        *pb = pack_bf16x2(wsc * (cv * bv.x + sv * bv.y), wsc * (-sv * bv.x + cv * bv.y));
+                        *pb = pack2(rot_t(unpack_bf16x2(*pb), cc, sn));
                         if (!SUMMARY) {
                             uint32_t* pc = reinterpret_cast<uint32_t*>(smem + OFF_C + off);
-                            const float2 cvv = unpack_bf16x2(*pc);
-                            *pc = pack_bf16x2(cv * cvv.x + sv * cvv.y, -sv * cvv.x + cv * cvv.y);
+                            *pc = pack2(rot_t(unpack_bf16x2(*pc), cc, sn));
                         }
                     }
                 }
@@ -490,47 +559,49 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!SUMMARY) {
             mbar_wait(&m->bar[BAR_G], par, m, status, 11);
             tc_fence_after();
-            // scale row `row` of B~ by w_t (the state contribution weight)
+            // scale this warpgroup's atom of row `row` of B~ by w_t
             {
                 const float wt = m->w[tr];
+                const float2 w2 = make_float2(wt, wt);
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    uint4* p = reinterpret_cast<uint4*>(smem + OFF_B + (c >> 3) * 16384 + sw128(row, c & 7));
-                    uint4 v = *p;
-                    float2 f;
-                    f = unpack_bf16x2(v.x); v.x = pack_bf16x2(wt * f.x, wt * f.y);
-                    f = unpack_bf16x2(v.y); v.y = pack_bf16x2(wt * f.x, wt * f.y);
-                    f = unpack_bf16x2(v.z); v.z = pack_bf16x2(wt * f.x, wt * f.y);
-                    f = unpack_bf16x2(v.w); v.w = pack_bf16x2(wt * f.x, wt * f.y);
-                    *p = v;
+                for (int c = 0; c < 8; ++c) {
+                    uint4* p = reinterpret_cast<uint4*>(smem + OFF_B + wg * 16384 + sw128(row, c));
+                    *p = scale_chunk(*p, w2);
                 }
             }
             fence_async_smem();
             mbar_arrive(&m->bar[BAR_BW]);
-            // P = (two-band decay mask) o G, bf16, K-major over C~'s smem
+            // P = (two-band decay mask) o G on this warpgroup's 64 columns,
+            // bf16, K-major over C~'s smem
             {
-                const float a_t = m->a[tr];
+                const float a2t = m->a2[tr];
 #pragma unroll 1
-                for (int cg = 0; cg < 4; ++cg) {
+                for (int cg = 0; cg < 2; ++cg) {
+                    const int col0 = wg * 64 + cg * 32;
                     float v[32];
-                    tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + cg * 32, v);
+                    tmem_ld32(tlane + col0, v);
 #pragma unroll
                     for (int j0 = 0; j0 < 32; j0 += R) {
-                        const int u = (cg * 32 + j0) / R;
+                        const int u = (col0 + j0) / R;
                         float mk = 0.f;
-                        if (u <= tr) mk = expf(a_t - m->a[u]) * (u == tr ? m->gam[u] : m->cf[u]);
+                        if (u <= tr) mk = exp2f(a2t - m->a2[u]) * (u == tr ? m->gam[u] : m->cf[u]);
+                        const float2 mk2 = make_float2(mk, mk);
 #pragma unroll
-                        for (int r = 0; r < R; ++r) v[j0 + r] *= mk;
+                        for (int r = 0; r < R; r += 2) {
+                            if (R == 1) {
+                                v[j0] *= mk;
+                            } else {
+                                const float2 g2 = __fmul2_rn(mk2, make_float2(v[j0 + r], v[j0 + r + 1]));
+                                v[j0 + r] = g2.x;
+                                v[j0 + r + 1] = g2.y;
+                            }
+                        }
                     }
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        const int cc = cg * 4 + c;      // 16-byte chunk over 128 columns
-                        uint4 o;
-                        o.x = pack_bf16x2(v[8 * c + 0], v[8 * c + 1]);
-                        o.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
-                        o.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
-                        o.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
-                        *reinterpret_cast<uint4*>(smem + OFF_C + (cc >> 3) * 16384 + sw128(row, cc & 7)) = o;
+                        const int cc = (col0 >> 3) + c;      // 16-byte chunk over 128 columns
+                        *reinterpret_cast<uint4*>(smem + OFF_C + (cc >> 3) * 16384 + sw128(row, cc & 7)) =
+                            pack_chunk(v + 8 * c);
                     }
                 }
             }
@@ -541,54 +612,49 @@ __global__ void __launch_bounds__(kThreads, 2)
 
         mbar_wait(&m->bar[BAR_Y], par, m, status, 12);
         tc_fence_after();
-        // state: S = e^{a_last} S + S_loc   (thread = state row)
+        // state: S = e^{a_last} S + S_loc  (thread = state row, this half's columns)
         {
             const float dec = m->scal[0];
+            const float2 dec2 = make_float2(dec, dec);
+            float v[32];
+            tmem_ld32(tlane + 128 + c0, v);
 #pragma unroll
-            for (int cg = 0; cg < 2; ++cg) {
-                float v[32];
-                tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + 128 + cg * 32, v);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) S[cg * 32 + j] = fmaf(dec, S[cg * 32 + j], v[j]);
+            for (int j = 0; j < 32; j += 2) {
+                const float2 s2 = __ffma2_rn(dec2, make_float2(S[j], S[j + 1]), make_float2(v[j], v[j + 1]));
+                S[j] = s2.x;
+                S[j + 1] = s2.y;
             }
             if (!SUMMARY) {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint4 v;
-                    v.x = pack_bf16x2(S[8 * c + 0], S[8 * c + 1]);
-                    v.y = pack_bf16x2(S[8 * c + 2], S[8 * c + 3]);
-                    v.z = pack_bf16x2(S[8 * c + 4], S[8 * c + 5]);
-                    v.w = pack_bf16x2(S[8 * c + 6], S[8 * c + 7]);
-                    *reinterpret_cast<uint4*>(smem + OFF_S + sw128(row, c)) = v;
-                }
+                for (int c = 0; c < 4; ++c)
+                    *reinterpret_cast<uint4*>(smem + OFF_S + sw128(row, 4 * wg + c)) = pack_chunk(S + 8 * c);
             }
         }
         if (!SUMMARY) {
-            // y = Y_intra + e^{a_t} Y_inter  (thread = tile row (t, r))
+            // y = Y_intra + e^{a_t} Y_inter  (thread = tile row (t, r), this half's columns)
             const float ea = m->ea[tr];
+            const float2 ea2 = make_float2(ea, ea);
 #pragma unroll 1
-            for (int cg = 0; cg < 2; ++cg) {
-                float yi[32], yx[32];
-                tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + cg * 32, yi);
-                tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + 192 + cg * 32, yx);
+            for (int hh = 0; hh < 2; ++hh) {
+                float yi[16], yx[16];
+                tmem_ld16(tlane + c0 + 16 * hh, yi);
+                tmem_ld16(tlane + 192 + c0 + 16 * hh, yx);
+#pragma unroll
+                for (int j = 0; j < 16; j += 2) {
+                    const float2 o2 = __ffma2_rn(ea2, make_float2(yx[j], yx[j + 1]), make_float2(yi[j], yi[j + 1]));
+                    yi[j] = o2.x;
+                    yi[j + 1] = o2.y;
+                }
                 if (tr < qc) {
                     uint4* dst = reinterpret_cast<uint4*>(
-                        yg + ((((size_t)b * L + t0 + tr) * H + h) * R + (row % R)) * kP + cg * 32);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint4 o;
-                        o.x = pack_bf16x2(fmaf(ea, yx[8 * c + 0], yi[8 * c + 0]), fmaf(ea, yx[8 * c + 1], yi[8 * c + 1]));
-                        o.y = pack_bf16x2(fmaf(ea, yx[8 * c + 2], yi[8 * c + 2]), fmaf(ea, yx[8 * c + 3], yi[8 * c + 3]));
-                        o.z = pack_bf16x2(fmaf(ea, yx[8 * c + 4], yi[8 * c + 4]), fmaf(ea, yx[8 * c + 5], yi[8 * c + 5]));
-                        o.w = pack_bf16x2(fmaf(ea, yx[8 * c + 6], yi[8 * c + 6]), fmaf(ea, yx[8 * c + 7], yi[8 * c + 7]));
-                        dst[c] = o;
-                    }
+                        yg + ((((size_t)b * L + t0 + tr) * H + h) * R + (row % R)) * kP + c0 + 16 * hh);
+                    dst[0] = pack_chunk(yi);
+                    dst[1] = pack_chunk(yi + 8);
                 }
             }
         }
         fence_async_smem();
         tc_fence_before();
-        mbar_arrive(&m->bar[BAR_FREE]);
     }
 
     // ---- epilogue of the segment
@@ -596,24 +662,24 @@ __global__ void __launch_bounds__(kThreads, 2)
         // an aborted tile may still have a TMA load in flight: let it land
         if (pending_load) mbar_wait_flag(&m->bar[BAR_LOAD], load_par, &m->drain_flag, nullptr, 0);
         // all MMAs this thread issued are complete before TMEM is freed
-        umma_commit(&m->bar[7]);
-        mbar_wait_flag(&m->bar[7], 0, &m->drain_flag, nullptr, 0);
+        umma_commit(&m->bar[BAR_DRAIN]);
+        mbar_wait_flag(&m->bar[BAR_DRAIN], 0, &m->drain_flag, nullptr, 0);
     }
     if (warp > 0) {
         const int n = row;
         if (SUMMARY) {
-            float4* dst = reinterpret_cast<float4*>(q.ws_sloc + (bhs * kN + n) * kP);
+            float4* dst = reinterpret_cast<float4*>(q.ws_sloc + (bhs * kN + n) * kP + c0);
 #pragma unroll
-            for (int c = 0; c < kP / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
+            for (int c = 0; c < kP / 8; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
             if (wk < 64) q.ws_phase[bhs * (kN / 2) + wk] = (float)m->phi[wk];
             if (wk == 0) q.ws_decay[bhs] = m->scal[1];
         } else if (seg == q.nseg - 1) {
             if (q.fin_h) {
                 float sv, cv;
                 sincosf((float)m->phi[n >> 1], &sv, &cv);
-                float* dst = q.fin_h + (bh * kN + n) * kP;
+                float* dst = q.fin_h + (bh * kN + n) * kP + c0;
 #pragma unroll
-                for (int p = 0; p < kP; ++p) {
+                for (int p = 0; p < kP / 2; ++p) {
                     const float other = __shfl_xor_sync(0xffffffffu, S[p], 1);
                     dst[p] = (n & 1) ? (sv * other + cv * S[p]) : (cv * S[p] - sv * other);
                 }
@@ -621,12 +687,12 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (q.fin_pB && L > 0) {
                 const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(q.B) + (((size_t)b * L + L - 1) * G + g) * R * kN;
                 __nv_bfloat16* o = static_cast<__nv_bfloat16*>(q.fin_pB) + bh * R * kN;
-                for (int e = wk; e < R * kN; e += 128) o[e] = s[e];
+                for (int e = wk; e < R * kN; e += kWorkers) o[e] = s[e];
             }
             if (q.fin_pX && L > 0) {
                 const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(q.x) + (((size_t)b * L + L - 1) * H + h) * R * kP;
                 __nv_bfloat16* o = static_cast<__nv_bfloat16*>(q.fin_pX) + bh * R * kP;
-                for (int e = wk; e < R * kP; e += 128) o[e] = s[e];
+                for (int e = wk; e < R * kP; e += kWorkers) o[e] = s[e];
             }
         }
     }
@@ -688,6 +754,9 @@ static cudaError_t launch_tc_R(const ScanParams& q, int* status, cudaStream_t st
         return cudaErrorInvalidValue;
     cudaFuncSetAttribute(scan_tc_kernel<R, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     cudaFuncSetAttribute(scan_tc_kernel<R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    // two CTAs per SM need the largest shared-memory carveout
+    cudaFuncSetAttribute(scan_tc_kernel<R, false>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    cudaFuncSetAttribute(scan_tc_kernel<R, true>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (q.nseg > 1) {
         scan_tc_kernel<R, true><<<dim3(q.nseg - 1, q.nheads, q.batch), kThreads, SMEM_BYTES, st>>>(mB, mC, mX, q, status);
         cudaError_t e = launch_scan_combine(q, st);
