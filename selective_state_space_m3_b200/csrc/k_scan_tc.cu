@@ -47,8 +47,11 @@ namespace tc {
 constexpr int kRows = 128;
 constexpr int kN = 128;
 constexpr int kP = 64;
-constexpr int kWorkers = 256;
+constexpr int kWG = 2;                 // worker warpgroups
+constexpr int kWorkers = 128 * kWG;
 constexpr int kThreads = 32 + kWorkers;
+constexpr int kNQ = kWorkers / 64;     // token groups of the phase pass
+constexpr int kSC = kP / kWG;          // state / y columns per warpgroup
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 // shared memory map (offsets from a 1024-byte aligned base)
@@ -57,7 +60,7 @@ constexpr int OFF_C = 32768;      // 32 KB: C~, later P
 constexpr int OFF_X = 65536;      // 16 KB: X
 constexpr int OFF_S = 81920;      // 16 KB: S_bf (rows n, 64 p)
 constexpr int OFF_MISC = 98304;
-constexpr int MISC_BYTES = 7168;
+constexpr int MISC_BYTES = 12288;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;   // + alignment slack
 
 struct Misc {
@@ -68,10 +71,11 @@ struct Misc {
     int pad[13];
     float dt[128], lam[128];
     float a[128], a2[128], gam[128], cf[128], w[128], ea[128];
-    float scan[8];
+    float scan[kWorkers / 32];
     float scal[4];                // [0] tile decay, [1] segment log-decay, [2..3] next dt/lambda
     double phi[64];               // phase carry per rotary pair (reduced)
-    double qsum[4][64];           // per-quarter phase totals of the current tile
+    double qsum[kNQ][64];         // per-token-group phase totals of the current tile
+    float msk[32 * 36];           // decay mask per (token, token), rows padded (R >= 4)
 };
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region too small");
 
@@ -103,8 +107,7 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
 
 // Bounded wait.  Returns false when the CTA is aborting (this wait or an
 // earlier one expired); the caller then carries on without waiting.
-__device__ __noinline__ bool mbar_wait_flag(uint64_t* b, uint32_t parity, int* abortp, int* status, int where) {
-    if (mbar_try(b, parity)) return true;
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* b, uint32_t parity, int* abortp, int* status, int where) {
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try(b, parity)) return true;
@@ -119,6 +122,12 @@ __device__ __noinline__ bool mbar_wait_flag(uint64_t* b, uint32_t parity, int* a
         }
     }
 }
+// the common case (the phase completes within try_wait's own suspend window)
+// stays inline; the bounded spin is out of line
+__device__ __forceinline__ bool mbar_wait_flag(uint64_t* b, uint32_t parity, int* abortp, int* status, int where) {
+    if (mbar_try(b, parity)) return true;
+    return mbar_wait_slow(b, parity, abortp, status, where);
+}
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Misc* m, int* status, int where) {
     return mbar_wait_flag(b, parity, &m->abort_flag, status, where);
 }
@@ -132,21 +141,24 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void workers_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-// all 256 workers get the OR of `cond` (named barrier 1 with a reduction), so
+__device__ __forceinline__ void workers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kWorkers) : "memory"); }
+// all workers get the OR of `cond` (named barrier 1 with a reduction), so
 // they take the same branch
 __device__ __forceinline__ int workers_any(int cond) {
     int r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.s32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, 1, 256, p;\n\t"
+        "bar.red.or.pred q, 1, %2, p;\n\t"
         "selp.s32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"(cond)
+        : "r"(cond), "n"(kWorkers)
         : "memory");
     return r;
 }
@@ -276,10 +288,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     scan_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
                    const __grid_constant__ CUtensorMap tmX, ScanParams q, int* status) {
     constexpr int T = kRows / R;       // tokens per tile
-    constexpr int TQ = T / 4;          // tokens per quarter tile (phase pass)
+    constexpr int TQ = T / kNQ;        // tokens per token group (phase pass)
     constexpr float kLog2e = 1.4426950408889634f;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned base for the SWIZZLE_128B tiles, derived by an offset
+    // from the shared array so that every access stays a 32-bit shared access
+    uint8_t* smem = smem_raw + ((1024u - (su32(smem_raw) & 1023u)) & 1023u);
     Misc* m = reinterpret_cast<Misc*>(smem + OFF_MISC);
     const uint32_t sbase = su32(smem);
 
@@ -318,24 +332,24 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int wg = wk >> 7;                   // warpgroup: column half of row work
     const int wq = warp & 3;                  // TMEM lane quarter of this warp
     const int row = wq * 32 + lane;           // tile row / state row owned in TMEM
-    const int c0 = wg * (kP / 2);             // this warpgroup's state / y columns
-    float S[kP / 2];                          // state row `row`, columns c0 .. c0+31
+    const int c0 = wg * kSC;                  // this warpgroup's state / y columns
+    float S[kSC];                             // state row `row`, columns c0 .. c0+kSC-1
     if (warp > 0) {
         if (wk < 64) m->phi[wk] = 0.0;
         const int n = row;
         if (SUMMARY) {
 #pragma unroll
-            for (int p = 0; p < kP / 2; ++p) S[p] = 0.f;
+            for (int p = 0; p < kSC; ++p) S[p] = 0.f;
         } else if (q.nseg > 1) {
             const float4* src = reinterpret_cast<const float4*>(q.ws_sin + (bhs * kN + n) * kP + c0);
 #pragma unroll
-            for (int c = 0; c < kP / 8; ++c) {
+            for (int c = 0; c < kSC / 4; ++c) {
                 const float4 v = src[c];
                 S[4 * c] = v.x; S[4 * c + 1] = v.y; S[4 * c + 2] = v.z; S[4 * c + 3] = v.w;
             }
         } else {
 #pragma unroll
-            for (int p = 0; p < kP / 2; ++p) S[p] = q.init_h ? q.init_h[(bh * kN + n) * kP + c0 + p] : 0.f;
+            for (int p = 0; p < kSC; ++p) S[p] = q.init_h ? q.init_h[(bh * kN + n) * kP + c0 + p] : 0.f;
             if (q.init_pB && q.init_pX) {
                 const float w0 = (1.f - q.lam[(size_t)b * L * H + h]) * q.dt[(size_t)b * L * H + h];
                 const __nv_bfloat16* pB = static_cast<const __nv_bfloat16*>(q.init_pB) + bh * R * kN;
@@ -343,19 +357,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int r = 0; r < R; ++r) {
                     const float bv = w0 * __bfloat162float(pB[r * kN + n]);
 #pragma unroll
-                    for (int p = 0; p < kP / 2; ++p) S[p] = fmaf(bv, __bfloat162float(pX[r * kP + c0 + p]), S[p]);
+                    for (int p = 0; p < kSC; ++p) S[p] = fmaf(bv, __bfloat162float(pX[r * kP + c0 + p]), S[p]);
                 }
             }
         }
         if (!SUMMARY) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < kSC / 8; ++c) {
                 uint4 v;
                 v.x = pack_bf16x2(S[8 * c + 0], S[8 * c + 1]);
                 v.y = pack_bf16x2(S[8 * c + 2], S[8 * c + 3]);
                 v.z = pack_bf16x2(S[8 * c + 4], S[8 * c + 5]);
                 v.w = pack_bf16x2(S[8 * c + 6], S[8 * c + 7]);
-                *reinterpret_cast<uint4*>(smem + OFF_S + sw128(n, 4 * wg + c)) = v;
+                *reinterpret_cast<uint4*>(smem + OFF_S + sw128(n, c0 / 8 + c)) = v;
             }
             fence_async_smem();
         }
@@ -366,10 +380,82 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t tmem = m->tmem_base;
     const uint32_t tlane = tmem + ((uint32_t)(wq * 32) << 16);   // this warp's lane quarter
 
-    const float* theta = q.theta;
-    const float* dtp = q.dt;
-    const float* lamp = q.lam;
     __nv_bfloat16* yg = static_cast<__nv_bfloat16*>(q.y);
+
+    // Per-tile inputs of the SIMT work (theta for this thread's rotary pair and
+    // token group, dt and lambda of token wk, the next token's dt/lambda).
+    // For R >= 2 they are loaded into registers one tile ahead, right after
+    // the previous tile's MMAs complete, so their latency overlaps that
+    // tile's epilogue; for R = 1 (32 theta values per thread) they are loaded
+    // at the tile's start after an L2 prefetch one tile ahead.
+    constexpr bool kRegPrefetch = (TQ <= 16);
+    const int pi = wk & 63, qt = wk >> 6;     // token work: rotary pair, token group
+    float th_n[TQ];
+    float dt_n = 0.f, lam_n = 1.f, dt_x = 0.f, lam_x = 1.f;
+    auto load_inputs = [&](int kn) {
+        const int t0n = tok0 + kn * T;
+        const int qcn = min(T, tok1 - t0n);
+#pragma unroll
+        for (int kk = 0; kk < TQ; ++kk) {
+            const int t = qt * TQ + kk;
+            th_n[kk] = (t < qcn) ? __ldg(q.theta + (((size_t)b * L + t0n + t) * G + g) * (kN / 2) + pi) : 0.f;
+        }
+        if (wk < T) {
+            const size_t o = ((size_t)b * L + t0n + wk) * H + h;
+            dt_n = (wk < qcn) ? __ldg(q.dt + o) : 0.f;
+            lam_n = (wk < qcn) ? __ldg(q.lam + o) : 1.f;
+        }
+        if (wk == 0) {
+            const int tn = t0n + qcn;
+            const size_t o = ((size_t)b * L + tn) * H + h;
+            dt_x = (tn < L) ? __ldg(q.dt + o) : 0.f;
+            lam_x = (tn < L) ? __ldg(q.lam + o) : 1.f;
+        }
+    };
+    auto prefetch_inputs = [&](int kn) {
+        const int tn0 = tok0 + kn * T;
+        const int qn = min(T, tok1 - tn0);
+        for (int j = wk; j < 4 * T; j += kWorkers) {
+            if (j < 2 * T) {
+                const int t = j >> 1;
+                if (t < qn) prefetch_l2(q.theta + (((size_t)b * L + tn0 + t) * G + g) * (kN / 2) + (j & 1) * 32);
+            } else {
+                const int t = (j - 2 * T) % T;
+                if (t < qn) prefetch_l2((j < 3 * T ? q.dt : q.lam) + ((size_t)b * L + tn0 + t) * H + h);
+            }
+        }
+    };
+    // y = Y_intra + e^{a_t} Y_inter of a finished tile (thread = tile row (t, r),
+    // this warpgroup's columns); run after the next tile's coefficient step
+    auto emit_y = [&](int t0y, int qcy, float eay) {
+        const float2 ea2 = make_float2(eay, eay);
+#pragma unroll 1
+        for (int hh = 0; hh < kSC / 16; ++hh) {
+            float yi[16], yx[16];
+            tmem_ld16(tlane + c0 + 16 * hh, yi);
+            tmem_ld16(tlane + 192 + c0 + 16 * hh, yx);
+#pragma unroll
+            for (int j = 0; j < 16; j += 2) {
+                const float2 o2 = __ffma2_rn(ea2, make_float2(yx[j], yx[j + 1]), make_float2(yi[j], yi[j + 1]));
+                yi[j] = o2.x;
+                yi[j + 1] = o2.y;
+            }
+            const int try_ = row / R;
+            if (try_ < qcy) {
+                uint4* dst = reinterpret_cast<uint4*>(
+                    yg + ((((size_t)b * L + t0y + try_) * H + h) * R + (row % R)) * kP + c0 + 16 * hh);
+                dst[0] = pack_chunk(yi);
+                dst[1] = pack_chunk(yi + 8);
+            }
+        }
+    };
+    bool y_pending = false;                   // a tile's y is waiting to be emitted
+    int y_t0 = 0, y_qc = 0;
+    float y_ea = 0.f;
+    if (warp > 0 && ntiles > 0) {
+        if (kRegPrefetch) load_inputs(0);
+        else if (ntiles > 1) prefetch_inputs(1);
+    }
 
     uint32_t pending_load = 0;   // control lane: a TMA load is in flight
     uint32_t load_par = 0;       // its mbarrier phase
@@ -449,24 +535,20 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
 
         // ---------------------------------------------------------- workers
-        // token work mapping: rotary pair pi, token quarter qt
-        const int pi = wk & 63, qt = wk >> 6;
+        if (!kRegPrefetch) {
+            load_inputs(k);
+            if (k + 2 < ntiles) prefetch_inputs(k + 2);
+        }
         float th[TQ];
 #pragma unroll
-        for (int kk = 0; kk < TQ; ++kk) {
-            const int t = qt * TQ + kk;
-            th[kk] = (t < qc) ? __ldg(theta + (((size_t)b * L + t0 + t) * G + g) * (kN / 2) + pi) : 0.f;
-        }
+        for (int kk = 0; kk < TQ; ++kk) th[kk] = th_n[kk];
         if (wk < T) {
-            const size_t o = ((size_t)b * L + t0 + wk) * H + h;
-            m->dt[wk] = (wk < qc) ? __ldg(dtp + o) : 0.f;
-            m->lam[wk] = (wk < qc) ? __ldg(lamp + o) : 1.f;
+            m->dt[wk] = dt_n;
+            m->lam[wk] = lam_n;
         }
         if (wk == 0) {
-            const int tn = t0 + qc;
-            const size_t o = ((size_t)b * L + tn) * H + h;
-            m->scal[2] = (tn < L) ? __ldg(dtp + o) : 0.f;
-            m->scal[3] = (tn < L) ? __ldg(lamp + o) : 1.f;
+            m->scal[2] = dt_x;
+            m->scal[3] = lam_x;
         }
         workers_sync();
         // a_t = sum_{s<=t} dt_s A (inclusive block scan over the tile's tokens)
@@ -503,6 +585,23 @@ __global__ void __launch_bounds__(kThreads, 2)
                 m->a2[wk] = a_last * kLog2e;
             }
         }
+        if (!SUMMARY && R >= 4) {
+            // decay mask per (token t, token u) of the tile, shared by the R x R
+            // rank block: e^{a_t - a_u} (gamma_u if u == t, c_u if u < t), 0 above
+            workers_sync();
+            constexpr int LD = T + 4;
+            for (int e = wk; e < T * T; e += kWorkers) {
+                const int t = e / T, u = e % T;
+                float v = 0.f;
+                if (u <= t) v = exp2f(m->a2[t] - m->a2[u]) * (u == t ? m->gam[u] : m->cf[u]);
+                m->msk[t * LD + u] = v;
+            }
+        }
+        // the previous tile's output, while this tile's TMA load lands
+        if (!SUMMARY && y_pending) {
+            emit_y(y_t0, y_qc, y_ea);
+            y_pending = false;
+        }
         // phase pass 1: this quarter's total
         const double carry = m->phi[pi];
         double acc = 0.0;
@@ -517,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         workers_sync();
         double start = carry;
         for (int j = 0; j < qt; ++j) start += m->qsum[j][pi];
-        if (qt == 3) m->phi[pi] = wrap_pi(start + acc);
+        if (qt == kNQ - 1) m->phi[pi] = wrap_pi(start + acc);
         // phase pass 2: rotate B (and C) rows (t, r) at pair pi, in place.
         // The start phase is exact (double, reduced); inside the quarter the
         // running phase is float, reduced every token.
@@ -553,6 +652,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
         fence_async_smem();
+        tc_fence_before();       // the deferred y's TMEM reads precede the next MMAs
         mbar_arrive(&m->bar[BAR_OPS]);
 
         const int tr = row / R;              // token of this thread's tile row
@@ -564,8 +664,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const float wt = m->w[tr];
                 const float2 w2 = make_float2(wt, wt);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint4* p = reinterpret_cast<uint4*>(smem + OFF_B + wg * 16384 + sw128(row, c));
+                for (int c = 0; c < 16 / kWG; ++c) {
+                    const int cc = wg * (16 / kWG) + c;   // 16-byte chunk of the 256-byte row
+                    uint4* p = reinterpret_cast<uint4*>(smem + OFF_B + (cc >> 3) * 16384 + sw128(row, cc & 7));
                     *p = scale_chunk(*p, w2);
                 }
             }
@@ -576,25 +677,35 @@ __global__ void __launch_bounds__(kThreads, 2)
             {
                 const float a2t = m->a2[tr];
 #pragma unroll 1
-                for (int cg = 0; cg < 2; ++cg) {
-                    const int col0 = wg * 64 + cg * 32;
+                for (int cg = 0; cg < 128 / kWG / 32; ++cg) {
+                    const int col0 = wg * (128 / kWG) + cg * 32;
                     float v[32];
                     tmem_ld32(tlane + col0, v);
+                    if (R >= 4) {
+                        // mask from the per-tile table, one value per R columns
+                        constexpr int LD = T + 4;
+                        const float4* mrow = reinterpret_cast<const float4*>(m->msk + tr * LD + col0 / R);
+                        float mk[32 / R];
 #pragma unroll
-                    for (int j0 = 0; j0 < 32; j0 += R) {
-                        const int u = (col0 + j0) / R;
-                        float mk = 0.f;
-                        if (u <= tr) mk = exp2f(a2t - m->a2[u]) * (u == tr ? m->gam[u] : m->cf[u]);
-                        const float2 mk2 = make_float2(mk, mk);
+                        for (int q4 = 0; q4 < 32 / R / 4; ++q4) {
+                            const float4 f = mrow[q4];
+                            mk[4 * q4] = f.x; mk[4 * q4 + 1] = f.y; mk[4 * q4 + 2] = f.z; mk[4 * q4 + 3] = f.w;
+                        }
 #pragma unroll
-                        for (int r = 0; r < R; r += 2) {
-                            if (R == 1) {
-                                v[j0] *= mk;
-                            } else {
-                                const float2 g2 = __fmul2_rn(mk2, make_float2(v[j0 + r], v[j0 + r + 1]));
-                                v[j0 + r] = g2.x;
-                                v[j0 + r + 1] = g2.y;
-                            }
+                        for (int j = 0; j < 32; j += 2) {
+                            const float2 g2 = __fmul2_rn(make_float2(mk[j / R], mk[(j + 1) / R]),
+                                                         make_float2(v[j], v[j + 1]));
+                            v[j] = g2.x;
+                            v[j + 1] = g2.y;
+                        }
+                    } else {
+                        const float a2t = m->a2[tr];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int u = (col0 + j) / R;
+                            const float mkv =
+                                (u <= tr) ? exp2f(a2t - m->a2[u]) * (u == tr ? m->gam[u] : m->cf[u]) : 0.f;
+                            v[j] *= mkv;
                         }
                     }
 #pragma unroll
@@ -612,46 +723,34 @@ __global__ void __launch_bounds__(kThreads, 2)
 
         mbar_wait(&m->bar[BAR_Y], par, m, status, 12);
         tc_fence_after();
+        if (kRegPrefetch && k + 1 < ntiles) load_inputs(k + 1);
         // state: S = e^{a_last} S + S_loc  (thread = state row, this half's columns)
         {
             const float dec = m->scal[0];
             const float2 dec2 = make_float2(dec, dec);
-            float v[32];
-            tmem_ld32(tlane + 128 + c0, v);
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                const float2 s2 = __ffma2_rn(dec2, make_float2(S[j], S[j + 1]), make_float2(v[j], v[j + 1]));
-                S[j] = s2.x;
-                S[j + 1] = s2.y;
+            for (int h16 = 0; h16 < kSC / 16; ++h16) {
+                float v[16];
+                tmem_ld16(tlane + 128 + c0 + 16 * h16, v);
+#pragma unroll
+                for (int j = 0; j < 16; j += 2) {
+                    const int jj = 16 * h16 + j;
+                    const float2 s2 = __ffma2_rn(dec2, make_float2(S[jj], S[jj + 1]), make_float2(v[j], v[j + 1]));
+                    S[jj] = s2.x;
+                    S[jj + 1] = s2.y;
+                }
             }
             if (!SUMMARY) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    *reinterpret_cast<uint4*>(smem + OFF_S + sw128(row, 4 * wg + c)) = pack_chunk(S + 8 * c);
+                for (int c = 0; c < kSC / 8; ++c)
+                    *reinterpret_cast<uint4*>(smem + OFF_S + sw128(row, c0 / 8 + c)) = pack_chunk(S + 8 * c);
             }
         }
         if (!SUMMARY) {
-            // y = Y_intra + e^{a_t} Y_inter  (thread = tile row (t, r), this half's columns)
-            const float ea = m->ea[tr];
-            const float2 ea2 = make_float2(ea, ea);
-#pragma unroll 1
-            for (int hh = 0; hh < 2; ++hh) {
-                float yi[16], yx[16];
-                tmem_ld16(tlane + c0 + 16 * hh, yi);
-                tmem_ld16(tlane + 192 + c0 + 16 * hh, yx);
-#pragma unroll
-                for (int j = 0; j < 16; j += 2) {
-                    const float2 o2 = __ffma2_rn(ea2, make_float2(yx[j], yx[j + 1]), make_float2(yi[j], yi[j + 1]));
-                    yi[j] = o2.x;
-                    yi[j + 1] = o2.y;
-                }
-                if (tr < qc) {
-                    uint4* dst = reinterpret_cast<uint4*>(
-                        yg + ((((size_t)b * L + t0 + tr) * H + h) * R + (row % R)) * kP + c0 + 16 * hh);
-                    dst[0] = pack_chunk(yi);
-                    dst[1] = pack_chunk(yi + 8);
-                }
-            }
+            y_pending = true;
+            y_t0 = t0;
+            y_qc = qc;
+            y_ea = m->ea[tr];
         }
         fence_async_smem();
         tc_fence_before();
@@ -665,12 +764,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         umma_commit(&m->bar[BAR_DRAIN]);
         mbar_wait_flag(&m->bar[BAR_DRAIN], 0, &m->drain_flag, nullptr, 0);
     }
+    if (warp > 0 && !SUMMARY && y_pending) emit_y(y_t0, y_qc, y_ea);
     if (warp > 0) {
+        workers_sync();          // the last tile's phase update is visible to all workers
         const int n = row;
         if (SUMMARY) {
             float4* dst = reinterpret_cast<float4*>(q.ws_sloc + (bhs * kN + n) * kP + c0);
 #pragma unroll
-            for (int c = 0; c < kP / 8; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
+            for (int c = 0; c < kSC / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
             if (wk < 64) q.ws_phase[bhs * (kN / 2) + wk] = (float)m->phi[wk];
             if (wk == 0) q.ws_decay[bhs] = m->scal[1];
         } else if (seg == q.nseg - 1) {
@@ -679,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 sincosf((float)m->phi[n >> 1], &sv, &cv);
                 float* dst = q.fin_h + (bh * kN + n) * kP + c0;
 #pragma unroll
-                for (int p = 0; p < kP / 2; ++p) {
+                for (int p = 0; p < kSC; ++p) {
                     const float other = __shfl_xor_sync(0xffffffffu, S[p], 1);
                     dst[p] = (n & 1) ? (sv * other + cv * S[p]) : (cv * S[p] - sv * other);
                 }

@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/m3.h"
+#include "m3.h"
 
 namespace m3 {
 

@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stddef.h>
 
-#include "../../include/m3.h"
+#include "m3.h"
 
 namespace m3 {
 
