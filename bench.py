@@ -48,6 +48,10 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the layer's batch (profiling captures of a smaller case)")
+    ap.add_argument("--workload", choices=["both", "prefill", "decode"], default="both",
+                    help="decode alone starts from a seeded random carry (profiling captures)")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="override the decode batch (profiling captures of a smaller case)")
     return ap.parse_args()
 
 
@@ -197,41 +201,47 @@ def cpu_baseline_sample():
 
 
 # ------------------------------------------------------------------ ours --
-def main():
-    args = parse()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
-        return run_reference(args, rank)
+class Ctx:
+    """Per-process state shared by the measured parts."""
 
-    import numpy as np
-    import torch
-    import torch.distributed as dist
+    def __init__(self, args):
+        import torch
+        import torch.distributed as dist
+        self.args = args
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(self.local)
+        if self.world > 1:
+            import datetime
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", self.local))
+        self.dist = dist
+        self.pk = peaks()
+        self.stream = torch.cuda.current_stream()
 
-    import m3_synth
-    import selective_state_space_m3_b200 as m3
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
 
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
+    def max_over_ranks(self, v: float) -> float:
+        import torch
+        if self.world == 1:
             return v
         t = torch.tensor([v], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
         return float(t.item())
 
-    pk = peaks()
+
+def run_prefill(cx, line):
+    """The chunked prefill of the 1.5B MIMO layer; fills the headline keys of
+    `line` and returns what the e2e and decode parts reuse."""
+    import torch
+    import m3_synth
+    import selective_state_space_m3_b200 as m3
+    args, pk, stream = cx.args, cx.pk, cx.stream
     s = m3_synth.CONFIGS[CFG]
-    s = m3_synth.shrink(s, seed=s.seed + 1000 * rank)     # each rank its own problem
+    s = m3_synth.shrink(s, seed=s.seed + 1000 * cx.rank)     # each rank its own problem
     if args.batch > 0:
         s = m3_synth.shrink(s, batch=args.batch)
     host = m3_synth.make_scan_inputs(s)
@@ -243,7 +253,6 @@ def main():
     fin = m3.Carry(torch.empty(s.batch, s.nheads, s.dstate, s.headdim, device="cuda"),
                    torch.empty(s.batch, s.nheads, s.rank, s.dstate, device="cuda", dtype=torch.bfloat16),
                    torch.empty(s.batch, s.nheads, s.rank, s.headdim, device="cuda", dtype=torch.bfloat16))
-    stream = torch.cuda.current_stream()
 
     def step():
         m3.m3_scan_fwd(d, dev["x"], dev["B"], dev["C"], dev["dt"], dev["A"], dev["lam"], dev["theta"],
@@ -256,9 +265,9 @@ def main():
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
-    with ClockSampler(local) as clk:
+    with ClockSampler(cx.local) as clk:
         clk.active = True
-        barrier()
+        cx.barrier()
         torch.cuda.synchronize()
         t_all0 = torch.cuda.Event(enable_timing=True)
         t_all1 = torch.cuda.Event(enable_timing=True)
@@ -269,130 +278,170 @@ def main():
             e1.record(stream)
         t_all1.record(stream)
         torch.cuda.synchronize()
-        barrier()
+        cx.barrier()
         clk.active = False
     assert m3.m3_device_status(ws) == m3.M3_OK
-    total_ms = max_over_ranks(t_all0.elapsed_time(t_all1))
+    total_ms = cx.max_over_ranks(t_all0.elapsed_time(t_all1))
     per_launch_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
     ms_per_step = total_ms / args.steps
     tokens = s.batch * s.seqlen
-    value = world * tokens * args.steps / (total_ms / 1e3)
+    value = cx.world * tokens * args.steps / (total_ms / 1e3)
 
     abytes = algorithmic_bytes(dev, y, fin)
     aflops = algorithmic_flops(s)
     achieved_gbs = abytes / (per_launch_ms / 1e3) / 1e9
     tflops = aflops / (per_launch_ms / 1e3) / 1e12
-    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": pk["hbm"], "unit": "GB/s",
-                "frac": achieved_gbs / pk["hbm"], "traffic": None,
-                "peak_source": pk["src"],
-                "kernel": "m3_scan_fwd (whole call: %d launch%s)" % (plan["launches"],
-                                                                     "" if plan["launches"] == 1 else "es"),
-                "algorithmic_bytes_per_launch": abytes,
-                "tensor_tflops": tflops, "tensor_frac_of_bf16_peak": tflops / pk["bf16"]}
+    line.update({
+        "value": value, "ms_per_step": ms_per_step,
+        "config": {"workload": m3_synth.CONFIG_NAMES[CFG], "global_batch": s.batch * cx.world,
+                   "seq_len": s.seqlen, "nheads": s.nheads, "headdim": s.headdim, "dstate": s.dstate,
+                   "rank": s.rank, "chunk": s.chunk,
+                   "parallelism": "replicas" if cx.world == 1 else f"dp{cx.world}",
+                   "l2": "inputs 3.5 GB per step >> 126 MB L2; no flush",
+                   "path": plan["path"], "segments": plan["segments"], "chunk_used": plan["chunk_used"]},
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": pk["hbm"], "unit": "GB/s",
+                     "frac": achieved_gbs / pk["hbm"], "traffic": None, "peak_source": pk["src"],
+                     "kernel": "m3_scan_fwd (whole call: %d launch%s)" % (
+                         plan["launches"], "" if plan["launches"] == 1 else "es"),
+                     "algorithmic_bytes_per_launch": abytes,
+                     "tensor_tflops": tflops, "tensor_frac_of_bf16_peak": tflops / pk["bf16"]},
+        "clocks": clk.summary(),
+        "gpu_launches": plan["launches"] * args.steps})
+    return dict(s=s, host=host, dev=dev, y=y, fin=fin, step=step, tokens=tokens)
 
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": m3_synth.CONFIG_NAMES[CFG], "global_batch": s.batch * world,
-                       "seq_len": s.seqlen, "nheads": s.nheads, "headdim": s.headdim, "dstate": s.dstate,
-                       "rank": s.rank, "chunk": s.chunk,
-                       "parallelism": "replicas" if world == 1 else f"dp{world}",
-                       "l2": "inputs 3.5 GB per step >> 126 MB L2; no flush",
-                       "path": plan["path"], "segments": plan["segments"], "chunk_used": plan["chunk_used"]},
-            "roofline": roofline, "clocks": clk.summary(),
-            "gpu_launches": plan["launches"] * args.steps}
 
-    # ---- end to end: pinned host buffers in, y out, copies inside the timed region
-    if not args.no_e2e:
-        pinned = {k: v.pin_memory() for k, v in host.items()}
-        y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-        h2d = sum(v.numel() * v.element_size() for v in pinned.values())
-        d2h = y_host.numel() * y_host.element_size()
-        ke = max(2, min(args.steps, 4))
+def run_e2e(cx, line, pf):
+    """Pinned host buffers in, y out, the copies inside the timed region."""
+    import torch
+    stream = cx.stream
+    pinned = {k: v.pin_memory() for k, v in pf["host"].items()}
+    y_host = torch.empty(pf["y"].shape, dtype=pf["y"].dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = y_host.numel() * y_host.element_size()
+    ke = max(2, min(cx.args.steps, 4))
 
-        def e2e_step():
-            for k, v in pinned.items():
-                dev[k].copy_(v, non_blocking=True)
-            step()
-            y_host.copy_(y, non_blocking=True)
+    def e2e_step():
+        for k, v in pinned.items():
+            pf["dev"][k].copy_(v, non_blocking=True)
+        pf["step"]()
+        y_host.copy_(pf["y"], non_blocking=True)
 
+    e2e_step()
+    torch.cuda.synchronize()
+    cx.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(ke):
         e2e_step()
-        torch.cuda.synchronize()
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(ke):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        ms = max_over_ranks(e0.elapsed_time(e1))
-        line["e2e"] = {"value": world * tokens * ke / (ms / 1e3), "unit": "tokens/s",
-                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke}
+    e1.record(stream)
+    torch.cuda.synchronize()
+    cx.barrier()
+    ms = cx.max_over_ranks(e0.elapsed_time(e1))
+    line["e2e"] = {"value": cx.world * pf["tokens"] * ke / (ms / 1e3), "unit": "tokens/s",
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke}
 
-    # ---- decode: m3_step x decode_steps in one CUDA graph, carry from the prefill
-    if not args.no_decode:
-        dec = m3_synth.DECODE
-        reps = -(-dec.batch // s.batch)
+
+def run_decode(cx, line, pf):
+    """m3_step x decode_steps captured in one CUDA graph; the carry comes from
+    the prefill's final state (tiled, sequence j <- batch row j mod 8), or
+    from a seeded random carry when the decode runs alone."""
+    import torch
+    import m3_synth
+    import selective_state_space_m3_b200 as m3
+    args, pk, stream = cx.args, cx.pk, cx.stream
+    dec = m3_synth.DecodeShape(seed=m3_synth.DECODE.seed + 1000 * cx.rank)
+    if args.decode_batch > 0:
+        dec = dataclasses_replace(dec, batch=args.decode_batch)
+    if pf is not None:
+        fin = pf["fin"]
+        reps = -(-dec.batch // fin.h.shape[0])
         state = m3.Carry(fin.h.repeat(reps, 1, 1, 1)[:dec.batch].contiguous(),
                          fin.prev_B.repeat(reps, 1, 1, 1)[:dec.batch].contiguous(),
                          fin.prev_x.repeat(reps, 1, 1, 1)[:dec.batch].contiguous())
-        pool = 64      # distinct tokens (22 MB each; 1.4 GB >> L2), cycled
-        toks = []
-        for k in range(pool):
-            t = m3_synth.make_decode_token(m3_synth.DecodeShape(seed=dec.seed + 1000 * rank), k)
-            toks.append({n: v.cuda() for n, v in t.items()})
-        Ad = dev["A"]
-        dd = m3.Dims(dec.batch, 1, dec.nheads, dec.ngroups, dec.headdim, dec.dstate, dec.rank, 1, m3.M3_BF16)
-        yd = torch.empty_like(toks[0]["x"])
-        S = args.decode_steps
+        Ad = pf["dev"]["A"]
+    else:
+        c = m3_synth.make_carry(dec.batch, dec.nheads, dec.dstate, dec.headdim, dec.rank, dec.dtype,
+                                dec.seed, scale=0.5)
+        state = m3.Carry(c["h"].cuda(), c["prev_B"].cuda(), c["prev_x"].cuda())
+        Ad = (-torch.exp(torch.linspace(-2, 1, dec.nheads))).cuda()
+    pool = 64      # distinct tokens (22 MB each at batch 256; 1.4 GB >> L2), cycled
+    toks = []
+    for k in range(pool):
+        t = m3_synth.make_decode_token(dec, k)
+        toks.append({n: v.cuda() for n, v in t.items()})
+    dd = m3.Dims(dec.batch, 1, dec.nheads, dec.ngroups, dec.headdim, dec.dstate, dec.rank, 1, m3.M3_BF16)
+    yd = torch.empty_like(toks[0]["x"])
+    S = args.decode_steps
 
-        def run_steps(n, st):
-            for k in range(n):
-                t = toks[k % pool]
-                m3.m3_step(dd, state, t["x"], t["B"], t["C"], t["dt"], Ad, t["lam"], t["theta"], yd, stream=st)
+    def run_steps(n, st):
+        for k in range(n):
+            t = toks[k % pool]
+            m3.m3_step(dd, state, t["x"], t["B"], t["C"], t["dt"], Ad, t["lam"], t["theta"], yd, stream=st)
 
-        run_steps(3, stream)
+    run_steps(3, stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run_steps(S, torch.cuda.current_stream())
+    g.replay()
+    torch.cuda.synchronize()
+    reps_t = 2
+    with ClockSampler(cx.local) as clk2:
+        clk2.active = True
+        cx.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps_t):
+            g.replay()
+        e1.record(stream)
         torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            run_steps(S, torch.cuda.current_stream())
-        g.replay()
-        torch.cuda.synchronize()
-        reps_t = 2
-        with ClockSampler(local) as clk2:
-            clk2.active = True
-            barrier()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(reps_t):
-                g.replay()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            barrier()
-            clk2.active = False
-        ms = max_over_ranks(e0.elapsed_time(e1))
-        per_step_us = ms * 1e3 / (reps_t * S)
-        t0 = toks[0]
-        step_bytes = (2 * state.h.numel() * 4 + 2 * (state.prev_B.numel() + state.prev_x.numel()) * 2 +
-                      sum(v.numel() * v.element_size() for v in t0.values()) + yd.numel() * 2 +
-                      Ad.numel() * 4)
-        gbs = step_bytes / (per_step_us * 1e-6) / 1e9
-        line["decode"] = {"workload": m3_synth.CONFIG_NAMES[4], "tokens_per_s": world * dec.batch / (per_step_us * 1e-6),
-                          "us_per_step": per_step_us, "steps_timed": reps_t * S,
-                          "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
-                                       "frac": gbs / pk["hbm"], "algorithmic_bytes_per_launch": step_bytes,
-                                       "traffic": None},
-                          "gpu_launches": reps_t * S, "clocks": clk2.summary(),
-                          "inputs": f"{pool} distinct tokens cycled ({pool * 22} MB > L2)"}
-        del g
+        cx.barrier()
+        clk2.active = False
+    ms = cx.max_over_ranks(e0.elapsed_time(e1))
+    per_step_us = ms * 1e3 / (reps_t * S)
+    t0 = toks[0]
+    step_bytes = (2 * state.h.numel() * 4 + 2 * (state.prev_B.numel() + state.prev_x.numel()) * 2 +
+                  sum(v.numel() * v.element_size() for v in t0.values()) + yd.numel() * 2 + Ad.numel() * 4)
+    gbs = step_bytes / (per_step_us * 1e-6) / 1e9
+    line["decode"] = {"workload": m3_synth.CONFIG_NAMES[4] if dec.batch == 256 else f"decode_b{dec.batch}",
+                      "tokens_per_s": cx.world * dec.batch / (per_step_us * 1e-6),
+                      "us_per_step": per_step_us, "steps_timed": reps_t * S,
+                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                                   "frac": gbs / pk["hbm"], "algorithmic_bytes_per_launch": step_bytes,
+                                   "traffic": None},
+                      "gpu_launches": reps_t * S, "clocks": clk2.summary(),
+                      "carry": "prefill final state" if pf is not None else "seeded random",
+                      "inputs": f"{pool} distinct tokens cycled"}
+    del g
 
-    if rank == 0 and not args.no_cpu:
+
+def dataclasses_replace(obj, **kw):
+    import dataclasses
+    return dataclasses.replace(obj, **kw)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    cx = Ctx(args)
+    line = {"metric": METRIC, "value": None, "unit": "tokens/s", "n_gpus": cx.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic"}
+    pf = None
+    if args.workload in ("both", "prefill"):
+        pf = run_prefill(cx, line)
+        if not args.no_e2e:
+            run_e2e(cx, line, pf)
+    if args.workload in ("both", "decode") and not args.no_decode:
+        run_decode(cx, line, pf)
+    if cx.rank == 0 and not args.no_cpu and args.workload != "decode":
         line["cpu_baseline"] = cpu_baseline_sample()
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank == 0:
+    if cx.world > 1:
+        cx.dist.barrier()
+        cx.dist.destroy_process_group()
+    if cx.rank == 0:
         print(json.dumps(line))
     return 0
 

@@ -156,6 +156,14 @@ m3_status m3_scan_plan(const m3_dims* dims, int* launches, int* segments,
  * bounded on-chip wait expired (that call's outputs are then invalid). */
 m3_status m3_device_status(void* workspace, void* stream);
 
+/* Diagnostic for the failure path: launches one small kernel whose single
+ * on-chip wait (the same bounded wait the prefill kernels use) is never
+ * satisfied, so it gives up after its limit (about 1 s) and records
+ * M3_ERR_DEVICE_TIMEOUT in the workspace status word, which
+ * m3_device_status then returns.  Nothing faults and the context stays
+ * usable.  `workspace` needs at least 256 bytes. */
+m3_status m3_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void* stream);
+
 /* Static, never NULL. */
 const char* m3_status_string(m3_status status);
 

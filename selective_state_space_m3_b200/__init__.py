@@ -55,6 +55,8 @@ def _load():
     IP = ctypes.POINTER(I)
     lib.m3_scan_plan.argtypes = [D, IP, IP, IP, IP]
     lib.m3_scan_plan.restype = I
+    lib.m3_selftest_bounded_wait.argtypes = [V, S, V]
+    lib.m3_selftest_bounded_wait.restype = I
     lib.m3_status_string.argtypes = [I]
     lib.m3_status_string.restype = ctypes.c_char_p
     for f in ("m3_scan_workspace_size", "m3_scan_fwd", "m3_step", "m3_rope_bc", "m3_device_status"):
@@ -66,7 +68,7 @@ _lib = _load()
 
 # every symbol include/m3.h declares (checked by the CPU test suite)
 ABI_SYMBOLS = ("m3_scan_workspace_size", "m3_scan_fwd", "m3_step", "m3_rope_bc",
-               "m3_scan_plan", "m3_device_status", "m3_status_string")
+               "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_status_string")
 
 
 @dataclasses.dataclass
@@ -182,11 +184,17 @@ def m3_device_status(workspace, stream=None) -> int:
     return int(_lib.m3_device_status(_ptr(workspace), _stream(stream)))
 
 
+def m3_selftest_bounded_wait(workspace, stream=None) -> None:
+    """Launch the bounded-wait diagnostic; read the result with m3_device_status."""
+    _check(_lib.m3_selftest_bounded_wait(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                         _stream(stream)), "m3_selftest_bounded_wait")
+
+
 def raw_lib():
     """The ctypes handle (for calls that pass raw pointers)."""
     return _lib
 
 
 __all__ = ["Dims", "Carry", "M3Error", "m3_scan_workspace_size", "m3_scan_fwd", "m3_step",
-           "m3_rope_bc", "m3_scan_plan", "m3_device_status", "m3_status_string", "io_dtype_of", "ABI_SYMBOLS",
+           "m3_rope_bc", "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_status_string", "io_dtype_of", "ABI_SYMBOLS",
            "M3_F32", "M3_BF16", "raw_lib", "LIB_PATH"]

@@ -837,6 +837,28 @@ static bool make_map(CUtensorMap* map, const void* base, int inner, int R, int g
 
 }  // namespace tc
 
+// Diagnostic: one CTA waits, through the same bounded-wait helper the scan
+// uses, on an mbarrier that no thread arrives at.  The wait gives up after
+// its limit, records M3_ERR_DEVICE_TIMEOUT (and where = 99) in `status` and
+// the kernel returns normally: the timeout path, exercised without a fault.
+__global__ void wait_selftest_kernel(int* status) {
+    __shared__ uint64_t bar;
+    __shared__ tc::Misc m;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bar, 1);
+        m.abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) tc::mbar_wait(&bar, 0, &m, status, 99);
+    __syncthreads();
+}
+
+cudaError_t launch_wait_selftest(int* status, cudaStream_t st) {
+    wait_selftest_kernel<<<1, 32, 0, st>>>(status);
+    return cudaGetLastError();
+}
+
 bool tc_eligible(const m3_dims& d) {
     return d.io_dtype == M3_BF16 && d.dstate == tc::kN && d.headdim == tc::kP &&
            (d.rank == 1 || d.rank == 2 || d.rank == 4 || d.rank == 8);

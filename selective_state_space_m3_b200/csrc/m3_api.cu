@@ -266,6 +266,13 @@ m3_status m3_rope_bc(const m3_dims* d, const void* B, const void* C, const float
     return launch_rope(*d, q, (cudaStream_t)stream);
 }
 
+m3_status m3_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void* stream) {
+    if (!workspace || !aligned16(workspace) || workspace_bytes < kWorkspaceHeaderBytes) return M3_ERR_WORKSPACE;
+    return launch_wait_selftest(reinterpret_cast<int*>(workspace), (cudaStream_t)stream) == cudaSuccess
+               ? M3_OK
+               : M3_ERR_CUDA;
+}
+
 m3_status m3_device_status(void* workspace, void* stream) {
     if (!workspace) return M3_ERR_INVALID_ARG;
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return M3_ERR_CUDA;

@@ -70,5 +70,6 @@ cudaError_t launch_scan_combine(const ScanParams& q, cudaStream_t st);
 bool tc_eligible(const m3_dims& d);
 int tc_tile_tokens(int rank);
 cudaError_t launch_scan_tc(const m3_dims& d, const ScanParams& q, int* status, cudaStream_t st);
+cudaError_t launch_wait_selftest(int* status, cudaStream_t st);
 
 }  // namespace m3

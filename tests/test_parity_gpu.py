@@ -296,3 +296,20 @@ def test_config4_decode_full_batch_sampled():
         torch.cuda.synchronize()
         _check(f"decode t{k} y", f64(y)[sample], yo, 2e-2)
     _check("decode h", f64(state.h)[sample], h, 2e-2)
+
+
+# ----------------------------------------------------------- failure path --
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A wait nobody satisfies gives up after its limit and reports
+    M3_ERR_DEVICE_TIMEOUT through the workspace status word; the status is
+    cleared on read and the device keeps working (a scan runs afterwards)."""
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    assert m3.m3_device_status(ws) == m3.M3_OK
+    m3.m3_selftest_bounded_wait(ws)
+    assert m3.m3_device_status(ws) == m3.M3_ERR_DEVICE_TIMEOUT
+    assert m3.m3_device_status(ws) == m3.M3_OK          # read-and-clear
+    shape = m3_synth.ScanShape(1, 100, 2, 2, 64, 128, 4, 64, "bf16", 0.0, 70)
+    inp = m3_synth.make_scan_inputs(shape)
+    y, fin = gpu_scan(shape, inp)
+    yo, ho, _, _ = _oracle_full(inp)
+    _check("after timeout y", f64(y), yo, 2e-2)
