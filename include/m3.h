@@ -164,6 +164,35 @@ m3_status m3_device_status(void* workspace, void* stream);
  * usable.  `workspace` needs at least 256 bytes. */
 m3_status m3_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void* stream);
 
+/* Prefill that allocates nothing and takes no workspace.
+ * The paper has no counterpart to this call: it exists for callers that
+ * cannot allocate device memory while they run -- for example a plugin
+ * hosted by an engine that owns all device memory and gives its plugins no
+ * allocator, or a latency-critical loop that must not enter the CUDA
+ * allocator after start-up -- and so cannot provide m3_scan_fwd's workspace.
+ * Same arguments and results as m3_scan_fwd minus the workspace.  The
+ * scratch it needs lives in one fixed array of M3_STATIC_SCRATCH_BYTES
+ * inside the library's device image; every GPU that loads the library holds
+ * that array until the process exits.  Sizes whose workspace
+ * (m3_scan_workspace_size) exceeds it return M3_ERR_WORKSPACE before any
+ * launch.  The call itself allocates nothing (no cudaMalloc, no cudaFree).
+ * The first call on each device looks up the array's device address with
+ * that device current and caches it; make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents (each call clears the status word it needs zeroed), so calls that
+ * overlap on the GPU -- on different streams, or on different host threads --
+ * race and must be serialised by the caller.  On-chip wait timeouts are
+ * recorded in the array's status word but not reported through this call;
+ * callers that need that report use m3_scan_fwd. */
+#define M3_STATIC_SCRATCH_BYTES (32u << 20)
+m3_status m3_scan_fwd_static(const m3_dims* dims,
+                             const void* x, const void* B, const void* C,
+                             const float* dt, const float* A, const float* lambda,
+                             const float* theta,
+                             const m3_carry* init,
+                             void* y, m3_carry* final_state,
+                             void* stream);
+
 /* Static, never NULL. */
 const char* m3_status_string(m3_status status);
 

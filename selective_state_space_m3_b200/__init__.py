@@ -55,6 +55,8 @@ def _load():
     IP = ctypes.POINTER(I)
     lib.m3_scan_plan.argtypes = [D, IP, IP, IP, IP]
     lib.m3_scan_plan.restype = I
+    lib.m3_scan_fwd_static.argtypes = [D, V, V, V, V, V, V, V, C, V, C, V]
+    lib.m3_scan_fwd_static.restype = I
     lib.m3_selftest_bounded_wait.argtypes = [V, S, V]
     lib.m3_selftest_bounded_wait.restype = I
     lib.m3_status_string.argtypes = [I]
@@ -68,7 +70,8 @@ _lib = _load()
 
 # every symbol include/m3.h declares (checked by the CPU test suite)
 ABI_SYMBOLS = ("m3_scan_workspace_size", "m3_scan_fwd", "m3_step", "m3_rope_bc",
-               "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_status_string")
+               "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_scan_fwd_static",
+               "m3_status_string")
 
 
 @dataclasses.dataclass
@@ -163,6 +166,20 @@ def m3_scan_fwd(dims: Dims, x, B, C, dt, A, lam, theta, y, workspace,
     _check(st, "m3_scan_fwd")
 
 
+def m3_scan_fwd_static(dims: Dims, x, B, C, dt, A, lam, theta, y,
+                       init: Optional[Carry] = None, final_state: Optional[Carry] = None, stream=None) -> None:
+    """m3_scan_fwd without a workspace, for callers that cannot allocate device
+    memory: the scratch is a fixed array inside the library (see include/m3.h
+    for the size limit and for why overlapping calls must be serialised)."""
+    d = dims.c()
+    ci = init.c() if init is not None else None
+    cf = final_state.c() if final_state is not None else None
+    st = _lib.m3_scan_fwd_static(ctypes.byref(d), _ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A), _ptr(lam),
+                                 _ptr(theta), ctypes.byref(ci) if ci is not None else None, _ptr(y),
+                                 ctypes.byref(cf) if cf is not None else None, _stream(stream))
+    _check(st, "m3_scan_fwd_static")
+
+
 def m3_step(dims: Dims, state: Carry, x, B, C, dt, A, lam, theta, y, stream=None) -> None:
     """One decode token; ``state`` is updated in place."""
     d = dims.c()
@@ -196,5 +213,5 @@ def raw_lib():
 
 
 __all__ = ["Dims", "Carry", "M3Error", "m3_scan_workspace_size", "m3_scan_fwd", "m3_step",
-           "m3_rope_bc", "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_status_string", "io_dtype_of", "ABI_SYMBOLS",
+           "m3_rope_bc", "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_scan_fwd_static", "m3_status_string", "io_dtype_of", "ABI_SYMBOLS",
            "M3_F32", "M3_BF16", "raw_lib", "LIB_PATH"]
