@@ -39,8 +39,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-decode", action="store_true")
@@ -52,6 +52,9 @@ def parse():
                     help="decode alone starts from a seeded random carry (profiling captures)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="override the decode batch (profiling captures of a smaller case)")
+    ap.add_argument("--config", type=int, choices=[1, 2, 3], default=CFG,
+                    help="prefill workload: 2 = the R=4 layer (default, the headline); 1 and 3 "
+                         "time the SISO layer and the long-context SISO layer")
     return ap.parse_args()
 
 
@@ -67,7 +70,7 @@ def peaks():
 
 # ------------------------------------------------------------ clocks (NVML) --
 class ClockSampler:
-    """Samples SM clock and clock-event reasons every 20 ms in a thread."""
+    """Samples SM clock and clock-event reasons every 5 ms in a thread."""
     BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
             0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks",
             0x1: "gpu_idle"}
@@ -101,7 +104,7 @@ class ClockSampler:
                     self.samples.append((mhz, bits, util))
             except Exception:  # noqa: BLE001
                 pass
-            time.sleep(0.02)
+            time.sleep(0.005)
 
     def __enter__(self):
         if self.ok:
@@ -202,23 +205,29 @@ def cpu_baseline_sample():
 
 # ------------------------------------------------------------------ ours --
 class Ctx:
-    """Per-process state shared by the measured parts."""
+    """Per-process state shared by the measured parts.  `device="cpu"` runs
+    the same rank plumbing over gloo (the host-logic tests use it)."""
 
-    def __init__(self, args):
+    def __init__(self, args, device: str = "cuda"):
         import torch
         import torch.distributed as dist
         self.args = args
+        self.device = device
         self.rank = int(os.environ.get("RANK", "0"))
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
-        torch.cuda.set_device(self.local)
+        if device == "cuda":
+            torch.cuda.set_device(self.local)
         if self.world > 1:
             import datetime
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                    device_id=torch.device("cuda", self.local))
+            if device == "cuda":
+                dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                        device_id=torch.device("cuda", self.local))
+            else:
+                dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
         self.dist = dist
         self.pk = peaks()
-        self.stream = torch.cuda.current_stream()
+        self.stream = torch.cuda.current_stream() if device == "cuda" else None
 
     def barrier(self):
         if self.world > 1:
@@ -228,31 +237,69 @@ class Ctx:
         import torch
         if self.world == 1:
             return v
-        t = torch.tensor([v], device="cuda", dtype=torch.float64)
+        t = torch.tensor([v], device=self.device, dtype=torch.float64)
         self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
         return float(t.item())
 
+    def close(self):
+        if self.world > 1:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+
+
+# DRAM bytes (read + write) of one scan_tc_kernel<4,0> launch, from the ncu
+# capture of the R=4 layer at batch 2 (the main pass of a 4-segment plan):
+# 749,579,520 + 122,186,752 bytes.  Traffic grows with the (batch, head) units
+# (each is one sequence read once), so a launch over `batch` sequences moves
+# batch / 2 times this.  The capture and its command are in profiles/.
+TRAFFIC_R4_B2 = 749_579_520 + 122_186_752
+L2_BYTES = 126 * 1024 * 1024
+
+
+def measured_traffic(s, plan):
+    if plan["path"] != "tcgen05" or s.rank != 4 or s.nheads != 32 or s.seqlen != 4096:
+        return None, "no capture for this shape"
+    return TRAFFIC_R4_B2 * s.batch / 2, "ncu dram bytes of the batch-2 capture x batch/2"
+
+
+def throughput(world: int, tokens_per_rank: int, steps: int, total_ms: float) -> float:
+    """Whole-job tokens/s: every rank processed `tokens_per_rank` per step and
+    the slowest rank's time is the job's time."""
+    return world * tokens_per_rank * steps / (total_ms / 1e3)
+
+
+def rank_shape(cfg: int, rank: int, batch: int = 0):
+    """Each rank runs its own seeded problem of the same shape (weak scaling)."""
+    import m3_synth
+    s = m3_synth.CONFIGS[cfg]
+    s = m3_synth.shrink(s, seed=s.seed + 1000 * rank)
+    if batch > 0:
+        s = m3_synth.shrink(s, batch=batch)
+    return s
+
 
 def run_prefill(cx, line):
-    """The chunked prefill of the 1.5B MIMO layer; fills the headline keys of
-    `line` and returns what the e2e and decode parts reuse."""
+    """The chunked prefill of one layer workload (default: the R=4 MIMO
+    layer); fills the headline keys of `line` and returns what the e2e and
+    decode parts reuse."""
     import torch
     import m3_synth
     import selective_state_space_m3_b200 as m3
     args, pk, stream = cx.args, cx.pk, cx.stream
-    s = m3_synth.CONFIGS[CFG]
-    s = m3_synth.shrink(s, seed=s.seed + 1000 * cx.rank)     # each rank its own problem
-    if args.batch > 0:
-        s = m3_synth.shrink(s, batch=args.batch)
+    s = rank_shape(args.config, cx.rank, args.batch)
     host = m3_synth.make_scan_inputs(s)
     dev = {k: v.cuda() for k, v in host.items()}
-    d = m3.Dims(s.batch, s.seqlen, s.nheads, s.ngroups, s.headdim, s.dstate, s.rank, s.chunk, m3.M3_BF16)
+    io = m3.M3_BF16 if s.dtype == "bf16" else m3.M3_F32
+    d = m3.Dims(s.batch, s.seqlen, s.nheads, s.ngroups, s.headdim, s.dstate, s.rank, s.chunk, io)
     plan = m3.m3_scan_plan(d)
     y = torch.empty_like(dev["x"])
     ws = torch.zeros(m3.m3_scan_workspace_size(d), dtype=torch.uint8, device="cuda")
     fin = m3.Carry(torch.empty(s.batch, s.nheads, s.dstate, s.headdim, device="cuda"),
-                   torch.empty(s.batch, s.nheads, s.rank, s.dstate, device="cuda", dtype=torch.bfloat16),
-                   torch.empty(s.batch, s.nheads, s.rank, s.headdim, device="cuda", dtype=torch.bfloat16))
+                   torch.empty(s.batch, s.nheads, s.rank, s.dstate, device="cuda", dtype=dev["x"].dtype),
+                   torch.empty(s.batch, s.nheads, s.rank, s.headdim, device="cuda", dtype=dev["x"].dtype))
+    abytes = algorithmic_bytes(dev, y, fin)
+    # inputs smaller than twice the L2 are evicted between timed launches
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda") if abytes < 2 * L2_BYTES else None
 
     def step():
         m3.m3_scan_fwd(d, dev["x"], dev["B"], dev["C"], dev["dt"], dev["A"], dev["lam"], dev["theta"],
@@ -273,6 +320,8 @@ def run_prefill(cx, line):
         t_all1 = torch.cuda.Event(enable_timing=True)
         t_all0.record(stream)
         for e0, e1 in ev:
+            if flush is not None:
+                flush.zero_()
             e0.record(stream)
             step()
             e1.record(stream)
@@ -281,26 +330,33 @@ def run_prefill(cx, line):
         cx.barrier()
         clk.active = False
     assert m3.m3_device_status(ws) == m3.M3_OK
-    total_ms = cx.max_over_ranks(t_all0.elapsed_time(t_all1))
-    per_launch_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    launch_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
+    per_launch_ms = statistics.mean(launch_ms)
+    # with a flush between launches the step time is the launches alone
+    own_ms = t_all0.elapsed_time(t_all1) if flush is None else sum(launch_ms)
+    total_ms = cx.max_over_ranks(own_ms)
     ms_per_step = total_ms / args.steps
     tokens = s.batch * s.seqlen
-    value = cx.world * tokens * args.steps / (total_ms / 1e3)
+    value = throughput(cx.world, tokens, args.steps, total_ms)
 
-    abytes = algorithmic_bytes(dev, y, fin)
     aflops = algorithmic_flops(s)
     achieved_gbs = abytes / (per_launch_ms / 1e3) / 1e9
     tflops = aflops / (per_launch_ms / 1e3) / 1e12
+    traffic, traffic_src = measured_traffic(s, plan)
     line.update({
         "value": value, "ms_per_step": ms_per_step,
-        "config": {"workload": m3_synth.CONFIG_NAMES[CFG], "global_batch": s.batch * cx.world,
+        "config": {"workload": m3_synth.CONFIG_NAMES[args.config] if args.batch <= 0 else
+                   m3_synth.CONFIG_NAMES[args.config] + f"_batch{s.batch}",
+                   "global_batch": s.batch * cx.world,
                    "seq_len": s.seqlen, "nheads": s.nheads, "headdim": s.headdim, "dstate": s.dstate,
                    "rank": s.rank, "chunk": s.chunk,
                    "parallelism": "replicas" if cx.world == 1 else f"dp{cx.world}",
-                   "l2": "inputs 3.5 GB per step >> 126 MB L2; no flush",
+                   "l2": ("inputs %.2f GB per step >> 126 MB L2; no flush" % (abytes / 1e9)) if flush is None
+                   else "L2 flushed (252 MB write) before every timed launch",
                    "path": plan["path"], "segments": plan["segments"], "chunk_used": plan["chunk_used"]},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": pk["hbm"], "unit": "GB/s",
-                     "frac": achieved_gbs / pk["hbm"], "traffic": None, "peak_source": pk["src"],
+                     "frac": achieved_gbs / pk["hbm"], "traffic": traffic, "traffic_source": traffic_src,
+                     "peak_source": pk["src"],
                      "kernel": "m3_scan_fwd (whole call: %d launch%s)" % (
                          plan["launches"], "" if plan["launches"] == 1 else "es"),
                      "algorithmic_bytes_per_launch": abytes,
@@ -352,7 +408,7 @@ def run_decode(cx, line, pf):
     dec = m3_synth.DecodeShape(seed=m3_synth.DECODE.seed + 1000 * cx.rank)
     if args.decode_batch > 0:
         dec = dataclasses_replace(dec, batch=args.decode_batch)
-    if pf is not None:
+    if pf is not None and args.config == CFG:
         fin = pf["fin"]
         reps = -(-dec.batch // fin.h.shape[0])
         state = m3.Carry(fin.h.repeat(reps, 1, 1, 1)[:dec.batch].contiguous(),
@@ -410,7 +466,8 @@ def run_decode(cx, line, pf):
                                    "frac": gbs / pk["hbm"], "algorithmic_bytes_per_launch": step_bytes,
                                    "traffic": None},
                       "gpu_launches": reps_t * S, "clocks": clk2.summary(),
-                      "carry": "prefill final state" if pf is not None else "seeded random",
+                      "carry": "prefill final state" if pf is not None and args.config == CFG
+                      else "seeded random",
                       "inputs": f"{pool} distinct tokens cycled"}
     del g
 
@@ -436,11 +493,9 @@ def main():
             run_e2e(cx, line, pf)
     if args.workload in ("both", "decode") and not args.no_decode:
         run_decode(cx, line, pf)
-    if cx.rank == 0 and not args.no_cpu and args.workload != "decode":
+    if cx.world == 1 and not args.no_cpu and args.workload != "decode" and args.config == CFG:
         line["cpu_baseline"] = cpu_baseline_sample()
-    if cx.world > 1:
-        cx.dist.barrier()
-        cx.dist.destroy_process_group()
+    cx.close()
     if cx.rank == 0:
         print(json.dumps(line))
     return 0

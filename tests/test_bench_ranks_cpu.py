@@ -1,0 +1,86 @@
+"""The multi-rank plumbing of bench.py, run as two gloo ranks on the CPU.
+
+With N GPUs the bench runs N independent replicas (one seeded problem per
+rank, no collective on the data path); the only collectives are the timing
+barrier and the max over ranks.  These tests run that plumbing with the gloo
+backend: the ranks agree on the slowest time, each rank draws a different
+problem of the same shape, and the reported value is the whole job's tokens
+over the slowest rank's time.
+"""
+import json
+import os
+import socket
+import sys
+import types
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import m3_synth
+    args = types.SimpleNamespace(config=bench.CFG, batch=1)
+    cx = bench.Ctx(args, device="cpu")
+    my_ms = 10.0 + 5.0 * rank                     # rank 1 is the slow one
+    cx.barrier()
+    slowest = cx.max_over_ranks(my_ms)
+    shape = bench.rank_shape(bench.CFG, cx.rank, batch=1)
+    small = m3_synth.shrink(shape, seqlen=8, nheads=2, ngroups=2)
+    x = m3_synth.make_scan_inputs(small)["x"].float()
+    cx.close()
+    with open(os.path.join(out_dir, f"r{rank}.json"), "w") as f:
+        json.dump({"slowest": slowest, "seed": shape.seed, "batch": shape.batch,
+                   "x0": x.flatten()[:4].tolist(), "world": cx.world}, f)
+
+
+def test_two_gloo_ranks_agree_on_the_slowest_time_and_draw_distinct_problems(tmp_path):
+    world = 2
+    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    r = [json.load(open(tmp_path / f"r{k}.json")) for k in range(world)]
+    assert r[0]["slowest"] == r[1]["slowest"] == 15.0
+    assert r[0]["world"] == r[1]["world"] == 2
+    assert r[0]["seed"] != r[1]["seed"]
+    assert r[0]["x0"] != r[1]["x0"]
+    assert r[0]["batch"] == r[1]["batch"] == 1
+
+
+def test_throughput_counts_every_rank_over_the_slowest_time():
+    # 2 ranks x 8 sequences x 4096 tokens, 10 steps, slowest rank 20 ms in total
+    v = bench.throughput(2, 8 * 4096, 10, 20.0)
+    assert v == pytest.approx(2 * 8 * 4096 * 10 / 0.020)
+    assert bench.throughput(1, 8 * 4096, 10, 20.0) == pytest.approx(v / 2)
+
+
+def test_single_rank_context_needs_no_process_group():
+    args = types.SimpleNamespace(config=bench.CFG, batch=0)
+    env = {k: os.environ.pop(k) for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK") if k in os.environ}
+    try:
+        cx = bench.Ctx(args, device="cpu")
+        assert cx.world == 1 and cx.max_over_ranks(3.5) == 3.5
+        cx.barrier()
+        cx.close()
+    finally:
+        os.environ.update(env)
+
+
+def test_traffic_is_reported_only_for_the_captured_shape():
+    import m3_synth
+    s = m3_synth.CONFIGS[bench.CFG]
+    t, _ = bench.measured_traffic(s, {"path": "tcgen05"})
+    assert t == pytest.approx(bench.TRAFFIC_R4_B2 * 4)
+    assert bench.measured_traffic(s, {"path": "simt"})[0] is None
+    assert bench.measured_traffic(m3_synth.CONFIGS[3], {"path": "tcgen05"})[0] is None

@@ -298,6 +298,52 @@ def test_config4_decode_full_batch_sampled():
     _check("decode h", f64(state.h)[sample], h, 2e-2)
 
 
+def test_decode_1000_steps_in_one_graph_as_timed():
+    """The decode workload as the bench times it: 256 sequences x 32 heads,
+    R=4, 1000 m3_step calls captured in one CUDA graph, 64 seeded tokens
+    cycled; sampled sequences are followed by the oracle through all 1000
+    steps and the last y and the final carry are compared."""
+    dec = m3_synth.DECODE
+    steps, pool = 1000, 64
+    c = m3_synth.make_carry(dec.batch, dec.nheads, dec.dstate, dec.headdim, dec.rank, dec.dtype,
+                            dec.seed, scale=0.5)
+    state = m3.Carry(c["h"].cuda(), c["prev_B"].cuda(), c["prev_x"].cuda())
+    A = -torch.exp(torch.linspace(-2, 1, dec.nheads))
+    Ad = A.cuda()
+    toks = [m3_synth.make_decode_token(dec, k) for k in range(pool)]
+    dtoks = [{n: v.cuda() for n, v in t.items()} for t in toks]
+    d = m3.Dims(dec.batch, 1, dec.nheads, dec.ngroups, dec.headdim, dec.dstate, dec.rank, 1, m3.M3_BF16)
+    y = torch.empty_like(dtoks[0]["x"])
+    sample = list(range(3, dec.batch, 37))
+    h, pB, pX = f64(c["h"])[sample], f64(c["prev_B"])[sample], f64(c["prev_x"])[sample]
+
+    # one step outside the capture, on a throwaway copy of the carry
+    warm = m3.Carry(state.h.clone(), state.prev_B.clone(), state.prev_x.clone())
+    t = dtoks[0]
+    m3.m3_step(d, warm, t["x"], t["B"], t["C"], t["dt"], Ad, t["lam"], t["theta"], y)
+    torch.cuda.synchronize()
+    del warm
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        st = torch.cuda.current_stream()
+        for k in range(steps):
+            t = dtoks[k % pool]
+            m3.m3_step(d, state, t["x"], t["B"], t["C"], t["dt"], Ad, t["lam"], t["theta"], y, stream=st)
+    g.replay()
+    torch.cuda.synchronize()
+
+    sub = [{n: f64(v[sample]) for n, v in t.items()} for t in toks]
+    Ao = f64(A)
+    for k in range(steps):
+        s = sub[k % pool]
+        yo, h, pB, pX = oracle.step(h, pB, pX, s["x"], s["B"], s["C"], s["dt"], Ao, s["lam"], s["theta"])
+    _check("graph decode y(last)", f64(y)[sample], yo, 2e-2)
+    _check("graph decode h", f64(state.h)[sample], h, 2e-2)
+    _check("graph decode prev_B", f64(state.prev_B)[sample], pB, 0.0)
+    _check("graph decode prev_x", f64(state.prev_x)[sample], pX, 0.0)
+    del g
+
+
 # ----------------------------------------------------------- failure path --
 def test_bounded_wait_reports_timeout_and_context_survives():
     """A wait nobody satisfies gives up after its limit and reports
