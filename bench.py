@@ -256,9 +256,14 @@ TRAFFIC_R4_B2 = 749_579_520 + 122_186_752
 L2_BYTES = 126 * 1024 * 1024
 
 
+TRAFFIC_CURRENT = False     # the capture predates the kernel now built
+
+
 def measured_traffic(s, plan):
     if plan["path"] != "tcgen05" or s.rank != 4 or s.nheads != 32 or s.seqlen != 4096:
         return None, "no capture for this shape"
+    if not TRAFFIC_CURRENT:
+        return None, "kernel changed since the last capture"
     return TRAFFIC_R4_B2 * s.batch / 2, "ncu dram bytes of the batch-2 capture x batch/2"
 
 

@@ -19,9 +19,11 @@
 //   TMA     B, C (bf16, SWIZZLE_128B, K-major: rows (t,r), 2 atoms of 64 n)
 //           and X (rows (t,r), 64 p) into shared memory; issued as soon as
 //           the previous tile's MMAs have read those buffers.
-//   workers dt/lambda -> a_t (block scan), gamma, c, w = e^{a_last-a}c, e^{a};
-//           cumulative phase per rotary pair (double running sum, one thread
-//           per (pair, quarter tile)); rotate B and C in place.
+//   workers dt/lambda -> a_t (warp scan, every warp keeps all tokens in
+//           registers), gamma, c, w = e^{a_last-a}c, e^{a}; cumulative phase
+//           per rotary pair (float, reduced to [-pi, pi] every token; the
+//           carry between tiles is reduced too); rotate B and C in place in
+//           bf16x2 arithmetic.  One worker barrier per tile.
 //   MMA 1   G = C~ B~^T (128x128, K=128)      -> TMEM cols [0,128)
 //           Y_inter = C~ S_bf (128x64, K=128) -> TMEM cols [192,256)
 //   workers scale B~ rows by w; P = mask o G -> bf16 over C~'s smem.
@@ -50,7 +52,7 @@ constexpr int kP = 64;
 constexpr int kWG = 2;                 // worker warpgroups
 constexpr int kWorkers = 128 * kWG;
 constexpr int kThreads = 32 + kWorkers;
-constexpr int kNQ = kWorkers / 64;     // token groups of the phase pass
+constexpr int kNE = kWorkers / 32;     // token groups of the phase / rotation pass (one per worker warp)
 constexpr int kSC = kP / kWG;          // state / y columns per warpgroup
 constexpr uint64_t kWaitNs = 1000000000ull;
 
@@ -60,7 +62,7 @@ constexpr int OFF_C = 32768;      // 32 KB: C~, later P
 constexpr int OFF_X = 65536;      // 16 KB: X
 constexpr int OFF_S = 81920;      // 16 KB: S_bf (rows n, 64 p)
 constexpr int OFF_MISC = 98304;
-constexpr int MISC_BYTES = 12288;
+constexpr int MISC_BYTES = 9216;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;   // + alignment slack
 
 struct Misc {
@@ -69,12 +71,7 @@ struct Misc {
     int abort_flag;
     int drain_flag;               // abort flag of the final drain waits (never set by others)
     int pad[13];
-    float dt[128], lam[128];
-    float a[128], a2[128], gam[128], cf[128], w[128], ea[128];
-    float scan[kWorkers / 32];
-    float scal[4];                // [0] tile decay, [1] segment log-decay, [2..3] next dt/lambda
-    double phi[64];               // phase carry per rotary pair (reduced)
-    double qsum[kNQ][64];         // per-token-group phase totals of the current tile
+    float2 qs[2][kNE][32];        // per token group: phase increments of pairs (2i, 2i+1), by tile parity
     float msk[32 * 36];           // decay mask per (token, token), rows padded (R >= 4)
 };
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region too small");
@@ -241,22 +238,37 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
-__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
-    // bf16 -> f32 is a 16-bit shift of the bit pattern
-    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
-}
-__device__ __forceinline__ uint32_t pack2(float2 v) { return pack_bf16x2(v.x, v.y); }
-// (x, y) -> (c x + s y, c y - s x): the transposed 2x2 rotation R(phi)^T
-__device__ __forceinline__ float2 rot_t(float2 v, float2 cc, float2 sn) {
-    // cc = (c, c), sn = (s, -s)
-    return __ffma2_rn(cc, v, __fmul2_rn(sn, make_float2(v.y, v.x)));
-}
-__device__ __forceinline__ uint4 scale_chunk(uint4 v, float2 w) {
-    v.x = pack2(__fmul2_rn(w, unpack_bf16x2(v.x)));
-    v.y = pack2(__fmul2_rn(w, unpack_bf16x2(v.y)));
-    v.z = pack2(__fmul2_rn(w, unpack_bf16x2(v.z)));
-    v.w = pack2(__fmul2_rn(w, unpack_bf16x2(v.w)));
+__device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t u) {
+    __nv_bfloat162 v;
+    memcpy(&v, &u, 4);
     return v;
+}
+__device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 v) {
+    uint32_t u;
+    memcpy(&u, &v, 4);
+    return u;
+}
+// one rotary pair in bf16x2: (x, y) -> (c x + s y, c y - s x), cc = (c, c),
+// sn = (s, -s); the product s*y is rounded to bf16 before the fused add
+__device__ __forceinline__ uint32_t rot_bf(uint32_t v, uint32_t cc, uint32_t sn) {
+    const uint32_t sw = __byte_perm(v, 0, 0x1032);          // (y, x)
+    return as_u32(__hfma2(as_bf2(cc), as_bf2(v), __hmul2(as_bf2(sn), as_bf2(sw))));
+}
+__device__ __forceinline__ uint4 scale_chunk(uint4 v, uint32_t w2) {
+    const __nv_bfloat162 w = as_bf2(w2);
+    v.x = as_u32(__hmul2(w, as_bf2(v.x)));
+    v.y = as_u32(__hmul2(w, as_bf2(v.y)));
+    v.z = as_u32(__hmul2(w, as_bf2(v.z)));
+    v.w = as_u32(__hmul2(w, as_bf2(v.w)));
+    return v;
+}
+// x[s] for a warp-uniform slice index s < NT (a select chain, no local memory)
+template <int NT>
+__device__ __forceinline__ float pick(const float (&x)[NT], int s) {
+    float r = x[0];
+#pragma unroll
+    for (int j = 1; j < NT; ++j) r = (s == j) ? x[j] : r;
+    return r;
 }
 // 8 consecutive floats -> one 16-byte chunk of bf16
 __device__ __forceinline__ uint4 pack_chunk(const float* f) {
@@ -281,14 +293,13 @@ __device__ __forceinline__ float wrap_pi_f(float x) {
 // Worker w (0..255) belongs to warpgroup wg = w / 128 and warp-in-group
 // wq = warp % 4, which is the TMEM lane quarter the warp may read.  "Row"
 // work (one tile row or state row per thread) is split between the two
-// warpgroups by columns; token work (coefficients, phases, rotation) is
-// split by (rotary pair, token quarter).
+// warpgroups by columns; the phase / rotation pass is split by token group
+// (one per worker warp) and rotary pair (two per lane).
 template <int R, bool SUMMARY>
 __global__ void __launch_bounds__(kThreads, 2)
     scan_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
                    const __grid_constant__ CUtensorMap tmX, ScanParams q, int* status) {
     constexpr int T = kRows / R;       // tokens per tile
-    constexpr int TQ = T / kNQ;        // tokens per token group (phase pass)
     constexpr float kLog2e = 1.4426950408889634f;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base for the SWIZZLE_128B tiles, derived by an offset
@@ -319,7 +330,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_init(&m->bar[BAR_DRAIN], 1);
         m->abort_flag = 0;
         m->drain_flag = 0;
-        m->scal[1] = 0.f;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_async_smem();
     }
@@ -335,7 +345,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int c0 = wg * kSC;                  // this warpgroup's state / y columns
     float S[kSC];                             // state row `row`, columns c0 .. c0+kSC-1
     if (warp > 0) {
-        if (wk < 64) m->phi[wk] = 0.0;
         const int n = row;
         if (SUMMARY) {
 #pragma unroll
@@ -382,51 +391,58 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     __nv_bfloat16* yg = static_cast<__nv_bfloat16*>(q.y);
 
-    // Per-tile inputs of the SIMT work (theta for this thread's rotary pair and
-    // token group, dt and lambda of token wk, the next token's dt/lambda).
-    // For R >= 2 they are loaded into registers one tile ahead, right after
-    // the previous tile's MMAs complete, so their latency overlaps that
-    // tile's epilogue; for R = 1 (32 theta values per thread) they are loaded
-    // at the tile's start after an L2 prefetch one tile ahead.
-    constexpr bool kRegPrefetch = (TQ <= 16);
-    const int pi = wk & 63, qt = wk >> 6;     // token work: rotary pair, token group
-    float th_n[TQ];
-    float dt_n = 0.f, lam_n = 1.f, dt_x = 0.f, lam_x = 1.f;
-    auto load_inputs = [&](int kn) {
+    // ---- token work of the workers
+    // Every worker warp keeps the whole tile's per-token coefficients in
+    // registers (lane l holds tokens l + 32 j, j < NT) and reads another
+    // token's value with a shuffle, so the coefficient step needs no shared
+    // memory and no barrier.  The phase / rotation pass gives worker warp qe
+    // the tokens [qe*TE, (qe+1)*TE) of the tile and lane l the rotary pairs
+    // 2l and 2l+1 (one 8-byte word of a B / C row).
+    constexpr int NT = (T + 31) / 32;
+    constexpr int TE = T / kNE;
+    constexpr bool kRegPrefetch = (TE <= 4);  // theta of the next tile held in registers
+    constexpr unsigned kFull = 0xffffffffu;
+    constexpr float kLn2 = 0.69314718055994531f;
+    const float A2 = Ah * kLog2e;             // decay per unit dt, log2 units
+    const int qe = warp - 1;                  // token group (warp-uniform)
+    const int g0 = qe * TE;                   // its first token
+    const int gsl = g0 >> 5, gln = g0 & 31;   // slice and lane holding that token
+    const int tr = row / R;                   // token of this thread's tile row
+    const int rsl = tr >> 5, rln = tr & 31;   // (rsl is warp-uniform for every R)
+    const float* th_base = q.theta + ((size_t)b * L * G + g) * (kN / 2) + 2 * lane;
+
+    float dt_n[NT], lam_n[NT], dx_n = 0.f, lx_n = 1.f;
+    float2 th_n[kRegPrefetch ? TE : 1];
+    auto load_tok = [&](int kn) {             // dt, lambda of tile kn and of the token after it
         const int t0n = tok0 + kn * T;
         const int qcn = min(T, tok1 - t0n);
 #pragma unroll
-        for (int kk = 0; kk < TQ; ++kk) {
-            const int t = qt * TQ + kk;
-            th_n[kk] = (t < qcn) ? __ldg(q.theta + (((size_t)b * L + t0n + t) * G + g) * (kN / 2) + pi) : 0.f;
+        for (int j = 0; j < NT; ++j) {
+            const int t = lane + 32 * j;
+            const size_t o = ((size_t)b * L + t0n + t) * H + h;
+            dt_n[j] = (t < qcn) ? __ldg(q.dt + o) : 0.f;
+            lam_n[j] = (t < qcn) ? __ldg(q.lam + o) : 1.f;
         }
-        if (wk < T) {
-            const size_t o = ((size_t)b * L + t0n + wk) * H + h;
-            dt_n = (wk < qcn) ? __ldg(q.dt + o) : 0.f;
-            lam_n = (wk < qcn) ? __ldg(q.lam + o) : 1.f;
-        }
-        if (wk == 0) {
-            const int tn = t0n + qcn;
-            const size_t o = ((size_t)b * L + tn) * H + h;
-            dt_x = (tn < L) ? __ldg(q.dt + o) : 0.f;
-            lam_x = (tn < L) ? __ldg(q.lam + o) : 1.f;
-        }
+        const int tn = t0n + qcn;
+        const size_t o = ((size_t)b * L + tn) * H + h;
+        dx_n = (tn < L) ? __ldg(q.dt + o) : 0.f;
+        lx_n = (tn < L) ? __ldg(q.lam + o) : 1.f;
     };
-    auto prefetch_inputs = [&](int kn) {
-        const int tn0 = tok0 + kn * T;
-        const int qn = min(T, tok1 - tn0);
-        for (int j = wk; j < 4 * T; j += kWorkers) {
-            if (j < 2 * T) {
-                const int t = j >> 1;
-                if (t < qn) prefetch_l2(q.theta + (((size_t)b * L + tn0 + t) * G + g) * (kN / 2) + (j & 1) * 32);
-            } else {
-                const int t = (j - 2 * T) % T;
-                if (t < qn) prefetch_l2((j < 3 * T ? q.dt : q.lam) + ((size_t)b * L + tn0 + t) * H + h);
-            }
+    auto theta_ld = [&](int t0n, int qcn, int kk) -> float2 {   // theta of pairs (2 lane, 2 lane + 1)
+        const int t = g0 + kk;
+        return (t < qcn) ? __ldg(reinterpret_cast<const float2*>(th_base + (size_t)(t0n + t) * G * (kN / 2)))
+                         : make_float2(0.f, 0.f);
+    };
+    auto prefetch_theta = [&](int kn) {       // L2 prefetch of a tile's theta rows (256 B per token)
+        const int t0n = tok0 + kn * T;
+        const int qn = min(T, tok1 - t0n);
+        for (int j = wk; j < 2 * T; j += kWorkers) {
+            const int t = j >> 1;
+            if (t < qn) prefetch_l2(q.theta + (((size_t)b * L + t0n + t) * G + g) * (kN / 2) + (j & 1) * 32);
         }
     };
     // y = Y_intra + e^{a_t} Y_inter of a finished tile (thread = tile row (t, r),
-    // this warpgroup's columns); run after the next tile's coefficient step
+    // this warpgroup's columns); run while the next tile's load lands
     auto emit_y = [&](int t0y, int qcy, float eay) {
         const float2 ea2 = make_float2(eay, eay);
 #pragma unroll 1
@@ -440,10 +456,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                 yi[j] = o2.x;
                 yi[j + 1] = o2.y;
             }
-            const int try_ = row / R;
-            if (try_ < qcy) {
+            if (tr < qcy) {
                 uint4* dst = reinterpret_cast<uint4*>(
-                    yg + ((((size_t)b * L + t0y + try_) * H + h) * R + (row % R)) * kP + c0 + 16 * hh);
+                    yg + ((((size_t)b * L + t0y + tr) * H + h) * R + (row % R)) * kP + c0 + 16 * hh);
                 dst[0] = pack_chunk(yi);
                 dst[1] = pack_chunk(yi + 8);
             }
@@ -452,9 +467,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     bool y_pending = false;                   // a tile's y is waiting to be emitted
     int y_t0 = 0, y_qc = 0;
     float y_ea = 0.f;
+    float2 carry = make_float2(0.f, 0.f);     // cumulative phase of pairs 2 lane, 2 lane + 1 (reduced)
+    float seg_a = 0.f;                        // log decay of the segment so far
     if (warp > 0 && ntiles > 0) {
-        if (kRegPrefetch) load_inputs(0);
-        else if (ntiles > 1) prefetch_inputs(1);
+        load_tok(0);
+        if (kRegPrefetch) {
+            const int qn = min(T, tok1 - tok0);
+#pragma unroll
+            for (int kk = 0; kk < TE; ++kk) th_n[kRegPrefetch ? kk : 0] = theta_ld(tok0, qn, kk);
+        } else if (ntiles > 1) {
+            prefetch_theta(1);
+        }
     }
 
     uint32_t pending_load = 0;   // control lane: a TMA load is in flight
@@ -464,13 +487,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int t0 = tok0 + k * T;
         const int qc = min(T, tok1 - t0);
         const uint32_t par = k & 1;
-        if (warp == 0) {
-            if (*(volatile int*)&m->abort_flag) break;
-        } else if (workers_any(*(volatile int*)&m->abort_flag)) {
-            break;
-        }
 
         if (warp == 0) {
+            // the whole warp takes the same exit (lanes 1..31 meet lane 0 at __syncwarp)
+            if (__any_sync(0xffffffffu, *(volatile int*)&m->abort_flag)) break;
             if (lane == 0) {
                 // ---------------- producer + MMA issuer
                 // The previous tile's MMAs are the last readers of B, C, X: once
@@ -488,8 +508,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tma_load_5d(sbase + OFF_X, &tmX, &m->bar[BAR_LOAD], 0, 0, h, t0, b);
                 pending_load = 1;
                 load_par = par;
-                mbar_wait(&m->bar[BAR_OPS], par, m, status, 2);
-                pending_load = 0;       // workers saw the load complete before arriving
+                // every worker saw the load complete before arriving here
+                if (mbar_wait(&m->bar[BAR_OPS], par, m, status, 2)) pending_load = 0;
                 tc_fence_after();
                 const uint32_t d_g = tmem, d_sl = tmem + 128, d_yx = tmem + 192;
                 if (!SUMMARY) {
@@ -535,118 +555,142 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
 
         // ---------------------------------------------------------- workers
-        if (!kRegPrefetch) {
-            load_inputs(k);
-            if (k + 2 < ntiles) prefetch_inputs(k + 2);
-        }
-        float th[TQ];
+        float dtv[NT], lmv[NT];
 #pragma unroll
-        for (int kk = 0; kk < TQ; ++kk) th[kk] = th_n[kk];
-        if (wk < T) {
-            m->dt[wk] = dt_n;
-            m->lam[wk] = lam_n;
+        for (int j = 0; j < NT; ++j) { dtv[j] = dt_n[j]; lmv[j] = lam_n[j]; }
+        const float dx = dx_n, lx = lx_n;
+        float2 th[kRegPrefetch ? TE : 1];
+        if (kRegPrefetch) {
+#pragma unroll
+            for (int kk = 0; kk < TE; ++kk) th[kRegPrefetch ? kk : 0] = th_n[kRegPrefetch ? kk : 0];
+        } else if (k + 2 < ntiles) {
+            prefetch_theta(k + 2);
         }
-        if (wk == 0) {
-            m->scal[2] = dt_x;
-            m->scal[3] = lam_x;
-        }
-        workers_sync();
-        // a_t = sum_{s<=t} dt_s A (inclusive block scan over the tile's tokens)
+        // theta of token g0 + kk: registers, or (long groups) an L1/L2-cached reload
+        auto th_at = [&](int kk) -> float2 { return kRegPrefetch ? th[kRegPrefetch ? kk : 0] : theta_ld(t0, qc, kk); };
+        // coefficients of every token (log2 units): a2 = inclusive scan of
+        // dt A, gamma = lambda dt, c = gamma + (1 - lambda') dt' with ' the
+        // next token (past the tile: the token after it, zero past the end)
+        float a2v[NT], gmv[NT], cfv[NT];
+        float a2_last;
         {
-            float v = (wk < qc) ? m->dt[wk] * Ah : 0.f;
+            float run = 0.f;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float u = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += u;
+            for (int j = 0; j < NT; ++j) {
+                float v = dtv[j] * A2;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float u = __shfl_up_sync(kFull, v, o);
+                    if (lane >= o) v += u;
+                }
+                a2v[j] = v + run;
+                run = __shfl_sync(kFull, a2v[j], 31);
             }
-            if (lane == 31) m->scan[warp - 1] = v;
-            workers_sync();
-            const int ww = warp - 1;
-            for (int j = 0; j < ww; ++j) v += m->scan[j];
-            if (wk < T) m->a[wk] = v;
-        }
-        workers_sync();
-        const float a_last = m->a[T - 1];
-        if (wk < T) {
-            if (wk < qc) {
-                const float d = m->dt[wk], lam = m->lam[wk];
-                const float gam = lam * d;
-                const float nxt = (wk + 1 < qc) ? (1.f - m->lam[wk + 1]) * m->dt[wk + 1]
-                                                : (1.f - m->scal[3]) * m->scal[2];
-                const float c = gam + nxt;
-                const float a = m->a[wk];
-                m->gam[wk] = gam;
-                m->cf[wk] = c;
-                m->w[wk] = exp2f((a_last - a) * kLog2e) * c;
-                m->ea[wk] = exp2f(a * kLog2e);
-                m->a2[wk] = a * kLog2e;
-            } else {
-                m->gam[wk] = 0.f; m->cf[wk] = 0.f; m->w[wk] = 0.f; m->ea[wk] = 0.f;
-                m->a2[wk] = a_last * kLog2e;
+            a2_last = run;
+            float up[NT];
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                gmv[j] = lmv[j] * dtv[j];
+                up[j] = (1.f - lmv[j]) * dtv[j];
+            }
+            const float ux = (1.f - lx) * dx;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                float nx = __shfl_down_sync(kFull, up[j], 1);
+                if (j + 1 < NT) {
+                    const float first = __shfl_sync(kFull, up[j + 1 < NT ? j + 1 : j], 0);
+                    if (lane == 31) nx = first;
+                }
+                if (lane + 32 * j + 1 == T) nx = ux;
+                cfv[j] = gmv[j] + nx;
             }
         }
         if (!SUMMARY && R >= 4) {
             // decay mask per (token t, token u) of the tile, shared by the R x R
             // rank block: e^{a_t - a_u} (gamma_u if u == t, c_u if u < t), 0 above
-            workers_sync();
             constexpr int LD = T + 4;
+#pragma unroll
             for (int e = wk; e < T * T; e += kWorkers) {
                 const int t = e / T, u = e % T;
-                float v = 0.f;
-                if (u <= t) v = exp2f(m->a2[t] - m->a2[u]) * (u == t ? m->gam[u] : m->cf[u]);
-                m->msk[t * LD + u] = v;
+                const float at = __shfl_sync(kFull, a2v[0], t), au = __shfl_sync(kFull, a2v[0], u);
+                const float gu = __shfl_sync(kFull, gmv[0], u), cu = __shfl_sync(kFull, cfv[0], u);
+                m->msk[t * LD + u] = (u <= t) ? exp2f(at - au) * (u == t ? gu : cu) : 0.f;
             }
+        }
+        // phase pass 1: this group's increments of pairs (2 lane, 2 lane + 1)
+        const float dsl = pick<NT>(dtv, gsl);
+        {
+            float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int kk = 0; kk < TE; ++kk) {
+                const float d = __shfl_sync(kFull, dsl, gln + kk);
+                const float2 tk = th_at(kk);
+                acc.x = fmaf(d, tk.x, acc.x);
+                acc.y = fmaf(d, tk.y, acc.y);
+            }
+            m->qs[par][qe][lane] = acc;
         }
         // the previous tile's output, while this tile's TMA load lands
         if (!SUMMARY && y_pending) {
             emit_y(y_t0, y_qc, y_ea);
             y_pending = false;
         }
-        // phase pass 1: this quarter's total
-        const double carry = m->phi[pi];
-        double acc = 0.0;
-#pragma unroll
-        for (int kk = 0; kk < TQ; ++kk) acc += (double)(m->dt[qt * TQ + kk] * th[kk]);
-        m->qsum[qt][pi] = acc;
-        if (wk == 0) {
-            m->scal[0] = exp2f(a_last * kLog2e);
-            m->scal[1] += a_last;
-        }
         mbar_wait(&m->bar[BAR_LOAD], par, m, status, 10);
-        workers_sync();
-        double start = carry;
-        for (int j = 0; j < qt; ++j) start += m->qsum[j][pi];
-        if (qt == kNQ - 1) m->phi[pi] = wrap_pi(start + acc);
-        // phase pass 2: rotate B (and C) rows (t, r) at pair pi, in place.
-        // The start phase is exact (double, reduced); inside the quarter the
-        // running phase is float, reduced every token.
+        // one barrier per tile: publishes qs and msk; all workers agree to stop
+        if (workers_any(*(volatile int*)&m->abort_flag)) break;
+        float2 ph = carry;
         {
-            const uint32_t atom = (uint32_t)(pi >> 5) * 16384u;
-            const int chunk = (pi & 31) >> 2;
-            const uint32_t inb = (uint32_t)(pi & 3) * 4u;
-            float ph = (float)wrap_pi(start);
+            float2 tot = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int kk = 0; kk < TQ; ++kk) {
-                const int t = qt * TQ + kk;
-                ph = wrap_pi_f(fmaf(m->dt[t], th[kk], ph));
-                if (t < qc) {
-                    float sv, cv;
-                    __sincosf(ph, &sv, &cv);
-                    float2 cc = make_float2(cv, cv), sn = make_float2(sv, -sv);
-                    if (SUMMARY) {
-                        const float wsc = m->w[t];
-                        cc = make_float2(wsc * cv, wsc * cv);
-                        sn = make_float2(wsc * sv, -wsc * sv);
-                    }
+            for (int j = 0; j < kNE; ++j) {
+                const float2 v = m->qs[par][j][lane];
+                if (j < qe) { ph.x += v.x; ph.y += v.y; }
+                tot.x += v.x;
+                tot.y += v.y;
+            }
+            carry = make_float2(wrap_pi_f(carry.x + tot.x), wrap_pi_f(carry.y + tot.y));
+        }
+        // phase pass 2: rotate rows (t, r) of B (and C) at pairs (2 lane,
+        // 2 lane + 1) in place, bf16x2; the running phase is reduced every token
+        {
+            const uint32_t atom = (uint32_t)(lane >> 4) * 16384u;
+            const int chunk = (lane & 15) >> 1;
+            const uint32_t inb = (uint32_t)(lane & 1) * 8u;
+            ph = make_float2(wrap_pi_f(ph.x), wrap_pi_f(ph.y));
+            const float a2sl = SUMMARY ? pick<NT>(a2v, gsl) : 0.f;
+            const float cfsl = SUMMARY ? pick<NT>(cfv, gsl) : 0.f;
 #pragma unroll
-                    for (int r = 0; r < R; ++r) {
-                        const uint32_t off = atom + sw128(t * R + r, chunk) + inb;
-                        uint32_t* pb = reinterpret_cast<uint32_t*>(smem + OFF_B + off);
-                        *pb = pack2(rot_t(unpack_bf16x2(*pb), cc, sn));
-                        if (!SUMMARY) {
-                            uint32_t* pc = reinterpret_cast<uint32_t*>(smem + OFF_C + off);
-                            *pc = pack2(rot_t(unpack_bf16x2(*pc), cc, sn));
-                        }
+            for (int kk = 0; kk < TE; ++kk) {
+                const int t = g0 + kk;
+                const float d = __shfl_sync(kFull, dsl, gln + kk);
+                const float2 tk = th_at(kk);
+                ph.x = wrap_pi_f(fmaf(d, tk.x, ph.x));
+                ph.y = wrap_pi_f(fmaf(d, tk.y, ph.y));
+                float s0, k0, s1, k1;
+                __sincosf(ph.x, &s0, &k0);
+                __sincosf(ph.y, &s1, &k1);
+                if (SUMMARY) {
+                    // the summary pass needs only w_t B~_t: fold w into the rotation
+                    const float wt = exp2f(a2_last - __shfl_sync(kFull, a2sl, gln + kk)) *
+                                     __shfl_sync(kFull, cfsl, gln + kk);
+                    s0 *= wt; k0 *= wt; s1 *= wt; k1 *= wt;
+                }
+                const uint32_t cc0 = pack_bf16x2(k0, k0), sn0 = pack_bf16x2(s0, -s0);
+                const uint32_t cc1 = pack_bf16x2(k1, k1), sn1 = pack_bf16x2(s1, -s1);
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const uint32_t off = atom + sw128(t * R + r, chunk) + inb;
+                    uint2* pb = reinterpret_cast<uint2*>(smem + OFF_B + off);
+                    uint2 vb = *pb;
+                    vb.x = rot_bf(vb.x, cc0, sn0);
+                    vb.y = rot_bf(vb.y, cc1, sn1);
+                    *pb = vb;
+                    if (!SUMMARY) {
+                        uint2* pc = reinterpret_cast<uint2*>(smem + OFF_C + off);
+                        uint2 vc = *pc;
+                        vc.x = rot_bf(vc.x, cc0, sn0);
+                        vc.y = rot_bf(vc.y, cc1, sn1);
+                        *pc = vc;
                     }
                 }
             }
@@ -655,14 +699,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_before();       // the deferred y's TMEM reads precede the next MMAs
         mbar_arrive(&m->bar[BAR_OPS]);
 
-        const int tr = row / R;              // token of this thread's tile row
+        // this thread's tile row: its token's log2 decay and pending weight
+        const float a2_tr = __shfl_sync(kFull, pick<NT>(a2v, rsl), rln);
         if (!SUMMARY) {
+            const float cf_tr = __shfl_sync(kFull, pick<NT>(cfv, rsl), rln);
             mbar_wait(&m->bar[BAR_G], par, m, status, 11);
             tc_fence_after();
-            // scale this warpgroup's atom of row `row` of B~ by w_t
+            // scale this warpgroup's half of row `row` of B~ by w_t
             {
-                const float wt = m->w[tr];
-                const float2 w2 = make_float2(wt, wt);
+                const float wt = exp2f(a2_last - a2_tr) * cf_tr;
+                const uint32_t w2 = pack_bf16x2(wt, wt);
 #pragma unroll
                 for (int c = 0; c < 16 / kWG; ++c) {
                     const int cc = wg * (16 / kWG) + c;   // 16-byte chunk of the 256-byte row
@@ -674,46 +720,50 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_arrive(&m->bar[BAR_BW]);
             // P = (two-band decay mask) o G on this warpgroup's 64 columns,
             // bf16, K-major over C~'s smem
-            {
-                const float a2t = m->a2[tr];
 #pragma unroll 1
-                for (int cg = 0; cg < 128 / kWG / 32; ++cg) {
-                    const int col0 = wg * (128 / kWG) + cg * 32;
-                    float v[32];
-                    tmem_ld32(tlane + col0, v);
-                    if (R >= 4) {
-                        // mask from the per-tile table, one value per R columns
-                        constexpr int LD = T + 4;
-                        const float4* mrow = reinterpret_cast<const float4*>(m->msk + tr * LD + col0 / R);
-                        float mk[32 / R];
-#pragma unroll
-                        for (int q4 = 0; q4 < 32 / R / 4; ++q4) {
-                            const float4 f = mrow[q4];
-                            mk[4 * q4] = f.x; mk[4 * q4 + 1] = f.y; mk[4 * q4 + 2] = f.z; mk[4 * q4 + 3] = f.w;
-                        }
-#pragma unroll
-                        for (int j = 0; j < 32; j += 2) {
-                            const float2 g2 = __fmul2_rn(make_float2(mk[j / R], mk[(j + 1) / R]),
-                                                         make_float2(v[j], v[j + 1]));
-                            v[j] = g2.x;
-                            v[j + 1] = g2.y;
-                        }
+            for (int cg = 0; cg < 128 / kWG / 16; ++cg) {
+                const int col0 = wg * (128 / kWG) + cg * 16;
+                float v[16];
+                tmem_ld16(tlane + col0, v);
+                if (R >= 4) {
+                    // mask from the per-tile table, one value per R columns
+                    constexpr int LD = T + 4;
+                    const float* mrow = m->msk + tr * LD + col0 / R;
+                    float mk[16 / R];
+                    if (R == 4) {
+                        const float4 f = *reinterpret_cast<const float4*>(mrow);
+                        mk[0] = f.x; mk[1] = f.y; mk[2 % (16 / R)] = f.z; mk[3 % (16 / R)] = f.w;
                     } else {
-                        const float a2t = m->a2[tr];
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int u = (col0 + j) / R;
-                            const float mkv =
-                                (u <= tr) ? exp2f(a2t - m->a2[u]) * (u == tr ? m->gam[u] : m->cf[u]) : 0.f;
-                            v[j] *= mkv;
-                        }
+                        const float2 f = *reinterpret_cast<const float2*>(mrow);
+                        mk[0] = f.x; mk[1] = f.y;
                     }
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int cc = (col0 >> 3) + c;      // 16-byte chunk over 128 columns
-                        *reinterpret_cast<uint4*>(smem + OFF_C + (cc >> 3) * 16384 + sw128(row, cc & 7)) =
-                            pack_chunk(v + 8 * c);
+                    for (int j = 0; j < 16; j += 2) {
+                        const float2 g2 = __fmul2_rn(make_float2(mk[j / R], mk[(j + 1) / R]),
+                                                     make_float2(v[j], v[j + 1]));
+                        v[j] = g2.x;
+                        v[j + 1] = g2.y;
                     }
+                } else {
+                    // columns u = (col0 + j) / R share one slice (warp-uniform)
+                    const int su = (col0 / R) >> 5, lu0 = (col0 / R) & 31;
+                    const float a2s = pick<NT>(a2v, su), gms = pick<NT>(gmv, su), cfs = pick<NT>(cfv, su);
+#pragma unroll
+                    for (int j = 0; j < 16; j += R) {
+                        const int u = col0 / R + j / R;
+                        const int lu = lu0 + j / R;
+                        const float au = __shfl_sync(kFull, a2s, lu);
+                        const float gu = __shfl_sync(kFull, gms, lu), cu = __shfl_sync(kFull, cfs, lu);
+                        const float mkv = (u <= tr) ? exp2f(a2_tr - au) * (u == tr ? gu : cu) : 0.f;
+#pragma unroll
+                        for (int rr = 0; rr < R; ++rr) v[j + rr] *= mkv;
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int cc = (col0 >> 3) + c;      // 16-byte chunk over 128 columns
+                    *reinterpret_cast<uint4*>(smem + OFF_C + (cc >> 3) * 16384 + sw128(row, cc & 7)) =
+                        pack_chunk(v + 8 * c);
                 }
             }
             fence_async_smem();
@@ -723,10 +773,17 @@ __global__ void __launch_bounds__(kThreads, 2)
 
         mbar_wait(&m->bar[BAR_Y], par, m, status, 12);
         tc_fence_after();
-        if (kRegPrefetch && k + 1 < ntiles) load_inputs(k + 1);
+        if (k + 1 < ntiles) {
+            load_tok(k + 1);
+            if (kRegPrefetch) {
+                const int t0n = t0 + T, qn = min(T, tok1 - t0n);
+#pragma unroll
+                for (int kk = 0; kk < TE; ++kk) th_n[kRegPrefetch ? kk : 0] = theta_ld(t0n, qn, kk);
+            }
+        }
         // state: S = e^{a_last} S + S_loc  (thread = state row, this half's columns)
         {
-            const float dec = m->scal[0];
+            const float dec = exp2f(a2_last);
             const float2 dec2 = make_float2(dec, dec);
 #pragma unroll
             for (int h16 = 0; h16 < kSC / 16; ++h16) {
@@ -746,11 +803,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                     *reinterpret_cast<uint4*>(smem + OFF_S + sw128(row, c0 / 8 + c)) = pack_chunk(S + 8 * c);
             }
         }
+        seg_a += a2_last * kLn2;
         if (!SUMMARY) {
             y_pending = true;
             y_t0 = t0;
             y_qc = qc;
-            y_ea = m->ea[tr];
+            y_ea = exp2f(a2_tr);
         }
         fence_async_smem();
         tc_fence_before();
@@ -766,22 +824,27 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     if (warp > 0 && !SUMMARY && y_pending) emit_y(y_t0, y_qc, y_ea);
     if (warp > 0) {
-        workers_sync();          // the last tile's phase update is visible to all workers
         const int n = row;
         if (SUMMARY) {
             float4* dst = reinterpret_cast<float4*>(q.ws_sloc + (bhs * kN + n) * kP + c0);
 #pragma unroll
             for (int c = 0; c < kSC / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
-            if (wk < 64) q.ws_phase[bhs * (kN / 2) + wk] = (float)m->phi[wk];
-            if (wk == 0) q.ws_decay[bhs] = m->scal[1];
+            if (qe == 0) {
+                q.ws_phase[bhs * (kN / 2) + 2 * lane] = carry.x;
+                q.ws_phase[bhs * (kN / 2) + 2 * lane + 1] = carry.y;
+            }
+            if (wk == 0) q.ws_decay[bhs] = seg_a;
         } else if (seg == q.nseg - 1) {
             if (q.fin_h) {
+                // phase of pair n/2 is held by lane n/4 of every worker warp
+                const float2 cv2 = make_float2(__shfl_sync(kFull, carry.x, n >> 2), __shfl_sync(kFull, carry.y, n >> 2));
+                const float phn = ((n >> 1) & 1) ? cv2.y : cv2.x;
                 float sv, cv;
-                sincosf((float)m->phi[n >> 1], &sv, &cv);
+                sincosf(phn, &sv, &cv);
                 float* dst = q.fin_h + (bh * kN + n) * kP + c0;
 #pragma unroll
                 for (int p = 0; p < kSC; ++p) {
-                    const float other = __shfl_xor_sync(0xffffffffu, S[p], 1);
+                    const float other = __shfl_xor_sync(kFull, S[p], 1);
                     dst[p] = (n & 1) ? (sv * other + cv * S[p]) : (cv * S[p] - sv * other);
                 }
             }
