@@ -26,8 +26,9 @@
 //           bf16x2 arithmetic.  One worker barrier per tile.
 //   MMA 1   G = C~ B~^T (128x128, K=128)      -> TMEM cols [0,128)
 //           Y_inter = C~ S_bf (128x64, K=128) -> TMEM cols [192,256)
-//   workers scale B~ rows by w; P = mask o G -> bf16 over C~'s smem.
-//   MMA 2   S_loc = (w B~)^T X (128x64, K=128) -> TMEM cols [128,192)
+//   workers w X -> the S_bf region (free after MMA 1); P = mask o G ->
+//           bf16 over C~'s smem.
+//   MMA 2   S_loc = B~^T (w X) (128x64, K=128) -> TMEM cols [128,192)
 //           Y_intra = P X (128x64, K=128)      -> TMEM cols [0,64)
 //   workers S = e^{a_last} S + S_loc (float32, registers, thread = state row);
 //           S_bf = bf16(S) for the next tile; y = Y_intra + e^{a_t} Y_inter.
@@ -401,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     constexpr int NT = (T + 31) / 32;
     constexpr int TE = T / kNE;
     constexpr bool kRegPrefetch = (TE <= 4);  // theta of the next tile held in registers
+    constexpr int kUnrollTE = kRegPrefetch ? TE : 4;
     constexpr unsigned kFull = 0xffffffffu;
     constexpr float kLn2 = 0.69314718055994531f;
     const float A2 = Ah * kLog2e;             // decay per unit dt, log2 units
@@ -411,6 +413,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int rsl = tr >> 5, rln = tr & 31;   // (rsl is warp-uniform for every R)
     const float* th_base = q.theta + ((size_t)b * L * G + g) * (kN / 2) + 2 * lane;
 
+    // Input loads read clamped (always valid) addresses and keep the raw
+    // values; tokens past the tile's end are masked where the values are
+    // used, so no instruction waits on a load right after issuing it.
     float dt_n[NT], lam_n[NT], dx_n = 0.f, lx_n = 1.f;
     float2 th_n[kRegPrefetch ? TE : 1];
     auto load_tok = [&](int kn) {             // dt, lambda of tile kn and of the token after it
@@ -418,20 +423,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int qcn = min(T, tok1 - t0n);
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
-            const int t = lane + 32 * j;
+            const int t = min(lane + 32 * j, qcn - 1);
             const size_t o = ((size_t)b * L + t0n + t) * H + h;
-            dt_n[j] = (t < qcn) ? __ldg(q.dt + o) : 0.f;
-            lam_n[j] = (t < qcn) ? __ldg(q.lam + o) : 1.f;
+            dt_n[j] = __ldg(q.dt + o);
+            lam_n[j] = __ldg(q.lam + o);
         }
-        const int tn = t0n + qcn;
+        const int tn = min(t0n + qcn, L - 1);
         const size_t o = ((size_t)b * L + tn) * H + h;
-        dx_n = (tn < L) ? __ldg(q.dt + o) : 0.f;
-        lx_n = (tn < L) ? __ldg(q.lam + o) : 1.f;
+        dx_n = __ldg(q.dt + o);
+        lx_n = __ldg(q.lam + o);
     };
-    auto theta_ld = [&](int t0n, int qcn, int kk) -> float2 {   // theta of pairs (2 lane, 2 lane + 1)
-        const int t = g0 + kk;
-        return (t < qcn) ? __ldg(reinterpret_cast<const float2*>(th_base + (size_t)(t0n + t) * G * (kN / 2)))
-                         : make_float2(0.f, 0.f);
+    auto theta_ld = [&](int t0n, int qcn, int kk) -> float2 {   // theta of pairs (2 lane, 2 lane + 1), raw
+        const int t = min(g0 + kk, qcn - 1);
+        return __ldg(reinterpret_cast<const float2*>(th_base + (size_t)(t0n + t) * G * (kN / 2)));
     };
     auto prefetch_theta = [&](int kn) {       // L2 prefetch of a tile's theta rows (256 B per token)
         const int t0n = tok0 + kn * T;
@@ -531,12 +535,15 @@ __global__ void __launch_bounds__(kThreads, 2)
                     mbar_wait(&m->bar[BAR_BW], par, m, status, 3);
                     tc_fence_after();
                 }
-                // S_loc = (w B~)^T X : A MN-major (M = n, two 64-wide blocks 16 KB apart),
-                // B MN-major (N = p); K = tile rows, 16 rows (2 KB) per instruction
+                // S_loc = B~^T (w X) : A MN-major (M = n, two 64-wide blocks 16 KB apart),
+                // B MN-major (N = p); K = tile rows, 16 rows (2 KB) per instruction.
+                // The summary pass has w folded into B~ and reads X; the main
+                // pass reads w X from the S_bf region.
                 constexpr uint32_t idS = idesc_bf16(128, 64, 1, 1);
+                const uint32_t off_wx = SUMMARY ? OFF_X : OFF_S;
                 for (int kk = 0; kk < 8; ++kk)
                     umma(d_sl, sdesc(sbase + OFF_B + kk * 2048, 16384, 1024),
-                         sdesc(sbase + OFF_X + kk * 2048, 8192, 1024), idS, kk > 0);
+                         sdesc(sbase + off_wx + kk * 2048, 8192, 1024), idS, kk > 0);
                 if (!SUMMARY) {
                     mbar_wait(&m->bar[BAR_P], par, m, status, 4);
                     tc_fence_after();
@@ -555,19 +562,30 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
 
         // ---------------------------------------------------------- workers
+        // this tile's inputs; tokens past the end count as dt = 0, lambda = 1
         float dtv[NT], lmv[NT];
 #pragma unroll
-        for (int j = 0; j < NT; ++j) { dtv[j] = dt_n[j]; lmv[j] = lam_n[j]; }
-        const float dx = dx_n, lx = lx_n;
-        float2 th[kRegPrefetch ? TE : 1];
+        for (int j = 0; j < NT; ++j) {
+            const bool in = lane + 32 * j < qc;
+            dtv[j] = in ? dt_n[j] : 0.f;
+            lmv[j] = in ? lam_n[j] : 1.f;
+        }
+        const bool nx_in = t0 + qc < L;
+        const float dx = nx_in ? dx_n : 0.f, lx = nx_in ? lx_n : 1.f;
+        float2 th[kRegPrefetch ? TE : 1];     // theta of tokens g0 + kk (zero past the end)
         if (kRegPrefetch) {
 #pragma unroll
-            for (int kk = 0; kk < TE; ++kk) th[kRegPrefetch ? kk : 0] = th_n[kRegPrefetch ? kk : 0];
+            for (int kk = 0; kk < TE; ++kk)
+                th[kRegPrefetch ? kk : 0] = (g0 + kk < qc) ? th_n[kRegPrefetch ? kk : 0] : make_float2(0.f, 0.f);
         } else if (k + 2 < ntiles) {
             prefetch_theta(k + 2);
         }
-        // theta of token g0 + kk: registers, or (long groups) an L1/L2-cached reload
-        auto th_at = [&](int kk) -> float2 { return kRegPrefetch ? th[kRegPrefetch ? kk : 0] : theta_ld(t0, qc, kk); };
+        // long token groups reload theta where it is used (L2, then L1)
+        auto th_at = [&](int kk) -> float2 {
+            if (kRegPrefetch) return th[kRegPrefetch ? kk : 0];
+            const float2 v = theta_ld(t0, qc, kk);
+            return (g0 + kk < qc) ? v : make_float2(0.f, 0.f);
+        };
         // coefficients of every token (log2 units): a2 = inclusive scan of
         // dt A, gamma = lambda dt, c = gamma + (1 - lambda') dt' with ' the
         // next token (past the tile: the token after it, zero past the end)
@@ -621,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const float dsl = pick<NT>(dtv, gsl);
         {
             float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
+#pragma unroll(kUnrollTE)
             for (int kk = 0; kk < TE; ++kk) {
                 const float d = __shfl_sync(kFull, dsl, gln + kk);
                 const float2 tk = th_at(kk);
@@ -659,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             ph = make_float2(wrap_pi_f(ph.x), wrap_pi_f(ph.y));
             const float a2sl = SUMMARY ? pick<NT>(a2v, gsl) : 0.f;
             const float cfsl = SUMMARY ? pick<NT>(cfv, gsl) : 0.f;
-#pragma unroll
+#pragma unroll(kUnrollTE)
             for (int kk = 0; kk < TE; ++kk) {
                 const int t = g0 + kk;
                 const float d = __shfl_sync(kFull, dsl, gln + kk);
@@ -705,15 +723,16 @@ __global__ void __launch_bounds__(kThreads, 2)
             const float cf_tr = __shfl_sync(kFull, pick<NT>(cfv, rsl), rln);
             mbar_wait(&m->bar[BAR_G], par, m, status, 11);
             tc_fence_after();
-            // scale this warpgroup's half of row `row` of B~ by w_t
+            // w_t X_t for the chunk-local state, into the S_bf region (free once
+            // G and Y_inter are done): this warpgroup's half of X row `row`
             {
                 const float wt = exp2f(a2_last - a2_tr) * cf_tr;
                 const uint32_t w2 = pack_bf16x2(wt, wt);
 #pragma unroll
-                for (int c = 0; c < 16 / kWG; ++c) {
-                    const int cc = wg * (16 / kWG) + c;   // 16-byte chunk of the 256-byte row
-                    uint4* p = reinterpret_cast<uint4*>(smem + OFF_B + (cc >> 3) * 16384 + sw128(row, cc & 7));
-                    *p = scale_chunk(*p, w2);
+                for (int c = 0; c < 8 / kWG; ++c) {
+                    const uint32_t off = sw128(row, wg * (8 / kWG) + c);   // 16-byte chunk of the 128-byte row
+                    *reinterpret_cast<uint4*>(smem + OFF_S + off) =
+                        scale_chunk(*reinterpret_cast<const uint4*>(smem + OFF_X + off), w2);
                 }
             }
             fence_async_smem();
@@ -810,8 +829,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             y_qc = qc;
             y_ea = exp2f(a2_tr);
         }
-        fence_async_smem();
-        tc_fence_before();
+        // (the S_bf stores and S_loc reads above are ordered before the next
+        // tile's MMAs by the fences ahead of that tile's OPS arrival)
     }
 
     // ---- epilogue of the segment
