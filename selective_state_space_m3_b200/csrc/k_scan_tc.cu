@@ -401,8 +401,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     // 2l and 2l+1 (one 8-byte word of a B / C row).
     constexpr int NT = (T + 31) / 32;
     constexpr int TE = T / kNE;
-    constexpr bool kRegPrefetch = (TE <= 4);  // theta of the next tile held in registers
-    constexpr int kUnrollTE = kRegPrefetch ? TE : 4;
+    constexpr bool kThReg = (TE <= 4);        // theta of the group held in registers for the tile
+    constexpr int kUnrollTE = kThReg ? TE : 4;
     constexpr unsigned kFull = 0xffffffffu;
     constexpr float kLn2 = 0.69314718055994531f;
     const float A2 = Ah * kLog2e;             // decay per unit dt, log2 units
@@ -411,13 +411,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int gsl = g0 >> 5, gln = g0 & 31;   // slice and lane holding that token
     const int tr = row / R;                   // token of this thread's tile row
     const int rsl = tr >> 5, rln = tr & 31;   // (rsl is warp-uniform for every R)
-    const float* th_base = q.theta + ((size_t)b * L * G + g) * (kN / 2) + 2 * lane;
 
     // Input loads read clamped (always valid) addresses and keep the raw
     // values; tokens past the tile's end are masked where the values are
     // used, so no instruction waits on a load right after issuing it.
     float dt_n[NT], lam_n[NT], dx_n = 0.f, lx_n = 1.f;
-    float2 th_n[kRegPrefetch ? TE : 1];
     auto load_tok = [&](int kn) {             // dt, lambda of tile kn and of the token after it
         const int t0n = tok0 + kn * T;
         const int qcn = min(T, tok1 - t0n);
@@ -435,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     };
     auto theta_ld = [&](int t0n, int qcn, int kk) -> float2 {   // theta of pairs (2 lane, 2 lane + 1), raw
         const int t = min(g0 + kk, qcn - 1);
-        return __ldg(reinterpret_cast<const float2*>(th_base + (size_t)(t0n + t) * G * (kN / 2)));
+        return __ldg(reinterpret_cast<const float2*>(q.theta + (((size_t)b * L + t0n + t) * G + g) * (kN / 2)) + lane);
     };
     auto prefetch_theta = [&](int kn) {       // L2 prefetch of a tile's theta rows (256 B per token)
         const int t0n = tok0 + kn * T;
@@ -468,20 +466,14 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
     };
-    bool y_pending = false;                   // a tile's y is waiting to be emitted
-    int y_t0 = 0, y_qc = 0;
-    float y_ea = 0.f;
+    int y_tile = -1;                          // tile whose y is waiting to be emitted (-1: none)
+    float y_ea = 0.f;                         // e^{a_t} of this thread's row in that tile
     float2 carry = make_float2(0.f, 0.f);     // cumulative phase of pairs 2 lane, 2 lane + 1 (reduced)
     float seg_a = 0.f;                        // log decay of the segment so far
     if (warp > 0 && ntiles > 0) {
         load_tok(0);
-        if (kRegPrefetch) {
-            const int qn = min(T, tok1 - tok0);
-#pragma unroll
-            for (int kk = 0; kk < TE; ++kk) th_n[kRegPrefetch ? kk : 0] = theta_ld(tok0, qn, kk);
-        } else if (ntiles > 1) {
-            prefetch_theta(1);
-        }
+        prefetch_theta(0);
+        if (ntiles > 1) prefetch_theta(1);
     }
 
     uint32_t pending_load = 0;   // control lane: a TMA load is in flight
@@ -572,18 +564,17 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         const bool nx_in = t0 + qc < L;
         const float dx = nx_in ? dx_n : 0.f, lx = nx_in ? lx_n : 1.f;
-        float2 th[kRegPrefetch ? TE : 1];     // theta of tokens g0 + kk (zero past the end)
-        if (kRegPrefetch) {
+        // theta of tokens g0 + kk (zero past the end): short groups load it
+        // here, ahead of its first use (L2 hits, prefetched two tiles ahead);
+        // long groups reload it where it is used
+        float2 th[kThReg ? TE : 1];
+        if (kThReg) {
 #pragma unroll
-            for (int kk = 0; kk < TE; ++kk)
-                th[kRegPrefetch ? kk : 0] = (g0 + kk < qc) ? th_n[kRegPrefetch ? kk : 0] : make_float2(0.f, 0.f);
-        } else if (k + 2 < ntiles) {
-            prefetch_theta(k + 2);
+            for (int kk = 0; kk < TE; ++kk) th[kThReg ? kk : 0] = theta_ld(t0, qc, kk);
         }
-        // long token groups reload theta where it is used (L2, then L1)
+        if (k + 2 < ntiles) prefetch_theta(k + 2);
         auto th_at = [&](int kk) -> float2 {
-            if (kRegPrefetch) return th[kRegPrefetch ? kk : 0];
-            const float2 v = theta_ld(t0, qc, kk);
+            const float2 v = kThReg ? th[kThReg ? kk : 0] : theta_ld(t0, qc, kk);
             return (g0 + kk < qc) ? v : make_float2(0.f, 0.f);
         };
         // coefficients of every token (log2 units): a2 = inclusive scan of
@@ -649,9 +640,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             m->qs[par][qe][lane] = acc;
         }
         // the previous tile's output, while this tile's TMA load lands
-        if (!SUMMARY && y_pending) {
-            emit_y(y_t0, y_qc, y_ea);
-            y_pending = false;
+        if (!SUMMARY && y_tile >= 0) {
+            emit_y(tok0 + y_tile * T, T, y_ea);     // a tile before the last is full
+            y_tile = -1;
         }
         mbar_wait(&m->bar[BAR_LOAD], par, m, status, 10);
         // one barrier per tile: publishes qs and msk; all workers agree to stop
@@ -794,11 +785,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
         if (k + 1 < ntiles) {
             load_tok(k + 1);
-            if (kRegPrefetch) {
-                const int t0n = t0 + T, qn = min(T, tok1 - t0n);
-#pragma unroll
-                for (int kk = 0; kk < TE; ++kk) th_n[kRegPrefetch ? kk : 0] = theta_ld(t0n, qn, kk);
-            }
         }
         // state: S = e^{a_last} S + S_loc  (thread = state row, this half's columns)
         {
@@ -824,9 +810,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         seg_a += a2_last * kLn2;
         if (!SUMMARY) {
-            y_pending = true;
-            y_t0 = t0;
-            y_qc = qc;
+            y_tile = k;
             y_ea = exp2f(a2_tr);
         }
         // (the S_bf stores and S_loc reads above are ordered before the next
@@ -841,7 +825,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         umma_commit(&m->bar[BAR_DRAIN]);
         mbar_wait_flag(&m->bar[BAR_DRAIN], 0, &m->drain_flag, nullptr, 0);
     }
-    if (warp > 0 && !SUMMARY && y_pending) emit_y(y_t0, y_qc, y_ea);
+    if (warp > 0 && !SUMMARY && y_tile >= 0) {
+        const int t0y = tok0 + y_tile * T;
+        emit_y(t0y, min(T, tok1 - t0y), y_ea);
+    }
     if (warp > 0) {
         const int n = row;
         if (SUMMARY) {
