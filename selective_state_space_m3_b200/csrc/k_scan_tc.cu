@@ -73,7 +73,10 @@ struct Misc {
     int drain_flag;               // abort flag of the final drain waits (never set by others)
     int pad[13];
     float2 qs[2][kNE][32];        // per token group: phase increments of pairs (2i, 2i+1), by tile parity
-    float msk[32 * 36];           // decay mask per (token, token), rows padded (R >= 4)
+    union {
+        float msk[32 * 36];       // R >= 4: decay mask per (token, token), rows padded
+        float cs[6][128];         // R < 4: c and gamma times e^{a_ref - a}, a_ref per block; a, gamma, c
+    } u;
 };
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region too small");
 
@@ -623,7 +626,29 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const int t = e / T, u = e % T;
                 const float at = __shfl_sync(kFull, a2v[0], t), au = __shfl_sync(kFull, a2v[0], u);
                 const float gu = __shfl_sync(kFull, gmv[0], u), cu = __shfl_sync(kFull, cfv[0], u);
-                m->msk[t * LD + u] = (u <= t) ? exp2f(at - au) * (u == t ? gu : cu) : 0.f;
+                m->u.msk[t * LD + u] = (u <= t) ? exp2f(at - au) * (u == t ? gu : cu) : 0.f;
+            }
+        }
+        if (!SUMMARY && R < 4 && qe == 0) {
+            // long tiles: the mask of a 16-column block (GT tokens) factors as
+            // e^{a_t - a_ref} x e^{a_ref - a_u} (gamma_u or c_u), a_ref = a at the
+            // block's first token, whenever the block's own decay is small
+            // enough that the second factor cannot overflow; such blocks get
+            // a_ref, the others +inf (element-wise path)
+            constexpr int GT = 16 / R;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                const int t = lane + 32 * j;
+                const float aref = __shfl_sync(kFull, a2v[j], lane & ~(GT - 1));
+                const float aend = __shfl_sync(kFull, a2v[j], lane | (GT - 1));
+                const bool ok = aref - aend <= 60.f;
+                const float colf = exp2f(aref - a2v[j]);
+                m->u.cs[0][t] = ok ? cfv[j] * colf : 0.f;
+                m->u.cs[1][t] = ok ? gmv[j] * colf : 0.f;
+                if ((lane & (GT - 1)) == 0) m->u.cs[2][t / GT] = ok ? aref : __int_as_float(0x7f800000);
+                m->u.cs[3][t] = a2v[j];
+                m->u.cs[4][t] = gmv[j];
+                m->u.cs[5][t] = cfv[j];
             }
         }
         // phase pass 1: this group's increments of pairs (2 lane, 2 lane + 1)
@@ -707,6 +732,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         fence_async_smem();
         tc_fence_before();       // the deferred y's TMEM reads precede the next MMAs
         mbar_arrive(&m->bar[BAR_OPS]);
+        // the next tile's dt / lambda: for short tiles their loads are issued
+        // here, while the tile's MMAs run (measured faster than after them)
+        if (R >= 4 && k + 1 < ntiles) load_tok(k + 1);
 
         // this thread's tile row: its token's log2 decay and pending weight
         const float a2_tr = __shfl_sync(kFull, pick<NT>(a2v, rsl), rln);
@@ -738,7 +766,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 if (R >= 4) {
                     // mask from the per-tile table, one value per R columns
                     constexpr int LD = T + 4;
-                    const float* mrow = m->msk + tr * LD + col0 / R;
+                    const float* mrow = m->u.msk + tr * LD + col0 / R;
                     float mk[16 / R];
                     if (R == 4) {
                         const float4 f = *reinterpret_cast<const float4*>(mrow);
@@ -755,18 +783,37 @@ __global__ void __launch_bounds__(kThreads, 2)
                         v[j + 1] = g2.y;
                     }
                 } else {
-                    // columns u = (col0 + j) / R share one slice (warp-uniform)
-                    const int su = (col0 / R) >> 5, lu0 = (col0 / R) & 31;
-                    const float a2s = pick<NT>(a2v, su), gms = pick<NT>(gmv, su), cfs = pick<NT>(cfv, su);
+                    constexpr int GT = 16 / R;            // tokens per 16-column block
+                    const int u0 = col0 / R;              // the block's first token (warp-uniform)
+                    const float aref = m->u.cs[2][u0 / GT];
+                    if (u0 > tr) {
 #pragma unroll
-                    for (int j = 0; j < 16; j += R) {
-                        const int u = col0 / R + j / R;
-                        const int lu = lu0 + j / R;
-                        const float au = __shfl_sync(kFull, a2s, lu);
-                        const float gu = __shfl_sync(kFull, gms, lu), cu = __shfl_sync(kFull, cfs, lu);
-                        const float mkv = (u <= tr) ? exp2f(a2_tr - au) * (u == tr ? gu : cu) : 0.f;
+                        for (int j = 0; j < 16; ++j) v[j] = 0.f;
+                    } else if (aref != __int_as_float(0x7f800000)) {
+                        const float rowf = exp2f(a2_tr - aref);
 #pragma unroll
-                        for (int rr = 0; rr < R; ++rr) v[j + rr] *= mkv;
+                        for (int i4 = 0; i4 < GT / 4; ++i4) {
+                            const float4 fc = reinterpret_cast<const float4*>(m->u.cs[0] + u0)[i4];
+                            const float4 fg = reinterpret_cast<const float4*>(m->u.cs[1] + u0)[i4];
+                            const float mc[4] = {fc.x, fc.y, fc.z, fc.w}, mg[4] = {fg.x, fg.y, fg.z, fg.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int u = u0 + 4 * i4 + e;
+                                const float mkv = rowf * ((u < tr) ? mc[e] : (u == tr ? mg[e] : 0.f));
+#pragma unroll
+                                for (int rr = 0; rr < R; ++rr) v[(4 * i4 + e) * R + rr] *= mkv;
+                            }
+                        }
+                    } else {
+                        // strong decay inside the block: element-wise
+#pragma unroll
+                        for (int j = 0; j < 16; j += R) {
+                            const int uu = u0 + j / R;
+                            const float au = m->u.cs[3][uu], gu = m->u.cs[4][uu], cu = m->u.cs[5][uu];
+                            const float mkv = (uu <= tr) ? exp2f(a2_tr - au) * (uu == tr ? gu : cu) : 0.f;
+#pragma unroll
+                            for (int rr = 0; rr < R; ++rr) v[j + rr] *= mkv;
+                        }
                     }
                 }
 #pragma unroll
@@ -783,9 +830,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
         mbar_wait(&m->bar[BAR_Y], par, m, status, 12);
         tc_fence_after();
-        if (k + 1 < ntiles) {
-            load_tok(k + 1);
-        }
+        if (R < 4 && k + 1 < ntiles) load_tok(k + 1);
         // state: S = e^{a_last} S + S_loc  (thread = state row, this half's columns)
         {
             const float dec = exp2f(a2_last);

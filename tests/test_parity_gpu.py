@@ -102,6 +102,25 @@ def test_tc_segments_and_ranks(R, nseg, monkeypatch):
     _check(f"tc R{R} nseg{nseg} h", f64(fin.h), ho, 2e-2)
 
 
+@pytest.mark.parametrize("R", [1, 2, 4])
+def test_tc_strong_decay(R):
+    """Heads whose decay inside a 16-column block of the mask is far beyond
+    the float range (A = -20 with dt ~ 0.7) next to ordinary heads: the
+    long-tile mask takes its element-wise path for the former and the
+    factored path for the latter."""
+    T = 128 // R
+    shape = m3_synth.ScanShape(2, 3 * T + 5, 4, 4, 64, 128, R, 64, "bf16", 0.0, 80 + R)
+    inp = m3_synth.make_scan_inputs(shape)
+    inp["A"] = inp["A"].clone()
+    inp["A"][0] = -20.0
+    inp["A"][2] = -6.0
+    assert m3.m3_scan_plan(dims_of(shape))["path"] == "tcgen05"
+    y, fin = gpu_scan(shape, inp)
+    yo, ho, _, _ = _oracle_full(inp)
+    _check(f"strong decay R{R} y", f64(y), yo, 2e-2)
+    _check(f"strong decay R{R} h", f64(fin.h), ho, 2e-2)
+
+
 def test_scan_with_initial_carry_bf16():
     shape = m3_synth.ScanShape(2, 190, 4, 4, 64, 128, 4, 64, "bf16", 0.0, 22)
     inp = m3_synth.make_scan_inputs(shape)
