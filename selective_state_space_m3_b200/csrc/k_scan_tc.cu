@@ -711,20 +711,27 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
                 const uint32_t cc0 = pack_bf16x2(k0, k0), sn0 = pack_bf16x2(s0, -s0);
                 const uint32_t cc1 = pack_bf16x2(k1, k1), sn1 = pack_bf16x2(s1, -s1);
+                // all loads of the token's rows first, then the stores: the
+                // compiler cannot tell that the swizzled rows do not overlap,
+                // so interleaving would serialise each row behind the last store
+                constexpr int NM = SUMMARY ? 1 : 2;      // B, and C in the main pass
+                uint2 vv[NM][R];
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
                     const uint32_t off = atom + sw128(t * R + r, chunk) + inb;
-                    uint2* pb = reinterpret_cast<uint2*>(smem + OFF_B + off);
-                    uint2 vb = *pb;
-                    vb.x = rot_bf(vb.x, cc0, sn0);
-                    vb.y = rot_bf(vb.y, cc1, sn1);
-                    *pb = vb;
-                    if (!SUMMARY) {
-                        uint2* pc = reinterpret_cast<uint2*>(smem + OFF_C + off);
-                        uint2 vc = *pc;
-                        vc.x = rot_bf(vc.x, cc0, sn0);
-                        vc.y = rot_bf(vc.y, cc1, sn1);
-                        *pc = vc;
+#pragma unroll
+                    for (int mt = 0; mt < NM; ++mt)
+                        vv[mt][r] = *reinterpret_cast<const uint2*>(smem + (mt ? OFF_C : OFF_B) + off);
+                }
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const uint32_t off = atom + sw128(t * R + r, chunk) + inb;
+#pragma unroll
+                    for (int mt = 0; mt < NM; ++mt) {
+                        uint2 v = vv[mt][r];
+                        v.x = rot_bf(v.x, cc0, sn0);
+                        v.y = rot_bf(v.y, cc1, sn1);
+                        *reinterpret_cast<uint2*>(smem + (mt ? OFF_C : OFF_B) + off) = v;
                     }
                 }
             }
@@ -747,12 +754,13 @@ __global__ void __launch_bounds__(kThreads, 2)
             {
                 const float wt = exp2f(a2_last - a2_tr) * cf_tr;
                 const uint32_t w2 = pack_bf16x2(wt, wt);
+                uint4 xv[8 / kWG];
 #pragma unroll
-                for (int c = 0; c < 8 / kWG; ++c) {
-                    const uint32_t off = sw128(row, wg * (8 / kWG) + c);   // 16-byte chunk of the 128-byte row
-                    *reinterpret_cast<uint4*>(smem + OFF_S + off) =
-                        scale_chunk(*reinterpret_cast<const uint4*>(smem + OFF_X + off), w2);
-                }
+                for (int c = 0; c < 8 / kWG; ++c)      // 16-byte chunks of the 128-byte row
+                    xv[c] = *reinterpret_cast<const uint4*>(smem + OFF_X + sw128(row, wg * (8 / kWG) + c));
+#pragma unroll
+                for (int c = 0; c < 8 / kWG; ++c)
+                    *reinterpret_cast<uint4*>(smem + OFF_S + sw128(row, wg * (8 / kWG) + c)) = scale_chunk(xv[c], w2);
             }
             fence_async_smem();
             mbar_arrive(&m->bar[BAR_BW]);
