@@ -685,7 +685,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             carry = make_float2(wrap_pi_f(carry.x + tot.x), wrap_pi_f(carry.y + tot.y));
         }
         // phase pass 2: rotate rows (t, r) of B (and C) at pairs (2 lane,
-        // 2 lane + 1) in place, bf16x2; the running phase is reduced every token
+        // 2 lane + 1) in place, bf16x2.  The running phase starts reduced to
+        // [-pi, pi] and grows by at most TE increments (|dt theta| each), a few
+        // tens of radians at most; at such arguments the fast sine / cosine
+        // err by ~1e-5 rad, far below the bf16 rounding of the rotated rows.
         {
             const uint32_t atom = (uint32_t)(lane >> 4) * 16384u;
             const int chunk = (lane & 15) >> 1;
@@ -698,8 +701,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const int t = g0 + kk;
                 const float d = __shfl_sync(kFull, dsl, gln + kk);
                 const float2 tk = th_at(kk);
-                ph.x = wrap_pi_f(fmaf(d, tk.x, ph.x));
-                ph.y = wrap_pi_f(fmaf(d, tk.y, ph.y));
+                ph.x = fmaf(d, tk.x, ph.x);
+                ph.y = fmaf(d, tk.y, ph.y);
                 float s0, k0, s1, k1;
                 __sincosf(ph.x, &s0, &k0);
                 __sincosf(ph.y, &s1, &k1);
