@@ -249,14 +249,17 @@ class Ctx:
 
 # DRAM bytes (read + write) of one scan_tc_kernel<4,0> launch, from the ncu
 # capture of the R=4 layer at batch 2 (the main pass of a 4-segment plan):
-# 749,579,520 + 122,186,752 bytes.  Traffic grows with the (batch, head) units
+# 754,761,984 + 120,160,512 bytes.  Traffic grows with the (batch, head) units
 # (each is one sequence read once), so a launch over `batch` sequences moves
 # batch / 2 times this.  The capture and its command are in profiles/.
-TRAFFIC_R4_B2 = 749_579_520 + 122_186_752
+TRAFFIC_R4_B2 = 754_761_984 + 120_160_512
+# DRAM bytes of one step_pipe_kernel launch (decode, batch 256, 32 heads,
+# R=4), from an ncu capture of that launch: 304,197,632 + 224,655,616 bytes.
+TRAFFIC_DECODE_B256 = 304_197_632 + 224_655_616
 L2_BYTES = 126 * 1024 * 1024
 
 
-TRAFFIC_CURRENT = False     # the capture predates the kernel now built
+TRAFFIC_CURRENT = True      # the captures match the kernels now built
 
 
 def measured_traffic(s, plan):
@@ -469,7 +472,8 @@ def run_decode(cx, line, pf):
                       "us_per_step": per_step_us, "steps_timed": reps_t * S,
                       "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
                                    "frac": gbs / pk["hbm"], "algorithmic_bytes_per_launch": step_bytes,
-                                   "traffic": None},
+                                   "traffic": TRAFFIC_DECODE_B256 if (dec.batch == 256 and TRAFFIC_CURRENT)
+                                   else None},
                       "gpu_launches": reps_t * S, "clocks": clk2.summary(),
                       "carry": "prefill final state" if pf is not None and args.config == CFG
                       else "seeded random",
