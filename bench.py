@@ -46,6 +46,7 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-rope", action="store_true", help="skip the m3_rope_bc measurement")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the layer's batch (profiling captures of a smaller case)")
     ap.add_argument("--workload", choices=["both", "prefill", "decode"], default="both",
@@ -405,6 +406,48 @@ def run_e2e(cx, line, pf):
                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke}
 
 
+def run_rope(cx, line, pf):
+    """m3_rope_bc (cumulative phase and rotated B, C per head) on the layer's
+    inputs: its own roofline, since it is the one standalone HBM-bound pass."""
+    import torch
+    import selective_state_space_m3_b200 as m3
+    args, pk, stream = cx.args, cx.pk, cx.stream
+    s, dev = pf["s"], pf["dev"]
+    io = dev["B"].dtype
+    Bo = torch.empty((s.batch, s.seqlen, s.nheads, s.rank, s.dstate), device="cuda", dtype=io)
+    Co = torch.empty_like(Bo)
+    ph = torch.empty((s.batch, s.seqlen, s.nheads, s.dstate // 2), device="cuda", dtype=torch.float32)
+    d = m3.Dims(s.batch, s.seqlen, s.nheads, s.ngroups, s.headdim, s.dstate, s.rank, s.chunk,
+                m3.M3_BF16 if s.dtype == "bf16" else m3.M3_F32)
+
+    def call():
+        m3.m3_rope_bc(d, dev["B"], dev["C"], dev["dt"], dev["theta"], Bo, Co, ph, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        call()
+    torch.cuda.synchronize()
+    n = max(5, min(args.steps, 20))
+    cx.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    cx.barrier()
+    ms = cx.max_over_ranks(e0.elapsed_time(e1)) / n
+    nbytes = sum(dev[k].numel() * dev[k].element_size() for k in ("B", "C", "dt", "theta"))
+    nbytes += sum(v.numel() * v.element_size() for v in (Bo, Co, ph))
+    gbs = nbytes / (ms / 1e3) / 1e9
+    line["rope"] = {"workload": "rope_bc_" + line["config"]["workload"], "ms_per_call": ms,
+                    "tokens_per_s": cx.world * s.batch * s.seqlen / (ms / 1e3),
+                    "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                                 "frac": gbs / pk["hbm"], "algorithmic_bytes_per_launch": nbytes,
+                                 "traffic": None},
+                    "gpu_launches": n, "l2": "inputs and outputs %.1f GB >> L2; no flush" % (nbytes / 1e9)}
+    del Bo, Co, ph
+
+
 def run_decode(cx, line, pf):
     """m3_step x decode_steps captured in one CUDA graph; the carry comes from
     the prefill's final state (tiled, sequence j <- batch row j mod 8), or
@@ -500,6 +543,8 @@ def main():
         pf = run_prefill(cx, line)
         if not args.no_e2e:
             run_e2e(cx, line, pf)
+        if not args.no_rope:
+            run_rope(cx, line, pf)
     if args.workload in ("both", "decode") and not args.no_decode:
         run_decode(cx, line, pf)
     if cx.world == 1 and not args.no_cpu and args.workload != "decode" and args.config == CFG:

@@ -208,6 +208,29 @@ def test_rope_bc_matches_oracle(dtype):
     assert np.max(np.abs(f64(ph))) <= np.pi + 1e-6
 
 
+def test_rope_bc_layer_shape_sampled():
+    """m3_rope_bc on the R=4 layer (8 x 4096 tokens, 32 heads, N=128, bf16) --
+    the launch the bench times -- against the oracle on sampled (b, h)."""
+    shape = m3_synth.CONFIGS[2]
+    inp = m3_synth.make_scan_inputs(shape)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    d = dims_of(shape)
+    b_, L, H, R, N = shape.batch, shape.seqlen, shape.nheads, shape.rank, shape.dstate
+    Bo = torch.empty((b_, L, H, R, N), device="cuda", dtype=torch.bfloat16)
+    Co = torch.empty_like(Bo)
+    ph = torch.empty((b_, L, H, N // 2), device="cuda", dtype=torch.float32)
+    m3.m3_rope_bc(d, dev["B"], dev["C"], dev["dt"], dev["theta"], Bo, Co, ph)
+    torch.cuda.synchronize()
+    for (b, h) in [(0, 0), (5, 19), (7, 31)]:
+        sl = lambda v: f64(v[b:b + 1, :, h:h + 1])
+        Bw, Cw, Pw = oracle.rope_bc(sl(inp["B"]), sl(inp["C"]), sl(inp["dt"]), sl(inp["theta"]), nheads=1)
+        _check(f"rope layer b{b} h{h} B", f64(Bo[b:b + 1, :, h:h + 1]), Bw, 2e-2)
+        _check(f"rope layer b{b} h{h} C", f64(Co[b:b + 1, :, h:h + 1]), Cw, 2e-2)
+        ang = np.angle(np.exp(1j * (f64(ph[b:b + 1, :, h:h + 1]) - Pw)))
+        print(f"rope layer b{b} h{h} phase max angular error {np.max(np.abs(ang)):.3e}")
+        assert np.max(np.abs(ang)) < 1e-5
+
+
 # ------------------------------------------------------------------ step --
 @pytest.mark.parametrize("dtype,R", [("f32", 1), ("f32", 2), ("bf16", 4), ("bf16", 1), ("bf16", 8)])
 def test_step_matches_oracle(dtype, R):
