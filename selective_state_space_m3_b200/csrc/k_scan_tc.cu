@@ -654,13 +654,20 @@ __global__ void __launch_bounds__(kThreads, 2)
         // phase pass 1: this group's increments of pairs (2 lane, 2 lane + 1)
         const float dsl = pick<NT>(dtv, gsl);
         {
+            // theta loads issued in batches of up to 8 tokens before their use
+            constexpr int KB = TE < 8 ? TE : 8;
             float2 acc = make_float2(0.f, 0.f);
-#pragma unroll(kUnrollTE)
-            for (int kk = 0; kk < TE; ++kk) {
-                const float d = __shfl_sync(kFull, dsl, gln + kk);
-                const float2 tk = th_at(kk);
-                acc.x = fmaf(d, tk.x, acc.x);
-                acc.y = fmaf(d, tk.y, acc.y);
+#pragma unroll
+            for (int k0 = 0; k0 < TE; k0 += KB) {
+                float2 thv[KB];
+#pragma unroll
+                for (int kk = 0; kk < KB; ++kk) thv[kk] = th_at(k0 + kk);
+#pragma unroll
+                for (int kk = 0; kk < KB; ++kk) {
+                    const float d = __shfl_sync(kFull, dsl, gln + k0 + kk);
+                    acc.x = fmaf(d, thv[kk].x, acc.x);
+                    acc.y = fmaf(d, thv[kk].y, acc.y);
+                }
             }
             m->qs[par][qe][lane] = acc;
         }
@@ -744,7 +751,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_arrive(&m->bar[BAR_OPS]);
         // the next tile's dt / lambda: for short tiles their loads are issued
         // here, while the tile's MMAs run (measured faster than after them)
-        if (R >= 4 && k + 1 < ntiles) load_tok(k + 1);
+        if (k + 1 < ntiles) load_tok(k + 1);
 
         // this thread's tile row: its token's log2 decay and pending weight
         const float a2_tr = __shfl_sync(kFull, pick<NT>(a2v, rsl), rln);
@@ -841,7 +848,6 @@ __global__ void __launch_bounds__(kThreads, 2)
 
         mbar_wait(&m->bar[BAR_Y], par, m, status, 12);
         tc_fence_after();
-        if (R < 4 && k + 1 < ntiles) load_tok(k + 1);
         // state: S = e^{a_last} S + S_loc  (thread = state row, this half's columns)
         {
             const float dec = exp2f(a2_last);
