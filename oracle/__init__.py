@@ -57,6 +57,8 @@ def _bind(lib):
     lib.oracle_scan.restype = ctypes.c_int
     lib.oracle_step.argtypes = [D] + [P] * 11
     lib.oracle_step.restype = ctypes.c_int
+    lib.oracle_scan_bwd.argtypes = [D] + [P] * 24
+    lib.oracle_scan_bwd.restype = ctypes.c_int
     lib.oracle_rope_bc.argtypes = [D] + [P] * 7
     lib.oracle_rope_bc.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
@@ -128,6 +130,31 @@ def scan(x, B, C, dt, A, lam, theta, init_h=None, init_pB=None, init_pX=None, li
     if rc != 0:
         raise ValueError("oracle_scan rejected its arguments")
     return y, hL, pB, pX
+
+
+def scan_bwd(x, B, C, dt, A, lam, theta, dy, init_h=None, init_pB=None, init_pX=None,
+             dh=None, dpB=None, dpX=None, lib=None):
+    """Gradients of J = sum <dy, y> + <dh, h_L> + <dpB, prev_B_L> + <dpX, prev_x_L>
+    with respect to every input of scan() (shapes as there).  Returns a dict
+    with dx, dB, dC (B and C summed over the heads of a group), ddt, dA, dlam,
+    dtheta, d_init_h, d_init_pB, d_init_pX."""
+    x, B, C, dt, A, lam, theta, dy = map(_f64, (x, B, C, dt, A, lam, theta, dy))
+    init_h, init_pB, init_pX, dh, dpB, dpX = map(_f64, (init_h, init_pB, init_pX, dh, dpB, dpX))
+    b, L, H, R, P = x.shape
+    G, N = B.shape[2], B.shape[4]
+    d = _Dims(b, L, H, G, P, N, R)
+    out = {"dx": np.zeros_like(x), "dB": np.zeros_like(B), "dC": np.zeros_like(C),
+           "ddt": np.zeros_like(dt), "dA": np.zeros_like(A), "dlam": np.zeros_like(lam),
+           "dtheta": np.zeros_like(theta), "d_init_h": np.zeros((b, H, N, P)),
+           "d_init_pB": np.zeros((b, H, R, N)), "d_init_pX": np.zeros((b, H, R, P))}
+    rc = (lib or _load()).oracle_scan_bwd(
+        ctypes.byref(d), _p(x), _p(B), _p(C), _p(dt), _p(A), _p(lam), _p(theta),
+        _p(init_h), _p(init_pB), _p(init_pX), _p(dy), _p(dh), _p(dpB), _p(dpX),
+        _p(out["dx"]), _p(out["dB"]), _p(out["dC"]), _p(out["ddt"]), _p(out["dA"]), _p(out["dlam"]),
+        _p(out["dtheta"]), _p(out["d_init_h"]), _p(out["d_init_pB"]), _p(out["d_init_pX"]))
+    if rc != 0:
+        raise ValueError("oracle_scan_bwd rejected its arguments")
+    return out
 
 
 def step(h, prev_B, prev_x, x, B, C, dt, A, lam, theta, lib=None):

@@ -225,6 +225,235 @@ int oracle_rope_bc(const oracle_dims* d,
     return 0;
 }
 
+/* Reverse-mode gradient of oracle_scan (the backward pass of the layer scan).
+ *
+ * Loss  J = sum_t <dy_t, y_t> + <dh, h_{L-1}> + <dpB, B_{L-1}> + <dpX, x_{L-1}>
+ * (dh, dpB, dpX: gradients arriving at the final carry; any may be NULL).
+ * Written out from the recurrence above by the chain rule, token by token in
+ * reverse.  With g_t = dJ/dh_t (the total adjoint of the state after token t),
+ * v_t = alpha_t h_{t-1} + beta_t B_{t-1} x_{t-1}^T (the state before R_t) and
+ * h_t = R_t v_t + gamma_t B_t x_t^T:
+ *   g_t      = C_t dy_t + alpha_{t+1} R_{t+1}^T g_{t+1}        (g_{L-1} starts at dh)
+ *   dC_t     = h_t dy_t^T
+ *   D_t      = gamma_t g_t + beta_{t+1} R_{t+1}^T g_{t+1}       (= dJ/d(B_t x_t^T))
+ *   dB_t     = D_t x_t,   dx_t = D_t^T B_t
+ *   dgamma_t = <g_t, B_t x_t^T>,  dalpha_t = <R_t^T g_t, h_{t-1}>,
+ *   dbeta_t  = <R_t^T g_t, B_{t-1} x_{t-1}^T>,
+ *   dphi_t[i] = sum_p g_t[pair i]^T R'(phi) v_t[pair i],  R' = dR/dphi,
+ * and, with alpha = e^{dt A}, beta = (1 - lam) dt alpha, gamma = lam dt,
+ * phi_i = dt theta_i:
+ *   ddt  = dalpha A alpha + dbeta (1 - lam)(alpha + dt A alpha) + dgamma lam + sum_i dphi_i theta_i
+ *   dA  += dalpha dt alpha + dbeta (1 - lam) dt^2 alpha
+ *   dlam = -dbeta dt alpha + dgamma dt,     dtheta_i = dphi_i dt.
+ * The carry-in gradients are g_{-1} = alpha_0 R_0^T g_0 (d init_h) and
+ * D_{-1} = beta_0 R_0^T g_0 (d init_pB = D_{-1} init_pX, d init_pX = D_{-1}^T init_pB).
+ *
+ * Outputs (overwritten; B, C and theta gradients are summed over the heads of
+ * a group, dA over batch and tokens): dx [b][t][h][r][p], dB, dC
+ * [b][t][g][r][n], ddt, dlam [b][t][h], dA [h], dtheta [b][t][g][N/2],
+ * d_init_h [b][h][n][p], d_init_pB [b][h][r][n], d_init_pX [b][h][r][p]
+ * (the d_init_* may be NULL).  Returns 0, or -1 on bad arguments. */
+int oracle_scan_bwd(const oracle_dims* d,
+                    const double* x, const double* B, const double* C,
+                    const double* dt, const double* A, const double* lam,
+                    const double* theta,
+                    const double* init_h, const double* init_pB, const double* init_pX,
+                    const double* dy, const double* dh, const double* dpB, const double* dpX,
+                    double* dx, double* dB, double* dC, double* ddt, double* dA,
+                    double* dlam, double* dtheta,
+                    double* d_init_h, double* d_init_pB, double* d_init_pX)
+{
+    if (!dims_ok(d) || !x || !B || !C || !dt || !A || !lam || !theta || !dy) return -1;
+    if (!dx || !dB || !dC || !ddt || !dA || !dlam || !dtheta) return -1;
+    const int Bn = d->batch, L = d->seqlen, H = d->nheads, G = d->ngroups;
+    const int P = d->headdim, N = d->dstate, R = d->rank;
+    const int hpg = H / G, NP = N * P;
+
+    /* per-head partial results, reduced over the heads of a group below */
+    double* dBh = (double*)calloc((size_t)Bn * L * H * R * N + 1, sizeof(double));
+    double* dCh = (double*)calloc((size_t)Bn * L * H * R * N + 1, sizeof(double));
+    double* dTh = (double*)calloc((size_t)Bn * L * H * (N / 2) + 1, sizeof(double));
+    double* dAh = (double*)calloc((size_t)Bn * H + 1, sizeof(double));
+    if (!dBh || !dCh || !dTh || !dAh) { free(dBh); free(dCh); free(dTh); free(dAh); return -1; }
+
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < Bn; ++b)
+        for (int h = 0; h < H; ++h) {
+            const int g = h / hpg;
+            const size_t bh = (size_t)b * H + h;
+            const double a = A[h];
+            /* forward: every state h_{t-1} .. h_{L-1}; hs[t + 1] = h_t, hs[0] = h_{-1} */
+            double* hs = (double*)calloc((size_t)(L + 1) * NP, sizeof(double));
+            double* PB0 = (double*)calloc((size_t)R * N, sizeof(double));
+            double* PX0 = (double*)calloc((size_t)R * P, sizeof(double));
+            double* PB = (double*)calloc((size_t)R * N, sizeof(double));
+            double* PX = (double*)calloc((size_t)R * P, sizeof(double));
+            double* yscratch = (double*)calloc((size_t)R * P, sizeof(double));
+            double* gk = (double*)calloc((size_t)NP, sizeof(double));
+            double* gv = (double*)calloc((size_t)NP, sizeof(double));
+            double* Db = (double*)calloc((size_t)NP, sizeof(double));
+            double* Dt = (double*)calloc((size_t)NP, sizeof(double));
+            double* v = (double*)calloc((size_t)NP, sizeof(double));
+            if (init_h) memcpy(hs, init_h + bh * NP, sizeof(double) * (size_t)NP);
+            if (init_pB) memcpy(PB0, init_pB + bh * R * N, sizeof(double) * (size_t)R * N);
+            if (init_pX) memcpy(PX0, init_pX + bh * R * P, sizeof(double) * (size_t)R * P);
+            memcpy(PB, PB0, sizeof(double) * (size_t)R * N);
+            memcpy(PX, PX0, sizeof(double) * (size_t)R * P);
+            for (int t = 0; t < L; ++t) {
+                const size_t bt = (size_t)b * L + t;
+                memcpy(hs + (size_t)(t + 1) * NP, hs + (size_t)t * NP, sizeof(double) * (size_t)NP);
+                step_bh(N, P, R, hs + (size_t)(t + 1) * NP, PB, PX,
+                        x + ((bt * H + h) * R) * P, B + ((bt * G + g) * R) * N, C + ((bt * G + g) * R) * N,
+                        dt[bt * H + h], a, lam[bt * H + h], theta + (bt * G + g) * (N / 2), yscratch);
+            }
+            /* reverse */
+            if (dh) memcpy(gk, dh + bh * NP, sizeof(double) * (size_t)NP);
+            for (int t = L - 1; t >= 0; --t) {
+                const size_t bt = (size_t)b * L + t;
+                const double* xt = x + ((bt * H + h) * R) * P;
+                const double* Bt = B + ((bt * G + g) * R) * N;
+                const double* Ct = C + ((bt * G + g) * R) * N;
+                const double* th = theta + (bt * G + g) * (N / 2);
+                const double* dyt = dy + ((bt * H + h) * R) * P;
+                const double* ht = hs + (size_t)(t + 1) * NP;
+                const double* hp = hs + (size_t)t * NP;
+                const double* pBt = t > 0 ? B + (((bt - 1) * G + g) * R) * N : PB0;
+                const double* pXt = t > 0 ? x + (((bt - 1) * H + h) * R) * P : PX0;
+                const double dd = dt[bt * H + h], lm = lam[bt * H + h];
+                const double al = exp(dd * a), be = (1.0 - lm) * dd * al, ga = lm * dd;
+                double* dxt = dx + ((bt * H + h) * R) * P;
+                double* dBt = dBh + ((bt * H + h) * R) * N;
+                double* dCt = dCh + ((bt * H + h) * R) * N;
+                double* dTt = dTh + (bt * H + h) * (N / 2);
+                memset(dxt, 0, sizeof(double) * (size_t)R * P);
+
+                /* readout: g_t += C_t dy_t,  dC_t = h_t dy_t^T */
+                for (int n = 0; n < N; ++n)
+                    for (int p = 0; p < P; ++p) {
+                        double acc = 0.0;
+                        for (int r = 0; r < R; ++r) acc += Ct[r * N + n] * dyt[r * P + p];
+                        gk[n * P + p] += acc;
+                    }
+                for (int r = 0; r < R; ++r)
+                    for (int n = 0; n < N; ++n) {
+                        double acc = 0.0;
+                        for (int p = 0; p < P; ++p) acc += ht[n * P + p] * dyt[r * P + p];
+                        dCt[r * N + n] = acc;
+                    }
+                /* the input term gamma_t B_t x_t^T and the beta term of token t+1 */
+                double dga = 0.0;
+                for (int n = 0; n < N; ++n)
+                    for (int p = 0; p < P; ++p) {
+                        double bx = 0.0;
+                        for (int r = 0; r < R; ++r) bx += Bt[r * N + n] * xt[r * P + p];
+                        dga += gk[n * P + p] * bx;
+                        Dt[n * P + p] = ga * gk[n * P + p] + Db[n * P + p];
+                    }
+                if (t == L - 1) {
+                    /* gradients arriving at the final (B, x) copies */
+                    if (dpB) for (int e = 0; e < R * N; ++e) dBt[e] += dpB[bh * R * N + e];
+                    if (dpX) for (int e = 0; e < R * P; ++e) dxt[e] += dpX[bh * R * P + e];
+                }
+                for (int r = 0; r < R; ++r) {
+                    for (int n = 0; n < N; ++n) {
+                        double acc = 0.0;
+                        for (int p = 0; p < P; ++p) acc += Dt[n * P + p] * xt[r * P + p];
+                        dBt[r * N + n] += acc;
+                    }
+                    for (int p = 0; p < P; ++p) {
+                        double acc = 0.0;
+                        for (int n = 0; n < N; ++n) acc += Dt[n * P + p] * Bt[r * N + n];
+                        dxt[r * P + p] += acc;
+                    }
+                }
+                /* v_t (the state before the rotation) */
+                for (int n = 0; n < N; ++n)
+                    for (int p = 0; p < P; ++p) {
+                        double bx = 0.0;
+                        for (int r = 0; r < R; ++r) bx += pBt[r * N + n] * pXt[r * P + p];
+                        v[n * P + p] = al * hp[n * P + p] + be * bx;
+                    }
+                /* rotation: dphi, and gv = R_t^T g_t */
+                double dphi_th = 0.0;
+                for (int i = 0; i < N / 2; ++i) {
+                    const double phi = dd * th[i];
+                    const double c = cos(phi), s = sin(phi);
+                    double dphi = 0.0;
+                    for (int p = 0; p < P; ++p) {
+                        const double g0 = gk[(2 * i) * P + p], g1 = gk[(2 * i + 1) * P + p];
+                        const double v0 = v[(2 * i) * P + p], v1 = v[(2 * i + 1) * P + p];
+                        dphi += g0 * (-s * v0 - c * v1) + g1 * (c * v0 - s * v1);
+                        gv[(2 * i) * P + p] = c * g0 + s * g1;
+                        gv[(2 * i + 1) * P + p] = -s * g0 + c * g1;
+                    }
+                    dTt[i] = dphi * dd;
+                    dphi_th += dphi * th[i];
+                }
+                double dal = 0.0, dbe = 0.0;
+                for (int n = 0; n < N; ++n)
+                    for (int p = 0; p < P; ++p) {
+                        double bx = 0.0;
+                        for (int r = 0; r < R; ++r) bx += pBt[r * N + n] * pXt[r * P + p];
+                        dal += gv[n * P + p] * hp[n * P + p];
+                        dbe += gv[n * P + p] * bx;
+                        Db[n * P + p] = be * gv[n * P + p];
+                        gk[n * P + p] = al * gv[n * P + p];
+                    }
+                ddt[bt * H + h] = dal * a * al + dbe * (1.0 - lm) * (al + dd * a * al) + dga * lm + dphi_th;
+                dAh[bh] += dal * dd * al + dbe * (1.0 - lm) * dd * dd * al;
+                dlam[bt * H + h] = -dbe * dd * al + dga * dd;
+            }
+            if (d_init_h) memcpy(d_init_h + bh * NP, gk, sizeof(double) * (size_t)NP);
+            if (d_init_pB)
+                for (int r = 0; r < R; ++r)
+                    for (int n = 0; n < N; ++n) {
+                        double acc = 0.0;
+                        for (int p = 0; p < P; ++p) acc += Db[n * P + p] * PX0[r * P + p];
+                        d_init_pB[bh * R * N + r * N + n] = acc;
+                    }
+            if (d_init_pX)
+                for (int r = 0; r < R; ++r)
+                    for (int p = 0; p < P; ++p) {
+                        double acc = 0.0;
+                        for (int n = 0; n < N; ++n) acc += Db[n * P + p] * PB0[r * N + n];
+                        d_init_pX[bh * R * P + r * P + p] = acc;
+                    }
+            free(hs); free(PB0); free(PX0); free(PB); free(PX); free(yscratch);
+            free(gk); free(gv); free(Db); free(Dt); free(v);
+        }
+    /* sum over the heads of each group (B, C, theta) and over the batch (A) */
+    for (int b = 0; b < Bn; ++b)
+        for (int t = 0; t < L; ++t)
+            for (int gi = 0; gi < G; ++gi) {
+                const size_t bg = ((size_t)b * L + t) * G + gi;
+                for (int e = 0; e < R * N; ++e) {
+                    double sb = 0.0, sc = 0.0;
+                    for (int k = 0; k < hpg; ++k) {
+                        const size_t bh = ((size_t)b * L + t) * H + gi * hpg + k;
+                        sb += dBh[bh * R * N + e];
+                        sc += dCh[bh * R * N + e];
+                    }
+                    dB[bg * R * N + e] = sb;
+                    dC[bg * R * N + e] = sc;
+                }
+                for (int i = 0; i < N / 2; ++i) {
+                    double st = 0.0;
+                    for (int k = 0; k < hpg; ++k) {
+                        const size_t bh = ((size_t)b * L + t) * H + gi * hpg + k;
+                        st += dTh[bh * (N / 2) + i];
+                    }
+                    dtheta[bg * (N / 2) + i] = st;
+                }
+            }
+    for (int h = 0; h < H; ++h) {
+        double s = 0.0;
+        for (int b = 0; b < Bn; ++b) s += dAh[(size_t)b * H + h];
+        dA[h] = s;
+    }
+    free(dBh); free(dCh); free(dTh); free(dAh);
+    return 0;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -528,3 +528,88 @@ def test_planted_mistakes_are_caught(name):
     lib = oracle.compile_variant(src, name)
     errs = (_pin_complex_err(lib), _pin_brute_err(lib))
     assert max(errs) > 1e-6, f"mutation {name} slipped through the pins: {errs}"
+
+
+# ------------------------------------------------------------- backward --
+def _fd_errors(lib, seed=7, b=2, L=6, H=2, G=1, P=3, N=4, R=2, carry=True):
+    """Relative error of the oracle's backward against central finite
+    differences of its forward, per input (random direction each)."""
+    rng = np.random.default_rng(seed)
+    rnd = lambda *s: rng.standard_normal(s)
+    inp = dict(x=rnd(b, L, H, R, P), B=rnd(b, L, G, R, N), C=rnd(b, L, G, R, N),
+               dt=np.log1p(np.exp(rnd(b, L, H))), A=-np.exp(rng.uniform(-2, 1, H)),
+               lam=1 / (1 + np.exp(-rnd(b, L, H))), theta=rng.uniform(-np.pi, np.pi, (b, L, G, N // 2)))
+    init = dict(init_h=rnd(b, H, N, P), init_pB=rnd(b, H, R, N), init_pX=rnd(b, H, R, P)) if carry else {}
+    dy = rnd(b, L, H, R, P)
+    fin = dict(dh=rnd(b, H, N, P), dpB=rnd(b, H, R, N), dpX=rnd(b, H, R, P)) if carry else {}
+
+    def J(i, n):
+        y, hL, pB, pX = oracle.scan(**i, **n, lib=lib)
+        j = float((dy * y).sum())
+        if carry:
+            j += float((fin["dh"] * hL).sum() + (fin["dpB"] * pB).sum() + (fin["dpX"] * pX).sum())
+        return j
+
+    g = oracle.scan_bwd(**inp, dy=dy, **init, **fin, lib=lib)
+    errs = {}
+    eps = 1e-6
+    for k in list(inp) + list(init):
+        tgt_inp, tgt_init = dict(inp), dict(init)
+        tgt = tgt_inp if k in inp else tgt_init
+        base = tgt[k]
+        v = rng.standard_normal(base.shape)
+        tgt[k] = base + eps * v
+        jp = J(tgt_inp, tgt_init)
+        tgt[k] = base - eps * v
+        jm = J(tgt_inp, tgt_init)
+        fd = (jp - jm) / (2 * eps)
+        an = float((g[{"init_h": "d_init_h", "init_pB": "d_init_pB", "init_pX": "d_init_pX"}.get(k, "d" + k)]
+                    * v).sum())
+        errs[k] = abs(fd - an) / max(abs(fd), 1e-12)
+    return errs
+
+
+@pytest.mark.parametrize("case", [
+    dict(),                                   # shared group (G=1 of 2 heads), MIMO R=2, carries
+    dict(G=2, R=1, seed=8),                   # SISO, one group per head
+    dict(carry=False, L=9, seed=9),           # no carry in or out
+    dict(R=3, N=6, P=2, seed=10),
+])
+def test_backward_matches_finite_differences(case):
+    """The oracle's backward (its own hand-written adjoint) against central
+    finite differences of the forward oracle: a directional derivative per
+    input, in float64."""
+    errs = _fd_errors(None, **case)
+    for k, e in errs.items():
+        assert e < 1e-6, (k, e, errs)
+
+
+_BWD_MUTATIONS = {
+    # the beta path of token t+1 left out of dJ/d(B_t x_t^T)
+    "bwd_no_beta_path": [("Dt[n * P + p] = ga * gk[n * P + p] + Db[n * P + p];",
+                          "Dt[n * P + p] = ga * gk[n * P + p];")],
+    # rotation derivative with the wrong sign
+    "bwd_dphi_sign": [("dphi += g0 * (-s * v0 - c * v1) + g1 * (c * v0 - s * v1);",
+                       "dphi += g0 * (s * v0 + c * v1) + g1 * (-c * v0 + s * v1);")],
+    # the phase term of d dt dropped
+    "bwd_ddt_no_phase": [("dga * lm + dphi_th;", "dga * lm;")],
+    # the adjoint not rotated back (R_t^T) before it is carried
+    "bwd_adjoint_unrotated": [("gk[n * P + p] = al * gv[n * P + p];", "gk[n * P + p] = al * gk[n * P + p];")],
+    # dA without the beta contribution
+    "bwd_dA_no_beta": [("dAh[bh] += dal * dd * al + dbe * (1.0 - lm) * dd * dd * al;",
+                        "dAh[bh] += dal * dd * al;")],
+    # the gradient arriving at the final prev_B ignored
+    "bwd_no_final_pB": [("if (dpB) for (int e = 0; e < R * N; ++e) dBt[e] += dpB[bh * R * N + e];",
+                         "/* dropped */")],
+}
+
+
+@pytest.mark.parametrize("name", sorted(_BWD_MUTATIONS))
+def test_backward_planted_mistakes_are_caught(name):
+    src = oracle.source_text()
+    for old, new in _BWD_MUTATIONS[name]:
+        assert src.count(old) == 1, old
+        src = src.replace(old, new)
+    lib = oracle.compile_variant(src, name)
+    errs = _fd_errors(lib)
+    assert max(errs.values()) > 1e-4, f"mutation {name} slipped through: {errs}"
