@@ -144,6 +144,45 @@ m3_status m3_rope_bc(const m3_dims* dims,
                      void* B_rot, void* C_rot, float* phase,
                      void* stream);
 
+/* Gradients arriving at, or leaving through, a carry (m3_scan_bwd).  All
+ * float32: h [b][h][n][p], prev_B [b][h][r][n], prev_x [b][h][r][p]; any
+ * member may be NULL (absent). */
+typedef struct m3_grad_carry {
+    float* h;
+    float* prev_B;
+    float* prev_x;
+} m3_grad_carry;
+
+/* Bytes of device workspace m3_scan_bwd needs for `dims` (host-only): a
+ * 256-byte header, the state checkpoints (one N x P float32 state per block
+ * of 32 tokens per (b, h)) and a per-(b, h) scratch of 32 states. */
+m3_status m3_scan_bwd_workspace_size(const m3_dims* dims, size_t* bytes);
+
+/* Backward pass of m3_scan_fwd: the gradient of
+ *   J = sum_t <dy_t, y_t> + <d_final.h, h_{L-1}> + <d_final.prev_B, B_{L-1}>
+ *       + <d_final.prev_x, x_{L-1}>
+ * with respect to every input, by reverse mode of the same recurrence
+ * ("Mamba-3" summary, b-lab.team, sections 1-3; the chain rule written out
+ * in k_bwd.cu).  Inputs as in m3_scan_fwd (same layouts, same `init`), plus
+ * dy ([b][t][h][r][p], io dtype) and d_final (nullable; members nullable).
+ * Outputs, all float32 and all overwritten: dx [b][t][h][r][p]; dB, dC
+ * [b][t][g][r][n] (summed over the heads of each group); ddt, dlambda
+ * [b][t][h]; dA [h] (summed over batch and tokens); dtheta [b][t][g][N/2]
+ * (summed over the heads of each group); d_init (nullable; members
+ * nullable): the gradient of the carry-in.
+ * Supported shapes: headdim 16, 32 or 64; rank 1..4; (N/2) * (P/16) <= 256.
+ * Others return M3_ERR_UNSUPPORTED.  Pointers 16-byte aligned.  The library
+ * zeroes the accumulated outputs on `stream` itself; all work is
+ * asynchronous on `stream`. */
+m3_status m3_scan_bwd(const m3_dims* dims,
+                      const void* x, const void* B, const void* C,
+                      const float* dt, const float* A, const float* lambda,
+                      const float* theta, const m3_carry* init,
+                      const void* dy, const m3_grad_carry* d_final,
+                      float* dx, float* dB, float* dC, float* ddt, float* dA,
+                      float* dlambda, float* dtheta, m3_grad_carry* d_init,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
 /* How m3_scan_fwd will run `dims` (host-only, nothing launched): the number
  * of kernel launches one call makes, the segments each (batch, head)
  * sequence is cut into, the chunk length the kernels use, and the path

@@ -59,6 +59,10 @@ def _load():
     lib.m3_scan_fwd_static.restype = I
     lib.m3_selftest_bounded_wait.argtypes = [V, S, V]
     lib.m3_selftest_bounded_wait.restype = I
+    lib.m3_scan_bwd_workspace_size.argtypes = [D, ctypes.POINTER(S)]
+    lib.m3_scan_bwd_workspace_size.restype = I
+    lib.m3_scan_bwd.argtypes = [D, V, V, V, V, V, V, V, C, V, C, V, V, V, V, V, V, V, C, V, S, V]
+    lib.m3_scan_bwd.restype = I
     lib.m3_status_string.argtypes = [I]
     lib.m3_status_string.restype = ctypes.c_char_p
     for f in ("m3_scan_workspace_size", "m3_scan_fwd", "m3_step", "m3_rope_bc", "m3_device_status"):
@@ -71,7 +75,7 @@ _lib = _load()
 # every symbol include/m3.h declares (checked by the CPU test suite)
 ABI_SYMBOLS = ("m3_scan_workspace_size", "m3_scan_fwd", "m3_step", "m3_rope_bc",
                "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_scan_fwd_static",
-               "m3_status_string")
+               "m3_scan_bwd_workspace_size", "m3_scan_bwd", "m3_status_string")
 
 
 @dataclasses.dataclass
@@ -207,11 +211,39 @@ def m3_selftest_bounded_wait(workspace, stream=None) -> None:
                                          _stream(stream)), "m3_selftest_bounded_wait")
 
 
+def m3_scan_bwd_workspace_size(dims: Dims) -> int:
+    n = ctypes.c_size_t(0)
+    d = dims.c()
+    _check(_lib.m3_scan_bwd_workspace_size(ctypes.byref(d), ctypes.byref(n)), "m3_scan_bwd_workspace_size")
+    return n.value
+
+
+def m3_scan_bwd(dims: Dims, x, B, C, dt, A, lam, theta, dy, grads: dict, workspace,
+                init: Optional[Carry] = None, d_final: Optional[Carry] = None,
+                d_init: Optional[Carry] = None, stream=None) -> None:
+    """Backward pass (see include/m3.h).  ``grads`` holds the float32 output
+    tensors dx, dB, dC, ddt, dA, dlam, dtheta; ``d_final`` / ``d_init`` are
+    Carry objects of float32 tensors (members may be None)."""
+    d = dims.c()
+    ci = init.c() if init is not None else None
+    cf = d_final.c() if d_final is not None else None
+    cd = d_init.c() if d_init is not None else None
+    g = grads
+    st = _lib.m3_scan_bwd(ctypes.byref(d), _ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A), _ptr(lam), _ptr(theta),
+                          ctypes.byref(ci) if ci is not None else None, _ptr(dy),
+                          ctypes.byref(cf) if cf is not None else None,
+                          _ptr(g["dx"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["ddt"]), _ptr(g["dA"]),
+                          _ptr(g["dlam"]), _ptr(g["dtheta"]), ctypes.byref(cd) if cd is not None else None,
+                          _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "m3_scan_bwd")
+
+
 def raw_lib():
     """The ctypes handle (for calls that pass raw pointers)."""
     return _lib
 
 
 __all__ = ["Dims", "Carry", "M3Error", "m3_scan_workspace_size", "m3_scan_fwd", "m3_step",
-           "m3_rope_bc", "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_scan_fwd_static", "m3_status_string", "io_dtype_of", "ABI_SYMBOLS",
+           "m3_rope_bc", "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_scan_fwd_static", "m3_scan_bwd_workspace_size", "m3_scan_bwd", "m3_status_string",
+           "io_dtype_of", "ABI_SYMBOLS",
            "M3_F32", "M3_BF16", "raw_lib", "LIB_PATH"]

@@ -1,0 +1,484 @@
+// k_bwd.cu -- backward pass of the Mamba-3 layer scan (sm_100a, SIMT, fp32).
+//
+// Reverse mode of the recurrence of "Mamba-3" summary (b-lab.team), section 1
+// (h_t = alpha h_{t-1} + beta B_{t-1} x_{t-1} + gamma B_t x_t) with the
+// rotation of section 2 (Proposition 2: R_t multiplies the t-1 -> t
+// transition) and the MIMO shapes of section 3.  With g_t = dJ/dh_t and
+// v_t = alpha_t h_{t-1} + beta_t B_{t-1} x_{t-1}^T (the state before R_t):
+//   g_t = C_t dy_t + alpha_{t+1} R_{t+1}^T g_{t+1},   dC_t = h_t dy_t^T,
+//   D_t = gamma_t g_t + beta_{t+1} R_{t+1}^T g_{t+1},  dB_t = D_t x_t,  dx_t = D_t^T B_t,
+//   dgamma = <g_t, B_t x_t^T>,  dalpha = <R_t^T g_t, h_{t-1}>,  dbeta = <R_t^T g_t, B_{t-1} x_{t-1}^T>,
+//   dphi_i = sum_p g_t[pair i]^T R'(phi_i) v_t[pair i],
+// then the chain to dt, lambda, A and theta through alpha = e^{dt A},
+// beta = (1 - lambda) dt alpha, gamma = lambda dt, phi_i = dt theta_i.
+//
+// The states h_t are needed in reverse order.  A first kernel runs the
+// recurrence forward and stores the state before every block of K tokens
+// (a checkpoint); the backward kernel, for each block from the last, runs
+// the block forward again from its checkpoint into a per-(b, h) scratch of
+// K states, then walks the block in reverse.  One CTA per (b, h); thread j
+// owns rotary pair i = j / (P/16) (rows 2i, 2i+1) and 16 columns of the
+// state, so rotations stay in the thread; reductions over columns use lane
+// shuffles, reductions over rows shared memory.  Gradients of B, C and theta
+// (shared by the heads of a group) and of A are accumulated with atomics
+// into zeroed float32 buffers.
+#include "m3_common.cuh"
+#include "m3_kernels.h"
+
+namespace m3 {
+namespace bwd {
+
+constexpr int kPW = 16;            // state columns per thread
+constexpr int kMaxThreads = 256;
+
+template <typename T> __device__ __forceinline__ void ld16(const T* p, float* f);
+template <> __device__ __forceinline__ void ld16<float>(const float* p, float* f) {
+    const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 v = q[i];
+        f[4 * i] = v.x; f[4 * i + 1] = v.y; f[4 * i + 2] = v.z; f[4 * i + 3] = v.w;
+    }
+}
+template <> __device__ __forceinline__ void ld16<__nv_bfloat16>(const __nv_bfloat16* p, float* f) {
+    const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const uint4 v = q[i];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            f[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+            f[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+        }
+    }
+}
+template <typename T> __device__ __forceinline__ float2 ld2(const T* p);
+template <> __device__ __forceinline__ float2 ld2<float>(const float* p) { return *reinterpret_cast<const float2*>(p); }
+template <> __device__ __forceinline__ float2 ld2<__nv_bfloat16>(const __nv_bfloat16* p) {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// Per-thread view of one token's inputs.
+template <int R>
+struct Tok {
+    float x[R][kPW];      // x_t[r][p] on the thread's columns
+    float2 b[R];          // (B_t[r][2i], B_t[r][2i+1])
+    float d, lam, th;     // dt, lambda, theta_t[i]
+};
+
+template <typename T, int R>
+__device__ __forceinline__ void load_tok(const BwdParams& q, int b, int h, int g, int t, int i, int p0, Tok<R>& k) {
+    const int L = q.seqlen, H = q.nheads, G = q.ngroups, N = q.dstate, P = q.headdim;
+    const size_t bt = (size_t)b * L + t;
+    const T* xs = static_cast<const T*>(q.x) + ((bt * H + h) * R) * P + p0;
+    const T* bs = static_cast<const T*>(q.B) + ((bt * G + g) * R) * N + 2 * i;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        ld16<T>(xs + (size_t)r * P, k.x[r]);
+        k.b[r] = ld2<T>(bs + (size_t)r * N);
+    }
+    k.d = q.dt[bt * H + h];
+    k.lam = q.lam[bt * H + h];
+    k.th = q.theta[(bt * G + g) * (N / 2) + i];
+}
+
+// The carry-in (B_{-1}, x_{-1}) in the same per-thread view (zeros if absent).
+template <typename T, int R>
+__device__ __forceinline__ void load_init_prev(const BwdParams& q, int b, int h, int i, int p0, Tok<R>& k) {
+    const int H = q.nheads, N = q.dstate, P = q.headdim;
+    const size_t bh = (size_t)b * H + h;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        if (q.init_pX) ld16<T>(static_cast<const T*>(q.init_pX) + (bh * R + r) * P + p0, k.x[r]);
+        else for (int c = 0; c < kPW; ++c) k.x[r][c] = 0.f;
+        k.b[r] = q.init_pB ? ld2<T>(static_cast<const T*>(q.init_pB) + (bh * R + r) * N + 2 * i) : make_float2(0.f, 0.f);
+    }
+}
+
+template <int R>
+__device__ __forceinline__ void zero_tok(Tok<R>& k) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        k.b[r] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < kPW; ++c) k.x[r][c] = 0.f;
+    }
+    k.d = 0.f; k.lam = 0.f; k.th = 0.f;
+}
+
+// One forward token on the thread's 2 x 16 state elements.
+template <int R>
+__device__ __forceinline__ void fwd_token(float (&h0)[kPW], float (&h1)[kPW], const Tok<R>& pv, const Tok<R>& cu,
+                                          float A) {
+    const float al = __expf(cu.d * A);
+    const float be = (1.f - cu.lam) * cu.d * al, ga = cu.lam * cu.d;
+    float s, c;
+    sincosf(cu.d * cu.th, &s, &c);
+#pragma unroll
+    for (int q = 0; q < kPW; ++q) {
+        float p0 = 0.f, p1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            p0 = fmaf(pv.b[r].x, pv.x[r][q], p0);
+            p1 = fmaf(pv.b[r].y, pv.x[r][q], p1);
+            b0 = fmaf(cu.b[r].x, cu.x[r][q], b0);
+            b1 = fmaf(cu.b[r].y, cu.x[r][q], b1);
+        }
+        const float v0 = fmaf(al, h0[q], be * p0), v1 = fmaf(al, h1[q], be * p1);
+        h0[q] = fmaf(ga, b0, c * v0 - s * v1);
+        h1[q] = fmaf(ga, b1, s * v0 + c * v1);
+    }
+}
+
+__device__ __forceinline__ void st_state(float* dst, int P, int i, int p0, const float (&h0)[kPW], const float (&h1)[kPW]) {
+    float4* r0 = reinterpret_cast<float4*>(dst + (size_t)(2 * i) * P + p0);
+    float4* r1 = reinterpret_cast<float4*>(dst + (size_t)(2 * i + 1) * P + p0);
+#pragma unroll
+    for (int c = 0; c < kPW / 4; ++c) {
+        r0[c] = make_float4(h0[4 * c], h0[4 * c + 1], h0[4 * c + 2], h0[4 * c + 3]);
+        r1[c] = make_float4(h1[4 * c], h1[4 * c + 1], h1[4 * c + 2], h1[4 * c + 3]);
+    }
+}
+__device__ __forceinline__ void ld_state(const float* src, int P, int i, int p0, float (&h0)[kPW], float (&h1)[kPW]) {
+    const float4* r0 = reinterpret_cast<const float4*>(src + (size_t)(2 * i) * P + p0);
+    const float4* r1 = reinterpret_cast<const float4*>(src + (size_t)(2 * i + 1) * P + p0);
+#pragma unroll
+    for (int c = 0; c < kPW / 4; ++c) {
+        const float4 a = r0[c], e = r1[c];
+        h0[4 * c] = a.x; h0[4 * c + 1] = a.y; h0[4 * c + 2] = a.z; h0[4 * c + 3] = a.w;
+        h1[4 * c] = e.x; h1[4 * c + 1] = e.y; h1[4 * c + 2] = e.z; h1[4 * c + 3] = e.w;
+    }
+}
+
+// Forward over the sequence, storing the state before every block of K tokens.
+template <typename T, int R>
+__global__ void __launch_bounds__(kMaxThreads) ckpt_kernel(BwdParams q) {
+    const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+    const int N = q.dstate, P = q.headdim, NPB = P / kPW, L = q.seqlen, K = q.K;
+    const int nck = (L + K - 1) / K;
+    const bool act = tid < (N / 2) * NPB;
+    const int i = act ? tid / NPB : 0, p0 = act ? (tid % NPB) * kPW : 0;
+    const int g = h / (q.nheads / q.ngroups);
+    const size_t bh = (size_t)b * q.nheads + h;
+    const float A = q.A[h];
+    float h0[kPW], h1[kPW];
+    if (q.init_h) ld_state(q.init_h + bh * N * P, P, i, p0, h0, h1);
+    else for (int c = 0; c < kPW; ++c) { h0[c] = 0.f; h1[c] = 0.f; }
+    Tok<R> pv, cu;
+    load_init_prev<T, R>(q, b, h, i, p0, pv);
+    for (int t = 0; t < L; ++t) {
+        if (t % K == 0 && act) st_state(q.ws_ckpt + (bh * nck + t / K) * N * P, P, i, p0, h0, h1);
+        load_tok<T, R>(q, b, h, g, t, i, p0, cu);
+        if (act) fwd_token<R>(h0, h1, pv, cu, A);
+        pv = cu;
+    }
+}
+
+// Reverse pass, one CTA per (b, h).
+template <typename T, int R>
+__global__ void __launch_bounds__(kMaxThreads) bwd_kernel(BwdParams q) {
+    __shared__ float sDx[2][4][kMaxThreads / 32 * 64];   // [parity][r][warp x column block x column]
+    __shared__ float sRed[2][8][4];             // [parity][warp][4 scalars]
+    const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int N = q.dstate, P = q.headdim, NPB = P / kPW, L = q.seqlen, K = q.K, H = q.nheads, G = q.ngroups;
+    const int nck = (L + K - 1) / K;
+    const int nact = (N / 2) * NPB;
+    const bool act = tid < nact;
+    const int i = act ? tid / NPB : 0, pb = act ? tid % NPB : 0, p0 = pb * kPW;
+    const int g = h / (H / G);
+    const size_t bh = (size_t)b * H + h;
+    const float A = q.A[h];
+    const int nwarps = (blockDim.x + 31) / 32;
+    float* scr = q.ws_scratch + bh * (size_t)K * N * P;
+
+    float g0[kPW], g1[kPW], db0[kPW], db1[kPW];
+    if (q.d_fin_h && act) ld_state(q.d_fin_h + bh * N * P, P, i, p0, g0, g1);
+    else for (int c = 0; c < kPW; ++c) { g0[c] = 0.f; g1[c] = 0.f; }
+    for (int c = 0; c < kPW; ++c) { db0[c] = 0.f; db1[c] = 0.f; }
+    float dA_acc = 0.f;
+    // gradients arriving at the final (B, x) copies: into dB_{L-1} (dx_{L-1} below)
+    if (q.d_fin_pB && L > 0)
+        for (int e = tid; e < R * N; e += blockDim.x)
+            atomicAdd(q.dB + (((size_t)b * L + L - 1) * G + g) * R * N + e, q.d_fin_pB[bh * R * N + e]);
+
+    int par = 0;
+    for (int c = nck - 1; c >= 0; --c) {
+        const int t0 = c * K, t1 = min(L, t0 + K);
+        // (a) the block forward again from its checkpoint: h_{t0} .. h_{t1-1} into scratch
+        {
+            float h0[kPW], h1[kPW];
+            if (act) ld_state(q.ws_ckpt + (bh * nck + c) * N * P, P, i, p0, h0, h1);
+            Tok<R> pv, cu;
+            if (t0 == 0) load_init_prev<T, R>(q, b, h, i, p0, pv);
+            else load_tok<T, R>(q, b, h, g, t0 - 1, i, p0, pv);
+            for (int t = t0; t < t1; ++t) {
+                load_tok<T, R>(q, b, h, g, t, i, p0, cu);
+                if (act) {
+                    fwd_token<R>(h0, h1, pv, cu, A);
+                    st_state(scr + (size_t)(t - t0) * N * P, P, i, p0, h0, h1);
+                }
+                pv = cu;
+            }
+        }
+        __syncthreads();      // (each thread reads back only what it wrote; kept for clarity of phases)
+        // (b) reverse over the block
+        for (int t = t1 - 1; t >= t0; --t) {
+            Tok<R> cu, pv;
+            load_tok<T, R>(q, b, h, g, t, i, p0, cu);
+            if (t == 0) load_init_prev<T, R>(q, b, h, i, p0, pv);
+            else load_tok<T, R>(q, b, h, g, t - 1, i, p0, pv);
+            const float d = cu.d, lm = cu.lam;      // token scalars (the same in every thread)
+            if (!act) { zero_tok<R>(cu); zero_tok<R>(pv); }   // idle threads carry zeros
+            const size_t bt = (size_t)b * L + t;
+            float ht0[kPW], ht1[kPW], hp0[kPW], hp1[kPW];
+            if (act) {
+                ld_state(scr + (size_t)(t - t0) * N * P, P, i, p0, ht0, ht1);
+                if (t > t0) ld_state(scr + (size_t)(t - 1 - t0) * N * P, P, i, p0, hp0, hp1);
+                else ld_state(q.ws_ckpt + (bh * nck + c) * N * P, P, i, p0, hp0, hp1);
+            } else {
+                for (int e = 0; e < kPW; ++e) { ht0[e] = ht1[e] = hp0[e] = hp1[e] = 0.f; }
+            }
+            float dy[R][kPW];
+            float2 cc[R];
+            {
+                const T* ys = static_cast<const T*>(q.dy) + ((bt * H + h) * R) * P + p0;
+                const T* cs = static_cast<const T*>(q.C) + ((bt * G + g) * R) * N + 2 * i;
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    ld16<T>(ys + (size_t)r * P, dy[r]);
+                    cc[r] = ld2<T>(cs + (size_t)r * N);
+                    if (!act) {
+                        cc[r] = make_float2(0.f, 0.f);
+#pragma unroll
+                        for (int e = 0; e < kPW; ++e) dy[r][e] = 0.f;
+                    }
+                }
+            }
+            const float al = __expf(d * A), be = (1.f - lm) * d * al, ga = lm * d;
+            float sn, cs_;
+            sincosf(act ? d * cu.th : 0.f, &sn, &cs_);
+            // readout: g += C dy, dC = h_t dy^T (this thread's columns)
+            float dcp[R][2];
+#pragma unroll
+            for (int r = 0; r < R; ++r) { dcp[r][0] = 0.f; dcp[r][1] = 0.f; }
+#pragma unroll
+            for (int e = 0; e < kPW; ++e) {
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    g0[e] = fmaf(cc[r].x, dy[r][e], g0[e]);
+                    g1[e] = fmaf(cc[r].y, dy[r][e], g1[e]);
+                    dcp[r][0] = fmaf(ht0[e], dy[r][e], dcp[r][0]);
+                    dcp[r][1] = fmaf(ht1[e], dy[r][e], dcp[r][1]);
+                }
+            }
+            // D = gamma g + beta' R'^T g' ; dB = D x ; dx = D^T B ; dgamma
+            float dbp[R][2], dxp[R][kPW];
+            float s_ga = 0.f, s_al = 0.f, s_be = 0.f, s_ph = 0.f;
+#pragma unroll
+            for (int r = 0; r < R; ++r) { dbp[r][0] = 0.f; dbp[r][1] = 0.f; }
+#pragma unroll
+            for (int e = 0; e < kPW; ++e) {
+                float bx0 = 0.f, bx1 = 0.f;
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    bx0 = fmaf(cu.b[r].x, cu.x[r][e], bx0);
+                    bx1 = fmaf(cu.b[r].y, cu.x[r][e], bx1);
+                }
+                s_ga = fmaf(g0[e], bx0, fmaf(g1[e], bx1, s_ga));
+                const float D0 = fmaf(ga, g0[e], db0[e]), D1 = fmaf(ga, g1[e], db1[e]);
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    dbp[r][0] = fmaf(D0, cu.x[r][e], dbp[r][0]);
+                    dbp[r][1] = fmaf(D1, cu.x[r][e], dbp[r][1]);
+                    dxp[r][e] = fmaf(D0, cu.b[r].x, D1 * cu.b[r].y);
+                }
+            }
+            // rotation: dphi, gv = R^T g ; dalpha, dbeta ; carry the adjoint
+            float dph = 0.f;
+#pragma unroll
+            for (int e = 0; e < kPW; ++e) {
+                float pbx0 = 0.f, pbx1 = 0.f;
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    pbx0 = fmaf(pv.b[r].x, pv.x[r][e], pbx0);
+                    pbx1 = fmaf(pv.b[r].y, pv.x[r][e], pbx1);
+                }
+                const float v0 = fmaf(al, hp0[e], be * pbx0), v1 = fmaf(al, hp1[e], be * pbx1);
+                dph += g0[e] * (-sn * v0 - cs_ * v1) + g1[e] * (cs_ * v0 - sn * v1);
+                const float gv0 = cs_ * g0[e] + sn * g1[e], gv1 = -sn * g0[e] + cs_ * g1[e];
+                s_al = fmaf(gv0, hp0[e], fmaf(gv1, hp1[e], s_al));
+                s_be = fmaf(gv0, pbx0, fmaf(gv1, pbx1, s_be));
+                db0[e] = be * gv0;
+                db1[e] = be * gv1;
+                g0[e] = al * gv0;
+                g1[e] = al * gv1;
+            }
+            if (!act) {
+                dph = 0.f; s_ga = s_al = s_be = 0.f;
+#pragma unroll
+                for (int r = 0; r < R; ++r) { dcp[r][0] = dcp[r][1] = dbp[r][0] = dbp[r][1] = 0.f; }
+            }
+            // reductions over the NPB column blocks of a row pair (adjacent lanes)
+            for (int o = 1; o < NPB; o <<= 1) {
+                dph += __shfl_xor_sync(0xffffffffu, dph, o);
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    dcp[r][0] += __shfl_xor_sync(0xffffffffu, dcp[r][0], o);
+                    dcp[r][1] += __shfl_xor_sync(0xffffffffu, dcp[r][1], o);
+                    dbp[r][0] += __shfl_xor_sync(0xffffffffu, dbp[r][0], o);
+                    dbp[r][1] += __shfl_xor_sync(0xffffffffu, dbp[r][1], o);
+                }
+            }
+            if (act && pb == 0) {
+                float* dCt = q.dC + (bt * G + g) * R * N + 2 * i;
+                float* dBt = q.dB + (bt * G + g) * R * N + 2 * i;
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    atomicAdd(dCt + (size_t)r * N, dcp[r][0]);
+                    atomicAdd(dCt + (size_t)r * N + 1, dcp[r][1]);
+                    atomicAdd(dBt + (size_t)r * N, dbp[r][0]);
+                    atomicAdd(dBt + (size_t)r * N + 1, dbp[r][1]);
+                }
+                atomicAdd(q.dtheta + (bt * G + g) * (N / 2) + i, dph * d);
+                s_ph = dph * cu.th;
+            }
+            // dx: reduce over the row pairs (lanes with the same column block, then warps)
+            for (int o = NPB; o < 32; o <<= 1) {
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+#pragma unroll
+                    for (int e = 0; e < kPW; ++e) dxp[r][e] += __shfl_xor_sync(0xffffffffu, dxp[r][e], o);
+            }
+            // scalars: reduce over the warp
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                s_ga += __shfl_xor_sync(0xffffffffu, s_ga, o);
+                s_al += __shfl_xor_sync(0xffffffffu, s_al, o);
+                s_be += __shfl_xor_sync(0xffffffffu, s_be, o);
+                s_ph += __shfl_xor_sync(0xffffffffu, s_ph, o);
+            }
+            if (lane < NPB) {
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+#pragma unroll
+                    for (int e = 0; e < kPW; ++e) sDx[par][r][(warp * NPB + lane) * kPW + e] = dxp[r][e];
+            }
+            if (lane == 0) {
+                sRed[par][warp][0] = s_ga;
+                sRed[par][warp][1] = s_al;
+                sRed[par][warp][2] = s_be;
+                sRed[par][warp][3] = s_ph;
+            }
+            __syncthreads();
+            // dx_t[r][p]: one thread per (r, p)
+            for (int e = tid; e < R * P; e += blockDim.x) {
+                const int r = e / P, p = e % P, pbk = p / kPW, col = p % kPW;
+                float acc = 0.f;
+                for (int w = 0; w < nwarps; ++w)
+                    if (w * 32 < nact) acc += sDx[par][r][(w * NPB + pbk) * kPW + col];
+                if (t == L - 1 && q.d_fin_pX) acc += q.d_fin_pX[bh * R * P + e];
+                q.dx[((bt * H + h) * R) * P + e] = acc;
+            }
+            if (tid == 0) {
+                float dga = 0.f, dal = 0.f, dbe = 0.f, dphth = 0.f;
+                for (int w = 0; w < nwarps; ++w) {
+                    dga += sRed[par][w][0];
+                    dal += sRed[par][w][1];
+                    dbe += sRed[par][w][2];
+                    dphth += sRed[par][w][3];
+                }
+                q.ddt[bt * H + h] = dal * A * al + dbe * (1.f - lm) * (al + d * A * al) + dga * lm + dphth;
+                q.dlam[bt * H + h] = -dbe * d * al + dga * d;
+                dA_acc += dal * d * al + dbe * (1.f - lm) * d * d * al;
+            }
+            par ^= 1;
+        }
+        __syncthreads();      // scratch is rewritten by the next block's forward
+    }
+    if (tid == 0) atomicAdd(q.dA + h, dA_acc);
+    // carry-in gradients: d h_{-1} = g ; d prev_B = D_{-1} prev_x ; d prev_x = D_{-1}^T prev_B
+    if (q.d_init_h && act) st_state(q.d_init_h + bh * N * P, P, i, p0, g0, g1);
+    if (q.d_init_pB || q.d_init_pX) {
+        Tok<R> pv;
+        load_init_prev<T, R>(q, b, h, i, p0, pv);
+        float dpb[R][2], dpx[R][kPW];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            dpb[r][0] = dpb[r][1] = 0.f;
+#pragma unroll
+            for (int e = 0; e < kPW; ++e) {
+                dpb[r][0] = fmaf(db0[e], pv.x[r][e], dpb[r][0]);
+                dpb[r][1] = fmaf(db1[e], pv.x[r][e], dpb[r][1]);
+                dpx[r][e] = act ? fmaf(db0[e], pv.b[r].x, db1[e] * pv.b[r].y) : 0.f;
+            }
+            if (!act) dpb[r][0] = dpb[r][1] = 0.f;
+        }
+        for (int o = 1; o < NPB; o <<= 1)
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                dpb[r][0] += __shfl_xor_sync(0xffffffffu, dpb[r][0], o);
+                dpb[r][1] += __shfl_xor_sync(0xffffffffu, dpb[r][1], o);
+            }
+        if (q.d_init_pB && act && pb == 0)
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                q.d_init_pB[(bh * R + r) * N + 2 * i] = dpb[r][0];
+                q.d_init_pB[(bh * R + r) * N + 2 * i + 1] = dpb[r][1];
+            }
+        for (int o = NPB; o < 32; o <<= 1)
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int e = 0; e < kPW; ++e) dpx[r][e] += __shfl_xor_sync(0xffffffffu, dpx[r][e], o);
+        if (lane < NPB)
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int e = 0; e < kPW; ++e) sDx[0][r][(warp * NPB + lane) * kPW + e] = dpx[r][e];
+        __syncthreads();
+        if (q.d_init_pX)
+            for (int e = tid; e < R * P; e += blockDim.x) {
+                const int r = e / P, p = e % P, pbk = p / kPW, col = p % kPW;
+                float acc = 0.f;
+                for (int w = 0; w < nwarps; ++w)
+                    if (w * 32 < nact) acc += sDx[0][r][(w * NPB + pbk) * kPW + col];
+                q.d_init_pX[(bh * R + r) * P + p] = acc;
+            }
+    }
+}
+
+template <typename T, int R>
+static cudaError_t launch_TR(const BwdParams& q, cudaStream_t st) {
+    const int threads = ((q.dstate / 2) * (q.headdim / kPW) + 31) / 32 * 32;
+    const dim3 grid((unsigned)q.nheads, (unsigned)q.batch);
+    ckpt_kernel<T, R><<<grid, threads, 0, st>>>(q);
+    bwd_kernel<T, R><<<grid, threads, 0, st>>>(q);
+    return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_T(const BwdParams& q, cudaStream_t st) {
+    switch (q.rank) {
+        case 1: return launch_TR<T, 1>(q, st);
+        case 2: return launch_TR<T, 2>(q, st);
+        case 3: return launch_TR<T, 3>(q, st);
+        case 4: return launch_TR<T, 4>(q, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace bwd
+
+bool bwd_supported(const m3_dims& d) {
+    const int P = d.headdim, N = d.dstate;
+    return (P == 16 || P == 32 || P == 64) && N % 2 == 0 && (N / 2) * (P / bwd::kPW) <= bwd::kMaxThreads &&
+           d.rank >= 1 && d.rank <= 4;
+}
+
+cudaError_t launch_bwd(const m3_dims& d, const BwdParams& q, cudaStream_t st) {
+    return d.io_dtype == M3_BF16 ? bwd::launch_T<__nv_bfloat16>(q, st) : bwd::launch_T<float>(q, st);
+}
+
+}  // namespace m3

@@ -266,6 +266,78 @@ m3_status m3_rope_bc(const m3_dims* d, const void* B, const void* C, const float
     return launch_rope(*d, q, (cudaStream_t)stream);
 }
 
+static constexpr int kBwdCkpt = 32;      // tokens between backward checkpoints
+
+static size_t bwd_ws_bytes(const m3_dims& d) {
+    const size_t units = (size_t)d.batch * d.nheads, NP = (size_t)d.dstate * d.headdim;
+    const size_t nck = d.seqlen > 0 ? (size_t)(d.seqlen + kBwdCkpt - 1) / kBwdCkpt : 0;
+    size_t off = kWorkspaceHeaderBytes;
+    off += (units * nck * NP * sizeof(float) + 255) & ~(size_t)255;
+    off += (units * kBwdCkpt * NP * sizeof(float) + 255) & ~(size_t)255;
+    return off;
+}
+
+m3_status m3_scan_bwd_workspace_size(const m3_dims* d, size_t* bytes) {
+    m3_status s = check_dims(d, true);
+    if (s != M3_OK) return s;
+    if (!bytes) return M3_ERR_INVALID_ARG;
+    if (!bwd_supported(*d)) return M3_ERR_UNSUPPORTED;
+    *bytes = bwd_ws_bytes(*d);
+    return M3_OK;
+}
+
+m3_status m3_scan_bwd(const m3_dims* d, const void* x, const void* B, const void* C, const float* dt,
+                      const float* A, const float* lambda, const float* theta, const m3_carry* init,
+                      const void* dy, const m3_grad_carry* d_final, float* dx, float* dB, float* dC, float* ddt,
+                      float* dA, float* dlambda, float* dtheta, m3_grad_carry* d_init, void* workspace,
+                      size_t ws_bytes, void* stream) {
+    m3_status s = check_dims(d, true);
+    if (s != M3_OK) return s;
+    if (!bwd_supported(*d)) return M3_ERR_UNSUPPORTED;
+    const bool work = d->batch > 0 && d->seqlen > 0;
+    if (!ptrs_ok({A, dA})) return M3_ERR_INVALID_ARG;
+    if (work && !ptrs_ok({x, B, C, dt, lambda, theta, dy, dx, dB, dC, ddt, dlambda, dtheta}))
+        return M3_ERR_INVALID_ARG;
+    if (init && !opt_ptrs_ok({init->h, init->prev_B, init->prev_x})) return M3_ERR_INVALID_ARG;
+    if (d_final && !opt_ptrs_ok({d_final->h, d_final->prev_B, d_final->prev_x})) return M3_ERR_INVALID_ARG;
+    if (d_init && !opt_ptrs_ok({d_init->h, d_init->prev_B, d_init->prev_x})) return M3_ERR_INVALID_ARG;
+    const size_t need = bwd_ws_bytes(*d);
+    if (!workspace || !aligned16(workspace) || ws_bytes < need) return M3_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t tokg = (size_t)d->batch * d->seqlen * d->ngroups;
+    // the accumulated outputs start at zero
+    if (cudaMemsetAsync(dA, 0, sizeof(float) * d->nheads, st) != cudaSuccess) return M3_ERR_CUDA;
+    if (work) {
+        if (cudaMemsetAsync(dB, 0, sizeof(float) * tokg * d->rank * d->dstate, st) != cudaSuccess ||
+            cudaMemsetAsync(dC, 0, sizeof(float) * tokg * d->rank * d->dstate, st) != cudaSuccess ||
+            cudaMemsetAsync(dtheta, 0, sizeof(float) * tokg * (d->dstate / 2), st) != cudaSuccess)
+            return M3_ERR_CUDA;
+    }
+    BwdParams q;
+    q.batch = d->batch; q.seqlen = d->seqlen; q.nheads = d->nheads; q.ngroups = d->ngroups;
+    q.headdim = d->headdim; q.dstate = d->dstate; q.rank = d->rank; q.K = kBwdCkpt;
+    q.x = x; q.B = B; q.C = C; q.dt = dt; q.A = A; q.lam = lambda; q.theta = theta;
+    q.init_h = init ? init->h : nullptr;
+    q.init_pB = init ? init->prev_B : nullptr;
+    q.init_pX = init ? init->prev_x : nullptr;
+    q.dy = dy;
+    q.d_fin_h = d_final ? d_final->h : nullptr;
+    q.d_fin_pB = d_final ? d_final->prev_B : nullptr;
+    q.d_fin_pX = d_final ? d_final->prev_x : nullptr;
+    q.dx = dx; q.dB = dB; q.dC = dC; q.ddt = ddt; q.dA = dA; q.dlam = dlambda; q.dtheta = dtheta;
+    q.d_init_h = d_init ? d_init->h : nullptr;
+    q.d_init_pB = d_init ? d_init->prev_B : nullptr;
+    q.d_init_pX = d_init ? d_init->prev_x : nullptr;
+    const size_t units = (size_t)d->batch * d->nheads, NP = (size_t)d->dstate * d->headdim;
+    const size_t nck = d->seqlen > 0 ? (size_t)(d->seqlen + kBwdCkpt - 1) / kBwdCkpt : 0;
+    char* base = static_cast<char*>(workspace);
+    q.ws_ckpt = reinterpret_cast<float*>(base + kWorkspaceHeaderBytes);
+    q.ws_scratch = reinterpret_cast<float*>(base + kWorkspaceHeaderBytes +
+                                            ((units * nck * NP * sizeof(float) + 255) & ~(size_t)255));
+    if (d->batch == 0) return M3_OK;
+    return launch_bwd(*d, q, st) == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
 m3_status m3_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void* stream) {
     if (!workspace || !aligned16(workspace) || workspace_bytes < kWorkspaceHeaderBytes) return M3_ERR_WORKSPACE;
     return launch_wait_selftest(reinterpret_cast<int*>(workspace), (cudaStream_t)stream) == cudaSuccess

@@ -60,6 +60,41 @@ struct ScanParams {
     float* ws_sin;     // [b][h][seg][N][P]
 };
 
+// backward pass (k_bwd.cu); gradients are float32, dB / dC / dtheta / dA
+// accumulated with atomics into buffers zeroed by the caller
+struct BwdParams {
+    int batch, seqlen, nheads, ngroups, headdim, dstate, rank;
+    int K;                     // checkpoint interval (tokens)
+    const void* x;
+    const void* B;
+    const void* C;
+    const float* dt;
+    const float* A;
+    const float* lam;
+    const float* theta;
+    const float* init_h;       // nullable
+    const void* init_pB;       // nullable
+    const void* init_pX;       // nullable
+    const void* dy;            // [b][t][h][r][p] io dtype
+    const float* d_fin_h;      // nullable [b][h][n][p]
+    const float* d_fin_pB;     // nullable [b][h][r][n]
+    const float* d_fin_pX;     // nullable [b][h][r][p]
+    float* dx;                 // [b][t][h][r][p]
+    float* dB;                 // [b][t][g][r][n]
+    float* dC;                 // [b][t][g][r][n]
+    float* ddt;                // [b][t][h]
+    float* dA;                 // [h]
+    float* dlam;               // [b][t][h]
+    float* dtheta;             // [b][t][g][n/2]
+    float* d_init_h;           // nullable
+    float* d_init_pB;          // nullable
+    float* d_init_pX;          // nullable
+    float* ws_ckpt;            // [b][h][ceil(L/K)][n][p]
+    float* ws_scratch;         // [b][h][K][n][p]
+};
+bool bwd_supported(const m3_dims& d);
+cudaError_t launch_bwd(const m3_dims& d, const BwdParams& q, cudaStream_t st);
+
 m3_status launch_step(const m3_dims& d, const StepParams& q, cudaStream_t st);
 m3_status launch_rope(const m3_dims& d, const RopeParams& q, cudaStream_t st);
 size_t simt_smem_bytes(int qs, int R, int N, int P, bool summary);

@@ -143,3 +143,22 @@ def test_plan_picks_the_tensor_core_path_for_bf16_layers():
         assert p["launches"] == (1 if p["segments"] == 1 else 3)
     # the 1.5B MIMO layer has 256 sequences: one segment each, one launch
     assert m3.m3_scan_plan(dims_of(m3_synth.CONFIGS[2]))["segments"] == 1
+
+
+def _bwd_status(d, ptr=GOOD, ws=GOOD, ws_bytes=1 << 34, dy=GOOD):
+    cd = d.c()
+    return LIB.m3_scan_bwd(ctypes.byref(cd), ptr, ptr, ptr, ptr, ptr, ptr, ptr, None, dy, None,
+                           ptr, ptr, ptr, ptr, ptr, ptr, ptr, None, ws, ws_bytes, None)
+
+
+def test_bwd_rejects_before_launching():
+    d = dims(headdim=16, dstate=16, rank=2)
+    n = m3.m3_scan_bwd_workspace_size(d)
+    assert n > 256
+    assert _bwd_status(dims(headdim=48)) == m3.M3_ERR_UNSUPPORTED       # P not 16/32/64
+    assert _bwd_status(dims(rank=5, headdim=16, dstate=16)) == m3.M3_ERR_UNSUPPORTED
+    assert _bwd_status(dims(nheads=3, ngroups=2)) == m3.M3_ERR_INVALID_ARG
+    assert _bwd_status(d, ptr=BAD) == m3.M3_ERR_INVALID_ARG
+    assert _bwd_status(d, dy=0) == m3.M3_ERR_INVALID_ARG
+    assert _bwd_status(d, ws_bytes=n - 1) == m3.M3_ERR_WORKSPACE
+    assert _bwd_status(d, ws=0) == m3.M3_ERR_WORKSPACE
