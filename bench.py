@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-rope", action="store_true", help="skip the m3_rope_bc measurement")
+    ap.add_argument("--bwd", action="store_true", help="also time the backward pass m3_scan_bwd")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the layer's batch (profiling captures of a smaller case)")
     ap.add_argument("--workload", choices=["both", "prefill", "decode"], default="both",
@@ -448,6 +449,52 @@ def run_rope(cx, line, pf):
     del Bo, Co, ph
 
 
+def run_bwd(cx, line, pf):
+    """m3_scan_bwd on the layer: the gradients of sum <dy, y> with respect to
+    every input (float32 outputs), dy seeded."""
+    import numpy as np
+    import torch
+    import selective_state_space_m3_b200 as m3
+    args, pk, stream = cx.args, cx.pk, cx.stream
+    s, dev = pf["s"], pf["dev"]
+    b, L, H, G, R, P, N = s.batch, s.seqlen, s.nheads, s.ngroups, s.rank, s.headdim, s.dstate
+    rng = np.random.default_rng(s.seed + 77)
+    dy = torch.from_numpy(rng.standard_normal((b, L, H, R, P)).astype(np.float32)).to(dev["x"].dtype).cuda()
+    f = dict(device="cuda", dtype=torch.float32)
+    g = {"dx": torch.empty(b, L, H, R, P, **f), "dB": torch.empty(b, L, G, R, N, **f),
+         "dC": torch.empty(b, L, G, R, N, **f), "ddt": torch.empty(b, L, H, **f), "dA": torch.empty(H, **f),
+         "dlam": torch.empty(b, L, H, **f), "dtheta": torch.empty(b, L, G, N // 2, **f)}
+    d = m3.Dims(b, L, H, G, P, N, R, s.chunk, m3.M3_BF16 if s.dtype == "bf16" else m3.M3_F32)
+    ws = torch.zeros(m3.m3_scan_bwd_workspace_size(d), dtype=torch.uint8, device="cuda")
+
+    def call():
+        m3.m3_scan_bwd(d, dev["x"], dev["B"], dev["C"], dev["dt"], dev["A"], dev["lam"], dev["theta"],
+                       dy, g, ws, stream=stream)
+
+    call()
+    torch.cuda.synchronize()
+    n = 3
+    cx.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    cx.barrier()
+    ms = cx.max_over_ranks(e0.elapsed_time(e1)) / n
+    nbytes = sum(dev[k].numel() * dev[k].element_size() for k in dev) + dy.numel() * dy.element_size()
+    nbytes += sum(v.numel() * v.element_size() for v in g.values())
+    gbs = nbytes / (ms / 1e3) / 1e9
+    line["bwd"] = {"workload": "scan_bwd_" + line["config"]["workload"], "ms_per_call": ms,
+                   "tokens_per_s": cx.world * b * L / (ms / 1e3),
+                   "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                                "frac": gbs / pk["hbm"], "algorithmic_bytes_per_launch": nbytes,
+                                "traffic": None},
+                   "gpu_launches": 2 * n, "kernels": "checkpoint forward + reverse (SIMT, float32)"}
+    del g, ws, dy
+
+
 def run_decode(cx, line, pf):
     """m3_step x decode_steps captured in one CUDA graph; the carry comes from
     the prefill's final state (tiled, sequence j <- batch row j mod 8), or
@@ -545,6 +592,8 @@ def main():
             run_e2e(cx, line, pf)
         if not args.no_rope:
             run_rope(cx, line, pf)
+        if args.bwd:
+            run_bwd(cx, line, pf)
     if args.workload in ("both", "decode") and not args.no_decode:
         run_decode(cx, line, pf)
     if cx.world == 1 and not args.no_cpu and args.workload != "decode" and args.config == CFG:

@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kMaxThreads) ckpt_kernel(BwdParams q) {
 
 // Reverse pass, one CTA per (b, h).
 template <typename T, int R>
-__global__ void __launch_bounds__(kMaxThreads) bwd_kernel(BwdParams q) {
+__global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
     __shared__ float sDx[2][4][kMaxThreads / 32 * 64];   // [parity][r][warp x column block x column]
     __shared__ float sRed[2][8][4];             // [parity][warp][4 scalars]
     const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -223,147 +223,161 @@ __global__ void __launch_bounds__(kMaxThreads) bwd_kernel(BwdParams q) {
             }
         }
         __syncthreads();      // (each thread reads back only what it wrote; kept for clarity of phases)
-        // (b) reverse over the block
+        // (b) reverse over the block.  The step runs in phases that each
+        // stream one rank's rows at a time, so few values are live at once.
         for (int t = t1 - 1; t >= t0; --t) {
-            Tok<R> cu, pv;
-            load_tok<T, R>(q, b, h, g, t, i, p0, cu);
-            if (t == 0) load_init_prev<T, R>(q, b, h, i, p0, pv);
-            else load_tok<T, R>(q, b, h, g, t - 1, i, p0, pv);
-            const float d = cu.d, lm = cu.lam;      // token scalars (the same in every thread)
-            if (!act) { zero_tok<R>(cu); zero_tok<R>(pv); }   // idle threads carry zeros
             const size_t bt = (size_t)b * L + t;
-            float ht0[kPW], ht1[kPW], hp0[kPW], hp1[kPW];
-            if (act) {
-                ld_state(scr + (size_t)(t - t0) * N * P, P, i, p0, ht0, ht1);
-                if (t > t0) ld_state(scr + (size_t)(t - 1 - t0) * N * P, P, i, p0, hp0, hp1);
-                else ld_state(q.ws_ckpt + (bh * nck + c) * N * P, P, i, p0, hp0, hp1);
-            } else {
-                for (int e = 0; e < kPW; ++e) { ht0[e] = ht1[e] = hp0[e] = hp1[e] = 0.f; }
-            }
-            float dy[R][kPW];
-            float2 cc[R];
+            const float d = q.dt[bt * H + h], lm = q.lam[bt * H + h];
+            const float th = q.theta[(bt * G + g) * (N / 2) + i];
+            const float al = __expf(d * A), be = (1.f - lm) * d * al, ga = lm * d;
+            float sn, cs_;
+            sincosf(act ? d * th : 0.f, &sn, &cs_);
+            const T* xs = static_cast<const T*>(q.x) + ((bt * H + h) * R) * P + p0;
+            const T* bs = static_cast<const T*>(q.B) + ((bt * G + g) * R) * N + 2 * i;
+            const T* ys = static_cast<const T*>(q.dy) + ((bt * H + h) * R) * P + p0;
+            const T* cs = static_cast<const T*>(q.C) + ((bt * G + g) * R) * N + 2 * i;
+
+            // phase 1 -- readout: g += C_t dy_t ; dC_t = h_t dy_t^T
             {
-                const T* ys = static_cast<const T*>(q.dy) + ((bt * H + h) * R) * P + p0;
-                const T* cs = static_cast<const T*>(q.C) + ((bt * G + g) * R) * N + 2 * i;
+                float ht0[kPW], ht1[kPW];
+                if (act) ld_state(scr + (size_t)(t - t0) * N * P, P, i, p0, ht0, ht1);
+                else for (int e = 0; e < kPW; ++e) ht0[e] = ht1[e] = 0.f;
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    ld16<T>(ys + (size_t)r * P, dy[r]);
-                    cc[r] = ld2<T>(cs + (size_t)r * N);
-                    if (!act) {
-                        cc[r] = make_float2(0.f, 0.f);
+                    float dy[kPW];
+                    ld16<T>(ys + (size_t)r * P, dy);
+                    float2 cr = ld2<T>(cs + (size_t)r * N);
+                    if (!act) cr = make_float2(0.f, 0.f);
+                    float dc0 = 0.f, dc1 = 0.f;
 #pragma unroll
-                        for (int e = 0; e < kPW; ++e) dy[r][e] = 0.f;
+                    for (int e = 0; e < kPW; ++e) {
+                        g0[e] = fmaf(cr.x, dy[e], g0[e]);
+                        g1[e] = fmaf(cr.y, dy[e], g1[e]);
+                        dc0 = fmaf(ht0[e], dy[e], dc0);
+                        dc1 = fmaf(ht1[e], dy[e], dc1);
+                    }
+                    for (int o = 1; o < NPB; o <<= 1) {
+                        dc0 += __shfl_xor_sync(0xffffffffu, dc0, o);
+                        dc1 += __shfl_xor_sync(0xffffffffu, dc1, o);
+                    }
+                    if (act && pb == 0) {
+                        float* dCt = q.dC + ((bt * G + g) * R + r) * N + 2 * i;
+                        atomicAdd(dCt, dc0);
+                        atomicAdd(dCt + 1, dc1);
                     }
                 }
             }
-            const float al = __expf(d * A), be = (1.f - lm) * d * al, ga = lm * d;
-            float sn, cs_;
-            sincosf(act ? d * cu.th : 0.f, &sn, &cs_);
-            // readout: g += C dy, dC = h_t dy^T (this thread's columns)
-            float dcp[R][2];
+            // phase 2 -- input terms: D = gamma g + beta' R'^T g' ; dB = D x ; dx = D^T B ;
+            // dgamma = <g, B x^T>
+            float s_ga = 0.f;
 #pragma unroll
-            for (int r = 0; r < R; ++r) { dcp[r][0] = 0.f; dcp[r][1] = 0.f; }
+            for (int r = 0; r < R; ++r) {
+                float xr[kPW];
+                ld16<T>(xs + (size_t)r * P, xr);
+                float2 br = ld2<T>(bs + (size_t)r * N);
+                if (!act) br = make_float2(0.f, 0.f);
+                float db_0 = 0.f, db_1 = 0.f, dxr[kPW];
 #pragma unroll
-            for (int e = 0; e < kPW; ++e) {
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    g0[e] = fmaf(cc[r].x, dy[r][e], g0[e]);
-                    g1[e] = fmaf(cc[r].y, dy[r][e], g1[e]);
-                    dcp[r][0] = fmaf(ht0[e], dy[r][e], dcp[r][0]);
-                    dcp[r][1] = fmaf(ht1[e], dy[r][e], dcp[r][1]);
+                for (int e = 0; e < kPW; ++e) {
+                    const float D0 = fmaf(ga, g0[e], db0[e]), D1 = fmaf(ga, g1[e], db1[e]);
+                    db_0 = fmaf(D0, xr[e], db_0);
+                    db_1 = fmaf(D1, xr[e], db_1);
+                    dxr[e] = act ? fmaf(D0, br.x, D1 * br.y) : 0.f;
+                    s_ga = fmaf(fmaf(g0[e], br.x, g1[e] * br.y), xr[e], s_ga);
                 }
+                for (int o = 1; o < NPB; o <<= 1) {
+                    db_0 += __shfl_xor_sync(0xffffffffu, db_0, o);
+                    db_1 += __shfl_xor_sync(0xffffffffu, db_1, o);
+                }
+                if (act && pb == 0) {
+                    float* dBt = q.dB + ((bt * G + g) * R + r) * N + 2 * i;
+                    atomicAdd(dBt, db_0);
+                    atomicAdd(dBt + 1, db_1);
+                }
+                // dx: over the row pairs (lanes with the same column block, then warps)
+                for (int o = NPB; o < 32; o <<= 1)
+#pragma unroll
+                    for (int e = 0; e < kPW; ++e) dxr[e] += __shfl_xor_sync(0xffffffffu, dxr[e], o);
+                if (lane < NPB)
+#pragma unroll
+                    for (int e = 0; e < kPW; ++e) sDx[par][r][(warp * NPB + lane) * kPW + e] = dxr[e];
             }
-            // D = gamma g + beta' R'^T g' ; dB = D x ; dx = D^T B ; dgamma
-            float dbp[R][2], dxp[R][kPW];
-            float s_ga = 0.f, s_al = 0.f, s_be = 0.f, s_ph = 0.f;
-#pragma unroll
-            for (int r = 0; r < R; ++r) { dbp[r][0] = 0.f; dbp[r][1] = 0.f; }
-#pragma unroll
-            for (int e = 0; e < kPW; ++e) {
-                float bx0 = 0.f, bx1 = 0.f;
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    bx0 = fmaf(cu.b[r].x, cu.x[r][e], bx0);
-                    bx1 = fmaf(cu.b[r].y, cu.x[r][e], bx1);
-                }
-                s_ga = fmaf(g0[e], bx0, fmaf(g1[e], bx1, s_ga));
-                const float D0 = fmaf(ga, g0[e], db0[e]), D1 = fmaf(ga, g1[e], db1[e]);
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    dbp[r][0] = fmaf(D0, cu.x[r][e], dbp[r][0]);
-                    dbp[r][1] = fmaf(D1, cu.x[r][e], dbp[r][1]);
-                    dxp[r][e] = fmaf(D0, cu.b[r].x, D1 * cu.b[r].y);
-                }
-            }
-            // rotation: dphi, gv = R^T g ; dalpha, dbeta ; carry the adjoint
-            float dph = 0.f;
+            if (!act) s_ga = 0.f;
+            // phase 3 -- the transition: gv = R_t^T g ; dphi ; dalpha = <gv, h_{t-1}> ;
+            // dbeta = <gv, B_{t-1} x_{t-1}^T> ; carry the adjoint
+            float s_al = 0.f, s_be = 0.f, dph = 0.f;
 #pragma unroll
             for (int e = 0; e < kPW; ++e) {
-                float pbx0 = 0.f, pbx1 = 0.f;
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    pbx0 = fmaf(pv.b[r].x, pv.x[r][e], pbx0);
-                    pbx1 = fmaf(pv.b[r].y, pv.x[r][e], pbx1);
-                }
-                const float v0 = fmaf(al, hp0[e], be * pbx0), v1 = fmaf(al, hp1[e], be * pbx1);
-                dph += g0[e] * (-sn * v0 - cs_ * v1) + g1[e] * (cs_ * v0 - sn * v1);
                 const float gv0 = cs_ * g0[e] + sn * g1[e], gv1 = -sn * g0[e] + cs_ * g1[e];
-                s_al = fmaf(gv0, hp0[e], fmaf(gv1, hp1[e], s_al));
-                s_be = fmaf(gv0, pbx0, fmaf(gv1, pbx1, s_be));
-                db0[e] = be * gv0;
-                db1[e] = be * gv1;
-                g0[e] = al * gv0;
-                g1[e] = al * gv1;
+                g0[e] = gv0;
+                g1[e] = gv1;
             }
-            if (!act) {
-                dph = 0.f; s_ga = s_al = s_be = 0.f;
+            {
+                float hp0[kPW], hp1[kPW];
+                if (act) {
+                    if (t > t0) ld_state(scr + (size_t)(t - 1 - t0) * N * P, P, i, p0, hp0, hp1);
+                    else ld_state(q.ws_ckpt + (bh * nck + c) * N * P, P, i, p0, hp0, hp1);
+                } else {
+                    for (int e = 0; e < kPW; ++e) hp0[e] = hp1[e] = 0.f;
+                }
 #pragma unroll
-                for (int r = 0; r < R; ++r) { dcp[r][0] = dcp[r][1] = dbp[r][0] = dbp[r][1] = 0.f; }
+                for (int e = 0; e < kPW; ++e) {
+                    s_al = fmaf(g0[e], hp0[e], fmaf(g1[e], hp1[e], s_al));
+                    dph = fmaf(g1[e], hp0[e], fmaf(-g0[e], hp1[e], dph));
+                }
+                dph *= al;
             }
-            // reductions over the NPB column blocks of a row pair (adjacent lanes)
-            for (int o = 1; o < NPB; o <<= 1) {
-                dph += __shfl_xor_sync(0xffffffffu, dph, o);
+            {
+                // the previous token's (B, x): the carry-in for t = 0
+                const T* pxs;
+                const T* pbs;
+                size_t pstride_b;
+                if (t > 0) {
+                    pxs = static_cast<const T*>(q.x) + (((bt - 1) * H + h) * R) * P + p0;
+                    pbs = static_cast<const T*>(q.B) + (((bt - 1) * G + g) * R) * N + 2 * i;
+                    pstride_b = (size_t)N;
+                } else {
+                    pxs = q.init_pX ? static_cast<const T*>(q.init_pX) + (bh * R) * P + p0 : nullptr;
+                    pbs = q.init_pB ? static_cast<const T*>(q.init_pB) + (bh * R) * N + 2 * i : nullptr;
+                    pstride_b = (size_t)N;
+                }
+                float dph_p = 0.f;
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    dcp[r][0] += __shfl_xor_sync(0xffffffffu, dcp[r][0], o);
-                    dcp[r][1] += __shfl_xor_sync(0xffffffffu, dcp[r][1], o);
-                    dbp[r][0] += __shfl_xor_sync(0xffffffffu, dbp[r][0], o);
-                    dbp[r][1] += __shfl_xor_sync(0xffffffffu, dbp[r][1], o);
+                    float px[kPW];
+                    if (pxs) ld16<T>(pxs + (size_t)r * P, px);
+                    else for (int e = 0; e < kPW; ++e) px[e] = 0.f;
+                    float2 pbr = pbs ? ld2<T>(pbs + (size_t)r * pstride_b) : make_float2(0.f, 0.f);
+                    if (!act) pbr = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int e = 0; e < kPW; ++e) {
+                        s_be = fmaf(fmaf(g0[e], pbr.x, g1[e] * pbr.y), px[e], s_be);
+                        dph_p = fmaf(fmaf(g1[e], pbr.x, -g0[e] * pbr.y), px[e], dph_p);
+                    }
                 }
+                dph = fmaf(be, dph_p, dph);
             }
+#pragma unroll
+            for (int e = 0; e < kPW; ++e) {
+                db0[e] = be * g0[e];
+                db1[e] = be * g1[e];
+                g0[e] *= al;
+                g1[e] *= al;
+            }
+            if (!act) { dph = 0.f; s_al = s_be = 0.f; }
+            for (int o = 1; o < NPB; o <<= 1) dph += __shfl_xor_sync(0xffffffffu, dph, o);
+            float s_ph = 0.f;
             if (act && pb == 0) {
-                float* dCt = q.dC + (bt * G + g) * R * N + 2 * i;
-                float* dBt = q.dB + (bt * G + g) * R * N + 2 * i;
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    atomicAdd(dCt + (size_t)r * N, dcp[r][0]);
-                    atomicAdd(dCt + (size_t)r * N + 1, dcp[r][1]);
-                    atomicAdd(dBt + (size_t)r * N, dbp[r][0]);
-                    atomicAdd(dBt + (size_t)r * N + 1, dbp[r][1]);
-                }
                 atomicAdd(q.dtheta + (bt * G + g) * (N / 2) + i, dph * d);
-                s_ph = dph * cu.th;
+                s_ph = dph * th;
             }
-            // dx: reduce over the row pairs (lanes with the same column block, then warps)
-            for (int o = NPB; o < 32; o <<= 1) {
-#pragma unroll
-                for (int r = 0; r < R; ++r)
-#pragma unroll
-                    for (int e = 0; e < kPW; ++e) dxp[r][e] += __shfl_xor_sync(0xffffffffu, dxp[r][e], o);
-            }
-            // scalars: reduce over the warp
+            // scalars: reduce over the warp, then over warps in shared memory
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 s_ga += __shfl_xor_sync(0xffffffffu, s_ga, o);
                 s_al += __shfl_xor_sync(0xffffffffu, s_al, o);
                 s_be += __shfl_xor_sync(0xffffffffu, s_be, o);
                 s_ph += __shfl_xor_sync(0xffffffffu, s_ph, o);
-            }
-            if (lane < NPB) {
-#pragma unroll
-                for (int r = 0; r < R; ++r)
-#pragma unroll
-                    for (int e = 0; e < kPW; ++e) sDx[par][r][(warp * NPB + lane) * kPW + e] = dxp[r][e];
             }
             if (lane == 0) {
                 sRed[par][warp][0] = s_ga;
