@@ -258,6 +258,9 @@ TRAFFIC_R4_B2 = 754_761_984 + 120_160_512
 # DRAM bytes of one step_pipe_kernel launch (decode, batch 256, 32 heads,
 # R=4), from an ncu capture of that launch: 304,197,632 + 224,655,616 bytes.
 TRAFFIC_DECODE_B256 = 304_197_632 + 224_655_616
+# DRAM bytes of one rope_block_kernel launch on the R=4 layer (batch 8), from
+# an ncu capture of that launch: 2,422,795,520 + 2,379,804,160 bytes.
+TRAFFIC_ROPE_LAYER = 2_422_795_520 + 2_379_804_160
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -444,7 +447,8 @@ def run_rope(cx, line, pf):
                     "tokens_per_s": cx.world * s.batch * s.seqlen / (ms / 1e3),
                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
                                  "frac": gbs / pk["hbm"], "algorithmic_bytes_per_launch": nbytes,
-                                 "traffic": None},
+                                 "traffic": TRAFFIC_ROPE_LAYER if (TRAFFIC_CURRENT and s.batch == 8 and
+                                                                   s.rank == 4 and s.seqlen == 4096) else None},
                     "gpu_launches": n, "l2": "inputs and outputs %.1f GB >> L2; no flush" % (nbytes / 1e9)}
     del Bo, Co, ph
 
