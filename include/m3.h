@@ -155,7 +155,8 @@ typedef struct m3_grad_carry {
 
 /* Bytes of device workspace m3_scan_bwd needs for `dims` (host-only): a
  * 256-byte header, the state checkpoints (one N x P float32 state per block
- * of 32 tokens per (b, h)) and a per-(b, h) scratch of 32 states. */
+ * of up to 16 tokens per (b, h)) and a per-(b, h) scratch of one block's
+ * states. */
 m3_status m3_scan_bwd_workspace_size(const m3_dims* dims, size_t* bytes);
 
 /* Backward pass of m3_scan_fwd: the gradient of

@@ -16,7 +16,9 @@
 // recurrence forward and stores the state before every block of K tokens
 // (a checkpoint); the backward kernel, for each block from the last, runs
 // the block forward again from its checkpoint into a per-(b, h) scratch of
-// K states, then walks the block in reverse.  One CTA per (b, h); thread j
+// K states, then walks the block in reverse.  Each block's token inputs
+// (and the token before it) are first staged in shared memory, so the
+// per-token steps read nothing from global memory but the states.  One CTA per (b, h); thread j
 // owns rotary pair i = j / (P/16) (rows 2i, 2i+1) and 16 columns of the
 // state, so rotations stay in the thread; reductions over columns use lane
 // shuffles, reductions over rows shared memory.  Gradients of B, C and theta
@@ -68,22 +70,6 @@ struct Tok {
     float d, lam, th;     // dt, lambda, theta_t[i]
 };
 
-template <typename T, int R>
-__device__ __forceinline__ void load_tok(const BwdParams& q, int b, int h, int g, int t, int i, int p0, Tok<R>& k) {
-    const int L = q.seqlen, H = q.nheads, G = q.ngroups, N = q.dstate, P = q.headdim;
-    const size_t bt = (size_t)b * L + t;
-    const T* xs = static_cast<const T*>(q.x) + ((bt * H + h) * R) * P + p0;
-    const T* bs = static_cast<const T*>(q.B) + ((bt * G + g) * R) * N + 2 * i;
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-        ld16<T>(xs + (size_t)r * P, k.x[r]);
-        k.b[r] = ld2<T>(bs + (size_t)r * N);
-    }
-    k.d = q.dt[bt * H + h];
-    k.lam = q.lam[bt * H + h];
-    k.th = q.theta[(bt * G + g) * (N / 2) + i];
-}
-
 // The carry-in (B_{-1}, x_{-1}) in the same per-thread view (zeros if absent).
 template <typename T, int R>
 __device__ __forceinline__ void load_init_prev(const BwdParams& q, int b, int h, int i, int p0, Tok<R>& k) {
@@ -94,41 +80,6 @@ __device__ __forceinline__ void load_init_prev(const BwdParams& q, int b, int h,
         if (q.init_pX) ld16<T>(static_cast<const T*>(q.init_pX) + (bh * R + r) * P + p0, k.x[r]);
         else for (int c = 0; c < kPW; ++c) k.x[r][c] = 0.f;
         k.b[r] = q.init_pB ? ld2<T>(static_cast<const T*>(q.init_pB) + (bh * R + r) * N + 2 * i) : make_float2(0.f, 0.f);
-    }
-}
-
-template <int R>
-__device__ __forceinline__ void zero_tok(Tok<R>& k) {
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-        k.b[r] = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < kPW; ++c) k.x[r][c] = 0.f;
-    }
-    k.d = 0.f; k.lam = 0.f; k.th = 0.f;
-}
-
-// One forward token on the thread's 2 x 16 state elements.
-template <int R>
-__device__ __forceinline__ void fwd_token(float (&h0)[kPW], float (&h1)[kPW], const Tok<R>& pv, const Tok<R>& cu,
-                                          float A) {
-    const float al = __expf(cu.d * A);
-    const float be = (1.f - cu.lam) * cu.d * al, ga = cu.lam * cu.d;
-    float s, c;
-    sincosf(cu.d * cu.th, &s, &c);
-#pragma unroll
-    for (int q = 0; q < kPW; ++q) {
-        float p0 = 0.f, p1 = 0.f, b0 = 0.f, b1 = 0.f;
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            p0 = fmaf(pv.b[r].x, pv.x[r][q], p0);
-            p1 = fmaf(pv.b[r].y, pv.x[r][q], p1);
-            b0 = fmaf(cu.b[r].x, cu.x[r][q], b0);
-            b1 = fmaf(cu.b[r].y, cu.x[r][q], b1);
-        }
-        const float v0 = fmaf(al, h0[q], be * p0), v1 = fmaf(al, h1[q], be * p1);
-        h0[q] = fmaf(ga, b0, c * v0 - s * v1);
-        h1[q] = fmaf(ga, b1, s * v0 + c * v1);
     }
 }
 
@@ -152,6 +103,115 @@ __device__ __forceinline__ void ld_state(const float* src, int P, int i, int p0,
     }
 }
 
+// Shared-memory staging of a block's token inputs.  Slot 0 holds the token
+// before the block (the carry-in for the first block), slot 1 + k token t0 + k.
+// Per slot: x [R][P], B [R][N], C [R][N], dy [R][P] (io dtype), theta [N/2],
+// then dt and lambda; every part starts on a 16-byte boundary.
+struct StageLayout {
+    int ox, ob, oc, oy, oth, osc, bytes;     // byte offsets inside a slot, slot size
+};
+__host__ __device__ inline StageLayout stage_layout(int R, int N, int P, int sz) {
+    StageLayout l;
+    l.ox = 0;
+    l.ob = l.ox + R * P * sz;
+    l.oc = l.ob + R * N * sz;
+    l.oy = l.oc + R * N * sz;
+    l.oth = l.oy + R * P * sz;
+    l.osc = l.oth + ((N / 2) * 4 + 15) / 16 * 16;
+    l.bytes = l.osc + 16;
+    return l;
+}
+
+// Copy tokens t0-1 .. t1-1 (x, B, theta, dt, lambda, and with `full` also C
+// and dy) into the stage; the carry-in fills slot 0 when t0 == 0.
+template <typename T, int R>
+__device__ void stage_block(const BwdParams& q, int b, int h, int g, int t0, int t1, uint8_t* stg,
+                            const StageLayout& sl, bool full) {
+    const int L = q.seqlen, H = q.nheads, G = q.ngroups, N = q.dstate, P = q.headdim;
+    const int nslot = t1 - t0 + 1;
+    const int ux = R * P * (int)sizeof(T) / 16, ub = R * N * (int)sizeof(T) / 16;
+    const int per = full ? 2 * ux + 2 * ub : ux + ub;          // 16-byte units per slot
+    for (int e = threadIdx.x; e < nslot * per; e += blockDim.x) {
+        const int sidx = e / per;
+        int u = e % per;
+        const int t = t0 - 1 + sidx;
+        uint8_t* slot = stg + (size_t)sidx * sl.bytes;
+        const size_t bt = (size_t)b * L + (t >= 0 ? t : 0);
+        const uint4* src;
+        uint4* dst;
+        if (u < ux) {
+            src = reinterpret_cast<const uint4*>(t >= 0 ? static_cast<const T*>(q.x) + ((bt * H + h) * R) * P
+                  : (q.init_pX ? static_cast<const T*>(q.init_pX) + (((size_t)b * H + h) * R) * P : nullptr));
+            dst = reinterpret_cast<uint4*>(slot + sl.ox);
+        } else if ((u -= ux) < ub) {
+            src = reinterpret_cast<const uint4*>(t >= 0 ? static_cast<const T*>(q.B) + ((bt * G + g) * R) * N
+                  : (q.init_pB ? static_cast<const T*>(q.init_pB) + (((size_t)b * H + h) * R) * N : nullptr));
+            dst = reinterpret_cast<uint4*>(slot + sl.ob);
+        } else if ((u -= ub) < ub) {
+            src = t >= 0 ? reinterpret_cast<const uint4*>(static_cast<const T*>(q.C) + ((bt * G + g) * R) * N) : nullptr;
+            dst = reinterpret_cast<uint4*>(slot + sl.oc);
+        } else {
+            u -= ub;
+            src = t >= 0 ? reinterpret_cast<const uint4*>(static_cast<const T*>(q.dy) + ((bt * H + h) * R) * P) : nullptr;
+            dst = reinterpret_cast<uint4*>(slot + sl.oy);
+        }
+        dst[u] = src ? src[u] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    {
+        for (int e = threadIdx.x; e < nslot * (N / 2 + 2); e += blockDim.x) {
+            const int sidx = e / (N / 2 + 2), u = e % (N / 2 + 2);
+            const int t = t0 - 1 + sidx;
+            uint8_t* slot = stg + (size_t)sidx * sl.bytes;
+            float v = 0.f;
+            if (t >= 0) {
+                const size_t bt = (size_t)b * L + t;
+                v = u < N / 2 ? q.theta[(bt * G + g) * (N / 2) + u] : (u == N / 2 ? q.dt[bt * H + h] : q.lam[bt * H + h]);
+            }
+            if (u < N / 2) reinterpret_cast<float*>(slot + sl.oth)[u] = v;
+            else reinterpret_cast<float*>(slot + sl.osc)[u - N / 2] = v;
+        }
+    }
+}
+
+// One forward token from stage slots (token t and token t - 1), streaming one
+// rank's rows at a time: h = R_t (alpha h + beta B_{t-1} x_{t-1}^T) + gamma B_t x_t^T.
+template <typename T, int R>
+__device__ __forceinline__ void fwd_token_stage(float (&h0)[kPW], float (&h1)[kPW], const uint8_t* pslot,
+                                                const uint8_t* slot, const StageLayout& sl, int N, int P, int i,
+                                                int p0, float A) {
+    const float* sc = reinterpret_cast<const float*>(slot + sl.osc);
+    const float d = sc[0], lm = sc[1], th = reinterpret_cast<const float*>(slot + sl.oth)[i];
+    const float al = __expf(d * A), be = (1.f - lm) * d * al, ga = lm * d;
+    float s, c;
+    sincosf(d * th, &s, &c);
+#pragma unroll
+    for (int e = 0; e < kPW; ++e) { h0[e] *= al; h1[e] *= al; }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        float px[kPW];
+        ld16<T>(reinterpret_cast<const T*>(pslot + sl.ox) + (size_t)r * P + p0, px);
+        const float2 pb = ld2<T>(reinterpret_cast<const T*>(pslot + sl.ob) + (size_t)r * N + 2 * i);
+        const float b0 = be * pb.x, b1 = be * pb.y;
+#pragma unroll
+        for (int e = 0; e < kPW; ++e) { h0[e] = fmaf(b0, px[e], h0[e]); h1[e] = fmaf(b1, px[e], h1[e]); }
+    }
+#pragma unroll
+    for (int e = 0; e < kPW; ++e) {
+        const float v0 = h0[e], v1 = h1[e];
+        h0[e] = c * v0 - s * v1;
+        h1[e] = s * v0 + c * v1;
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        float xr[kPW];
+        ld16<T>(reinterpret_cast<const T*>(slot + sl.ox) + (size_t)r * P + p0, xr);
+        const float2 bb = ld2<T>(reinterpret_cast<const T*>(slot + sl.ob) + (size_t)r * N + 2 * i);
+        const float b0 = ga * bb.x, b1 = ga * bb.y;
+#pragma unroll
+        for (int e = 0; e < kPW; ++e) { h0[e] = fmaf(b0, xr[e], h0[e]); h1[e] = fmaf(b1, xr[e], h1[e]); }
+    }
+}
+
 // Forward over the sequence, storing the state before every block of K tokens.
 template <typename T, int R>
 __global__ void __launch_bounds__(kMaxThreads) ckpt_kernel(BwdParams q) {
@@ -166,13 +226,18 @@ __global__ void __launch_bounds__(kMaxThreads) ckpt_kernel(BwdParams q) {
     float h0[kPW], h1[kPW];
     if (q.init_h) ld_state(q.init_h + bh * N * P, P, i, p0, h0, h1);
     else for (int c = 0; c < kPW; ++c) { h0[c] = 0.f; h1[c] = 0.f; }
-    Tok<R> pv, cu;
-    load_init_prev<T, R>(q, b, h, i, p0, pv);
-    for (int t = 0; t < L; ++t) {
-        if (t % K == 0 && act) st_state(q.ws_ckpt + (bh * nck + t / K) * N * P, P, i, p0, h0, h1);
-        load_tok<T, R>(q, b, h, g, t, i, p0, cu);
-        if (act) fwd_token<R>(h0, h1, pv, cu, A);
-        pv = cu;
+    extern __shared__ __align__(16) uint8_t stg[];
+    const StageLayout sl = stage_layout(R, N, P, (int)sizeof(T));
+    for (int c = 0; c < nck; ++c) {
+        const int t0 = c * K, t1 = min(L, t0 + K);
+        if (act) st_state(q.ws_ckpt + (bh * nck + c) * N * P, P, i, p0, h0, h1);
+        stage_block<T, R>(q, b, h, g, t0, t1, stg, sl, false);
+        __syncthreads();
+        if (act)
+            for (int t = t0; t < t1; ++t)
+                fwd_token_stage<T, R>(h0, h1, stg + (size_t)(t - t0) * sl.bytes, stg + (size_t)(t - t0 + 1) * sl.bytes,
+                                      sl, N, P, i, p0, A);
+        __syncthreads();
     }
 }
 
@@ -203,39 +268,42 @@ __global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
         for (int e = tid; e < R * N; e += blockDim.x)
             atomicAdd(q.dB + (((size_t)b * L + L - 1) * G + g) * R * N + e, q.d_fin_pB[bh * R * N + e]);
 
+    extern __shared__ __align__(16) uint8_t stg[];
+    const StageLayout sl = stage_layout(R, N, P, (int)sizeof(T));
     int par = 0;
     for (int c = nck - 1; c >= 0; --c) {
         const int t0 = c * K, t1 = min(L, t0 + K);
+        // every input of the block (and of the token before it) into shared memory
+        stage_block<T, R>(q, b, h, g, t0, t1, stg, sl, true);
+        __syncthreads();
         // (a) the block forward again from its checkpoint: h_{t0} .. h_{t1-1} into scratch
         {
             float h0[kPW], h1[kPW];
-            if (act) ld_state(q.ws_ckpt + (bh * nck + c) * N * P, P, i, p0, h0, h1);
-            Tok<R> pv, cu;
-            if (t0 == 0) load_init_prev<T, R>(q, b, h, i, p0, pv);
-            else load_tok<T, R>(q, b, h, g, t0 - 1, i, p0, pv);
-            for (int t = t0; t < t1; ++t) {
-                load_tok<T, R>(q, b, h, g, t, i, p0, cu);
-                if (act) {
-                    fwd_token<R>(h0, h1, pv, cu, A);
+            if (act) {
+                ld_state(q.ws_ckpt + (bh * nck + c) * N * P, P, i, p0, h0, h1);
+                for (int t = t0; t < t1; ++t) {
+                    fwd_token_stage<T, R>(h0, h1, stg + (size_t)(t - t0) * sl.bytes,
+                                          stg + (size_t)(t - t0 + 1) * sl.bytes, sl, N, P, i, p0, A);
                     st_state(scr + (size_t)(t - t0) * N * P, P, i, p0, h0, h1);
                 }
-                pv = cu;
             }
         }
-        __syncthreads();      // (each thread reads back only what it wrote; kept for clarity of phases)
         // (b) reverse over the block.  The step runs in phases that each
         // stream one rank's rows at a time, so few values are live at once.
         for (int t = t1 - 1; t >= t0; --t) {
             const size_t bt = (size_t)b * L + t;
-            const float d = q.dt[bt * H + h], lm = q.lam[bt * H + h];
-            const float th = q.theta[(bt * G + g) * (N / 2) + i];
+            const uint8_t* slot = stg + (size_t)(t - t0 + 1) * sl.bytes;       // token t
+            const uint8_t* pslot = stg + (size_t)(t - t0) * sl.bytes;          // token t - 1 (or the carry-in)
+            const float d = reinterpret_cast<const float*>(slot + sl.osc)[0];
+            const float lm = reinterpret_cast<const float*>(slot + sl.osc)[1];
+            const float th = reinterpret_cast<const float*>(slot + sl.oth)[i];
             const float al = __expf(d * A), be = (1.f - lm) * d * al, ga = lm * d;
             float sn, cs_;
             sincosf(act ? d * th : 0.f, &sn, &cs_);
-            const T* xs = static_cast<const T*>(q.x) + ((bt * H + h) * R) * P + p0;
-            const T* bs = static_cast<const T*>(q.B) + ((bt * G + g) * R) * N + 2 * i;
-            const T* ys = static_cast<const T*>(q.dy) + ((bt * H + h) * R) * P + p0;
-            const T* cs = static_cast<const T*>(q.C) + ((bt * G + g) * R) * N + 2 * i;
+            const T* xs = reinterpret_cast<const T*>(slot + sl.ox) + p0;
+            const T* bs = reinterpret_cast<const T*>(slot + sl.ob) + 2 * i;
+            const T* ys = reinterpret_cast<const T*>(slot + sl.oy) + p0;
+            const T* cs = reinterpret_cast<const T*>(slot + sl.oc) + 2 * i;
 
             // phase 1 -- readout: g += C_t dy_t ; dC_t = h_t dy_t^T
             {
@@ -328,26 +396,16 @@ __global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
                 dph *= al;
             }
             {
-                // the previous token's (B, x): the carry-in for t = 0
-                const T* pxs;
-                const T* pbs;
-                size_t pstride_b;
-                if (t > 0) {
-                    pxs = static_cast<const T*>(q.x) + (((bt - 1) * H + h) * R) * P + p0;
-                    pbs = static_cast<const T*>(q.B) + (((bt - 1) * G + g) * R) * N + 2 * i;
-                    pstride_b = (size_t)N;
-                } else {
-                    pxs = q.init_pX ? static_cast<const T*>(q.init_pX) + (bh * R) * P + p0 : nullptr;
-                    pbs = q.init_pB ? static_cast<const T*>(q.init_pB) + (bh * R) * N + 2 * i : nullptr;
-                    pstride_b = (size_t)N;
-                }
+                // the previous token's (B, x): the carry-in for t = 0 (zeros if absent)
+                const T* pxs = reinterpret_cast<const T*>(pslot + sl.ox) + p0;
+                const T* pbs = reinterpret_cast<const T*>(pslot + sl.ob) + 2 * i;
+                const size_t pstride_b = (size_t)N;
                 float dph_p = 0.f;
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
                     float px[kPW];
-                    if (pxs) ld16<T>(pxs + (size_t)r * P, px);
-                    else for (int e = 0; e < kPW; ++e) px[e] = 0.f;
-                    float2 pbr = pbs ? ld2<T>(pbs + (size_t)r * pstride_b) : make_float2(0.f, 0.f);
+                    ld16<T>(pxs + (size_t)r * P, px);
+                    float2 pbr = ld2<T>(pbs + (size_t)r * pstride_b);
                     if (!act) pbr = make_float2(0.f, 0.f);
 #pragma unroll
                     for (int e = 0; e < kPW; ++e) {
@@ -467,8 +525,11 @@ template <typename T, int R>
 static cudaError_t launch_TR(const BwdParams& q, cudaStream_t st) {
     const int threads = ((q.dstate / 2) * (q.headdim / kPW) + 31) / 32 * 32;
     const dim3 grid((unsigned)q.nheads, (unsigned)q.batch);
-    ckpt_kernel<T, R><<<grid, threads, 0, st>>>(q);
-    bwd_kernel<T, R><<<grid, threads, 0, st>>>(q);
+    const size_t smem = (size_t)(q.K + 1) * stage_layout(R, q.dstate, q.headdim, (int)sizeof(T)).bytes;
+    cudaFuncSetAttribute(ckpt_kernel<T, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(bwd_kernel<T, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    ckpt_kernel<T, R><<<grid, threads, smem, st>>>(q);
+    bwd_kernel<T, R><<<grid, threads, smem, st>>>(q);
     return cudaGetLastError();
 }
 
@@ -487,8 +548,18 @@ static cudaError_t launch_T(const BwdParams& q, cudaStream_t st) {
 
 bool bwd_supported(const m3_dims& d) {
     const int P = d.headdim, N = d.dstate;
-    return (P == 16 || P == 32 || P == 64) && N % 2 == 0 && (N / 2) * (P / bwd::kPW) <= bwd::kMaxThreads &&
+    return (P == 16 || P == 32 || P == 64) && N % 8 == 0 && (N / 2) * (P / bwd::kPW) <= bwd::kMaxThreads &&
            d.rank >= 1 && d.rank <= 4;
+}
+
+// Tokens per block (the checkpoint interval and the shared-memory stage):
+// 16, or fewer when a block's inputs would not fit in 160 KB.
+int bwd_block_tokens(const m3_dims& d) {
+    const int sz = d.io_dtype == M3_BF16 ? 2 : 4;
+    const int bytes = bwd::stage_layout(d.rank, d.dstate, d.headdim, sz).bytes;
+    int k = 16;
+    while (k > 1 && (k + 1) * bytes > 160 * 1024) k >>= 1;
+    return k;
 }
 
 cudaError_t launch_bwd(const m3_dims& d, const BwdParams& q, cudaStream_t st) {

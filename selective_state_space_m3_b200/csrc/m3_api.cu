@@ -266,9 +266,8 @@ m3_status m3_rope_bc(const m3_dims* d, const void* B, const void* C, const float
     return launch_rope(*d, q, (cudaStream_t)stream);
 }
 
-static constexpr int kBwdCkpt = 32;      // tokens between backward checkpoints
-
 static size_t bwd_ws_bytes(const m3_dims& d) {
+    const size_t kBwdCkpt = (size_t)bwd_block_tokens(d);     // tokens between checkpoints
     const size_t units = (size_t)d.batch * d.nheads, NP = (size_t)d.dstate * d.headdim;
     const size_t nck = d.seqlen > 0 ? (size_t)(d.seqlen + kBwdCkpt - 1) / kBwdCkpt : 0;
     size_t off = kWorkspaceHeaderBytes;
@@ -315,6 +314,7 @@ m3_status m3_scan_bwd(const m3_dims* d, const void* x, const void* B, const void
     }
     BwdParams q;
     q.batch = d->batch; q.seqlen = d->seqlen; q.nheads = d->nheads; q.ngroups = d->ngroups;
+    const int kBwdCkpt = bwd_block_tokens(*d);
     q.headdim = d->headdim; q.dstate = d->dstate; q.rank = d->rank; q.K = kBwdCkpt;
     q.x = x; q.B = B; q.C = C; q.dt = dt; q.A = A; q.lam = lambda; q.theta = theta;
     q.init_h = init ? init->h : nullptr;

@@ -93,6 +93,7 @@ struct BwdParams {
     float* ws_scratch;         // [b][h][K][n][p]
 };
 bool bwd_supported(const m3_dims& d);
+int bwd_block_tokens(const m3_dims& d);
 cudaError_t launch_bwd(const m3_dims& d, const BwdParams& q, cudaStream_t st);
 
 m3_status launch_step(const m3_dims& d, const StepParams& q, cudaStream_t st);
