@@ -31,7 +31,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "tokens/sec per SSM layer (chunked fwd, decode step) and % of roofline on 1 B200"
-CFG = 2                      # the 1.5B-like MIMO layer
+LAYER = "mimo_r4_layer"       # the 1.5B-like MIMO layer
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -54,9 +54,9 @@ def parse():
                     help="decode alone starts from a seeded random carry (profiling captures)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="override the decode batch (profiling captures of a smaller case)")
-    ap.add_argument("--config", type=int, choices=[1, 2, 3], default=CFG,
-                    help="prefill workload: 2 = the R=4 layer (default, the headline); 1 and 3 "
-                         "time the SISO layer and the long-context SISO layer")
+    ap.add_argument("--layer", choices=["siso_layer", "mimo_r4_layer", "long_siso"], default=LAYER,
+                    help="prefill workload: the R=4 MIMO layer (default, the headline), the SISO "
+                         "layer or the long-context SISO layer")
     return ap.parse_args()
 
 
@@ -160,7 +160,7 @@ def run_reference(args, rank):
     import torch
     import m3_synth
     import oracle
-    s = m3_synth.CONFIGS[CFG]
+    s = m3_synth.LAYERS[LAYER]
     # bounded sample: batch row 0, all heads, the whole sequence (about 11
     # CPU-seconds per step at ~0.35 s per head)
     sub = m3_synth.shrink(s, batch=1)
@@ -178,7 +178,7 @@ def run_reference(args, rank):
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": m3_synth.CONFIG_NAMES[CFG], "global_batch": s.batch, "seq_len": s.seqlen,
+            "config": {"workload": m3_synth.NAMES[LAYER], "global_batch": s.batch, "seq_len": s.seqlen,
                        "sample": "batch row 0 of 8, all 32 heads, full L=4096 per step"},
             "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": "1 of 8 batch rows (32 heads x 4096 tokens) per step"},
@@ -193,7 +193,7 @@ def cpu_baseline_sample():
     import torch
     import m3_synth
     import oracle
-    s = m3_synth.CONFIGS[CFG]
+    s = m3_synth.LAYERS[LAYER]
     sub = m3_synth.shrink(s, batch=2)
     inp = m3_synth.make_scan_inputs(sub)
     f = {k: v.to(torch.float64).numpy() for k, v in inp.items()}
@@ -281,10 +281,10 @@ def throughput(world: int, tokens_per_rank: int, steps: int, total_ms: float) ->
     return world * tokens_per_rank * steps / (total_ms / 1e3)
 
 
-def rank_shape(cfg: int, rank: int, batch: int = 0):
+def rank_shape(layer: str, rank: int, batch: int = 0):
     """Each rank runs its own seeded problem of the same shape (weak scaling)."""
     import m3_synth
-    s = m3_synth.CONFIGS[cfg]
+    s = m3_synth.LAYERS[layer]
     s = m3_synth.shrink(s, seed=s.seed + 1000 * rank)
     if batch > 0:
         s = m3_synth.shrink(s, batch=batch)
@@ -299,7 +299,7 @@ def run_prefill(cx, line):
     import m3_synth
     import selective_state_space_m3_b200 as m3
     args, pk, stream = cx.args, cx.pk, cx.stream
-    s = rank_shape(args.config, cx.rank, args.batch)
+    s = rank_shape(args.layer, cx.rank, args.batch)
     host = m3_synth.make_scan_inputs(s)
     dev = {k: v.cuda() for k, v in host.items()}
     io = m3.M3_BF16 if s.dtype == "bf16" else m3.M3_F32
@@ -358,8 +358,8 @@ def run_prefill(cx, line):
     traffic, traffic_src = measured_traffic(s, plan)
     line.update({
         "value": value, "ms_per_step": ms_per_step,
-        "config": {"workload": m3_synth.CONFIG_NAMES[args.config] if args.batch <= 0 else
-                   m3_synth.CONFIG_NAMES[args.config] + f"_batch{s.batch}",
+        "config": {"workload": m3_synth.NAMES[args.layer] if args.batch <= 0 else
+                   m3_synth.NAMES[args.layer] + f"_batch{s.batch}",
                    "global_batch": s.batch * cx.world,
                    "seq_len": s.seqlen, "nheads": s.nheads, "headdim": s.headdim, "dstate": s.dstate,
                    "rank": s.rank, "chunk": s.chunk,
@@ -510,7 +510,7 @@ def run_decode(cx, line, pf):
     dec = m3_synth.DecodeShape(seed=m3_synth.DECODE.seed + 1000 * cx.rank)
     if args.decode_batch > 0:
         dec = dataclasses_replace(dec, batch=args.decode_batch)
-    if pf is not None and args.config == CFG:
+    if pf is not None and args.layer == LAYER:
         fin = pf["fin"]
         reps = -(-dec.batch // fin.h.shape[0])
         state = m3.Carry(fin.h.repeat(reps, 1, 1, 1)[:dec.batch].contiguous(),
@@ -561,7 +561,7 @@ def run_decode(cx, line, pf):
     step_bytes = (2 * state.h.numel() * 4 + 2 * (state.prev_B.numel() + state.prev_x.numel()) * 2 +
                   sum(v.numel() * v.element_size() for v in t0.values()) + yd.numel() * 2 + Ad.numel() * 4)
     gbs = step_bytes / (per_step_us * 1e-6) / 1e9
-    line["decode"] = {"workload": m3_synth.CONFIG_NAMES[4] if dec.batch == 256 else f"decode_b{dec.batch}",
+    line["decode"] = {"workload": m3_synth.NAMES["decode"] if dec.batch == 256 else f"decode_b{dec.batch}",
                       "tokens_per_s": cx.world * dec.batch / (per_step_us * 1e-6),
                       "us_per_step": per_step_us, "steps_timed": reps_t * S,
                       "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
@@ -569,7 +569,7 @@ def run_decode(cx, line, pf):
                                    "traffic": TRAFFIC_DECODE_B256 if (dec.batch == 256 and TRAFFIC_CURRENT)
                                    else None},
                       "gpu_launches": reps_t * S, "clocks": clk2.summary(),
-                      "carry": "prefill final state" if pf is not None and args.config == CFG
+                      "carry": "prefill final state" if pf is not None and args.layer == LAYER
                       else "seeded random",
                       "inputs": f"{pool} distinct tokens cycled"}
     del g
@@ -600,7 +600,7 @@ def main():
             run_bwd(cx, line, pf)
     if args.workload in ("both", "decode") and not args.no_decode:
         run_decode(cx, line, pf)
-    if cx.world == 1 and not args.no_cpu and args.workload != "decode" and args.config == CFG:
+    if cx.world == 1 and not args.no_cpu and args.workload != "decode" and args.layer == LAYER:
         line["cpu_baseline"] = cpu_baseline_sample()
     cx.close()
     if cx.rank == 0:

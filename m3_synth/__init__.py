@@ -45,20 +45,21 @@ class ScanShape:
     seed: int = 0
 
 
-# The five workloads of the Mamba-3 layer-scan study (sizes of 1.5B-scale
-# layers, plus a tiny fp32 case and a decode case).
-CONFIGS = {
-    0: ScanShape(1, 256, 1, 1, 16, 16, 1, 32, "f32", 0.0, 0),
-    1: ScanShape(4, 2048, 8, 1, 64, 128, 1, 64, "bf16", 0.0, 1),
-    2: ScanShape(8, 4096, 32, 32, 64, 128, 4, 64, "bf16", 0.0, 2),
-    3: ScanShape(1, 32768, 32, 32, 64, 128, 1, 128, "bf16", -1.0, 3),
-}
-CONFIG_NAMES = {
-    0: "siso_tiny_b1_h1_L256_P16_N16_Q32_f32",
-    1: "siso_layer_b4_h8_g1_L2048_P64_N128_Q64_bf16",
-    2: "mimo_r4_layer_b8_h32_L4096_P64_N128_Q64_bf16",
-    3: "long_siso_b1_h32_L32768_P64_N128_Q128_bf16",
-    4: "decode_mimo_r4_b256_h32_P64_N128_x1000",
+# The workloads of the Mamba-3 layer-scan study: a tiny fp32 case, three
+# layers of 1.5B-scale models (seeds 1, 2, 3) and a decode case (below).
+SISO_TINY = ScanShape(1, 256, 1, 1, 16, 16, 1, 32, "f32", 0.0, 0)
+SISO_LAYER = ScanShape(4, 2048, 8, 1, 64, 128, 1, 64, "bf16", 0.0, 1)
+MIMO_R4_LAYER = ScanShape(8, 4096, 32, 32, 64, 128, 4, 64, "bf16", 0.0, 2)
+LONG_SISO = ScanShape(1, 32768, 32, 32, 64, 128, 1, 128, "bf16", -1.0, 3)
+# short names (command lines) and full names (reports)
+LAYERS = {"siso_tiny": SISO_TINY, "siso_layer": SISO_LAYER, "mimo_r4_layer": MIMO_R4_LAYER,
+          "long_siso": LONG_SISO}
+NAMES = {
+    "siso_tiny": "siso_tiny_b1_h1_L256_P16_N16_Q32_f32",
+    "siso_layer": "siso_layer_b4_h8_g1_L2048_P64_N128_Q64_bf16",
+    "mimo_r4_layer": "mimo_r4_layer_b8_h32_L4096_P64_N128_Q64_bf16",
+    "long_siso": "long_siso_b1_h32_L32768_P64_N128_Q128_bf16",
+    "decode": "decode_mimo_r4_b256_h32_P64_N128_x1000",
 }
 
 
@@ -73,7 +74,7 @@ class DecodeShape:
     steps: int = 1000
     dtype: str = "bf16"
     seed: int = 4
-    init_from: int = 2   # carry initialised from this scan config's final state
+    # the carry starts from the final state of the MIMO R=4 layer's prefill
 
 
 DECODE = DecodeShape()
@@ -117,7 +118,7 @@ def make_scan_inputs(s: ScanShape) -> dict:
 
 def make_decode_token(d: DecodeShape, k: int, batch: Optional[int] = None) -> dict:
     """Per-token inputs of decode step ``k`` (fresh draws, generator seeded by
-    (seed, k)); distributions as the scan configs.  ``batch`` may shrink the
+    (seed, k)); distributions as the scan workloads.  ``batch`` may shrink the
     batch for small tests (the first ``batch`` rows of the same draw order are
     NOT preserved: a smaller batch is a different draw)."""
     b = d.batch if batch is None else batch

@@ -133,16 +133,15 @@ def test_null_dims():
 def test_plan_picks_the_tensor_core_path_for_bf16_layers():
     import m3_synth
     from tests._util import dims_of
-    p0 = m3.m3_scan_plan(dims_of(m3_synth.CONFIGS[0]))
+    p0 = m3.m3_scan_plan(dims_of(m3_synth.SISO_TINY))
     assert p0["path"] == "simt" and p0["chunk_used"] == 32
-    for cfg in (1, 2, 3):
-        s = m3_synth.CONFIGS[cfg]
+    for s in (m3_synth.SISO_LAYER, m3_synth.MIMO_R4_LAYER, m3_synth.LONG_SISO):
         p = m3.m3_scan_plan(dims_of(s))
         assert p["path"] == "tcgen05"
         assert p["chunk_used"] == 128 // s.rank
         assert p["launches"] == (1 if p["segments"] == 1 else 3)
     # the 1.5B MIMO layer has 256 sequences: one segment each, one launch
-    assert m3.m3_scan_plan(dims_of(m3_synth.CONFIGS[2]))["segments"] == 1
+    assert m3.m3_scan_plan(dims_of(m3_synth.MIMO_R4_LAYER))["segments"] == 1
 
 
 def _bwd_status(d, ptr=GOOD, ws=GOOD, ws_bytes=1 << 34, dy=GOOD):

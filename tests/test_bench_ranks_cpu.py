@@ -32,12 +32,12 @@ def _rank_main(rank, world, port, out_dir):
     os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
                       MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import m3_synth
-    args = types.SimpleNamespace(config=bench.CFG, batch=1)
+    args = types.SimpleNamespace(layer=bench.LAYER, batch=1)
     cx = bench.Ctx(args, device="cpu")
     my_ms = 10.0 + 5.0 * rank                     # rank 1 is the slow one
     cx.barrier()
     slowest = cx.max_over_ranks(my_ms)
-    shape = bench.rank_shape(bench.CFG, cx.rank, batch=1)
+    shape = bench.rank_shape(bench.LAYER, cx.rank, batch=1)
     small = m3_synth.shrink(shape, seqlen=8, nheads=2, ngroups=2)
     x = m3_synth.make_scan_inputs(small)["x"].float()
     cx.close()
@@ -66,7 +66,7 @@ def test_throughput_counts_every_rank_over_the_slowest_time():
 
 
 def test_single_rank_context_needs_no_process_group():
-    args = types.SimpleNamespace(config=bench.CFG, batch=0)
+    args = types.SimpleNamespace(layer=bench.LAYER, batch=0)
     env = {k: os.environ.pop(k) for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK") if k in os.environ}
     try:
         cx = bench.Ctx(args, device="cpu")
@@ -79,11 +79,11 @@ def test_single_rank_context_needs_no_process_group():
 
 def test_traffic_is_reported_only_for_the_captured_shape():
     import m3_synth
-    s = m3_synth.CONFIGS[bench.CFG]
+    s = m3_synth.LAYERS[bench.LAYER]
     t, _ = bench.measured_traffic(s, {"path": "tcgen05"})
     if bench.TRAFFIC_CURRENT:
         assert t == pytest.approx(bench.TRAFFIC_R4_B2 * 4)
     else:
         assert t is None
     assert bench.measured_traffic(s, {"path": "simt"})[0] is None
-    assert bench.measured_traffic(m3_synth.CONFIGS[3], {"path": "tcgen05"})[0] is None
+    assert bench.measured_traffic(m3_synth.LONG_SISO, {"path": "tcgen05"})[0] is None

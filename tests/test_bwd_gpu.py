@@ -59,7 +59,7 @@ def _compare(tag, g, ref, tol=1e-4, skip=(), di=None):
 
 
 CASES = [
-    # several 32-token checkpoint blocks and a ragged tail; shared group
+    # several 16-token checkpoint blocks and a ragged tail; shared group
     (m3_synth.ScanShape(2, 100, 2, 1, 16, 16, 2, 32, "f32", 0.0, 91), "f32_mimo_shared"),
     (m3_synth.ScanShape(1, 70, 3, 3, 64, 128, 4, 64, "bf16", 0.0, 92), "bf16_r4_layer_dims"),
     (m3_synth.ScanShape(2, 45, 4, 2, 32, 32, 1, 64, "bf16", -1.0, 93), "bf16_siso"),
@@ -94,7 +94,7 @@ def test_scan_bwd_layer_shape_sampled():
     """The R=4 layer's full shape (8 x 4096 tokens, 32 heads, one group per
     head), sampled (b, h) against the oracle run on that slice alone.  dA
     sums over the batch, so it is compared through its own slice sum."""
-    shape = m3_synth.CONFIGS[2]
+    shape = m3_synth.MIMO_R4_LAYER
     inp = m3_synth.make_scan_inputs(shape)
     b, L, H, R, P = shape.batch, shape.seqlen, shape.nheads, shape.rank, shape.headdim
     rng = np.random.default_rng(2024)

@@ -40,7 +40,7 @@ def _check(name, got, want, tol):
 # ------------------------------------------------------------ small cases --
 SMALL = [
     # shape, id  -- span several chunks and a ragged tail
-    (m3_synth.ScanShape(1, 256, 1, 1, 16, 16, 1, 32, "f32", 0.0, 0), "cfg0_full"),
+    (m3_synth.ScanShape(1, 256, 1, 1, 16, 16, 1, 32, "f32", 0.0, 0), "siso_tiny_full"),
     (m3_synth.ScanShape(2, 300, 4, 2, 16, 16, 2, 32, "f32", 0.0, 11), "f32_mimo_ragged"),
     (m3_synth.ScanShape(2, 333, 4, 2, 64, 128, 1, 64, "bf16", 0.0, 12), "bf16_siso_ragged"),
     (m3_synth.ScanShape(1, 200, 3, 3, 64, 128, 4, 64, "bf16", 0.0, 13), "bf16_mimo_r4"),
@@ -211,7 +211,7 @@ def test_rope_bc_matches_oracle(dtype):
 def test_rope_bc_layer_shape_sampled():
     """m3_rope_bc on the R=4 layer (8 x 4096 tokens, 32 heads, N=128, bf16) --
     the launch the bench times -- against the oracle on sampled (b, h)."""
-    shape = m3_synth.CONFIGS[2]
+    shape = m3_synth.MIMO_R4_LAYER
     inp = m3_synth.make_scan_inputs(shape)
     dev = {k: v.cuda() for k, v in inp.items()}
     d = dims_of(shape)
@@ -278,40 +278,40 @@ def test_scan_then_steps_equals_longer_scan():
 
 
 # ----------------------------------------------- full-size, sampled outputs --
-def _sampled_full(cfg, samples):
-    shape = m3_synth.CONFIGS[cfg]
+def _sampled_full(name, samples):
+    shape = m3_synth.LAYERS[name]
     inp = m3_synth.make_scan_inputs(shape)
     y, fin = gpu_scan(shape, inp)
     tol = tol_for(shape.dtype)
     for (b, h) in samples:
         one = slice_bh(inp, shape, b, h)
         yo, ho, _, _ = oracle.scan(**one)
-        _check(f"cfg{cfg} b{b} h{h} y", f64(y[b:b + 1, :, h:h + 1]), yo, tol)
-        _check(f"cfg{cfg} b{b} h{h} h", f64(fin.h[b:b + 1, h:h + 1]), ho, tol)
+        _check(f"{name} b{b} h{h} y", f64(y[b:b + 1, :, h:h + 1]), yo, tol)
+        _check(f"{name} b{b} h{h} h", f64(fin.h[b:b + 1, h:h + 1]), ho, tol)
 
 
-def test_config0_full_size():
-    _sampled_full(0, [(0, 0)])
+def test_siso_tiny_full_size():
+    _sampled_full("siso_tiny", [(0, 0)])
 
 
-def test_config1_full_size_sampled():
-    _sampled_full(1, [(0, 0), (1, 5), (3, 7)])
+def test_siso_layer_full_size_sampled():
+    _sampled_full("siso_layer", [(0, 0), (1, 5), (3, 7)])
 
 
-def test_config2_full_size_sampled():
-    _sampled_full(2, [(0, 0), (3, 17), (7, 31)])
+def test_mimo_r4_layer_full_size_sampled():
+    _sampled_full("mimo_r4_layer", [(0, 0), (3, 17), (7, 31)])
 
 
-def test_config3_full_size_sampled():
-    _sampled_full(3, [(0, 0), (0, 21)])
+def test_long_siso_full_size_sampled():
+    _sampled_full("long_siso", [(0, 0), (0, 21)])
 
 
-def test_config4_decode_full_batch_sampled():
+def test_decode_full_batch_sampled():
     """Decode at the full batch (256 sequences, 32 heads, R=4) for 32 tokens,
-    from the oracle's final carry of config 2's first batch row (tiled over
+    from the oracle's final carry of the R=4 layer's first batch row (tiled over
     the 256 sequences), sampled sequences compared with the oracle."""
     dec = m3_synth.DECODE
-    c2 = m3_synth.CONFIGS[2]
+    c2 = m3_synth.MIMO_R4_LAYER
     inp2 = m3_synth.make_scan_inputs(c2)
     one = {k: f64(v[0:1]) if k != "A" else f64(v) for k, v in inp2.items()}
     _, h0, pB0, pX0 = oracle.scan(**one)                       # [1][32][...]
