@@ -251,10 +251,10 @@ class Ctx:
 
 # DRAM bytes (read + write) of one scan_tc_kernel<4,0> launch, from the ncu
 # capture of the R=4 layer at batch 2 (the main pass of a 4-segment plan):
-# 754,761,984 + 120,160,512 bytes.  Traffic grows with the (batch, head) units
+# 754,940,416 + 120,642,816 bytes.  Traffic grows with the (batch, head) units
 # (each is one sequence read once), so a launch over `batch` sequences moves
 # batch / 2 times this.  The capture and its command are in profiles/.
-TRAFFIC_R4_B2 = 754_761_984 + 120_160_512
+TRAFFIC_R4_B2 = 754_940_416 + 120_642_816
 # DRAM bytes of one step_pipe_kernel launch (decode, batch 256, 32 heads,
 # R=4), from an ncu capture of that launch: 304,197,632 + 224,655,616 bytes.
 TRAFFIC_DECODE_B256 = 304_197_632 + 224_655_616
