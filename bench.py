@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-rope", action="store_true", help="skip the m3_rope_bc measurement")
     ap.add_argument("--bwd", action="store_true", help="also time the backward pass m3_scan_bwd")
+    ap.add_argument("--phase", action="store_true", help="also time two phase interventions")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the layer's batch (profiling captures of a smaller case)")
     ap.add_argument("--workload", choices=["both", "prefill", "decode"], default="both",
@@ -499,6 +500,48 @@ def run_bwd(cx, line, pf):
     del g, ws, dy
 
 
+def run_phase(cx, line, pf):
+    """m3_scan_fwd_phase on the layer for two interventions (reversed phase:
+    a theta rewrite; rotation on readout only: m3_rope_bc plus a theta = 0
+    scan), against the prefill's algorithmic bytes."""
+    import torch
+    import selective_state_space_m3_b200 as m3
+    args, pk, stream = cx.args, cx.pk, cx.stream
+    s, dev = pf["s"], pf["dev"]
+    d = m3.Dims(s.batch, s.seqlen, s.nheads, s.ngroups, s.headdim, s.dstate, s.rank, s.chunk,
+                m3.M3_BF16 if s.dtype == "bf16" else m3.M3_F32)
+    y = torch.empty_like(dev["x"])
+    out = {}
+    for name, mode in (("reverse", m3.M3_PHASE_REVERSE), ("read_only", m3.M3_PHASE_READ_ONLY)):
+        ws = torch.zeros(m3.m3_scan_phase_workspace_size(d, mode), dtype=torch.uint8, device="cuda")
+
+        def call():
+            m3.m3_scan_fwd_phase(d, mode, dev["x"], dev["B"], dev["C"], dev["dt"], dev["A"], dev["lam"],
+                                 dev["theta"], y, ws, stream=stream)
+
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        n = 10
+        cx.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        cx.barrier()
+        assert m3.m3_device_status(ws) == m3.M3_OK
+        ms = cx.max_over_ranks(e0.elapsed_time(e1)) / n
+        gbs = line["roofline"]["algorithmic_bytes_per_launch"] / (ms / 1e3) / 1e9
+        out[name] = {"ms_per_call": ms, "tokens_per_s": cx.world * s.batch * s.seqlen / (ms / 1e3),
+                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                                  "frac": gbs / pk["hbm"], "traffic": None,
+                                  "algorithmic_bytes_per_launch": line["roofline"]["algorithmic_bytes_per_launch"]}}
+        del ws
+    line["phase"] = out
+
+
 def run_decode(cx, line, pf):
     """m3_step x decode_steps captured in one CUDA graph; the carry comes from
     the prefill's final state (tiled, sequence j <- batch row j mod 8), or
@@ -598,6 +641,8 @@ def main():
             run_rope(cx, line, pf)
         if args.bwd:
             run_bwd(cx, line, pf)
+        if args.phase:
+            run_phase(cx, line, pf)
     if args.workload in ("both", "decode") and not args.no_decode:
         run_decode(cx, line, pf)
     if cx.world == 1 and not args.no_cpu and args.workload != "decode" and args.layer == LAYER:

@@ -184,6 +184,45 @@ m3_status m3_scan_bwd(const m3_dims* dims,
                       float* dlambda, float* dtheta, m3_grad_carry* d_init,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* Phase interventions ("Understanding Mamba-3 Through Oscillatory Dynamics",
+ * section 5.3 and appendix D.4; fixed rotations, section 4.3).  The first
+ * five rewrite theta before the scan; the last two keep the rotation on one
+ * side of the state only, in the form of Proposition 3 ("Mamba-3" summary,
+ * b-lab.team, section 2):  y_t = C'_t^T h'_t with h' the theta = 0 recurrence
+ * driven by B', where B' = B~ (rotated by the cumulative phase) or B, and
+ * C' = C~ or C. */
+typedef enum m3_phase_mode {
+    M3_PHASE_NATIVE = 0,      /* theta as given                                   */
+    M3_PHASE_ZERO = 1,        /* theta := 0 (no rotation)                         */
+    M3_PHASE_REVERSE = 2,     /* theta := -theta                                  */
+    M3_PHASE_SHUFFLE = 3,     /* theta_t[i] := theta_t[perm[i]], every token      */
+    M3_PHASE_FIXED = 4,       /* theta_t[i] := freq[g][i], the same every token   */
+    M3_PHASE_WRITE_ONLY = 5,  /* rotation on writing (B~), none on readout (C)    */
+    M3_PHASE_READ_ONLY = 6    /* rotation on readout (C~), none on writing (B)    */
+} m3_phase_mode;
+
+/* Bytes of device workspace m3_scan_fwd_phase needs (host-only). */
+m3_status m3_scan_phase_workspace_size(const m3_dims* dims, int mode, size_t* bytes);
+
+/* m3_scan_fwd under a phase intervention.  Arguments as m3_scan_fwd, plus:
+ *   mode  an m3_phase_mode;
+ *   perm  (SHUFFLE) HOST array of N/2 int32, a permutation of 0..N/2-1
+ *         (checked; M3_ERR_INVALID_ARG otherwise); NULL for other modes;
+ *   freq  (FIXED) HOST array [G][N/2] of float32 phase increments per unit
+ *         dt; NULL for other modes.
+ * Both are copied into the workspace on `stream`.  For ZERO, REVERSE,
+ * SHUFFLE and FIXED the carry (init / final_state) means what it means for
+ * m3_scan_fwd.  For WRITE_ONLY and READ_ONLY the state is that of the
+ * theta = 0 recurrence on (B', C'), i.e. the rotated frame of Proposition 3
+ * without the final rotation back, and `init` is read in that frame.  The
+ * device status word is the workspace's first 256 bytes, as for m3_scan_fwd. */
+m3_status m3_scan_fwd_phase(const m3_dims* dims, int mode, const int* perm, const float* freq,
+                            const void* x, const void* B, const void* C,
+                            const float* dt, const float* A, const float* lambda,
+                            const float* theta, const m3_carry* init, void* y,
+                            m3_carry* final_state, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
 /* How m3_scan_fwd will run `dims` (host-only, nothing launched): the number
  * of kernel launches one call makes, the segments each (batch, head)
  * sequence is cut into, the chunk length the kernels use, and the path

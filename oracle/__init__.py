@@ -157,6 +157,42 @@ def scan_bwd(x, B, C, dt, A, lam, theta, dy, init_h=None, init_pB=None, init_pX=
     return out
 
 
+PHASE_MODES = ("native", "zero", "reverse", "shuffle", "fixed", "write_only", "read_only")
+
+
+def scan_phase(mode, x, B, C, dt, A, lam, theta, perm=None, freq=None, init_h=None, init_pB=None,
+               init_pX=None, lib=None):
+    """The scan under a phase intervention ("Understanding Mamba-3 Through
+    Oscillatory Dynamics", section 5.3, appendix D.4; fixed rotations,
+    section 4.3), written as its definition: the first five modes change
+    theta and run scan(); write_only / read_only run the theta = 0 scan on
+    per-head operands of which one side is rotated by the cumulative phase
+    (rope_bc, Proposition 3) and the other is not.  Returns scan()'s tuple."""
+    mode = PHASE_MODES.index(mode) if isinstance(mode, str) else int(mode)
+    x, B, C, dt, A, lam, theta = map(_f64, (x, B, C, dt, A, lam, theta))
+    kw = dict(init_h=init_h, init_pB=init_pB, init_pX=init_pX, lib=lib)
+    if mode == 0:
+        return scan(x, B, C, dt, A, lam, theta, **kw)
+    if mode == 1:
+        return scan(x, B, C, dt, A, lam, np.zeros_like(theta), **kw)
+    if mode == 2:
+        return scan(x, B, C, dt, A, lam, -theta, **kw)
+    if mode == 3:
+        return scan(x, B, C, dt, A, lam, theta[..., np.asarray(perm)], **kw)
+    if mode == 4:
+        fq = np.asarray(freq, dtype=np.float64)            # [G][N/2]
+        return scan(x, B, C, dt, A, lam, np.broadcast_to(fq, theta.shape).copy(), **kw)
+    H = x.shape[2]
+    G = B.shape[2]
+    Br, Cr, _ = rope_bc(B, C, dt, theta, nheads=H, lib=lib)
+    Bh = np.repeat(B, H // G, axis=2)
+    Ch = np.repeat(C, H // G, axis=2)
+    th0 = np.zeros(theta.shape[:2] + (H, theta.shape[3]))
+    if mode == 5:
+        return scan(x, Br, Ch, dt, A, lam, th0, **kw)
+    return scan(x, Bh, Cr, dt, A, lam, th0, **kw)
+
+
 def step(h, prev_B, prev_x, x, B, C, dt, A, lam, theta, lib=None):
     """One decode token.  h [b,h,n,p], prev_B [b,h,r,n], prev_x [b,h,r,p];
     x [b,h,r,p]; B, C [b,g,r,n]; dt, lam [b,h]; A [h]; theta [b,g,n/2].

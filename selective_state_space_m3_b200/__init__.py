@@ -15,6 +15,7 @@ import dataclasses
 import os
 from typing import Optional
 
+import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -63,6 +64,10 @@ def _load():
     lib.m3_scan_bwd_workspace_size.restype = I
     lib.m3_scan_bwd.argtypes = [D, V, V, V, V, V, V, V, C, V, C, V, V, V, V, V, V, V, C, V, S, V]
     lib.m3_scan_bwd.restype = I
+    lib.m3_scan_phase_workspace_size.argtypes = [D, I, ctypes.POINTER(S)]
+    lib.m3_scan_phase_workspace_size.restype = I
+    lib.m3_scan_fwd_phase.argtypes = [D, I, V, V, V, V, V, V, V, V, V, C, V, C, V, S, V]
+    lib.m3_scan_fwd_phase.restype = I
     lib.m3_status_string.argtypes = [I]
     lib.m3_status_string.restype = ctypes.c_char_p
     for f in ("m3_scan_workspace_size", "m3_scan_fwd", "m3_step", "m3_rope_bc", "m3_device_status"):
@@ -75,7 +80,8 @@ _lib = _load()
 # every symbol include/m3.h declares (checked by the CPU test suite)
 ABI_SYMBOLS = ("m3_scan_workspace_size", "m3_scan_fwd", "m3_step", "m3_rope_bc",
                "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_scan_fwd_static",
-               "m3_scan_bwd_workspace_size", "m3_scan_bwd", "m3_status_string")
+               "m3_scan_bwd_workspace_size", "m3_scan_bwd", "m3_scan_phase_workspace_size",
+               "m3_scan_fwd_phase", "m3_status_string")
 
 
 @dataclasses.dataclass
@@ -238,6 +244,40 @@ def m3_scan_bwd(dims: Dims, x, B, C, dt, A, lam, theta, dy, grads: dict, workspa
     _check(st, "m3_scan_bwd")
 
 
+M3_PHASE_NATIVE, M3_PHASE_ZERO, M3_PHASE_REVERSE, M3_PHASE_SHUFFLE, M3_PHASE_FIXED, \
+    M3_PHASE_WRITE_ONLY, M3_PHASE_READ_ONLY = range(7)
+
+
+def m3_scan_phase_workspace_size(dims: Dims, mode: int) -> int:
+    n = ctypes.c_size_t(0)
+    d = dims.c()
+    _check(_lib.m3_scan_phase_workspace_size(ctypes.byref(d), int(mode), ctypes.byref(n)),
+           "m3_scan_phase_workspace_size")
+    return n.value
+
+
+def m3_scan_fwd_phase(dims: Dims, mode: int, x, B, C, dt, A, lam, theta, y, workspace, perm=None, freq=None,
+                      init: Optional[Carry] = None, final_state: Optional[Carry] = None, stream=None) -> None:
+    """m3_scan_fwd under a phase intervention (see include/m3.h).  ``perm``
+    (SHUFFLE) and ``freq`` (FIXED) are host sequences / arrays."""
+    d = dims.c()
+    ci = init.c() if init is not None else None
+    cf = final_state.c() if final_state is not None else None
+    perm_c = (ctypes.c_int * len(perm))(*[int(v) for v in perm]) if perm is not None else None
+    freq_c = None
+    if freq is not None:
+        flat = [float(v) for v in np.asarray(freq, dtype=np.float32).ravel()]
+        freq_c = (ctypes.c_float * len(flat))(*flat)
+    st = _lib.m3_scan_fwd_phase(ctypes.byref(d), int(mode),
+                                ctypes.cast(perm_c, ctypes.c_void_p) if perm_c is not None else None,
+                                ctypes.cast(freq_c, ctypes.c_void_p) if freq_c is not None else None,
+                                _ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A), _ptr(lam), _ptr(theta),
+                                ctypes.byref(ci) if ci is not None else None, _ptr(y),
+                                ctypes.byref(cf) if cf is not None else None, _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "m3_scan_fwd_phase")
+
+
 def raw_lib():
     """The ctypes handle (for calls that pass raw pointers)."""
     return _lib
@@ -245,5 +285,5 @@ def raw_lib():
 
 __all__ = ["Dims", "Carry", "M3Error", "m3_scan_workspace_size", "m3_scan_fwd", "m3_step",
            "m3_rope_bc", "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_scan_fwd_static", "m3_scan_bwd_workspace_size", "m3_scan_bwd", "m3_status_string",
-           "io_dtype_of", "ABI_SYMBOLS",
+           "m3_scan_phase_workspace_size", "m3_scan_fwd_phase", "io_dtype_of", "ABI_SYMBOLS",
            "M3_F32", "M3_BF16", "raw_lib", "LIB_PATH"]

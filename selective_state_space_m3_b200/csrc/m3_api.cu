@@ -4,6 +4,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <vector>
+
 #include "m3_common.cuh"
 #include "m3_kernels.h"
 
@@ -336,6 +338,119 @@ m3_status m3_scan_bwd(const m3_dims* d, const void* x, const void* B, const void
                                             ((units * nck * NP * sizeof(float) + 255) & ~(size_t)255));
     if (d->batch == 0) return M3_OK;
     return launch_bwd(*d, q, st) == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+// ------------------------------------------------------- phase interventions
+struct PhaseLayout {
+    size_t inner, perm, freq, theta, brot, crot, expd, total;
+};
+
+static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static m3_status phase_layout(const m3_dims& d, int mode, PhaseLayout* l) {
+    if (mode < M3_PHASE_NATIVE || mode > M3_PHASE_READ_ONLY) return M3_ERR_INVALID_ARG;
+    const bool onesided = mode == M3_PHASE_WRITE_ONLY || mode == M3_PHASE_READ_ONLY;
+    m3_dims di = d;
+    if (onesided) di.ngroups = d.nheads;
+    size_t inner = 0;
+    m3_status s = m3_scan_workspace_size(&di, &inner);
+    if (s != M3_OK) return s;
+    const size_t NH = d.dstate / 2, tok = (size_t)d.batch * d.seqlen;
+    const size_t io = d.io_dtype == M3_BF16 ? 2 : 4;
+    l->inner = 0;
+    size_t off = up256(inner);
+    l->perm = off;  off = up256(off + (mode == M3_PHASE_SHUFFLE ? NH * sizeof(int) : 0));
+    l->freq = off;  off = up256(off + (mode == M3_PHASE_FIXED ? (size_t)d.ngroups * NH * sizeof(float) : 0));
+    const size_t th_groups = onesided ? (size_t)d.nheads : (size_t)d.ngroups;
+    l->theta = off; off = up256(off + (mode == M3_PHASE_NATIVE ? 0 : tok * th_groups * NH * sizeof(float)));
+    const size_t per_head = onesided ? tok * d.nheads * (size_t)d.rank * d.dstate * io : 0;
+    l->brot = off;  off = up256(off + per_head);
+    l->crot = off;  off = up256(off + per_head);
+    l->expd = off;  off = up256(off + (onesided && d.ngroups != d.nheads ? per_head : 0));
+    l->total = off;
+    return M3_OK;
+}
+
+m3_status m3_scan_phase_workspace_size(const m3_dims* d, int mode, size_t* bytes) {
+    m3_status s = check_dims(d, true);
+    if (s != M3_OK) return s;
+    if (!bytes) return M3_ERR_INVALID_ARG;
+    PhaseLayout l;
+    s = phase_layout(*d, mode, &l);
+    if (s != M3_OK) return s;
+    *bytes = l.total;
+    return M3_OK;
+}
+
+m3_status m3_scan_fwd_phase(const m3_dims* d, int mode, const int* perm, const float* freq, const void* x,
+                            const void* B, const void* C, const float* dt, const float* A, const float* lambda,
+                            const float* theta, const m3_carry* init, void* y, m3_carry* final_state,
+                            void* workspace, size_t ws_bytes, void* stream) {
+    m3_status s = check_dims(d, true);
+    if (s != M3_OK) return s;
+    PhaseLayout l;
+    s = phase_layout(*d, mode, &l);
+    if (s != M3_OK) return s;
+    const int NH = d->dstate / 2;
+    if (mode == M3_PHASE_SHUFFLE) {
+        if (!perm) return M3_ERR_INVALID_ARG;
+        std::vector<char> seen(NH, 0);
+        for (int i = 0; i < NH; ++i) {
+            if (perm[i] < 0 || perm[i] >= NH || seen[perm[i]]) return M3_ERR_INVALID_ARG;
+            seen[perm[i]] = 1;
+        }
+    }
+    if (mode == M3_PHASE_FIXED && !freq) return M3_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace) || ws_bytes < l.total) return M3_ERR_WORKSPACE;
+    const bool work = d->batch > 0 && d->seqlen > 0;
+    if (work && !ptrs_ok({x, B, C, dt, A, lambda, theta, y})) return M3_ERR_INVALID_ARG;
+    if (mode == M3_PHASE_NATIVE)
+        return m3_scan_fwd(d, x, B, C, dt, A, lambda, theta, init, y, final_state, workspace, ws_bytes, stream);
+    cudaStream_t st = (cudaStream_t)stream;
+    char* base = static_cast<char*>(workspace);
+    const size_t tok = (size_t)d->batch * d->seqlen;
+    const size_t inner_bytes = l.perm;            // the inner scan's workspace comes first
+    if (mode == M3_PHASE_WRITE_ONLY || mode == M3_PHASE_READ_ONLY) {
+        m3_dims di = *d;
+        di.ngroups = d->nheads;
+        void* brot = base + l.brot;
+        void* crot = base + l.crot;
+        float* th0 = reinterpret_cast<float*>(base + l.theta);
+        if (work) {
+            s = m3_rope_bc(d, B, C, dt, theta, brot, crot, nullptr, stream);
+            if (s != M3_OK) return s;
+            if (cudaMemsetAsync(th0, 0, tok * d->nheads * NH * sizeof(float), st) != cudaSuccess) return M3_ERR_CUDA;
+        }
+        // the side that keeps no rotation, one copy per head
+        const void* plain = mode == M3_PHASE_WRITE_ONLY ? C : B;
+        const void* plain_h = plain;
+        if (work && d->ngroups != d->nheads) {
+            const size_t row = (size_t)d->rank * d->dstate * (d->io_dtype == M3_BF16 ? 2 : 4);
+            if (launch_expand_heads(plain, base + l.expd, tok, d->nheads, d->ngroups, row, st) != cudaSuccess)
+                return M3_ERR_CUDA;
+            plain_h = base + l.expd;
+        }
+        const void* Bp = mode == M3_PHASE_WRITE_ONLY ? brot : plain_h;
+        const void* Cp = mode == M3_PHASE_WRITE_ONLY ? plain_h : crot;
+        return m3_scan_fwd(&di, x, work ? Bp : B, work ? Cp : C, dt, A, lambda, work ? th0 : theta, init, y,
+                           final_state, workspace, inner_bytes, stream);
+    }
+    // zero / reverse / shuffle / fixed: rewrite theta, then the ordinary scan
+    int* dperm = reinterpret_cast<int*>(base + l.perm);
+    float* dfreq = reinterpret_cast<float*>(base + l.freq);
+    float* th = reinterpret_cast<float*>(base + l.theta);
+    if (mode == M3_PHASE_SHUFFLE &&
+        cudaMemcpyAsync(dperm, perm, NH * sizeof(int), cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return M3_ERR_CUDA;
+    if (mode == M3_PHASE_FIXED &&
+        cudaMemcpyAsync(dfreq, freq, (size_t)d->ngroups * NH * sizeof(float), cudaMemcpyHostToDevice, st) !=
+            cudaSuccess)
+        return M3_ERR_CUDA;
+    if (work && launch_theta_transform(mode, theta, dperm, dfreq, th, tok * d->ngroups, d->ngroups, NH, st) !=
+                    cudaSuccess)
+        return M3_ERR_CUDA;
+    return m3_scan_fwd(d, x, B, C, dt, A, lambda, work ? th : theta, init, y, final_state, workspace, inner_bytes,
+                       stream);
 }
 
 m3_status m3_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void* stream) {

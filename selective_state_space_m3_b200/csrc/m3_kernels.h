@@ -96,6 +96,12 @@ bool bwd_supported(const m3_dims& d);
 int bwd_block_tokens(const m3_dims& d);
 cudaError_t launch_bwd(const m3_dims& d, const BwdParams& q, cudaStream_t st);
 
+// phase interventions (k_phase.cu)
+cudaError_t launch_theta_transform(int mode, const float* in, const int* perm, const float* freq, float* out,
+                                   size_t rows, int G, int NH, cudaStream_t st);
+cudaError_t launch_expand_heads(const void* src, void* dst, size_t bt_count, int H, int G, size_t row_bytes,
+                                cudaStream_t st);
+
 m3_status launch_step(const m3_dims& d, const StepParams& q, cudaStream_t st);
 m3_status launch_rope(const m3_dims& d, const RopeParams& q, cudaStream_t st);
 size_t simt_smem_bytes(int qs, int R, int N, int P, bool summary);

@@ -161,3 +161,24 @@ def test_bwd_rejects_before_launching():
     assert _bwd_status(d, dy=0) == m3.M3_ERR_INVALID_ARG
     assert _bwd_status(d, ws_bytes=n - 1) == m3.M3_ERR_WORKSPACE
     assert _bwd_status(d, ws=0) == m3.M3_ERR_WORKSPACE
+
+
+def _phase_status(d, mode, perm=None, freq=None, ws_bytes=1 << 34):
+    cd = d.c()
+    pc = (ctypes.c_int * len(perm))(*perm) if perm is not None else None
+    fc = (ctypes.c_float * len(freq))(*freq) if freq is not None else None
+    return LIB.m3_scan_fwd_phase(ctypes.byref(cd), mode, ctypes.cast(pc, ctypes.c_void_p) if pc else None,
+                                 ctypes.cast(fc, ctypes.c_void_p) if fc else None,
+                                 GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, None, GOOD, None, GOOD, ws_bytes, None)
+
+
+def test_phase_rejects_before_launching():
+    d = dims(dstate=16)                        # 8 rotary pairs
+    assert _phase_status(d, 7) == m3.M3_ERR_INVALID_ARG
+    assert _phase_status(d, m3.M3_PHASE_SHUFFLE) == m3.M3_ERR_INVALID_ARG                 # no perm
+    assert _phase_status(d, m3.M3_PHASE_SHUFFLE, perm=[0, 1, 2, 3, 4, 5, 6, 6]) == m3.M3_ERR_INVALID_ARG
+    assert _phase_status(d, m3.M3_PHASE_SHUFFLE, perm=[0, 1, 2, 3, 4, 5, 6, 8]) == m3.M3_ERR_INVALID_ARG
+    assert _phase_status(d, m3.M3_PHASE_FIXED) == m3.M3_ERR_INVALID_ARG                   # no freq
+    n = m3.m3_scan_phase_workspace_size(d, m3.M3_PHASE_READ_ONLY)
+    assert n > m3.m3_scan_workspace_size(d)
+    assert _phase_status(d, m3.M3_PHASE_READ_ONLY, ws_bytes=n - 1) == m3.M3_ERR_WORKSPACE

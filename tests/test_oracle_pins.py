@@ -613,3 +613,46 @@ def test_backward_planted_mistakes_are_caught(name):
     lib = oracle.compile_variant(src, name)
     errs = _fd_errors(lib)
     assert max(errs.values()) > 1e-4, f"mutation {name} slipped through: {errs}"
+
+
+# --------------------------------------------------- phase interventions --
+def test_phase_modes_reduce_to_native_where_they_must():
+    """With theta == 0 every intervention is the native scan; an identity
+    permutation and a 'fixed' frequency equal to the given theta are too."""
+    I = rand_inputs(31, b=1, L=30, H=4, G=2, P=3, N=8, R=2)
+    I0 = dict(I, theta=np.zeros_like(I["theta"]))
+    y0 = oracle.scan(**I0)[0]
+    for mode in ("zero", "reverse", "write_only", "read_only"):
+        assert rel(oracle.scan_phase(mode, **I0)[0], y0) < 1e-12, mode
+    y = oracle.scan(**I)[0]
+    assert rel(oracle.scan_phase("shuffle", **I, perm=[0, 1, 2, 3])[0], y) < 1e-12
+    Ic = dict(I, theta=np.broadcast_to(np.array([[0.3, -1.1, 2.0, 0.7], [1.5, 0.2, -0.4, 3.0]]),
+                                       I["theta"].shape).copy())
+    assert rel(oracle.scan_phase("fixed", **Ic, freq=[[0.3, -1.1, 2.0, 0.7], [1.5, 0.2, -0.4, 3.0]])[0],
+               oracle.scan(**Ic)[0]) < 1e-12
+    # reverse equals the native scan on the mirrored pairs (conjugate rotation)
+    Im = dict(I, B=I["B"][..., [1, 0, 3, 2, 5, 4, 7, 6]], C=I["C"][..., [1, 0, 3, 2, 5, 4, 7, 6]])
+    yr = oracle.scan_phase("reverse", **I)[0]
+    assert rel(yr, oracle.scan(**Im)[0]) < 1e-12
+
+
+@pytest.mark.parametrize("mode", ["write_only", "read_only"])
+def test_one_sided_rotation_is_the_dense_two_band_form(mode):
+    """write_only / read_only against the dense two-band SSD matrix built here
+    with only one of B, C rotated by the cumulative phase (complex multiply)."""
+    I = rand_inputs(32, b=1, L=18, H=1, G=1, P=2, N=4, R=2)
+    y = oracle.scan_phase(mode, **I)[0]
+    L, R, P, N = 18, 2, 2, 4
+    dt, lam, A = I["dt"][0, :, 0], I["lam"][0, :, 0], I["A"][0]
+    a = np.cumsum(dt * A)
+    M = np.tril(np.exp(a[:, None] - a[None, :])) @ (
+        np.diag(lam * dt) + np.diag(((1 - lam) * dt * np.exp(dt * A))[1:], k=-1))
+    Phi = np.cumsum(dt[:, None] * I["theta"][0, :, 0], axis=0)
+    rot = lambda v: to_complex(v) * np.exp(-1j * Phi)[:, None, :]
+    Bc = rot(I["B"][0, :, 0]) if mode == "write_only" else to_complex(I["B"][0, :, 0])
+    Cc = to_complex(I["C"][0, :, 0]) if mode == "write_only" else rot(I["C"][0, :, 0])
+    Bt = np.stack([Bc.real, Bc.imag], -1).reshape(L, R, N)
+    Ct = np.stack([Cc.real, Cc.imag], -1).reshape(L, R, N)
+    Gm = np.einsum("trn,usn->trus", Ct, Bt).reshape(L * R, L * R)
+    Y = (np.kron(M, np.ones((R, R))) * Gm) @ I["x"][0, :, 0].reshape(L * R, P)
+    assert np.max(np.abs(y[0, :, 0].reshape(L * R, P) - Y)) < 1e-10
