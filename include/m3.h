@@ -36,10 +36,13 @@
  * bfloat16 operands with float32 accumulation on the bfloat16 path).
  *
  * Ownership and threading.  Every pointer is a device pointer owned by the
- * caller (except m3_scan_workspace_size's output and the dims/carry structs,
- * which are host memory read during the call).  The library allocates no
+ * caller (except the size outputs of the *_workspace_size calls, the
+ * dims/carry structs and m3_scan_fwd_phase's perm / freq arrays, which are
+ * host memory read during the call).  The library allocates no
  * device memory, keeps no state between calls apart from cached device
- * attributes, and never synchronises the stream except in m3_device_status.
+ * attributes, and never synchronises the stream except in m3_device_status
+ * and in m3_scan_fwd_phase's copy of its host arrays (SHUFFLE / FIXED modes:
+ * a copy from pageable host memory may wait for the stream).
  * Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
  * stream).  Calls on different streams are independent if they share no
  * buffers.  Device pointers must be 16-byte aligned.
