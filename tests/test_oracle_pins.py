@@ -656,3 +656,21 @@ def test_one_sided_rotation_is_the_dense_two_band_form(mode):
     Gm = np.einsum("trn,usn->trus", Ct, Bt).reshape(L * R, L * R)
     Y = (np.kron(M, np.ones((R, R))) * Gm) @ I["x"][0, :, 0].reshape(L * R, P)
     assert np.max(np.abs(y[0, :, 0].reshape(L * R, P) - Y)) < 1e-10
+
+
+def test_backward_homogeneity_identities():
+    """Exact identities, no finite differences: with a zero carry-in the loss
+    J = sum <dy, y> is linear in x, in B and in C separately (homogeneous of
+    degree one), so <dJ/dx, x> = <dJ/dB, B> = <dJ/dC, C> = J; and the carry-in
+    state enters linearly, so adding h_{-1} adds exactly <dJ/dh_{-1}, h_{-1}>."""
+    I = rand_inputs(41, b=2, L=12, H=2, G=1, P=3, N=6, R=2)
+    rng = np.random.default_rng(410)
+    dy = rng.standard_normal((2, 12, 2, 2, 3))
+    y = oracle.scan(**I)[0]
+    J = float((dy * y).sum())
+    g = oracle.scan_bwd(**I, dy=dy)
+    for k in ("x", "B", "C"):
+        assert abs(float((g["d" + k] * I[k]).sum()) - J) < 1e-10 * max(1.0, abs(J)), k
+    h0 = rng.standard_normal((2, 2, 6, 3))
+    J1 = float((dy * oracle.scan(**I, init_h=h0)[0]).sum())
+    assert abs((J1 - J) - float((g["d_init_h"] * h0).sum())) < 1e-10 * max(1.0, abs(J1))
