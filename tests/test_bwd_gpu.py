@@ -125,3 +125,32 @@ def test_scan_bwd_empty_sequence():
     assert torch.equal(di.h, dh)
     assert torch.count_nonzero(g["dA"]) == 0
     assert torch.count_nonzero(di.prev_B) == 0 and torch.count_nonzero(di.prev_x) == 0
+
+
+def test_scan_bwd_layer_homogeneity_full_size():
+    """At the R=4 layer's full size, identities that need no oracle: with no
+    carry-in, J = sum <dy, y> is linear in x, in B and in C, so the backward's
+    <dx, x>, <dB, B> and <dC, C> are the same number, J.  Against J computed
+    from the forward's y the bound is the forward's own: |J_fwd - J| is at most
+    the y error (relative L2 2e-2) times ||y|| ||dy|| (Cauchy-Schwarz); the sum
+    cancels heavily, so J_fwd alone is a loose check."""
+    shape = m3_synth.MIMO_R4_LAYER
+    inp = m3_synth.make_scan_inputs(shape)
+    b, L, H, R, P = shape.batch, shape.seqlen, shape.nheads, shape.rank, shape.headdim
+    rng = np.random.default_rng(77)
+    dy = torch.from_numpy(rng.standard_normal((b, L, H, R, P)).astype(np.float32)).to(torch.bfloat16)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    d = dims_of(shape)
+    y = torch.empty_like(dev["x"])
+    ws = torch.zeros(m3.m3_scan_workspace_size(d), dtype=torch.uint8, device="cuda")
+    m3.m3_scan_fwd(d, dev["x"], dev["B"], dev["C"], dev["dt"], dev["A"], dev["lam"], dev["theta"], y, ws)
+    dyd = dy.cuda().double()
+    J_fwd = float((y.double() * dyd).sum())
+    bound = 2e-2 * float(y.double().norm()) * float(dyd.norm())
+    g, _ = _gpu_bwd(shape, inp, dy)
+    v = {k: float((g["d" + k].double() * dev[k].double()).sum()) for k in ("x", "B", "C")}
+    print(f"homogeneity: <dx,x>={v['x']:.6e} <dB,B>={v['B']:.6e} <dC,C>={v['C']:.6e} J_fwd={J_fwd:.6e} "
+          f"bound={bound:.3e}")
+    assert abs(v["B"] - v["x"]) <= 1e-3 * abs(v["x"]), v
+    assert abs(v["C"] - v["x"]) <= 1e-3 * abs(v["x"]), v
+    assert abs(v["x"] - J_fwd) <= bound, (v, J_fwd, bound)
