@@ -87,3 +87,11 @@ def test_traffic_is_reported_only_for_the_captured_shape():
         assert t is None
     assert bench.measured_traffic(s, {"path": "simt"})[0] is None
     assert bench.measured_traffic(m3_synth.LONG_SISO, {"path": "tcgen05"})[0] is None
+
+
+def test_bench_defaults_are_one_gpu_and_minutes_of_work(monkeypatch):
+    monkeypatch.setattr(sys, "argv", ["bench.py"])
+    a = bench.parse()
+    assert a.gpus == 1 and a.warmup >= 3 and 1 <= a.steps <= 200
+    assert a.impl == "ours" and a.layer == bench.LAYER and a.decode_steps == 1000
+    assert not a.bwd and not a.phase          # the optional measurements stay off by default
