@@ -201,9 +201,34 @@ def cpu_baseline_sample():
     t0 = time.perf_counter()
     oracle.scan(**f)
     dt = time.perf_counter() - t0
-    return {"value": sub.batch * sub.seqlen / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "sample": f"2 of 8 batch rows (64 head-sequences x 4096 tokens), {dt:.1f} s wall"}
+    out = {"value": sub.batch * sub.seqlen / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
+           "kind": "oracle",
+           "sample": f"2 of 8 batch rows (64 head-sequences x 4096 tokens), {dt:.1f} s wall"}
+    out["single_thread"] = oracle_single_thread()
+    return out
+
+
+def oracle_single_thread():
+    """The oracle on one host thread, on the two small SISO workloads in full
+    (the tiny one and the 4 x 2048-token, 8-head layer): a per-core figure
+    beside the all-cores sample."""
+    import torch
+    import m3_synth
+    import oracle
+    res = {}
+    cores = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        for name in ("siso_tiny", "siso_layer"):
+            s = m3_synth.LAYERS[name]
+            f = {k: v.to(torch.float64).numpy() for k, v in m3_synth.make_scan_inputs(s).items()}
+            t0 = time.perf_counter()
+            oracle.scan(**f)
+            dt = time.perf_counter() - t0
+            res[name] = {"tokens_per_s": s.batch * s.seqlen / dt, "seconds": dt}
+    finally:
+        oracle.set_num_threads(cores)
+    return res
 
 
 # ------------------------------------------------------------------ ours --

@@ -63,6 +63,8 @@ def _bind(lib):
     lib.oracle_rope_bc.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+    lib.oracle_set_num_threads.restype = None
     return lib
 
 
@@ -106,6 +108,12 @@ def _f64(a):
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """OpenMP threads of later oracle calls (timing only: every (b, h) is
+    computed by one thread, so the results do not depend on it)."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def scan(x, B, C, dt, A, lam, theta, init_h=None, init_pB=None, init_pX=None, lib=None):

@@ -463,3 +463,15 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* Sets the OpenMP thread count of later calls (n >= 1); timing only, the
+ * results do not depend on it (each (b, h) is computed by one thread). */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

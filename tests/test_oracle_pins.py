@@ -441,6 +441,27 @@ def test_oracle_rejects_bad_arguments():
                     I["theta"][..., :1])          # odd N
 
 
+def test_thread_count_does_not_change_results():
+    """Each (b, h) is one thread's sequential loop, so one thread and all of
+    them give bit-identical outputs, forward and backward (the bench times the
+    oracle both ways)."""
+    I = rand_inputs(14, b=3, L=9, H=4, G=2, P=3, N=4, R=2)
+    dy = np.random.default_rng(140).standard_normal(I["x"].shape)
+    cores = oracle.num_threads()
+    try:
+        oracle.set_num_threads(1)
+        one = oracle.scan(**I), oracle.scan_bwd(**I, dy=dy)
+        oracle.set_num_threads(max(cores, 2))
+        many = oracle.scan(**I), oracle.scan_bwd(**I, dy=dy)
+    finally:
+        oracle.set_num_threads(cores)
+    for a, b in zip(one[0], many[0]):
+        np.testing.assert_array_equal(a, b)
+    assert one[1].keys() == many[1].keys()
+    for k in one[1]:
+        np.testing.assert_array_equal(one[1][k], many[1][k])
+
+
 # ------------------------------------------------------- planted mistakes --
 def _pin_complex_err(lib):
     """max |oracle - native complex SSM| on time-varying inputs (Prop. 2 reading)."""
