@@ -377,6 +377,25 @@ def run_prefill(cx, line):
     ms_per_step = total_ms / args.steps
     tokens = s.batch * s.seqlen
     value = throughput(cx.world, tokens, args.steps, total_ms)
+    unflushed = None
+    if flush is not None:
+        # the same launches back to back, inputs left in L2: reported beside
+        # the flushed figure, never as the value
+        cx.barrier()
+        torch.cuda.synchronize()
+        u0 = torch.cuda.Event(enable_timing=True)
+        u1 = torch.cuda.Event(enable_timing=True)
+        u0.record(stream)
+        for _ in range(args.steps):
+            step()
+        u1.record(stream)
+        torch.cuda.synchronize()
+        cx.barrier()
+        assert m3.m3_device_status(ws) == m3.M3_OK
+        u_ms = cx.max_over_ranks(u0.elapsed_time(u1))
+        unflushed = {"ms_per_step": u_ms / args.steps,
+                     "tokens_per_s": throughput(cx.world, tokens, args.steps, u_ms),
+                     "l2": "not flushed: inputs stay in L2 between launches"}
 
     aflops = algorithmic_flops(s)
     achieved_gbs = abytes / (per_launch_ms / 1e3) / 1e9
@@ -402,6 +421,8 @@ def run_prefill(cx, line):
                      "tensor_tflops": tflops, "tensor_frac_of_bf16_peak": tflops / pk["bf16"]},
         "clocks": clk.summary(),
         "gpu_launches": plan["launches"] * args.steps})
+    if unflushed is not None:
+        line["unflushed"] = unflushed
     return dict(s=s, host=host, dev=dev, y=y, fin=fin, step=step, tokens=tokens)
 
 
