@@ -182,3 +182,20 @@ def test_phase_rejects_before_launching():
     n = m3.m3_scan_phase_workspace_size(d, m3.M3_PHASE_READ_ONLY)
     assert n > m3.m3_scan_workspace_size(d)
     assert _phase_status(d, m3.M3_PHASE_READ_ONLY, ws_bytes=n - 1) == m3.M3_ERR_WORKSPACE
+
+
+def test_empty_problems_return_ok_before_touching_anything():
+    """batch = 0 (and L = 0 for the per-sequence calls) is a valid call with
+    nothing to do: it returns M3_OK with null data pointers and enqueues no
+    kernel; the plan reports zero launches."""
+    e = dims(batch=0)
+    assert scan_status(e, ptr=0, y=0) == m3.M3_OK
+    assert m3.m3_scan_plan(e)["launches"] == 0
+    assert m3.m3_scan_plan(dims(seqlen=0))["launches"] == 0
+    d = e.c()
+    assert LIB.m3_step(ctypes.byref(d), ctypes.byref(m3._Carry(None, None, None)), *([None] * 8),
+                       None) == m3.M3_OK
+    for empty in (e, dims(seqlen=0)):
+        d = empty.c()
+        assert LIB.m3_rope_bc(ctypes.byref(d), None, None, None, None, None, None, None,
+                              None) == m3.M3_OK
