@@ -53,6 +53,10 @@
  * wait on on-chip barriers bound every wait; on expiry they record
  * M3_ERR_DEVICE_TIMEOUT in the workspace's status word and return early,
  * which m3_device_status reports.  No C++ exception crosses this boundary.
+ * Buffer extents cannot be checked through plain pointers: every buffer must
+ * hold at least the elements its layout gives for `dims` (nothing is read
+ * from a buffer whose extent for `dims` is zero); a smaller buffer is read or
+ * written out of bounds.
  */
 #ifndef M3_H_
 #define M3_H_
