@@ -95,3 +95,16 @@ def test_bench_defaults_are_one_gpu_and_minutes_of_work(monkeypatch):
     assert a.gpus == 1 and a.warmup >= 3 and 1 <= a.steps <= 200
     assert a.impl == "ours" and a.layer == bench.LAYER and a.decode_steps == 1000
     assert not a.bwd and not a.phase          # the optional measurements stay off by default
+
+
+def test_reference_arm_prints_on_rank_0_only():
+    """Under torchrun the oracle arm runs on rank 0 alone; another rank exits 0
+    at once, prints nothing and joins no process group."""
+    import subprocess
+    env = {**os.environ, "RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1",
+           "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(_free_port())}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "3"], env=env, cwd=ROOT, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""
