@@ -181,7 +181,8 @@ def run_reference(args, rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": m3_synth.NAMES[LAYER], "global_batch": s.batch, "seq_len": s.seqlen,
                        "sample": "batch row 0 of 8, all 32 heads, full L=4096 per step"},
-            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "host_cpus": os.cpu_count(),
+                             "kind": "oracle",
                              "sample": "1 of 8 batch rows (32 heads x 4096 tokens) per step"},
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
@@ -202,7 +203,7 @@ def cpu_baseline_sample():
     oracle.scan(**f)
     dt = time.perf_counter() - t0
     out = {"value": sub.batch * sub.seqlen / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
-           "kind": "oracle",
+           "host_cpus": os.cpu_count(), "kind": "oracle",
            "sample": f"2 of 8 batch rows (64 head-sequences x 4096 tokens), {dt:.1f} s wall"}
     out["single_thread"] = oracle_single_thread()
     return out
