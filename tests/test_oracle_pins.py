@@ -383,6 +383,25 @@ def test_mimo_is_sum_of_siso_runs():
     np.testing.assert_allclose(hL, hsum, rtol=1e-11, atol=1e-11)
 
 
+def test_output_is_linear_in_x_and_the_carry():
+    """y and the final state are linear in (x, h_-1, x_-1) jointly, with B, C
+    and the coefficients fixed [M3 s1]: nothing in the recurrence adds a term
+    that does not carry exactly one factor of the state or of x."""
+    I = rand_inputs(15, b=2, L=23, H=2, G=1, P=3, N=6, R=2)
+    rng = np.random.default_rng(150)
+    x2 = rng.standard_normal(I["x"].shape)
+    h1, h2 = rng.standard_normal((2, 2, 2, 6, 3))
+    pB = rng.standard_normal((2, 2, 2, 6))
+    p1, p2 = rng.standard_normal((2, 2, 2, 2, 3))
+    rest = {k: v for k, v in I.items() if k != "x"}
+    ya, ha, _, _ = oracle.scan(x=I["x"], **rest, init_h=h1, init_pB=pB, init_pX=p1)
+    yb, hb, _, _ = oracle.scan(x=x2, **rest, init_h=h2, init_pB=pB, init_pX=p2)
+    yc, hc, _, _ = oracle.scan(x=I["x"] - 2.5 * x2, **rest, init_h=h1 - 2.5 * h2, init_pB=pB,
+                               init_pX=p1 - 2.5 * p2)
+    np.testing.assert_allclose(yc, ya - 2.5 * yb, rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(hc, ha - 2.5 * hb, rtol=1e-11, atol=1e-11)
+
+
 def test_rank1_equals_siso_shape():
     I = rand_inputs(9, b=1, L=20, H=1, G=1, P=4, N=4, R=1)
     y, hL, _, _ = oracle.scan(**I)
