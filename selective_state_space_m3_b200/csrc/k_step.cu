@@ -435,17 +435,6 @@ static cudaError_t launch_T(const StepParams& q, int R, int npt, int threads, si
 
 constexpr int kPipeStages = 3;
 
-static int sm_count_step() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0, v = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
-        n = v;
-    }
-    return n;
-}
-
 template <typename T, int R>
 static cudaError_t launch_pipe_R(const m3_dims& d, const StepParams& q, cudaStream_t st) {
     constexpr int N = 128, P = 64;
@@ -460,7 +449,7 @@ static cudaError_t launch_pipe_R(const m3_dims& d, const StepParams& q, cudaStre
     int per_sm = 0;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
     if (per_sm < 1) per_sm = 1;
-    int grid = sm_count_step() * per_sm;
+    int grid = device_sm_count() * per_sm;
     if (grid > units) grid = units;
     kern<<<grid, 256, smem, st>>>(q, units);
     return cudaGetLastError();

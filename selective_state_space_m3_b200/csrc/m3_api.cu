@@ -4,6 +4,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <vector>
 
 #include "m3_common.cuh"
@@ -60,18 +61,19 @@ static bool env_is(const char* name, const char* val) {
     return v && strcmp(v, val) == 0;
 }
 
-// SM count of the current device (a cached device attribute; 148 on B200
-// and when no device can be queried)
-static int sm_count() {
-    static int cached[64] = {0};
+// SM count of the current device: a device attribute cached per device
+// (atomics: calls may come from several host threads); 148, the B200's
+// count, when no device can be queried
+int device_sm_count() {
+    static std::atomic<int> cached[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (cached[dev] == 0) {
-        int n = 0;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cached[dev] = n;
+        cached[dev].store(n, std::memory_order_relaxed);
     }
-    return cached[dev];
+    return n;
 }
 
 // Path and chunking.  tcgen05 path: a chunk is one 128-row UMMA tile
@@ -95,7 +97,7 @@ static m3_status make_plan(const m3_dims& d, Plan* pl) {
     }
     const long long nchunks = d.seqlen > 0 ? (d.seqlen + qs - 1) / qs : 0;
     const long long units = (long long)d.batch * d.nheads;
-    const long long sms = sm_count();
+    const long long sms = device_sm_count();
     int nseg = 1;
     if (units > 0 && units < sms && nchunks >= 4) {
         long long want = (2 * sms) / units;

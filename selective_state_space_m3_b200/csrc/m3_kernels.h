@@ -102,6 +102,9 @@ cudaError_t launch_theta_transform(int mode, const float* in, const int* perm, c
 cudaError_t launch_expand_heads(const void* src, void* dst, size_t bt_count, int H, int G, size_t row_bytes,
                                 cudaStream_t st);
 
+// SM count of the current device, cached per device (148 if it cannot be queried)
+int device_sm_count();
+
 m3_status launch_step(const m3_dims& d, const StepParams& q, cudaStream_t st);
 m3_status launch_rope(const m3_dims& d, const RopeParams& q, cudaStream_t st);
 size_t simt_smem_bytes(int qs, int R, int N, int P, bool summary);
