@@ -108,3 +108,27 @@ def test_reference_arm_prints_on_rank_0_only():
                        timeout=300)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_prefill_roofline_arithmetic():
+    """The algorithmic bytes and FLOPs of the R=4 layer prefill, from tensor
+    shapes alone (meta tensors): 3336 B per token-head (x 512, y 512, B and C
+    2048, theta 256, dt and lambda 8) plus A and the final carry once, and
+    (Q+1) R^2 (N+P) + 4 R N P = 330,752 FLOP per token-head at Q = 64."""
+    import torch
+    import m3_synth
+    s = m3_synth.MIMO_R4_LAYER
+    b, L, H, G, R, P, N = s.batch, s.seqlen, s.nheads, s.ngroups, s.rank, s.headdim, s.dstate
+
+    def m(*shape, dtype=torch.float32):
+        return torch.empty(*shape, dtype=dtype, device="meta")
+
+    bf = torch.bfloat16
+    t = {"x": m(b, L, H, R, P, dtype=bf), "B": m(b, L, G, R, N, dtype=bf), "C": m(b, L, G, R, N, dtype=bf),
+         "dt": m(b, L, H), "A": m(H), "lam": m(b, L, H), "theta": m(b, L, G, N // 2)}
+    fin = types.SimpleNamespace(h=m(b, H, N, P), prev_B=m(b, H, R, N, dtype=bf), prev_x=m(b, H, R, P, dtype=bf))
+    token_heads = b * L * H
+    carry = b * H * (N * P * 4 + R * N * 2 + R * P * 2)
+    got = bench.algorithmic_bytes(t, m(b, L, H, R, P, dtype=bf), fin)
+    assert got == 3336 * token_heads + 4 * H + carry == 3_506_831_488
+    assert bench.algorithmic_flops(s) == 330_752 * token_heads
