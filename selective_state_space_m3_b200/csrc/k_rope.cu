@@ -161,8 +161,6 @@ __global__ void __launch_bounds__(256) rope_block_kernel(RopeParams q) {
     const T* __restrict__ Cin = static_cast<const T*>(q.C);
     T* __restrict__ Bo = static_cast<T*>(q.B_rot);
     T* __restrict__ Co = static_cast<T*>(q.C_rot);
-    // a null output (internal callers only) skips that side entirely
-    const bool doB = Bo != nullptr, doC = Co != nullptr;
     // theta and dt of a block: 4 theta values and (first 64 threads) one dt per
     // thread, loaded one block ahead into registers (clamped addresses, masked
     // when stored to shared memory)
@@ -223,8 +221,8 @@ __global__ void __launch_bounds__(256) rope_block_kernel(RopeParams q) {
                 const int e = min(e0 + tid + 256 * u, items - 1);
                 const int v = e % NV, kr = e / NV, r = kr % R, k = kr / R;
                 const size_t src = ((((size_t)b * L + t0 + k) * G + g) * R + r) * N + 2 * (i0 + v * VP);
-                vb[u] = doB ? *reinterpret_cast<const uint4*>(Bin + src) : make_uint4(0u, 0u, 0u, 0u);
-                vc[u] = doC ? *reinterpret_cast<const uint4*>(Cin + src) : make_uint4(0u, 0u, 0u, 0u);
+                vb[u] = *reinterpret_cast<const uint4*>(Bin + src);
+                vc[u] = *reinterpret_cast<const uint4*>(Cin + src);
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -244,8 +242,8 @@ __global__ void __launch_bounds__(256) rope_block_kernel(RopeParams q) {
                     fc[2 * j] = cs.x * c0 + cs.y * c1;
                     fc[2 * j + 1] = cs.x * c1 - cs.y * c0;
                 }
-                if (doB) *reinterpret_cast<uint4*>(Bo + dst) = Vec16<T>::pack(fb);
-                if (doC) *reinterpret_cast<uint4*>(Co + dst) = Vec16<T>::pack(fc);
+                *reinterpret_cast<uint4*>(Bo + dst) = Vec16<T>::pack(fb);
+                *reinterpret_cast<uint4*>(Co + dst) = Vec16<T>::pack(fc);
             }
         }
         __syncthreads();                                 // before the next block overwrites sTh / sCS

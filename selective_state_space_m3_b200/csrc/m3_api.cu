@@ -419,15 +419,7 @@ m3_status m3_scan_fwd_phase(const m3_dims* d, int mode, const int* perm, const f
         void* crot = base + l.crot;
         float* th0 = reinterpret_cast<float*>(base + l.theta);
         if (work) {
-            // only the rotated side is produced (a null output skips the other)
-            RopeParams rq;
-            rq.batch = d->batch; rq.seqlen = d->seqlen; rq.nheads = d->nheads; rq.ngroups = d->ngroups;
-            rq.dstate = d->dstate; rq.rank = d->rank;
-            rq.B = B; rq.C = C; rq.dt = dt; rq.theta = theta; rq.phase = nullptr;
-            rq.B_rot = mode == M3_PHASE_WRITE_ONLY ? brot : nullptr;
-            rq.C_rot = mode == M3_PHASE_READ_ONLY ? crot : nullptr;
-            s = (d->dstate / 2) % 16 == 0 ? launch_rope(*d, rq, st)
-                                          : m3_rope_bc(d, B, C, dt, theta, brot, crot, nullptr, stream);
+            s = m3_rope_bc(d, B, C, dt, theta, brot, crot, nullptr, stream);
             if (s != M3_OK) return s;
             if (cudaMemsetAsync(th0, 0, tok * d->nheads * NH * sizeof(float), st) != cudaSuccess) return M3_ERR_CUDA;
         }
