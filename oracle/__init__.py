@@ -16,6 +16,10 @@ Passages followed (page titles and sections):
     (block-diagonal R(dt theta[i]) rotations, y = C^T h) and Proposition 3
     (the rotation moved onto B and C as a cumulative phase, oracle_rope_bc).
   * same page, section 3 "MIMO": B, C in R^{N x R}, x in R^{P x R}.
+  * "Understanding Mamba-3 Through Oscillatory Dynamics", sections 2.2, 4.1,
+    4.2 and appendix C.2: the damping-regime variants (scan_damped).
+  * the low-rank reflection extension's abstract (listed on the same paper's
+    page) and appendix C.4 of that paper: scan_reflect.
 """
 from __future__ import annotations
 
@@ -61,6 +65,10 @@ def _bind(lib):
     lib.oracle_scan_bwd.restype = ctypes.c_int
     lib.oracle_rope_bc.argtypes = [D] + [P] * 7
     lib.oracle_rope_bc.restype = ctypes.c_int
+    lib.oracle_scan_damped.argtypes = [D, ctypes.c_int] + [P] * 14
+    lib.oracle_scan_damped.restype = ctypes.c_int
+    lib.oracle_scan_reflect.argtypes = [D] + [P] * 15
+    lib.oracle_scan_reflect.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
@@ -79,15 +87,18 @@ def _load():
 def compile_variant(source_text: str, tag: str):
     """Compile a modified copy of the oracle source (tests plant mistakes in
     it to show that the pins catch them) and return a ctypes handle usable as
-    the ``lib=`` argument of scan/step/rope_bc."""
-    os.makedirs(_BUILD, exist_ok=True)
-    src = os.path.join(_BUILD, f"variant_{tag}_{os.getpid()}.c")
-    so = src[:-2] + ".so"
-    with open(src, "w") as f:
-        f.write(source_text)
-    subprocess.run(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-std=c99",
-                    "-o", so, src, "-lm"], check=True)
-    return _bind(ctypes.CDLL(so))
+    the ``lib=`` argument of scan/step/rope_bc.  The copy is built in a
+    temporary directory that is removed once the library is loaded (the
+    loaded image stays valid after its file is unlinked)."""
+    import tempfile
+    with tempfile.TemporaryDirectory(prefix=f"m3oracle_{tag}_") as tmp:
+        src = os.path.join(tmp, "variant.c")
+        so = os.path.join(tmp, "variant.so")
+        with open(src, "w") as f:
+            f.write(source_text)
+        subprocess.run(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-std=c99",
+                        "-o", so, src, "-lm"], check=True)
+        return _bind(ctypes.CDLL(so))
 
 
 def source_text() -> str:
@@ -163,6 +174,48 @@ def scan_bwd(x, B, C, dt, A, lam, theta, dy, init_h=None, init_pB=None, init_pX=
     if rc != 0:
         raise ValueError("oracle_scan_bwd rejected its arguments")
     return out
+
+
+DAMPING_REGIMES = ("under", "critical", "over")
+
+
+def _scan_variant(fn, lead, x, B, C, dt, A, lam, theta, init_h, init_pB, init_pX):
+    x, B, C, dt, A, lam, theta = map(_f64, (x, B, C, dt, A, lam, theta))
+    init_h, init_pB, init_pX = map(_f64, (init_h, init_pB, init_pX))
+    b, L, H, R, P = x.shape
+    G, N = B.shape[2], B.shape[4]
+    d = _Dims(b, L, H, G, P, N, R)
+    y = np.zeros((b, L, H, R, P))
+    hL = np.zeros((b, H, N, P))
+    pB = np.zeros((b, H, R, N))
+    pX = np.zeros((b, H, R, P))
+    rc = fn(ctypes.byref(d), *lead, _p(x), _p(B), _p(C), _p(dt), _p(A), _p(lam), _p(theta),
+            _p(init_h), _p(init_pB), _p(init_pX), _p(y), _p(hL), _p(pB), _p(pX))
+    if rc != 0:
+        raise ValueError(f"{fn.__name__} rejected its arguments")
+    return y, hL, pB, pX
+
+
+def scan_damped(regime, x, B, C, dt, A, lam, theta, init_h=None, init_pB=None, init_pX=None, lib=None):
+    """Damping-regime variant ("Understanding Mamba-3 Through Oscillatory
+    Dynamics", sections 2.2, 4.1, 4.2, appendix C.2): rotary pair i of token t
+    evolves under dt (A I + theta[i] K_s), K_s = [[0, -1], [s, 0]], with
+    s = +1 (under, Mamba-3), 0 (critical), -1 (over); inputs, layouts and
+    returns as scan().  ``regime`` is a DAMPING_REGIMES name or 0/1/2."""
+    rg = DAMPING_REGIMES.index(regime) if isinstance(regime, str) else int(regime)
+    lb = lib or _load()
+    return _scan_variant(lb.oracle_scan_damped, (ctypes.c_int(rg),), x, B, C, dt, A, lam, theta,
+                         init_h, init_pB, init_pX)
+
+
+def scan_reflect(u, x, B, C, dt, A, lam, theta, init_h=None, init_pB=None, init_pX=None, lib=None):
+    """Low-rank reflection extension: Mamba-3's transition with the diagonal
+    alpha_t I replaced by alpha_t (I - 2 u u^T / u^T u), u [b,t,g,n] an
+    input-dependent direction (u = 0: no reflection); otherwise as scan()."""
+    u = _f64(u)
+    lb = lib or _load()
+    return _scan_variant(lb.oracle_scan_reflect, (_p(u),), x, B, C, dt, A, lam, theta,
+                         init_h, init_pB, init_pX)
 
 
 PHASE_MODES = ("native", "zero", "reverse", "shuffle", "fixed", "write_only", "read_only")

@@ -29,6 +29,13 @@
  *   which Proposition 3 (data-dependent RoPE on B and C) holds with every B_s
  *   rotated by its own cumulative phase.
  *
+ * Two transition variants follow the main scan further down:
+ * oracle_scan_damped (damping regimes: the rotation block of every pair
+ * replaced by the critically damped shear or the overdamped hyperbolic
+ * block, same input rule) and oracle_scan_reflect (a rank-one Householder
+ * reflection added to the diagonal part of the transition).  Their readings
+ * are stated above each.
+ *
  * Layouts (row-major, innermost last):
  *   x      [b][t][h][r][p]        y      [b][t][h][r][p]
  *   B, C   [b][t][g][r][n]        theta  [b][t][g][N/2]
@@ -452,6 +459,180 @@ int oracle_scan_bwd(const oracle_dims* d,
     }
     free(dBh); free(dCh); free(dTh); free(dAh);
     return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Damping-regime variants ("Understanding Mamba-3 Through Oscillatory
+ * Dynamics", section 2.2 and Table 1 (the three regimes of a damped
+ * second-order system), section 4.1 (variants with the same coupled 2-D
+ * state, input-update rule and state dimension, the damping parameter
+ * selecting the regime around a shared spectral centre), section 4.2 and
+ * appendix C.2 (mode persistence)).
+ *
+ * Reading: rotary pair i of token t evolves, over its interval, under the
+ * generator dt_t (A_h I + theta_t[i] K_s) with K_s = [[0, -1], [s, 0]]:
+ *   s = +1  underdamped  (eigenvalues A +- i theta: Mamba-3's decay-rotation),
+ *   s =  0  critically damped (double eigenvalue A, one eigenvector),
+ *   s = -1  overdamped   (real eigenvalues A +- theta),
+ * so the centre A of the eigenvalue pair is the same in every regime.  Since
+ * K_s^2 = -s I, exp(phi K_s) = c(phi) I + sn(phi) K_s with
+ *   (c, sn) = (cos, sin) for s = +1, (1, phi) for s = 0, (cosh, sinh) for
+ *   s = -1,
+ * i.e. the 2x2 block T = [[c, -sn], [s sn, c]], phi = dt_t theta_t[i].  The
+ * input-update rule is Mamba-3's exponential-trapezoidal one with T_t in
+ * place of R_t:
+ *   h_t = T_t (alpha_t h_{t-1} + beta_t B_{t-1} X_{t-1}^T) + gamma_t B_t X_t^T,
+ *   y_t = C_t^T h_t.
+ * regime: 0 = underdamped, 1 = critically damped, 2 = overdamped.
+ * Written on its own (not through step_bh), so that the underdamped regime
+ * checks the general 2x2 block against step_bh's rotation.
+ * ---------------------------------------------------------------------- */
+static void pair_block(int regime, double phi, double* c, double* sn, double* sg)
+{
+    if (regime == 0) { *c = cos(phi); *sn = sin(phi); *sg = 1.0; }
+    else if (regime == 1) { *c = 1.0; *sn = phi; *sg = 0.0; }
+    else { *c = cosh(phi); *sn = sinh(phi); *sg = -1.0; }
+}
+
+/* One token of either variant for one (b, h).  regime selects the pair block
+ * (damped variants); u (length N, may be NULL) is the reflection direction
+ * of the reflection variant, which then uses the underdamped block. */
+static void step_bh_general(int N, int P, int R, int regime, const double* u,
+                            double* H, double* PB, double* PX,
+                            const double* xt, const double* Bt, const double* Ct,
+                            double d, double a, double lam, const double* th,
+                            double* yt)
+{
+    const double alpha = exp(d * a);
+    const double beta = (1.0 - lam) * d * alpha;
+    const double gamma = lam * d;
+
+    /* v = alpha h + beta B_{t-1} X_{t-1}^T */
+    for (int n = 0; n < N; ++n)
+        for (int p = 0; p < P; ++p) {
+            double pend = 0.0;
+            for (int r = 0; r < R; ++r) pend += PX[r * P + p] * PB[r * N + n];
+            H[n * P + p] = alpha * H[n * P + p] + beta * pend;
+        }
+
+    /* reflection v <- (I - 2 u u^T / u^T u) v, column by column (u = 0: none) */
+    if (u) {
+        double uu = 0.0;
+        for (int n = 0; n < N; ++n) uu += u[n] * u[n];
+        if (uu > 0.0) {
+            for (int p = 0; p < P; ++p) {
+                double dot = 0.0;
+                for (int n = 0; n < N; ++n) dot += u[n] * H[n * P + p];
+                const double f = 2.0 * dot / uu;
+                for (int n = 0; n < N; ++n) H[n * P + p] -= f * u[n];
+            }
+        }
+    }
+
+    /* pair blocks T (regime) on rows (2i, 2i+1) */
+    for (int i = 0; i < N / 2; ++i) {
+        double c, sn, sg;
+        pair_block(regime, d * th[i], &c, &sn, &sg);
+        for (int p = 0; p < P; ++p) {
+            const double u0 = H[(2 * i) * P + p];
+            const double u1 = H[(2 * i + 1) * P + p];
+            H[(2 * i) * P + p] = c * u0 - sn * u1;
+            H[(2 * i + 1) * P + p] = sg * sn * u0 + c * u1;
+        }
+    }
+
+    /* + gamma B_t X_t^T */
+    for (int n = 0; n < N; ++n)
+        for (int p = 0; p < P; ++p) {
+            double cur = 0.0;
+            for (int r = 0; r < R; ++r) cur += xt[r * P + p] * Bt[r * N + n];
+            H[n * P + p] += gamma * cur;
+        }
+
+    for (int r = 0; r < R; ++r)
+        for (int p = 0; p < P; ++p) {
+            double out = 0.0;
+            for (int n = 0; n < N; ++n) out += H[n * P + p] * Ct[r * N + n];
+            yt[r * P + p] = out;
+        }
+
+    memcpy(PB, Bt, (size_t)R * N * sizeof(double));
+    memcpy(PX, xt, (size_t)R * P * sizeof(double));
+}
+
+static int scan_general(const oracle_dims* d, int regime, const double* u,
+                        const double* x, const double* B, const double* C,
+                        const double* dt, const double* A, const double* lam,
+                        const double* theta,
+                        const double* init_h, const double* init_pB, const double* init_pX,
+                        double* y, double* out_h, double* out_pB, double* out_pX)
+{
+    if (!dims_ok(d) || !x || !B || !C || !dt || !A || !lam || !theta || !y) return -1;
+    if (regime < 0 || regime > 2) return -1;
+    const int Bn = d->batch, L = d->seqlen, H = d->nheads, G = d->ngroups;
+    const int P = d->headdim, N = d->dstate, R = d->rank;
+    const int hpg = H / G;
+
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < Bn; ++b)
+        for (int h = 0; h < H; ++h) {
+            const int g = h / hpg;
+            double* Hs = (double*)calloc((size_t)N * P, sizeof(double));
+            double* PB = (double*)calloc((size_t)R * N, sizeof(double));
+            double* PX = (double*)calloc((size_t)R * P, sizeof(double));
+            const size_t bh = (size_t)b * H + h;
+            if (init_h) memcpy(Hs, init_h + bh * N * P, sizeof(double) * (size_t)N * P);
+            if (init_pB) memcpy(PB, init_pB + bh * R * N, sizeof(double) * (size_t)R * N);
+            if (init_pX) memcpy(PX, init_pX + bh * R * P, sizeof(double) * (size_t)R * P);
+            for (int t = 0; t < L; ++t) {
+                const size_t bt = (size_t)b * L + t;
+                step_bh_general(N, P, R, regime, u ? u + (bt * G + g) * N : NULL, Hs, PB, PX,
+                                x + ((bt * H + h) * R) * P, B + ((bt * G + g) * R) * N,
+                                C + ((bt * G + g) * R) * N, dt[bt * H + h], A[h], lam[bt * H + h],
+                                theta + (bt * G + g) * (N / 2), y + ((bt * H + h) * R) * P);
+            }
+            if (out_h) memcpy(out_h + bh * N * P, Hs, sizeof(double) * (size_t)N * P);
+            if (out_pB) memcpy(out_pB + bh * R * N, PB, sizeof(double) * (size_t)R * N);
+            if (out_pX) memcpy(out_pX + bh * R * P, PX, sizeof(double) * (size_t)R * P);
+            free(Hs); free(PB); free(PX);
+        }
+    return 0;
+}
+
+/* Damping-regime variant of oracle_scan (regime 0, 1, 2 as above); same
+ * arguments and layouts otherwise. */
+int oracle_scan_damped(const oracle_dims* d, int regime,
+                       const double* x, const double* B, const double* C,
+                       const double* dt, const double* A, const double* lam,
+                       const double* theta,
+                       const double* init_h, const double* init_pB, const double* init_pX,
+                       double* y, double* out_h, double* out_pB, double* out_pX)
+{
+    return scan_general(d, regime, NULL, x, B, C, dt, A, lam, theta, init_h, init_pB, init_pX,
+                        y, out_h, out_pB, out_pX);
+}
+
+/* Low-rank reflection extension (abstract of the extension of Mamba-3's
+ * diagonal transition with an input-dependent rank-one reflection term,
+ * listed on "Understanding Mamba-3 Through Oscillatory Dynamics"; two
+ * reflections compose to a rotation, appendix C.4 of that paper).
+ * Reading: the diagonal part alpha_t I of the transition becomes
+ * alpha_t (I - 2 u_t u_t^T / u_t^T u_t), a Householder reflection along the
+ * input-dependent direction u_t (per token and group, like B), and the
+ * exponential-trapezoidal rule, the rotation R_t and the readout stay:
+ *   h_t = R_t H_t (alpha_t h_{t-1} + beta_t B_{t-1} X_{t-1}^T) + gamma_t B_t X_t^T,
+ *   H_t = I - 2 u_t u_t^T / (u_t^T u_t)   (H_t = I where u_t = 0).
+ * u: [b][t][g][N]. */
+int oracle_scan_reflect(const oracle_dims* d, const double* u,
+                        const double* x, const double* B, const double* C,
+                        const double* dt, const double* A, const double* lam,
+                        const double* theta,
+                        const double* init_h, const double* init_pB, const double* init_pX,
+                        double* y, double* out_h, double* out_pB, double* out_pX)
+{
+    if (!u) return -1;
+    return scan_general(d, 0, u, x, B, C, dt, A, lam, theta, init_h, init_pB, init_pX,
+                        y, out_h, out_pB, out_pX);
 }
 
 int oracle_num_threads(void)
