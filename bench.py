@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-rope", action="store_true", help="skip the m3_rope_bc measurement")
     ap.add_argument("--bwd", action="store_true", help="also time the backward pass m3_scan_bwd")
     ap.add_argument("--phase", action="store_true", help="also time two phase interventions")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the damping-regime and reflection variants")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the layer's batch (profiling captures of a smaller case)")
     ap.add_argument("--workload", choices=["both", "prefill", "decode"], default="both",
@@ -605,6 +607,83 @@ def run_phase(cx, line, pf):
     line["phase"] = out
 
 
+def fp32_peak_tflops(sm_max_mhz) -> float:
+    """FP32 FMA roofline of the CUDA cores: 148 SMs x 128 FP32 lanes x 2 FLOP
+    per FMA x the maximum SM clock (1965 MHz on this machine's B200s)."""
+    return 148 * 128 * 2 * float(sm_max_mhz or 1965) * 1e6 / 1e12
+
+
+def variant_flops(s, reflect: bool) -> float:
+    """Algorithmic FLOPs of the token-by-token recurrence per call: per state
+    element and token, the pending beta term (2R + 1), the 2x2 pair block (3),
+    the input term (2R + 1) and the readout (2R); the reflection adds its
+    projection and update (4)."""
+    per = 6 * s.rank + 5 + (4 if reflect else 0)
+    return float(per) * s.dstate * s.headdim * s.batch * s.seqlen * s.nheads
+
+
+def run_variants(cx, line):
+    """The transition variants on the SISO layer workload (batch 4, 8 heads,
+    L = 2048, bf16): the critically damped and overdamped regimes
+    (m3_scan_fwd_damped) and the low-rank reflection (m3_scan_fwd_reflect),
+    token by token in float32 on the CUDA cores (roofline: FP32 FMA rate).
+    The 25 MB of inputs are evicted from L2 before every timed launch."""
+    import torch
+    import m3_synth
+    import selective_state_space_m3_b200 as m3
+    args, pk, stream = cx.args, cx.pk, cx.stream
+    s = m3_synth.shrink(m3_synth.SISO_LAYER, seed=m3_synth.SISO_LAYER.seed + 1000 * cx.rank)
+    host = m3_synth.make_scan_inputs(s)
+    dev = {k: v.cuda() for k, v in host.items()}
+    theta_over = m3_synth.overdamped_theta(host, s).cuda()
+    u = m3_synth.make_reflect_direction(s).cuda()
+    d = m3.Dims(s.batch, s.seqlen, s.nheads, s.ngroups, s.headdim, s.dstate, s.rank, s.chunk, m3.M3_BF16)
+    y = torch.empty_like(dev["x"])
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    nbytes = sum(v.numel() * v.element_size() for v in dev.values()) + y.numel() * y.element_size()
+    out = {}
+    calls = {
+        "critical": lambda: m3.m3_scan_fwd_damped(d, m3.M3_DAMP_CRITICAL, dev["x"], dev["B"], dev["C"], dev["dt"],
+                                                  dev["A"], dev["lam"], dev["theta"], y, stream=stream),
+        "over": lambda: m3.m3_scan_fwd_damped(d, m3.M3_DAMP_OVER, dev["x"], dev["B"], dev["C"], dev["dt"],
+                                              dev["A"], dev["lam"], theta_over, y, stream=stream),
+        "reflect": lambda: m3.m3_scan_fwd_reflect(d, u, dev["x"], dev["B"], dev["C"], dev["dt"], dev["A"],
+                                                  dev["lam"], dev["theta"], y, stream=stream),
+    }
+    with ClockSampler(cx.local) as clk:
+        for name, call in calls.items():
+            for _ in range(3):
+                call()
+            torch.cuda.synchronize()
+            n = 10
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+            cx.barrier()
+            clk.active = True
+            for e0, e1 in ev:
+                flush.zero_()
+                e0.record(stream)
+                call()
+                e1.record(stream)
+            torch.cuda.synchronize()
+            clk.active = False
+            cx.barrier()
+            ms = cx.max_over_ranks(statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev))
+            fl = variant_flops(s, name == "reflect")
+            peak = fp32_peak_tflops(clk.max_mhz if clk.ok else None)
+            tf = fl / (ms / 1e3) / 1e12
+            out[name] = {"ms_per_call": ms, "tokens_per_s": cx.world * s.batch * s.seqlen / (ms / 1e3),
+                         "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                                      "frac": tf / peak, "algorithmic_flops_per_launch": fl,
+                                      "peak_source": "148 SMs x 128 FP32 lanes x 2 x max SM clock",
+                                      "hbm_frac": nbytes / (ms / 1e3) / 1e9 / pk["hbm"], "traffic": None},
+                         "gpu_launches": n}
+    out["workload"] = m3_synth.NAMES["siso_layer"]
+    out["l2"] = "L2 flushed (252 MB write) before every timed launch"
+    out["clocks"] = clk.summary()
+    line["variants"] = out
+    del flush
+
+
 def run_decode(cx, line, pf):
     """m3_step x decode_steps captured in one CUDA graph; the carry comes from
     the prefill's final state (tiled, sequence j <- batch row j mod 8), or
@@ -708,6 +787,8 @@ def main():
             run_phase(cx, line, pf)
     if args.workload in ("both", "decode") and not args.no_decode:
         run_decode(cx, line, pf)
+    if args.workload == "both" and not args.no_variants:
+        run_variants(cx, line)
     if cx.world == 1 and not args.no_cpu and args.workload != "decode" and args.layer == LAYER:
         line["cpu_baseline"] = cpu_baseline_sample()
     cx.close()

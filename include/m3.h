@@ -237,6 +237,58 @@ m3_status m3_scan_fwd_phase(const m3_dims* dims, int mode, const int* perm, cons
                             m3_carry* final_state, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/* Damping-regime variants ("Understanding Mamba-3 Through Oscillatory
+ * Dynamics", section 2.2 and Table 1, section 4.1, section 4.2, appendix
+ * C.2).  Rotary pair i of token t evolves over its interval under the
+ * generator dt_t (A_h I + theta_t[i] K_s), K_s = [[0, -1], [s, 0]], so the
+ * eigenvalue pair is centred on A_h in every regime:
+ *   M3_DAMP_UNDER     s = +1: block R(phi) (Mamba-3 itself),
+ *   M3_DAMP_CRITICAL  s =  0: block [[1, -phi], [0, 1]] (a shear),
+ *   M3_DAMP_OVER      s = -1: block [[cosh phi, -sinh phi], [-sinh phi, cosh phi]],
+ * phi = dt_t theta_t[i]; the exponential-trapezoidal input rule and the
+ * readout are unchanged:
+ *   h_t = T_t (alpha_t h_{t-1} + beta_t B_{t-1} X_{t-1}^T) + gamma_t B_t X_t^T,
+ *   y_t = C_t^T h_t.
+ * (This library's reading: the pages name the regimes and fix the shared
+ * centre, the state structure and the input rule, not the block itself.) */
+typedef enum m3_damping {
+    M3_DAMP_UNDER = 0,
+    M3_DAMP_CRITICAL = 1,
+    M3_DAMP_OVER = 2
+} m3_damping;
+
+/* The scan under a damping regime.  Arguments, layouts, carry and results as
+ * m3_scan_fwd (the carry's h is in the original frame), plus `regime` (an
+ * m3_damping); no workspace.  The recurrence runs token by token in float32
+ * (the chunked form of m3_scan_fwd needs the inverse of every prefix of
+ * transitions, which grows like e^{|Phi|} or |Phi| outside the underdamped
+ * regime).  Overdamped pairs grow like e^{dt (A + |theta|)}: inputs with
+ * |theta| > |A| leave the regime and make the state grow.  Supported shapes:
+ * rank 1, 2 or 4; dstate a multiple of 8 and at most 256; headdim a multiple
+ * of 16; others return M3_ERR_UNSUPPORTED.  dims->chunk is ignored. */
+m3_status m3_scan_fwd_damped(const m3_dims* dims, int regime,
+                             const void* x, const void* B, const void* C,
+                             const float* dt, const float* A, const float* lambda,
+                             const float* theta, const m3_carry* init,
+                             void* y, m3_carry* final_state, void* stream);
+
+/* Low-rank reflection extension (the extension's abstract listed on
+ * "Understanding Mamba-3 Through Oscillatory Dynamics": an input-dependent
+ * rank-one reflection added to Mamba-3's diagonal transition, keeping the
+ * exponential-trapezoidal rule, RoPE and the readout; appendix C.4 of that
+ * paper: two reflections compose to a rotation).  Reading:
+ *   h_t = R_t H_t (alpha_t h_{t-1} + beta_t B_{t-1} X_{t-1}^T) + gamma_t B_t X_t^T,
+ *   H_t = I - 2 u_t u_t^T / (u_t^T u_t),   H_t = I where u_t = 0,
+ * with u_t [batch][seqlen][ngroups][dstate] in the io dtype (per token and
+ * group, like B; only its direction matters; required, like the other
+ * inputs, whenever there are tokens).  Everything else as
+ * m3_scan_fwd_damped (token by token, float32, no workspace, same shapes). */
+m3_status m3_scan_fwd_reflect(const m3_dims* dims, const void* u,
+                              const void* x, const void* B, const void* C,
+                              const float* dt, const float* A, const float* lambda,
+                              const float* theta, const m3_carry* init,
+                              void* y, m3_carry* final_state, void* stream);
+
 /* How m3_scan_fwd will run `dims` (host-only, nothing launched): the number
  * of kernel launches one call makes, the segments each (batch, head)
  * sequence is cut into, the chunk length the kernels use, and the path

@@ -151,6 +151,30 @@ def make_carry(batch: int, nheads: int, dstate: int, headdim: int, rank: int,
     return {"h": torch.from_numpy(h), "prev_B": _store(pB, dtype), "prev_x": _store(pX, dtype)}
 
 
+def make_reflect_direction(s: ScanShape, zero_tokens=()) -> torch.Tensor:
+    """Reflection directions u [b][t][g][n] for the low-rank reflection
+    variant: N(0, 1) draws (generator seeded by (seed, 4099)), stored in the
+    io dtype; the tokens listed in ``zero_tokens`` get u = 0 (no reflection).
+    Only the direction of u matters to the method."""
+    rng = np.random.Generator(np.random.PCG64([s.seed, 4099]))
+    u = rng.standard_normal((s.batch, s.seqlen, s.ngroups, s.dstate), dtype=np.float32)
+    for t in zero_tokens:
+        if 0 <= t < s.seqlen:
+            u[:, t] = 0.0
+    return _store(u, s.dtype)
+
+
+def overdamped_theta(inp: dict, s: ScanShape, margin: float = 0.9) -> torch.Tensor:
+    """theta rescaled for the overdamped regime: theta ~ U(-pi, pi) mapped to
+    U(-margin m, margin m) with m the smallest |A| of the group's heads, so
+    that every pair keeps both eigenvalues A +- theta below zero (the regime's
+    stable range).  Returns a new float32 tensor."""
+    H, G = s.nheads, s.ngroups
+    A = inp["A"].to(torch.float64).abs().reshape(G, H // G).min(dim=1).values      # per group
+    th = inp["theta"].to(torch.float64) / math.pi * margin * A.reshape(1, 1, G, 1)
+    return th.to(torch.float32).contiguous()
+
+
 def shrink(s: ScanShape, **kw) -> ScanShape:
     """Same distributions and seed, other sizes (parity cases the oracle runs
     in seconds)."""

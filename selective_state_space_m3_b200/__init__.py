@@ -68,6 +68,10 @@ def _load():
     lib.m3_scan_phase_workspace_size.restype = I
     lib.m3_scan_fwd_phase.argtypes = [D, I, V, V, V, V, V, V, V, V, V, C, V, C, V, S, V]
     lib.m3_scan_fwd_phase.restype = I
+    lib.m3_scan_fwd_damped.argtypes = [D, I, V, V, V, V, V, V, V, C, V, C, V]
+    lib.m3_scan_fwd_damped.restype = I
+    lib.m3_scan_fwd_reflect.argtypes = [D, V, V, V, V, V, V, V, V, C, V, C, V]
+    lib.m3_scan_fwd_reflect.restype = I
     lib.m3_status_string.argtypes = [I]
     lib.m3_status_string.restype = ctypes.c_char_p
     for f in ("m3_scan_workspace_size", "m3_scan_fwd", "m3_step", "m3_rope_bc", "m3_device_status"):
@@ -81,7 +85,7 @@ _lib = _load()
 ABI_SYMBOLS = ("m3_scan_workspace_size", "m3_scan_fwd", "m3_step", "m3_rope_bc",
                "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_scan_fwd_static",
                "m3_scan_bwd_workspace_size", "m3_scan_bwd", "m3_scan_phase_workspace_size",
-               "m3_scan_fwd_phase", "m3_status_string")
+               "m3_scan_fwd_phase", "m3_scan_fwd_damped", "m3_scan_fwd_reflect", "m3_status_string")
 
 
 @dataclasses.dataclass
@@ -278,6 +282,35 @@ def m3_scan_fwd_phase(dims: Dims, mode: int, x, B, C, dt, A, lam, theta, y, work
     _check(st, "m3_scan_fwd_phase")
 
 
+M3_DAMP_UNDER, M3_DAMP_CRITICAL, M3_DAMP_OVER = range(3)
+
+
+def m3_scan_fwd_damped(dims: Dims, regime: int, x, B, C, dt, A, lam, theta, y,
+                       init: Optional[Carry] = None, final_state: Optional[Carry] = None, stream=None) -> None:
+    """The scan under a damping regime (M3_DAMP_UNDER / CRITICAL / OVER; see
+    include/m3.h).  No workspace."""
+    d = dims.c()
+    ci = init.c() if init is not None else None
+    cf = final_state.c() if final_state is not None else None
+    st = _lib.m3_scan_fwd_damped(ctypes.byref(d), int(regime), _ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A),
+                                 _ptr(lam), _ptr(theta), ctypes.byref(ci) if ci is not None else None, _ptr(y),
+                                 ctypes.byref(cf) if cf is not None else None, _stream(stream))
+    _check(st, "m3_scan_fwd_damped")
+
+
+def m3_scan_fwd_reflect(dims: Dims, u, x, B, C, dt, A, lam, theta, y,
+                        init: Optional[Carry] = None, final_state: Optional[Carry] = None, stream=None) -> None:
+    """The scan with the low-rank reflection term; ``u`` [b][t][g][n] in the
+    io dtype (see include/m3.h).  No workspace."""
+    d = dims.c()
+    ci = init.c() if init is not None else None
+    cf = final_state.c() if final_state is not None else None
+    st = _lib.m3_scan_fwd_reflect(ctypes.byref(d), _ptr(u), _ptr(x), _ptr(B), _ptr(C), _ptr(dt), _ptr(A),
+                                  _ptr(lam), _ptr(theta), ctypes.byref(ci) if ci is not None else None, _ptr(y),
+                                  ctypes.byref(cf) if cf is not None else None, _stream(stream))
+    _check(st, "m3_scan_fwd_reflect")
+
+
 def raw_lib():
     """The ctypes handle (for calls that pass raw pointers)."""
     return _lib
@@ -285,5 +318,6 @@ def raw_lib():
 
 __all__ = ["Dims", "Carry", "M3Error", "m3_scan_workspace_size", "m3_scan_fwd", "m3_step",
            "m3_rope_bc", "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_scan_fwd_static", "m3_scan_bwd_workspace_size", "m3_scan_bwd", "m3_status_string",
-           "m3_scan_phase_workspace_size", "m3_scan_fwd_phase", "io_dtype_of", "ABI_SYMBOLS",
+           "m3_scan_phase_workspace_size", "m3_scan_fwd_phase", "m3_scan_fwd_damped", "m3_scan_fwd_reflect",
+           "M3_DAMP_UNDER", "M3_DAMP_CRITICAL", "M3_DAMP_OVER", "io_dtype_of", "ABI_SYMBOLS",
            "M3_F32", "M3_BF16", "raw_lib", "LIB_PATH"]

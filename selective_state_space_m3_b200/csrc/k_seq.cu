@@ -1,0 +1,423 @@
+// k_seq.cu -- token-by-token scan kernels of the two transition variants of
+// the Mamba-3 layer: the damping regimes and the low-rank reflection.
+//
+// Damping regimes ("Understanding Mamba-3 Through Oscillatory Dynamics",
+// section 2.2 and Table 1, section 4.1, section 4.2 and appendix C.2): rotary
+// pair i of token t evolves over its interval under dt (A I + theta[i] K_s),
+// K_s = [[0, -1], [s, 0]]; its 2x2 block is [[c, -sn], [s sn, c]] with
+// (c, sn) = (cos phi, sin phi) for s = +1 (underdamped, Mamba-3 itself),
+// (1, phi) for s = 0 (critically damped), (cosh phi, sinh phi) for s = -1
+// (overdamped), phi = dt theta[i].  The input rule is Mamba-3's
+// exponential-trapezoidal one ("Mamba-3" summary, b-lab.team, section 1):
+//   h_t = T_t (alpha_t h_{t-1} + beta_t B_{t-1} X_{t-1}^T) + gamma_t B_t X_t^T,
+//   y_t = C_t^T h_t   (section 3, MIMO rank R).
+// Low-rank reflection (the extension's abstract listed on the same paper's
+// page; appendix C.4 for two reflections making a rotation): the diagonal
+// alpha_t I of the transition becomes alpha_t (I - 2 u u^T / u^T u), the
+// rotation R_t and the rest stay: h_t = R_t H_t (alpha h + beta B X^T) + ...
+//
+// Why token by token.  The chunked prefill moves the rotation onto B and C
+// as a cumulative phase (Proposition 3), which needs the inverse of every
+// prefix of transitions: for the overdamped block those grow like e^{|Phi|}
+// and for the critical shear like |Phi|, and the reflection is not diagonal
+// in any fixed basis, so neither has the chunked tensor-core form.  This
+// kernel runs the recurrence directly in float32.
+//
+// Mapping.  State columns p evolve independently (the transition acts on the
+// rows n).  A warp owns PC = 4 columns of one (batch, head) and every row:
+// lane l holds the rotary pairs i = l + 32 k (k < KP), i.e. rows 2i and 2i+1,
+// so a pair block never leaves its thread.  Readout and reflection sums over
+// n are warp shuffles; nothing crosses warps.  A CTA of 4 warps covers 16
+// columns and stages each token's B, C (and u), theta, dt, lambda and its 16
+// columns of x in shared memory with cp.async, a chunk of TK tokens ahead of
+// use (two buffers).
+#include "m3_common.cuh"
+#include "m3_kernels.h"
+
+namespace m3 {
+namespace seq {
+
+constexpr int kWarps = 4;
+constexpr int kPC = 4;                     // columns per warp
+constexpr int kCB = kWarps * kPC;          // columns per CTA
+constexpr int kThreads = 32 * kWarps;
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+                 "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+                 "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// Byte layout of one token's slot in shared memory (all offsets multiples of 16).
+struct Slot {
+    int B, C, U, TH, X, DL, bytes;
+};
+__host__ __device__ inline Slot slot_layout(int R, int N, int es, bool refl) {
+    Slot s;
+    int o = 0;
+    s.B = o;  o += R * N * es;
+    s.C = o;  o += R * N * es;
+    s.U = o;  o += refl ? N * es : 0;
+    s.TH = o; o += (N / 2) * 4;
+    s.X = o;  o += R * kCB * es;
+    s.DL = o; o += 16;                      // dt, lambda
+    s.bytes = (o + 15) & ~15;
+    return s;
+}
+
+template <typename T> __device__ __forceinline__ float2 ld2(const T* p);   // rows (2i, 2i+1)
+template <> __device__ __forceinline__ float2 ld2<float>(const float* p) { return *reinterpret_cast<const float2*>(p); }
+template <> __device__ __forceinline__ float2 ld2<__nv_bfloat16>(const __nv_bfloat16* p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+
+// Sum over the warp of NV values per lane.  Afterwards lane l holds the total
+// of value index l / (32 / NV) in v[0] (NV a power of two, <= 32): each
+// halving step keeps one half and adds the partner lane's other half.
+template <int NV>
+__device__ __forceinline__ void reduce_scatter(float (&v)[NV], int lane) {
+    int m = NV;
+    int o = 16;
+#pragma unroll
+    for (int step = 0; step < 5; ++step, o >>= 1) {
+        if (m > 1) {
+            const int half = m >> 1;
+            const bool upper = (lane & o) != 0;
+#pragma unroll
+            for (int j = 0; j < NV / 2; ++j) {
+                if (j < half) {
+                    const float send = upper ? v[j] : v[j + half];
+                    const float keep = upper ? v[j + half] : v[j];
+                    v[j] = keep + __shfl_xor_sync(kFull, send, o);
+                }
+            }
+            m = half;
+        } else {
+            v[0] += __shfl_xor_sync(kFull, v[0], o);
+        }
+    }
+}
+
+// (c, sn, s) of one pair block for the regime (0 under, 1 critical, 2 over)
+__device__ __forceinline__ void pair_block(int regime, float phi, float& c, float& sn, float& sg) {
+    if (regime == 0) {
+        sincosf(phi, &sn, &c);
+        sg = 1.f;
+    } else if (regime == 1) {
+        c = 1.f;
+        sn = phi;
+        sg = 0.f;
+    } else {
+        c = coshf(phi);
+        sn = sinhf(phi);
+        sg = -1.f;
+    }
+}
+
+template <typename T, int R, int KP, bool REFL>
+__global__ void __launch_bounds__(kThreads) seq_kernel(SeqParams q, int TK) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c0 = blockIdx.x * kCB;            // first column of the CTA
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int L = q.seqlen, H = q.nheads, G = q.ngroups, N = q.dstate, P = q.headdim;
+    const int NH = N / 2;
+    const int g = h / (H / G);
+    const size_t bh = (size_t)b * H + h;
+    const int cw = c0 + warp * kPC;             // first column of this warp
+    const bool wact = cw < P;                   // warp has columns (P is a multiple of 16)
+    const float Ah = q.A[h];
+    const T* xg = static_cast<const T*>(q.x);
+    const T* Bg = static_cast<const T*>(q.B);
+    const T* Cg = static_cast<const T*>(q.C);
+    const T* Ug = static_cast<const T*>(q.u);
+    constexpr int es = sizeof(T);
+    const Slot sl = slot_layout(R, N, es, REFL);
+
+    // ---- staging of a chunk of tokens (cp.async, 16-byte pieces)
+    auto stage = [&](int chunk, int buf) {
+        const int t0 = chunk * TK;
+        const int nt = min(TK, L - t0);
+        uint8_t* base = smem + (size_t)buf * TK * sl.bytes;
+        const int pB = R * N * es / 16, pU = REFL ? N * es / 16 : 0, pT = NH * 4 / 16;
+        const int pX = kCB * es / 16;                    // per rank
+        const int per = 2 * pB + pU + pT + R * pX;
+        for (int e = tid; e < nt * per; e += kThreads) {
+            const int tt = e / per;
+            int k = e % per;
+            const size_t bt = (size_t)b * L + t0 + tt;
+            uint8_t* s = base + (size_t)tt * sl.bytes;
+            if (k < pB) {
+                cp_async16(s + sl.B + 16 * k, reinterpret_cast<const uint8_t*>(Bg + (bt * G + g) * R * N) + 16 * k);
+                continue;
+            }
+            k -= pB;
+            if (k < pB) {
+                cp_async16(s + sl.C + 16 * k, reinterpret_cast<const uint8_t*>(Cg + (bt * G + g) * R * N) + 16 * k);
+                continue;
+            }
+            k -= pB;
+            if (k < pU) {
+                cp_async16(s + sl.U + 16 * k, reinterpret_cast<const uint8_t*>(Ug + (bt * G + g) * N) + 16 * k);
+                continue;
+            }
+            k -= pU;
+            if (k < pT) {
+                cp_async16(s + sl.TH + 16 * k, reinterpret_cast<const uint8_t*>(q.theta + (bt * G + g) * NH) + 16 * k);
+                continue;
+            }
+            k -= pT;
+            const int r = k / pX, kk = k % pX;
+            if (c0 + kk * 16 / es < P)
+                cp_async16(s + sl.X + r * kCB * es + 16 * kk,
+                           reinterpret_cast<const uint8_t*>(xg + ((bt * H + h) * R + r) * P + c0) + 16 * kk);
+        }
+        for (int tt = tid; tt < nt; tt += kThreads) {
+            const size_t o = ((size_t)b * L + t0 + tt) * H + h;
+            uint8_t* s = base + (size_t)tt * sl.bytes + sl.DL;
+            cp_async4(s, q.dt + o);
+            cp_async4(s + 4, q.lam + o);
+        }
+    };
+
+    // ---- carry in
+    float hs[KP][2][kPC];
+    float pb[KP][2][R];
+    float px[R][kPC];
+#pragma unroll
+    for (int k = 0; k < KP; ++k) {
+        const int i = lane + 32 * k;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+#pragma unroll
+            for (int c = 0; c < kPC; ++c)
+                hs[k][e][c] = (q.init_h && i < NH && wact) ? q.init_h[(bh * N + 2 * i + e) * P + cw + c] : 0.f;
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                pb[k][e][r] = (q.init_pB && i < NH) ? ld_io(static_cast<const T*>(q.init_pB) + (bh * R + r) * N + 2 * i + e)
+                                                    : 0.f;
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int c = 0; c < kPC; ++c)
+            px[r][c] = (q.init_pX && wact) ? ld_io(static_cast<const T*>(q.init_pX) + (bh * R + r) * P + cw + c) : 0.f;
+
+    const int nchunks = (L + TK - 1) / TK;
+    stage(0, 0);
+    cp_async_commit();
+    constexpr int NV = R * kPC;                 // readout values per lane
+    for (int ch = 0; ch < nchunks; ++ch) {
+        if (ch + 1 < nchunks) stage(ch + 1, (ch + 1) & 1);
+        cp_async_commit();
+        cp_async_wait_prev();
+        __syncthreads();
+        const int t0 = ch * TK;
+        const int nt = min(TK, L - t0);
+        const uint8_t* base = smem + (size_t)(ch & 1) * TK * sl.bytes;
+        for (int tt = 0; tt < nt; ++tt) {
+            const uint8_t* s = base + (size_t)tt * sl.bytes;
+            const float d = reinterpret_cast<const float*>(s + sl.DL)[0];
+            const float lm = reinterpret_cast<const float*>(s + sl.DL)[1];
+            const float al = expf(d * Ah);
+            const float be = (1.f - lm) * d * al;
+            const float ga = lm * d;
+            // this token's x for the warp's columns (same for every lane)
+            float xc[R][kPC];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int c = 0; c < kPC; ++c)
+                    xc[r][c] = ld_io(reinterpret_cast<const T*>(s + sl.X) + r * kCB + warp * kPC + c);
+            // v = alpha h + beta B_{t-1} X_{t-1}^T
+#pragma unroll
+            for (int k = 0; k < KP; ++k)
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+#pragma unroll
+                    for (int c = 0; c < kPC; ++c) {
+                        float pend = 0.f;
+#pragma unroll
+                        for (int r = 0; r < R; ++r) pend = fmaf(pb[k][e][r], px[r][c], pend);
+                        hs[k][e][c] = fmaf(be, pend, al * hs[k][e][c]);
+                    }
+            if (REFL) {
+                // v <- v - (2 / u^T u) u (u^T v), column by column (u = 0: no reflection)
+                float uv[KP][2];
+                float uu = 0.f;
+#pragma unroll
+                for (int k = 0; k < KP; ++k) {
+                    const int i = lane + 32 * k;
+                    const float2 u2 = i < NH ? ld2(reinterpret_cast<const T*>(s + sl.U) + 2 * i) : make_float2(0.f, 0.f);
+                    uv[k][0] = u2.x;
+                    uv[k][1] = u2.y;
+                    uu = fmaf(u2.x, u2.x, fmaf(u2.y, u2.y, uu));
+                }
+                float dot[kPC + 1];
+#pragma unroll
+                for (int c = 0; c < kPC; ++c) {
+                    float a = 0.f;
+#pragma unroll
+                    for (int k = 0; k < KP; ++k) a = fmaf(uv[k][0], hs[k][0][c], fmaf(uv[k][1], hs[k][1][c], a));
+                    dot[c] = a;
+                }
+                dot[kPC] = uu;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1)
+#pragma unroll
+                    for (int c = 0; c <= kPC; ++c) dot[c] += __shfl_xor_sync(kFull, dot[c], o);
+                const float f = dot[kPC] > 0.f ? 2.f / dot[kPC] : 0.f;
+#pragma unroll
+                for (int c = 0; c < kPC; ++c) {
+                    const float fd = f * dot[c];
+#pragma unroll
+                    for (int k = 0; k < KP; ++k) {
+                        hs[k][0][c] = fmaf(-fd, uv[k][0], hs[k][0][c]);
+                        hs[k][1][c] = fmaf(-fd, uv[k][1], hs[k][1][c]);
+                    }
+                }
+            }
+            // pair blocks T_t (the rotation R_t in the reflection variant)
+#pragma unroll
+            for (int k = 0; k < KP; ++k) {
+                const int i = lane + 32 * k;
+                const float th = i < NH ? reinterpret_cast<const float*>(s + sl.TH)[i] : 0.f;
+                float cc, sn, sg;
+                pair_block(REFL ? 0 : q.regime, d * th, cc, sn, sg);
+#pragma unroll
+                for (int c = 0; c < kPC; ++c) {
+                    const float v0 = hs[k][0][c], v1 = hs[k][1][c];
+                    hs[k][0][c] = fmaf(cc, v0, -sn * v1);
+                    hs[k][1][c] = fmaf(sg * sn, v0, cc * v1);
+                }
+            }
+            // + gamma B_t X_t^T; then y = C_t^T h (partial over this lane's rows)
+            float bt_[KP][2][R], yv[NV];
+#pragma unroll
+            for (int j = 0; j < NV; ++j) yv[j] = 0.f;
+#pragma unroll
+            for (int k = 0; k < KP; ++k) {
+                const int i = lane + 32 * k;
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const float2 b2 = i < NH ? ld2(reinterpret_cast<const T*>(s + sl.B) + r * N + 2 * i) : make_float2(0.f, 0.f);
+                    bt_[k][0][r] = b2.x;
+                    bt_[k][1][r] = b2.y;
+                }
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+#pragma unroll
+                    for (int c = 0; c < kPC; ++c) {
+                        float cur = 0.f;
+#pragma unroll
+                        for (int r = 0; r < R; ++r) cur = fmaf(bt_[k][e][r], xc[r][c], cur);
+                        hs[k][e][c] = fmaf(ga, cur, hs[k][e][c]);
+                    }
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const float2 c2 = i < NH ? ld2(reinterpret_cast<const T*>(s + sl.C) + r * N + 2 * i) : make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int c = 0; c < kPC; ++c)
+                        yv[r * kPC + c] = fmaf(c2.x, hs[k][0][c], fmaf(c2.y, hs[k][1][c], yv[r * kPC + c]));
+                }
+            }
+            reduce_scatter<NV>(yv, lane);
+            constexpr int SPAN = 32 / NV;          // lanes holding one value's total
+            if (wact && (lane % SPAN) == 0) {
+                const int idx = lane / SPAN, r = idx / kPC, c = idx % kPC;
+                st_io(static_cast<T*>(q.y) + ((((size_t)b * L + t0 + tt) * H + h) * R + r) * P + cw + c, yv[0]);
+            }
+#pragma unroll
+            for (int k = 0; k < KP; ++k)
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+#pragma unroll
+                    for (int r = 0; r < R; ++r) pb[k][e][r] = bt_[k][e][r];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int c = 0; c < kPC; ++c) px[r][c] = xc[r][c];
+        }
+        __syncthreads();   // every warp is done with this buffer before it is staged again
+    }
+
+    // ---- carry out: the state is in the original frame
+#pragma unroll
+    for (int k = 0; k < KP; ++k) {
+        const int i = lane + 32 * k;
+        if (i >= NH) continue;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            if (q.fin_h && wact)
+#pragma unroll
+                for (int c = 0; c < kPC; ++c) q.fin_h[(bh * N + 2 * i + e) * P + cw + c] = hs[k][e][c];
+            if (q.fin_pB && blockIdx.x == 0 && warp == 0)
+#pragma unroll
+                for (int r = 0; r < R; ++r) st_io(static_cast<T*>(q.fin_pB) + (bh * R + r) * N + 2 * i + e, pb[k][e][r]);
+        }
+    }
+    if (q.fin_pX && wact && lane == 0)
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int c = 0; c < kPC; ++c) st_io(static_cast<T*>(q.fin_pX) + (bh * R + r) * P + cw + c, px[r][c]);
+}
+
+template <typename T, int R, int KP, bool REFL>
+static cudaError_t launch_t(const SeqParams& q, cudaStream_t st) {
+    const Slot sl = slot_layout(R, q.dstate, sizeof(T), REFL);
+    // tokens per staged chunk: up to 16, two buffers within 96 KB
+    int TK = (96 * 1024) / (2 * sl.bytes);
+    if (TK > 16) TK = 16;
+    if (TK < 1) return cudaErrorInvalidValue;
+    const size_t smem = (size_t)2 * TK * sl.bytes;
+    cudaError_t e = cudaFuncSetAttribute(seq_kernel<T, R, KP, REFL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((q.headdim + kCB - 1) / kCB, q.nheads, q.batch);
+    seq_kernel<T, R, KP, REFL><<<grid, kThreads, smem, st>>>(q, TK);
+    return cudaGetLastError();
+}
+
+template <typename T, bool REFL>
+static cudaError_t launch_rk(const SeqParams& q, cudaStream_t st) {
+    const int KP = (q.dstate / 2 + 31) / 32;
+    switch (q.rank * 8 + KP) {
+        case 1 * 8 + 1: return launch_t<T, 1, 1, REFL>(q, st);
+        case 1 * 8 + 2: return launch_t<T, 1, 2, REFL>(q, st);
+        case 1 * 8 + 4: return launch_t<T, 1, 4, REFL>(q, st);
+        case 2 * 8 + 1: return launch_t<T, 2, 1, REFL>(q, st);
+        case 2 * 8 + 2: return launch_t<T, 2, 2, REFL>(q, st);
+        case 2 * 8 + 4: return launch_t<T, 2, 4, REFL>(q, st);
+        case 4 * 8 + 1: return launch_t<T, 4, 1, REFL>(q, st);
+        case 4 * 8 + 2: return launch_t<T, 4, 2, REFL>(q, st);
+        case 4 * 8 + 4: return launch_t<T, 4, 4, REFL>(q, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace seq
+
+bool seq_supported(const m3_dims& d) {
+    const int KP = (d.dstate / 2 + 31) / 32;
+    return (d.rank == 1 || d.rank == 2 || d.rank == 4) && d.dstate % 8 == 0 && (KP == 1 || KP == 2 || KP == 4) &&
+           d.headdim % seq::kCB == 0;
+}
+
+cudaError_t launch_seq(const m3_dims& d, const SeqParams& q, cudaStream_t st) {
+    const bool refl = q.u != nullptr;
+    if (d.io_dtype == M3_BF16)
+        return refl ? seq::launch_rk<__nv_bfloat16, true>(q, st) : seq::launch_rk<__nv_bfloat16, false>(q, st);
+    return refl ? seq::launch_rk<float, true>(q, st) : seq::launch_rk<float, false>(q, st);
+}
+
+}  // namespace m3

@@ -455,6 +455,65 @@ m3_status m3_scan_fwd_phase(const m3_dims* d, int mode, const int* perm, const f
                        stream);
 }
 
+// ------------------------------------------------- transition variants --
+// carry pass-through of an empty call (no tokens): shared by the variants
+static m3_status carry_passthrough(const m3_dims* d, const m3_carry* init, m3_carry* fin, cudaStream_t st) {
+    if (!fin || d->batch == 0) return M3_OK;
+    const size_t units = (size_t)d->batch * d->nheads;
+    const size_t hb = units * d->dstate * d->headdim * sizeof(float);
+    const size_t bb = units * d->rank * d->dstate * io_bytes(*d);
+    const size_t xb = units * d->rank * d->headdim * io_bytes(*d);
+    cudaError_t e = cudaSuccess;
+    if (fin->h)
+        e = (init && init->h) ? cudaMemcpyAsync(fin->h, init->h, hb, cudaMemcpyDeviceToDevice, st)
+                              : cudaMemsetAsync(fin->h, 0, hb, st);
+    if (e == cudaSuccess && fin->prev_B)
+        e = (init && init->prev_B) ? cudaMemcpyAsync(fin->prev_B, init->prev_B, bb, cudaMemcpyDeviceToDevice, st)
+                                   : cudaMemsetAsync(fin->prev_B, 0, bb, st);
+    if (e == cudaSuccess && fin->prev_x)
+        e = (init && init->prev_x) ? cudaMemcpyAsync(fin->prev_x, init->prev_x, xb, cudaMemcpyDeviceToDevice, st)
+                                   : cudaMemsetAsync(fin->prev_x, 0, xb, st);
+    return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+static m3_status scan_variant(const m3_dims* d, int regime, const void* u, const void* x, const void* B,
+                              const void* C, const float* dt, const float* A, const float* lambda,
+                              const float* theta, const m3_carry* init, void* y, m3_carry* fin, void* stream) {
+    m3_status s = check_dims(d, true);
+    if (s != M3_OK) return s;
+    if (regime < 0 || regime > 2) return M3_ERR_INVALID_ARG;
+    if (!seq_supported(*d)) return M3_ERR_UNSUPPORTED;
+    const bool work = d->batch > 0 && d->seqlen > 0;
+    if (work && !ptrs_ok({x, B, C, dt, A, lambda, theta, y})) return M3_ERR_INVALID_ARG;
+    if (init && !opt_ptrs_ok({init->h, init->prev_B, init->prev_x})) return M3_ERR_INVALID_ARG;
+    if (fin && !opt_ptrs_ok({fin->h, fin->prev_B, fin->prev_x})) return M3_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (!work) return carry_passthrough(d, init, fin, st);
+    SeqParams q;
+    memset(&q, 0, sizeof(q));
+    q.batch = d->batch; q.seqlen = d->seqlen; q.nheads = d->nheads; q.ngroups = d->ngroups;
+    q.headdim = d->headdim; q.dstate = d->dstate; q.rank = d->rank; q.regime = regime;
+    q.x = x; q.B = B; q.C = C; q.u = u; q.dt = dt; q.A = A; q.lam = lambda; q.theta = theta;
+    if (init) { q.init_h = init->h; q.init_pB = init->prev_B; q.init_pX = init->prev_x; }
+    q.y = y;
+    if (fin) { q.fin_h = fin->h; q.fin_pB = fin->prev_B; q.fin_pX = fin->prev_x; }
+    return launch_seq(*d, q, st) == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+m3_status m3_scan_fwd_damped(const m3_dims* d, int regime, const void* x, const void* B, const void* C,
+                             const float* dt, const float* A, const float* lambda, const float* theta,
+                             const m3_carry* init, void* y, m3_carry* final_state, void* stream) {
+    return scan_variant(d, regime, nullptr, x, B, C, dt, A, lambda, theta, init, y, final_state, stream);
+}
+
+m3_status m3_scan_fwd_reflect(const m3_dims* d, const void* u, const void* x, const void* B, const void* C,
+                              const float* dt, const float* A, const float* lambda, const float* theta,
+                              const m3_carry* init, void* y, m3_carry* final_state, void* stream) {
+    // u is read only when there are tokens (like the other inputs)
+    if (d && d->batch > 0 && d->seqlen > 0 && !ptrs_ok({u})) return M3_ERR_INVALID_ARG;
+    return scan_variant(d, 0, u, x, B, C, dt, A, lambda, theta, init, y, final_state, stream);
+}
+
 m3_status m3_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void* stream) {
     if (!workspace || !aligned16(workspace) || workspace_bytes < kWorkspaceHeaderBytes) return M3_ERR_WORKSPACE;
     return launch_wait_selftest(reinterpret_cast<int*>(workspace), (cudaStream_t)stream) == cudaSuccess

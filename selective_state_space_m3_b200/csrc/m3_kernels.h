@@ -60,6 +60,30 @@ struct ScanParams {
     float* ws_sin;     // [b][h][seg][N][P]
 };
 
+// token-by-token scan of the transition variants (k_seq.cu): damping regimes
+// (u == nullptr, regime 0/1/2) and the low-rank reflection (u != nullptr)
+struct SeqParams {
+    int batch, seqlen, nheads, ngroups, headdim, dstate, rank;
+    int regime;          // 0 under, 1 critical, 2 over (ignored with u)
+    const void* x;
+    const void* B;
+    const void* C;
+    const void* u;       // [b][t][g][n] io, or null
+    const float* dt;
+    const float* A;
+    const float* lam;
+    const float* theta;
+    const float* init_h;
+    const void* init_pB;
+    const void* init_pX;
+    void* y;
+    float* fin_h;
+    void* fin_pB;
+    void* fin_pX;
+};
+bool seq_supported(const m3_dims& d);
+cudaError_t launch_seq(const m3_dims& d, const SeqParams& q, cudaStream_t st);
+
 // backward pass (k_bwd.cu); gradients are float32, dB / dC / dtheta / dA
 // accumulated with atomics into buffers zeroed by the caller
 struct BwdParams {

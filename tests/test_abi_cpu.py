@@ -199,3 +199,32 @@ def test_empty_problems_return_ok_before_touching_anything():
         d = empty.c()
         assert LIB.m3_rope_bc(ctypes.byref(d), None, None, None, None, None, None, None,
                               None) == m3.M3_OK
+
+
+def _variant_status(d, regime=0, u=GOOD, ptr=GOOD, reflect=False):
+    cd = d.c()
+    if reflect:
+        return LIB.m3_scan_fwd_reflect(ctypes.byref(cd), u, ptr, ptr, ptr, ptr, ptr, ptr, ptr, None, ptr, None,
+                                       None)
+    return LIB.m3_scan_fwd_damped(ctypes.byref(cd), regime, ptr, ptr, ptr, ptr, ptr, ptr, ptr, None, ptr, None,
+                                  None)
+
+
+def test_variants_reject_before_launching():
+    """Damped and reflection scans: a bad regime, unsupported shapes (rank 3,
+    dstate not a multiple of 8 or above 256, headdim not a multiple of 16),
+    null or misaligned pointers all return before any launch; an empty call
+    is OK with null pointers."""
+    d = dims(headdim=16, dstate=16, rank=2)
+    assert _variant_status(d, regime=3) == m3.M3_ERR_INVALID_ARG
+    assert _variant_status(d, regime=-1) == m3.M3_ERR_INVALID_ARG
+    assert _variant_status(dims(rank=3)) == m3.M3_ERR_UNSUPPORTED
+    assert _variant_status(dims(dstate=12)) == m3.M3_ERR_UNSUPPORTED
+    assert _variant_status(dims(dstate=512)) == m3.M3_ERR_UNSUPPORTED
+    assert _variant_status(dims(headdim=24)) == m3.M3_ERR_UNSUPPORTED
+    assert _variant_status(d, ptr=BAD) == m3.M3_ERR_INVALID_ARG
+    assert _variant_status(d, reflect=True, u=BAD) == m3.M3_ERR_INVALID_ARG
+    assert _variant_status(d, reflect=True, u=None) == m3.M3_ERR_INVALID_ARG
+    for e in (dims(batch=0), dims(seqlen=0)):
+        assert _variant_status(e, ptr=None) == m3.M3_OK
+        assert _variant_status(e, ptr=None, reflect=True, u=None) == m3.M3_OK
