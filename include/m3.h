@@ -59,7 +59,9 @@
  * the prefill (m3_scan_fwd and the calls built on it) to the float32 SIMT
  * kernels even where the tensor-core path applies; M3_SCAN_NSEG=n (n >= 1)
  * cuts each sequence into n segments (at most one per chunk) instead of the
- * planner's choice.
+ * planner's choice; M3_TC_KERNEL=persistent runs the tensor-core prefill on
+ * the persistent warp-specialised kernel (one CTA per SM, tiles pipelined
+ * across roles) instead of the default tile kernel.
  * Buffer extents cannot be checked through plain pointers: every buffer must
  * hold at least the elements its layout gives for `dims` (nothing is read
  * from a buffer whose extent for `dims` is zero); a smaller buffer is read or

@@ -39,10 +39,8 @@
 // Every wait on an mbarrier is bounded (1 s); on expiry the kernel records
 // M3_ERR_DEVICE_TIMEOUT in the workspace status word, finishes the tile with
 // no further waiting and returns after freeing its TMEM.
-#include <cuda.h>
-
-#include "m3_common.cuh"
 #include "m3_kernels.h"
+#include "tc_ptx.cuh"
 
 namespace m3 {
 namespace tc {
@@ -55,7 +53,6 @@ constexpr int kWorkers = 128 * kWG;
 constexpr int kThreads = 32 + kWorkers;
 constexpr int kNE = kWorkers / 32;     // token groups of the phase / rotation pass (one per worker warp)
 constexpr int kSC = kP / kWG;          // state / y columns per warpgroup
-constexpr uint64_t kWaitNs = 1000000000ull;
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr int OFF_B = 0;          // 32 KB: B~ (two 16 KB atoms)
@@ -83,71 +80,12 @@ static_assert(sizeof(Misc) <= MISC_BYTES, "misc region too small");
 enum { BAR_LOAD = 0, BAR_OPS, BAR_G, BAR_BW, BAR_P, BAR_Y, BAR_DRAIN };
 
 // ------------------------------------------------------------ PTX wrappers --
-__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+using namespace ptx;
 
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(su32(b)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait.  Returns false when the CTA is aborting (this wait or an
-// earlier one expired); the caller then carries on without waiting.
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* b, uint32_t parity, int* abortp, int* status, int where) {
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
-        if (mbar_try(b, parity)) return true;
-        if (*(volatile int*)abortp) return false;
-        if (globaltimer_ns() - t0 > kWaitNs) {
-            *(volatile int*)abortp = 1;
-            if (status) {
-                atomicCAS(status, 0, (int)M3_ERR_DEVICE_TIMEOUT);
-                status[1] = where;
-            }
-            return false;
-        }
-    }
-}
-// the common case (the phase completes within try_wait's own suspend window)
-// stays inline; the bounded spin is out of line
-__device__ __forceinline__ bool mbar_wait_flag(uint64_t* b, uint32_t parity, int* abortp, int* status, int where) {
-    if (mbar_try(b, parity)) return true;
-    return mbar_wait_slow(b, parity, abortp, status, where);
-}
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Misc* m, int* status, int where) {
     return mbar_wait_flag(b, parity, &m->abort_flag, status, where);
 }
 
-__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
-                                            int c2, int c3, int c4) {
-    asm volatile(
-        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
-        ::"r"(dst), "l"((uint64_t)map), "r"(su32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
-        : "memory");
-}
-
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void workers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kWorkers) : "memory"); }
 // all workers get the OR of `cond` (named barrier 1 with a reduction), so
 // they take the same branch
@@ -162,135 +100,6 @@ __device__ __forceinline__ int workers_any(int cond) {
         : "r"(cond), "n"(kWorkers)
         : "memory");
     return r;
-}
-
-__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(dst)), "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-// D[tmem] (+)= A[smem desc] x B[smem desc], bf16 inputs, fp32 accumulate
-__device__ __forceinline__ void umma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc)
-        : "memory");
-}
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
-                 : "memory");
-}
-
-// 32 lanes x 32 consecutive fp32 columns; thread = lane
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-}
-
-// 32 lanes x 16 consecutive fp32 columns; thread = lane
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-          "=r"(r[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
-}
-
-// Shared-memory matrix descriptor, SWIZZLE_128B (sm_100 layout: start>>4,
-// LBO>>4 at bit 16, SBO>>4 at bit 32, version 1 at bit 46, swizzle 2 at 61).
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
-}
-// Instruction descriptor, kind::f16: D f32, A/B bf16, majors, N>>3, M>>4.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
-           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-// byte offset of 16-byte chunk `c` (0..7) of row `row` inside a 128-row
-// SWIZZLE_128B atom (rows of 128 bytes, chunk index XOR row%8)
-__device__ __forceinline__ uint32_t sw128(int row, int c) { return (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4)); }
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t u) {
-    __nv_bfloat162 v;
-    memcpy(&v, &u, 4);
-    return v;
-}
-__device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 v) {
-    uint32_t u;
-    memcpy(&u, &v, 4);
-    return u;
-}
-// one rotary pair in bf16x2: (x, y) -> (c x + s y, c y - s x), cc = (c, c),
-// sn = (s, -s); the product s*y is rounded to bf16 before the fused add
-__device__ __forceinline__ uint32_t rot_bf(uint32_t v, uint32_t cc, uint32_t sn) {
-    const uint32_t sw = __byte_perm(v, 0, 0x1032);          // (y, x)
-    return as_u32(__hfma2(as_bf2(cc), as_bf2(v), __hmul2(as_bf2(sn), as_bf2(sw))));
-}
-__device__ __forceinline__ uint4 scale_chunk(uint4 v, uint32_t w2) {
-    const __nv_bfloat162 w = as_bf2(w2);
-    v.x = as_u32(__hmul2(w, as_bf2(v.x)));
-    v.y = as_u32(__hmul2(w, as_bf2(v.y)));
-    v.z = as_u32(__hmul2(w, as_bf2(v.z)));
-    v.w = as_u32(__hmul2(w, as_bf2(v.w)));
-    return v;
-}
-// x[s] for a warp-uniform slice index s < NT (a select chain, no local memory)
-template <int NT>
-__device__ __forceinline__ float pick(const float (&x)[NT], int s) {
-    float r = x[0];
-#pragma unroll
-    for (int j = 1; j < NT; ++j) r = (s == j) ? x[j] : r;
-    return r;
-}
-// 8 consecutive floats -> one 16-byte chunk of bf16
-__device__ __forceinline__ uint4 pack_chunk(const float* f) {
-    uint4 o;
-    o.x = pack_bf16x2(f[0], f[1]);
-    o.y = pack_bf16x2(f[2], f[3]);
-    o.z = pack_bf16x2(f[4], f[5]);
-    o.w = pack_bf16x2(f[6], f[7]);
-    return o;
-}
-// reduce a float angle to [-pi, pi] (two-constant additive reduction:
-// 2*pi split into a float head and tail so k*2pi is formed exactly enough)
-__device__ __forceinline__ float wrap_pi_f(float x) {
-    constexpr float kInv2Pi = 0.15915494309189535f;
-    constexpr float k2PiHi = 6.28318548202514648f;      // float(2 pi)
-    constexpr float k2PiLo = -1.7484555314695172e-7f;   // 2 pi - float(2 pi)
-    const float k = rintf(x * kInv2Pi);
-    return fmaf(-k, k2PiLo, fmaf(-k, k2PiHi, x));
 }
 
 // ------------------------------------------------------------------ kernel --
@@ -951,8 +760,11 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
+}  // namespace tc
+
 // 5-D map over [b][t][grp][r][inner] with a box of (64 inner, R, 1, T, 1)
-static bool make_map(CUtensorMap* map, const void* base, int inner, int R, int grp, int L, int batch, int T) {
+bool make_tile_map(CUtensorMap* map, const void* base, int inner, int R, int grp, int L, int batch, int T) {
+    using namespace tc;
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[5] = {(cuuint64_t)inner, (cuuint64_t)R, (cuuint64_t)grp, (cuuint64_t)L, (cuuint64_t)batch};
@@ -965,8 +777,6 @@ static bool make_map(CUtensorMap* map, const void* base, int inner, int R, int g
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-}  // namespace tc
 
 // Diagnostic: one CTA waits, through the same bounded-wait helper the scan
 // uses, on an mbarrier that no thread arrives at.  The wait gives up after
@@ -1002,9 +812,9 @@ static cudaError_t launch_tc_R(const ScanParams& q, int* status, cudaStream_t st
     using namespace tc;
     constexpr int T = kRows / R;
     CUtensorMap mB, mC, mX;
-    if (!make_map(&mB, q.B, kN, R, q.ngroups, q.seqlen, q.batch, T) ||
-        !make_map(&mC, q.C, kN, R, q.ngroups, q.seqlen, q.batch, T) ||
-        !make_map(&mX, q.x, kP, R, q.nheads, q.seqlen, q.batch, T))
+    if (!make_tile_map(&mB, q.B, kN, R, q.ngroups, q.seqlen, q.batch, T) ||
+        !make_tile_map(&mC, q.C, kN, R, q.ngroups, q.seqlen, q.batch, T) ||
+        !make_tile_map(&mX, q.x, kP, R, q.nheads, q.seqlen, q.batch, T))
         return cudaErrorInvalidValue;
     cudaFuncSetAttribute(scan_tc_kernel<R, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     cudaFuncSetAttribute(scan_tc_kernel<R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
@@ -1018,6 +828,33 @@ static cudaError_t launch_tc_R(const ScanParams& q, int* status, cudaStream_t st
     }
     scan_tc_kernel<R, false><<<dim3(q.nseg, q.nheads, q.batch), kThreads, SMEM_BYTES, st>>>(mB, mC, mX, q, status);
     return cudaGetLastError();
+}
+
+template <int R>
+static cudaError_t launch_tc_summary_R(const ScanParams& q, int* status, cudaStream_t st) {
+    using namespace tc;
+    constexpr int T = kRows / R;
+    CUtensorMap mB, mC, mX;
+    if (!make_tile_map(&mB, q.B, kN, R, q.ngroups, q.seqlen, q.batch, T) ||
+        !make_tile_map(&mC, q.C, kN, R, q.ngroups, q.seqlen, q.batch, T) ||
+        !make_tile_map(&mX, q.x, kP, R, q.nheads, q.seqlen, q.batch, T))
+        return cudaErrorInvalidValue;
+    cudaFuncSetAttribute(scan_tc_kernel<R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaFuncSetAttribute(scan_tc_kernel<R, true>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    scan_tc_kernel<R, true><<<dim3(q.nseg - 1, q.nheads, q.batch), kThreads, SMEM_BYTES, st>>>(mB, mC, mX, q, status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_scan_combine(q, st);
+}
+
+cudaError_t launch_scan_tc_summary(const m3_dims& d, const ScanParams& q, int* status, cudaStream_t st) {
+    switch (d.rank) {
+        case 1: return launch_tc_summary_R<1>(q, status, st);
+        case 2: return launch_tc_summary_R<2>(q, status, st);
+        case 4: return launch_tc_summary_R<4>(q, status, st);
+        case 8: return launch_tc_summary_R<8>(q, status, st);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t launch_scan_tc(const m3_dims& d, const ScanParams& q, int* status, cudaStream_t st) {

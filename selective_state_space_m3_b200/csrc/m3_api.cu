@@ -48,6 +48,11 @@ struct Plan {
     int qs;      // chunk length the kernels use (tokens)
     int nseg;    // segments per (b, h)
     int cps;     // chunks per segment
+    int kernel;  // tcgen05 path: 1 = tile kernel (k_scan_tc.cu), 2 = persistent kernel (k_scan_ws.cu)
+    int wmode;   // persistent kernel: 0 = ranges with hand-off, 1 = one segment per CTA
+    int grid;    // persistent kernel: CTAs
+    int M;       // persistent kernel, mode 0: tiles per CTA
+    int nt;      // tiles (chunks) per sequence
 };
 
 static int env_int(const char* name, int dflt) {
@@ -86,6 +91,57 @@ int device_sm_count() {
 static m3_status make_plan(const m3_dims& d, Plan* pl) {
     const size_t kMaxSmem = 200 * 1024;
     const bool tc = tc_eligible(d) && !env_is("M3_SCAN_PATH", "simt");
+    // tcgen05 path: the tile kernel (two CTAs per SM, one sequence or
+    // segment each) unless M3_TC_KERNEL=persistent asks for the persistent
+    // warp-specialised kernel (one CTA per SM; measured slower on every layer
+    // workload, kept as an option)
+    pl->kernel = tc ? (env_is("M3_TC_KERNEL", "persistent") ? 2 : 1) : 0;
+    pl->wmode = 0;
+    pl->grid = 0;
+    pl->M = 0;
+    if (pl->kernel == 2) {
+        // persistent kernel: one CTA per SM.  With at least as many (b, h)
+        // sequences as SMs the concatenated tiles are cut into one range per
+        // CTA (a sequence split by a range boundary hands its state from its
+        // head to its tail); with fewer, each sequence is cut into segments
+        // (at most one CTA each, all resident) whose incoming states come from
+        // a summary pass.  M3_SCAN_NSEG forces segments.
+        const int qs = tc_tile_tokens(d.rank);
+        const long long nt = d.seqlen > 0 ? (d.seqlen + qs - 1) / qs : 0;
+        const long long units = (long long)d.batch * d.nheads;
+        const long long sms = device_sm_count();
+        const int forced = env_int("M3_SCAN_NSEG", 0);
+        pl->path = 1;
+        pl->qs = qs;
+        pl->nt = (int)nt;
+        if (forced <= 0 && units >= sms && nt > 0) {
+            const long long total = units * nt;
+            if (total > (1LL << 30)) return M3_ERR_UNSUPPORTED;
+            pl->wmode = 0;
+            pl->M = (int)((total + sms - 1) / sms);
+            pl->grid = (int)sms;
+            pl->nseg = 1;
+            pl->cps = (int)nt;
+            return M3_OK;
+        }
+        long long nseg = 1;
+        if (forced > 0) {
+            nseg = forced;
+        } else if (units > 0) {
+            nseg = sms / units;
+            if (nseg > nt / 2) nseg = nt / 2;
+        }
+        if (nseg < 1) nseg = 1;
+        if (nt > 0 && nseg > nt) nseg = nt;
+        const long long cps = nt > 0 ? (nt + nseg - 1) / nseg : 1;
+        if (nt > 0) nseg = (nt + cps - 1) / cps;
+        if (units * nseg > 0x7fffffffLL) return M3_ERR_UNSUPPORTED;
+        pl->wmode = 1;
+        pl->nseg = (int)nseg;
+        pl->cps = (int)cps;
+        pl->grid = (int)(units * nseg);
+        return M3_OK;
+    }
     int qs;
     if (tc) {
         qs = tc_tile_tokens(d.rank);
@@ -117,7 +173,7 @@ static m3_status make_plan(const m3_dims& d, Plan* pl) {
 }
 
 struct WsLayout {
-    size_t sloc, decay, phase, sin, total;
+    size_t sloc, decay, phase, sin, ho_state, ho_flag, total;
 };
 
 static size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -131,6 +187,9 @@ static WsLayout ws_layout(const m3_dims& d, const Plan& pl) {
     w.decay = off; off = round256(off + units * sizeof(float));
     w.phase = off; off = round256(off + units * (d.dstate / 2) * sizeof(float));
     w.sin = off;   off = round256(off + units * NP * sizeof(float));
+    const size_t slots = (pl.kernel == 2 && pl.wmode == 0) ? (size_t)pl.grid : 0;
+    w.ho_state = off; off = round256(off + slots * NP * sizeof(float));
+    w.ho_flag = off;  off = round256(off + slots * sizeof(int));
     w.total = off;
     return w;
 }
@@ -171,7 +230,7 @@ m3_status m3_scan_plan(const m3_dims* d, int* launches, int* segments, int* chun
     s = make_plan(*d, &pl);
     if (s != M3_OK) return s;
     const bool work = d->batch > 0 && d->seqlen > 0;
-    if (launches) *launches = work ? (pl.nseg > 1 ? 3 : 1) : 0;
+    if (launches) *launches = work ? (pl.nseg > 1 ? 3 : 1) : 0;   // summary, combine, main
     if (segments) *segments = pl.nseg;
     if (chunk_used) *chunk_used = pl.qs;
     if (path) *path = pl.path;
@@ -233,8 +292,29 @@ m3_status m3_scan_fwd(const m3_dims* d, const void* x, const void* B, const void
     q.ws_decay = reinterpret_cast<float*>(ws + w.decay);
     q.ws_phase = reinterpret_cast<float*>(ws + w.phase);
     q.ws_sin = reinterpret_cast<float*>(ws + w.sin);
-    cudaError_t e = pl.path == 1 ? launch_scan_tc(*d, q, reinterpret_cast<int*>(workspace), st)
-                                 : launch_scan_simt(*d, q, st);
+    int* status = reinterpret_cast<int*>(workspace);
+    cudaError_t e;
+    if (pl.kernel == 2) {
+        e = cudaSuccess;
+        if (pl.wmode == 1 && pl.nseg > 1) e = launch_scan_tc_summary(*d, q, status, st);
+        if (e == cudaSuccess) {
+            static std::atomic<int> calls{0};
+            int id = calls.fetch_add(1, std::memory_order_relaxed) + 1;
+            id = (id & 0x3fffffff) + 1;            // never 0: a cleared flag never matches
+            WsPlanArgs pa;
+            pa.mode = pl.wmode;
+            pa.nt = pl.nt;
+            pa.M = pl.M;
+            pa.total = pl.nt * (int)units;
+            pa.grid = pl.grid;
+            pa.call_id = id;
+            pa.ho_state = reinterpret_cast<float*>(ws + w.ho_state);
+            pa.ho_flag = reinterpret_cast<int*>(ws + w.ho_flag);
+            e = launch_scan_ws(*d, q, pa, status, st);
+        }
+    } else {
+        e = pl.path == 1 ? launch_scan_tc(*d, q, status, st) : launch_scan_simt(*d, q, st);
+    }
     return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }
 

@@ -140,5 +140,20 @@ bool tc_eligible(const m3_dims& d);
 int tc_tile_tokens(int rank);
 cudaError_t launch_scan_tc(const m3_dims& d, const ScanParams& q, int* status, cudaStream_t st);
 cudaError_t launch_wait_selftest(int* status, cudaStream_t st);
+// the summary pass of the tile kernel only (segments), then the combine
+cudaError_t launch_scan_tc_summary(const m3_dims& d, const ScanParams& q, int* status, cudaStream_t st);
+
+// persistent warp-specialised prefill (k_scan_ws.cu): mode 0 cuts the
+// concatenated chains of tiles into one range per CTA and hands states from
+// a chain's head to its tail (cooperative launch); mode 1 runs one segment
+// per CTA with its incoming state from the summary pass
+struct WsPlanArgs {
+    int mode, nt, M, total, grid, call_id;
+    float* ho_state;   // [grid][N][P]
+    int* ho_flag;      // [grid]
+};
+int ws_smem_bytes();
+cudaError_t launch_scan_ws(const m3_dims& d, const ScanParams& q, const WsPlanArgs& pa, int* status,
+                           cudaStream_t st);
 
 }  // namespace m3
