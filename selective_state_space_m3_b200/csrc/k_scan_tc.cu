@@ -316,6 +316,21 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tma_load_5d(sbase + OFF_X, &tmX, &m->bar[BAR_LOAD], 0, 0, h, t0, b);
                 pending_load = 1;
                 load_par = par;
+                // the next tile into L2: its load, issued once this tile's MMAs
+                // are done, then waits for L2 instead of DRAM.  Only for cut
+                // sequences: there the grid holds few CTAs and each tile's load
+                // latency sits on the critical path; with one segment per
+                // sequence the SMs hold enough CTAs to hide it.
+                if (q.nseg > 1 && k + 1 < ntiles) {
+                    const int tn = t0 + T;
+                    tma_prefetch_5d(&tmB, 0, 0, g, tn, b);
+                    tma_prefetch_5d(&tmB, 64, 0, g, tn, b);
+                    if (!SUMMARY) {
+                        tma_prefetch_5d(&tmC, 0, 0, g, tn, b);
+                        tma_prefetch_5d(&tmC, 64, 0, g, tn, b);
+                    }
+                    tma_prefetch_5d(&tmX, 0, 0, h, tn, b);
+                }
                 // every worker saw the load complete before arriving here
                 if (mbar_wait(&m->bar[BAR_OPS], par, m, status, 2)) pending_load = 0;
                 tc_fence_after();
