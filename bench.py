@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-rope", action="store_true", help="skip the m3_rope_bc measurement")
+    ap.add_argument("--no-layers", action="store_true",
+                    help="skip the SISO and long-context SISO prefill objects")
     ap.add_argument("--bwd", action="store_true", help="also time the backward pass m3_scan_bwd")
     ap.add_argument("--phase", action="store_true", help="also time two phase interventions")
     ap.add_argument("--no-variants", action="store_true",
@@ -146,52 +148,68 @@ def algorithmic_bytes(t: dict, y, fin) -> int:
     return n
 
 
-def algorithmic_flops(s, tile_rows=128) -> float:
-    """Causal chunked-scan FLOPs per token-head: intra-chunk Gram + masked
-    product ((Q+1) R^2 (N+P) with Q the chunk), plus the state terms
-    (chunk output C~ S and chunk state B~^T X: 4 R N P)."""
-    Q, R, N, P = s.chunk, s.rank, s.dstate, s.headdim
+def algorithmic_flops(s, chunk: int) -> float:
+    """Causal chunked-scan FLOPs per token-head at chunk length `chunk` (the
+    one the plan runs): intra-chunk Gram + masked product ((Q+1) R^2 (N+P)),
+    plus the state terms (chunk output C~ S and chunk state B~^T X: 4 R N P)."""
+    Q, R, N, P = chunk, s.rank, s.dstate, s.headdim
     per = (Q + 1) * R * R * (N + P) + 4 * R * N * P
     return float(per) * s.batch * s.seqlen * s.nheads
 
 
 # ------------------------------------------------------------- reference --
-def run_reference(args, rank):
-    if rank != 0:
-        return 0
+def oracle_sample_timing(budget_s: float, min_calls: int = 2, max_calls: int = 20, fixed_calls: int = 0,
+                         warmup: int = 1):
+    """The fp64 oracle on a bounded sample of the headline workload: batch row
+    0 of 8, the whole sequence, all heads (fewer heads when one call would not
+    fit the budget).  `warmup` untimed calls, then timed calls: `fixed_calls`
+    if given, else as many as fit in `budget_s` (between min_calls and
+    max_calls).  Returns (layer tokens per second, seconds per call, calls,
+    heads)."""
     import numpy as np
     import torch
     import m3_synth
     import oracle
     s = m3_synth.LAYERS[LAYER]
-    # bounded sample: batch row 0, the whole sequence, all heads -- or fewer
-    # heads when the first warm-up step shows that steps + warm-up would take
-    # more than about two minutes on this host
     sub = m3_synth.shrink(s, batch=1)
-    inp = m3_synth.make_scan_inputs(sub)
-    f = {k: v.to(torch.float64).numpy() for k, v in inp.items()}
+    f = {k: v.to(torch.float64).numpy() for k, v in m3_synth.make_scan_inputs(sub).items()}
     t0 = time.perf_counter()
     oracle.scan(**f)
     first = time.perf_counter() - t0
     heads = s.nheads
-    budget_s = 120.0
-    if (args.steps + args.warmup) * first > budget_s:
-        # the oracle runs one (b, h) per thread, so a step costs whole rounds of
+    calls = fixed_calls if fixed_calls > 0 else int(min(max_calls, max(min_calls, budget_s // max(first, 1e-6))))
+    if (calls + warmup) * first > 1.5 * budget_s:
+        # the oracle runs one (b, h) per thread, so a call costs whole rounds of
         # `cores` heads: keep as many rounds as fit in the budget (at least one)
         cores = max(1, oracle.num_threads())
         rounds_all = -(-s.nheads // cores)
-        rounds = int(rounds_all * budget_s / ((args.steps + args.warmup) * first))
+        rounds = int(rounds_all * budget_s / ((calls + warmup) * first))
         heads = max(1, min(s.nheads, max(rounds, 1) * cores))
         assert s.ngroups == s.nheads          # one group per head: heads and groups slice together
         f = {k: (v[:heads] if k == "A" else np.ascontiguousarray(v[:, :, :heads])) for k, v in f.items()}
-    for _ in range(max(args.warmup - 1, 0)):
+    for _ in range(max(warmup - 1, 0)):
         oracle.scan(**f)
     t0 = time.perf_counter()
-    for _ in range(args.steps):
+    for _ in range(calls):
         oracle.scan(**f)
-    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    dt = (time.perf_counter() - t0) / max(calls, 1)
     toks = sub.batch * sub.seqlen * heads / s.nheads      # layer tokens: all heads of a token
-    val = toks / dt
+    return toks / dt, dt, calls, heads
+
+
+def oracle_sample_text(heads: int, calls: int) -> str:
+    return (f"batch row 0 of 8 ({heads} of 32 heads x 4096 tokens) per call, {calls} timed calls after "
+            "a warm-up call, scaled to layer tokens")
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return 0
+    import m3_synth
+    import oracle
+    s = m3_synth.LAYERS[LAYER]
+    val, dt, calls, heads = oracle_sample_timing(budget_s=120.0, fixed_calls=args.steps,
+                                                 warmup=max(args.warmup, 1))
     cores = oracle.num_threads()
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
@@ -199,30 +217,20 @@ def run_reference(args, rank):
             "config": {"workload": m3_synth.NAMES[LAYER], "global_batch": s.batch, "seq_len": s.seqlen,
                        "sample": f"batch row 0 of 8, {heads} of 32 heads, full L=4096 per step"},
             "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "host_cpus": os.cpu_count(),
-                             "kind": "oracle",
-                             "sample": f"1 of 8 batch rows ({heads} of 32 heads x 4096 tokens) per step, "
-                                       "scaled to layer tokens"},
+                             "kind": "oracle", "sample": oracle_sample_text(heads, calls)},
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
     return 0
 
 
 def cpu_baseline_sample():
-    """The oracle on a bounded sample of the same workload (batch rows 0-1,
-    all heads, full L), timed on this host's cores."""
-    import torch
-    import m3_synth
+    """The oracle on a bounded sample of the same workload, timed on this
+    host's cores the same way as the reference arm (warm-up call, then about
+    15 s of timed calls)."""
     import oracle
-    s = m3_synth.LAYERS[LAYER]
-    sub = m3_synth.shrink(s, batch=2)
-    inp = m3_synth.make_scan_inputs(sub)
-    f = {k: v.to(torch.float64).numpy() for k, v in inp.items()}
-    t0 = time.perf_counter()
-    oracle.scan(**f)
-    dt = time.perf_counter() - t0
-    out = {"value": sub.batch * sub.seqlen / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
-           "host_cpus": os.cpu_count(), "kind": "oracle",
-           "sample": f"2 of 8 batch rows (64 head-sequences x 4096 tokens), {dt:.1f} s wall"}
+    val, dt, calls, heads = oracle_sample_timing(budget_s=15.0)
+    out = {"value": val, "unit": "tokens/s", "cores": oracle.num_threads(), "host_cpus": os.cpu_count(),
+           "kind": "oracle", "sample": oracle_sample_text(heads, calls), "seconds_per_call": dt}
     out["single_thread"] = oracle_single_thread()
     return out
 
@@ -294,30 +302,50 @@ class Ctx:
             self.dist.destroy_process_group()
 
 
-# DRAM bytes (read + write) of one scan_tc_kernel<4,0> launch, from the ncu
-# capture of the R=4 layer at batch 2 (the main pass of a 4-segment plan):
-# 754,940,416 + 120,642,816 bytes.  Traffic grows with the (batch, head) units
-# (each is one sequence read once), so a launch over `batch` sequences moves
-# batch / 2 times this.  The capture and its command are in profiles/.
-TRAFFIC_R4_B2 = 754_940_416 + 120_642_816
-# DRAM bytes of one step_pipe_kernel launch (decode, batch 256, 32 heads,
-# R=4), from an ncu capture of that launch: 304,197,632 + 224,655,616 bytes.
-TRAFFIC_DECODE_B256 = 304_197_632 + 224_655_616
-# DRAM bytes of one rope_block_kernel launch on the R=4 layer (batch 8), from
-# an ncu capture of that launch: 2,422,795,520 + 2,379,804,160 bytes.
-TRAFFIC_ROPE_LAYER = 2_422_795_520 + 2_379_804_160
 L2_BYTES = 126 * 1024 * 1024
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum of one launch,
+# from ncu) of the dominant kernel of each measured part, keyed to what was
+# captured: the kernel, the workload and plan it ran, and a digest of the
+# kernel's sources at capture time.  A figure is reported only while the
+# built sources still have that digest and the timed launch has that
+# workload and plan; otherwise "traffic" is null and the reason is given.
+# The ncu commands are in profiles/.
+KERNEL_SOURCES = {
+    "scan_tc_kernel": ("k_scan_tc.cu", "tc_ptx.cuh", "m3_common.cuh", "m3_kernels.h"),
+    "step_pipe_kernel": ("k_step.cu", "m3_common.cuh", "m3_kernels.h"),
+    "rope_block_kernel": ("k_rope.cu", "m3_common.cuh", "m3_kernels.h"),
+}
+CAPTURES = {
+    # kernel: (workload, plan segments or None, bytes per launch, source digest)
+    "scan_tc_kernel": None,
+    "step_pipe_kernel": None,
+    "rope_block_kernel": None,
+}
 
-TRAFFIC_CURRENT = True      # the captures match the kernels now built
+
+def source_digest(kernel: str) -> str:
+    """sha256 (first 16 hex digits) of the kernel's source files, in order."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "selective_state_space_m3_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
-def measured_traffic(s, plan):
-    if plan["path"] != "tcgen05" or s.rank != 4 or s.nheads != 32 or s.seqlen != 4096:
-        return None, "no capture for this shape"
-    if not TRAFFIC_CURRENT:
-        return None, "kernel changed since the last capture"
-    return TRAFFIC_R4_B2 * s.batch / 2, "ncu dram bytes of the batch-2 capture x batch/2"
+def captured_traffic(kernel: str, workload: str, segments=None, captures=None):
+    """(bytes per launch, source) of the capture that matches, else (None, why)."""
+    cap = (CAPTURES if captures is None else captures).get(kernel)
+    if cap is None:
+        return None, "no ncu capture of this kernel on the current sources"
+    c_work, c_seg, c_bytes, c_digest = cap
+    if c_work != workload or (c_seg is not None and c_seg != segments):
+        return None, f"capture is of {c_work} (segments {c_seg}), not of this launch"
+    digest = source_digest(kernel)
+    if digest != c_digest:
+        return None, f"kernel sources changed since the capture (digest {digest}, captured {c_digest})"
+    return c_bytes, f"ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch, sources {digest}"
 
 
 def throughput(world: int, tokens_per_rank: int, steps: int, total_ms: float) -> float:
@@ -416,14 +444,16 @@ def run_prefill(cx, line):
                      "tokens_per_s": throughput(cx.world, tokens, args.steps, u_ms),
                      "l2": "not flushed: inputs stay in L2 between launches"}
 
-    aflops = algorithmic_flops(s)
+    aflops = algorithmic_flops(s, plan["chunk_used"])
     achieved_gbs = abytes / (per_launch_ms / 1e3) / 1e9
     tflops = aflops / (per_launch_ms / 1e3) / 1e12
-    traffic, traffic_src = measured_traffic(s, plan)
+    workload = m3_synth.NAMES[args.layer] if args.batch <= 0 else m3_synth.NAMES[args.layer] + f"_batch{s.batch}"
+    traffic, traffic_src = captured_traffic("scan_tc_kernel", workload, plan["segments"])
+    if plan["launches"] != 1:
+        traffic, traffic_src = None, "plan has several launches; capture covers one kernel launch"
     line.update({
         "value": value, "ms_per_step": ms_per_step,
-        "config": {"workload": m3_synth.NAMES[args.layer] if args.batch <= 0 else
-                   m3_synth.NAMES[args.layer] + f"_batch{s.batch}",
+        "config": {"workload": workload,
                    "global_batch": s.batch * cx.world,
                    "seq_len": s.seqlen, "nheads": s.nheads, "headdim": s.headdim, "dstate": s.dstate,
                    "rank": s.rank, "chunk": s.chunk,
@@ -443,6 +473,86 @@ def run_prefill(cx, line):
     if unflushed is not None:
         line["unflushed"] = unflushed
     return dict(s=s, host=host, dev=dev, y=y, fin=fin, step=step, tokens=tokens)
+
+
+def run_layer(cx, name):
+    """m3_scan_fwd on another prefill workload (the SISO layer, or the
+    long-context SISO layer), timed like the headline: CUDA events around
+    each call on the launching stream, L2 flushed before each call when the
+    inputs are smaller than twice the L2.  Each call is timed twice: launched
+    eagerly, and captured once in a CUDA graph and replayed (the plan's
+    launches then follow each other on the device with no host in between);
+    the graph figure is the object's ms_per_call."""
+    import torch
+    import m3_synth
+    import selective_state_space_m3_b200 as m3
+    args, pk, stream = cx.args, cx.pk, cx.stream
+    s = rank_shape(name, cx.rank)
+    dev = {k: v.cuda() for k, v in m3_synth.make_scan_inputs(s).items()}
+    io = m3.M3_BF16 if s.dtype == "bf16" else m3.M3_F32
+    d = m3.Dims(s.batch, s.seqlen, s.nheads, s.ngroups, s.headdim, s.dstate, s.rank, s.chunk, io)
+    plan = m3.m3_scan_plan(d)
+    y = torch.empty_like(dev["x"])
+    ws = torch.zeros(m3.m3_scan_workspace_size(d), dtype=torch.uint8, device="cuda")
+    fin = m3.Carry(torch.empty(s.batch, s.nheads, s.dstate, s.headdim, device="cuda"),
+                   torch.empty(s.batch, s.nheads, s.rank, s.dstate, device="cuda", dtype=dev["x"].dtype),
+                   torch.empty(s.batch, s.nheads, s.rank, s.headdim, device="cuda", dtype=dev["x"].dtype))
+    abytes = algorithmic_bytes(dev, y, fin)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda") if abytes < 2 * L2_BYTES else None
+
+    def call(st):
+        m3.m3_scan_fwd(d, dev["x"], dev["B"], dev["C"], dev["dt"], dev["A"], dev["lam"], dev["theta"],
+                       y, ws, final_state=fin, stream=st)
+
+    for _ in range(max(3, args.warmup)):
+        call(stream)
+    torch.cuda.synchronize()
+    assert m3.m3_device_status(ws) == m3.M3_OK
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call(torch.cuda.current_stream())
+    g.replay()
+    torch.cuda.synchronize()
+    n = max(5, min(args.steps, 20))
+
+    def timed(fn):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        cx.barrier()
+        torch.cuda.synchronize()
+        for e0, e1 in ev:
+            if flush is not None:
+                flush.zero_()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        cx.barrier()
+        return cx.max_over_ranks(statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev))
+
+    with ClockSampler(cx.local) as clk:
+        clk.active = True
+        eager_ms = timed(lambda: call(stream))
+        graph_ms = timed(g.replay)
+        clk.active = False
+    assert m3.m3_device_status(ws) == m3.M3_OK
+    del g
+    gbs = abytes / (graph_ms / 1e3) / 1e9
+    tflops = algorithmic_flops(s, plan["chunk_used"]) / (graph_ms / 1e3) / 1e12
+    out = {"workload": m3_synth.NAMES[name], "ms_per_call": graph_ms, "eager_ms_per_call": eager_ms,
+           "tokens_per_s": cx.world * s.batch * s.seqlen / (graph_ms / 1e3),
+           "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                        "frac": gbs / pk["hbm"], "peak_source": pk["src"], "algorithmic_bytes_per_launch": abytes,
+                        "traffic": None, "traffic_source": "no ncu capture of this workload on the current sources",
+                        "kernel": "m3_scan_fwd (whole call: %d launch%s, CUDA graph)" % (
+                            plan["launches"], "" if plan["launches"] == 1 else "es"),
+                        "tensor_tflops": tflops, "tensor_frac_of_bf16_peak": tflops / pk["bf16"]},
+           "plan": {"path": plan["path"], "segments": plan["segments"], "launches": plan["launches"],
+                    "chunk_used": plan["chunk_used"]},
+           "l2": ("inputs %.2f GB >> 126 MB L2; no flush" % (abytes / 1e9)) if flush is None
+           else "L2 flushed (252 MB write) before every timed call",
+           "clocks": clk.summary(), "gpu_launches": 2 * n * plan["launches"], "calls_timed": n}
+    del flush, ws, dev
+    return out
 
 
 def run_e2e(cx, line, pf):
@@ -509,12 +619,12 @@ def run_rope(cx, line, pf):
     nbytes = sum(dev[k].numel() * dev[k].element_size() for k in ("B", "C", "dt", "theta"))
     nbytes += sum(v.numel() * v.element_size() for v in (Bo, Co, ph))
     gbs = nbytes / (ms / 1e3) / 1e9
+    rope_traffic, rope_src = captured_traffic("rope_block_kernel", line["config"]["workload"])
     line["rope"] = {"workload": "rope_bc_" + line["config"]["workload"], "ms_per_call": ms,
                     "tokens_per_s": cx.world * s.batch * s.seqlen / (ms / 1e3),
                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
                                  "frac": gbs / pk["hbm"], "algorithmic_bytes_per_launch": nbytes,
-                                 "traffic": TRAFFIC_ROPE_LAYER if (TRAFFIC_CURRENT and s.batch == 8 and
-                                                                   s.rank == 4 and s.seqlen == 4096) else None},
+                                 "traffic": rope_traffic, "traffic_source": rope_src},
                     "gpu_launches": n, "l2": "inputs and outputs %.1f GB >> L2; no flush" % (nbytes / 1e9)}
     del Bo, Co, ph
 
@@ -746,13 +856,14 @@ def run_decode(cx, line, pf):
     step_bytes = (2 * state.h.numel() * 4 + 2 * (state.prev_B.numel() + state.prev_x.numel()) * 2 +
                   sum(v.numel() * v.element_size() for v in t0.values()) + yd.numel() * 2 + Ad.numel() * 4)
     gbs = step_bytes / (per_step_us * 1e-6) / 1e9
-    line["decode"] = {"workload": m3_synth.NAMES["decode"] if dec.batch == 256 else f"decode_b{dec.batch}",
+    dec_work = m3_synth.NAMES["decode"] if dec.batch == 256 else f"decode_b{dec.batch}"
+    dec_traffic, dec_src = captured_traffic("step_pipe_kernel", dec_work)
+    line["decode"] = {"workload": dec_work,
                       "tokens_per_s": cx.world * dec.batch / (per_step_us * 1e-6),
                       "us_per_step": per_step_us, "steps_timed": reps_t * S,
                       "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
                                    "frac": gbs / pk["hbm"], "algorithmic_bytes_per_launch": step_bytes,
-                                   "traffic": TRAFFIC_DECODE_B256 if (dec.batch == 256 and TRAFFIC_CURRENT)
-                                   else None},
+                                   "traffic": dec_traffic, "traffic_source": dec_src},
                       "gpu_launches": reps_t * S, "clocks": clk2.summary(),
                       "carry": "prefill final state" if pf is not None and args.layer == LAYER
                       else "seeded random",
@@ -785,6 +896,9 @@ def main():
             run_bwd(cx, line, pf)
         if args.phase:
             run_phase(cx, line, pf)
+        if args.layer == LAYER and not args.no_layers:
+            # the other two prefill workloads, each in its own object
+            line["layers"] = {n: run_layer(cx, n) for n in ("siso_layer", "long_siso")}
     if args.workload in ("both", "decode") and not args.no_decode:
         run_decode(cx, line, pf)
     if args.workload == "both" and not args.no_variants:

@@ -95,7 +95,12 @@ typedef struct m3_dims {
     int headdim;    /* P >= 1                                                  */
     int dstate;     /* N >= 2, even (N/2 rotary pairs)                         */
     int rank;       /* R >= 1 (1 = SISO)                                       */
-    int chunk;      /* Q >= 1: chunk length of the chunked prefill            */
+    int chunk;      /* Q >= 1: chunk length of the chunked prefill on the
+                     * float32 SIMT path (shortened to fit shared memory);
+                     * the tcgen05 path ignores it and uses chunks of 128/R
+                     * tokens (one 128-row tile).  The result is the same
+                     * recurrence either way; m3_scan_plan reports the
+                     * chunk actually used.                                   */
     int io_dtype;   /* m3_dtype of x, B, C, y, prev_B, prev_x                  */
 } m3_dims;
 
@@ -325,7 +330,9 @@ m3_status m3_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void
  * launch.  The call itself allocates nothing (no cudaMalloc, no cudaFree).
  * The first call on each device looks up the array's device address with
  * that device current and caches it; make that first call before any stream
- * capture.  All calls share the one array and it keeps the last call's
+ * capture.  The cached address belongs to the device's primary context:
+ * after cudaDeviceReset it is stale, so call m3_static_forget_device with
+ * that device current before the next m3_scan_fwd_static on it.  All calls share the one array and it keeps the last call's
  * contents (each call clears the status word it needs zeroed), so calls that
  * overlap on the GPU -- on different streams, or on different host threads --
  * race and must be serialised by the caller.  On-chip wait timeouts are
@@ -339,6 +346,13 @@ m3_status m3_scan_fwd_static(const m3_dims* dims,
                              const m3_carry* init,
                              void* y, m3_carry* final_state,
                              void* stream);
+
+/* Drops the cached device address of the static scratch array for the
+ * current device (needed only after cudaDeviceReset: the next
+ * m3_scan_fwd_static looks it up again).  Must not overlap a running
+ * m3_scan_fwd_static on that device.  Host-only; M3_ERR_CUDA if no device
+ * is current. */
+m3_status m3_static_forget_device(void);
 
 /* Static, never NULL. */
 const char* m3_status_string(m3_status status);

@@ -58,6 +58,8 @@ def _load():
     lib.m3_scan_plan.restype = I
     lib.m3_scan_fwd_static.argtypes = [D, V, V, V, V, V, V, V, C, V, C, V]
     lib.m3_scan_fwd_static.restype = I
+    lib.m3_static_forget_device.argtypes = []
+    lib.m3_static_forget_device.restype = I
     lib.m3_selftest_bounded_wait.argtypes = [V, S, V]
     lib.m3_selftest_bounded_wait.restype = I
     lib.m3_scan_bwd_workspace_size.argtypes = [D, ctypes.POINTER(S)]
@@ -84,7 +86,7 @@ _lib = _load()
 # every symbol include/m3.h declares (checked by the CPU test suite)
 ABI_SYMBOLS = ("m3_scan_workspace_size", "m3_scan_fwd", "m3_step", "m3_rope_bc",
                "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_scan_fwd_static",
-               "m3_scan_bwd_workspace_size", "m3_scan_bwd", "m3_scan_phase_workspace_size",
+               "m3_static_forget_device", "m3_scan_bwd_workspace_size", "m3_scan_bwd", "m3_scan_phase_workspace_size",
                "m3_scan_fwd_phase", "m3_scan_fwd_damped", "m3_scan_fwd_reflect", "m3_status_string")
 
 
@@ -192,6 +194,12 @@ def m3_scan_fwd_static(dims: Dims, x, B, C, dt, A, lam, theta, y,
                                  _ptr(theta), ctypes.byref(ci) if ci is not None else None, _ptr(y),
                                  ctypes.byref(cf) if cf is not None else None, _stream(stream))
     _check(st, "m3_scan_fwd_static")
+
+
+def m3_static_forget_device() -> None:
+    """Drop the static scratch array's cached address for the current device
+    (only needed after a device reset)."""
+    _check(_lib.m3_static_forget_device(), "m3_static_forget_device")
 
 
 def m3_step(dims: Dims, state: Carry, x, B, C, dt, A, lam, theta, y, stream=None) -> None:
@@ -317,7 +325,8 @@ def raw_lib():
 
 
 __all__ = ["Dims", "Carry", "M3Error", "m3_scan_workspace_size", "m3_scan_fwd", "m3_step",
-           "m3_rope_bc", "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_scan_fwd_static", "m3_scan_bwd_workspace_size", "m3_scan_bwd", "m3_status_string",
+           "m3_rope_bc", "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_scan_fwd_static",
+           "m3_static_forget_device", "m3_scan_bwd_workspace_size", "m3_scan_bwd", "m3_status_string",
            "m3_scan_phase_workspace_size", "m3_scan_fwd_phase", "m3_scan_fwd_damped", "m3_scan_fwd_reflect",
            "M3_DAMP_UNDER", "M3_DAMP_CRITICAL", "M3_DAMP_OVER", "io_dtype_of", "ABI_SYMBOLS",
            "M3_F32", "M3_BF16", "raw_lib", "LIB_PATH"]

@@ -20,8 +20,8 @@
 
 namespace {
 
-// Largest workspace the static variant can serve (see M3_STATIC_SCRATCH_BYTES).
-constexpr size_t kScratchBytes = 32u << 20;
+// Largest workspace the static variant can serve: the public limit itself.
+constexpr size_t kScratchBytes = M3_STATIC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_m3_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -43,6 +43,14 @@ m3_status scratch_address(void** out) {
 }
 
 }  // namespace
+
+extern "C" m3_status m3_static_forget_device(void) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return M3_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    g_addr[dev] = nullptr;
+    return M3_OK;
+}
 
 extern "C" m3_status m3_scan_fwd_static(const m3_dims* dims, const void* x, const void* B, const void* C,
                                         const float* dt, const float* A, const float* lambda,

@@ -77,16 +77,24 @@ def test_single_rank_context_needs_no_process_group():
         os.environ.update(env)
 
 
-def test_traffic_is_reported_only_for_the_captured_shape():
-    import m3_synth
-    s = m3_synth.LAYERS[bench.LAYER]
-    t, _ = bench.measured_traffic(s, {"path": "tcgen05"})
-    if bench.TRAFFIC_CURRENT:
-        assert t == pytest.approx(bench.TRAFFIC_R4_B2 * 4)
-    else:
-        assert t is None
-    assert bench.measured_traffic(s, {"path": "simt"})[0] is None
-    assert bench.measured_traffic(m3_synth.LONG_SISO, {"path": "tcgen05"})[0] is None
+def test_traffic_is_reported_only_for_the_captured_sources_and_plan():
+    d = bench.source_digest("scan_tc_kernel")
+    assert len(d) == 16 and d == bench.source_digest("scan_tc_kernel")
+    assert d != bench.source_digest("step_pipe_kernel")
+    caps = {"scan_tc_kernel": ("mimo_r4_layer", 1, 123, d)}
+    t, src = bench.captured_traffic("scan_tc_kernel", "mimo_r4_layer", 1, captures=caps)
+    assert t == 123 and d in src
+    # another plan, another workload, other sources, no capture: no figure
+    assert bench.captured_traffic("scan_tc_kernel", "mimo_r4_layer", 4, captures=caps)[0] is None
+    assert bench.captured_traffic("scan_tc_kernel", "long_siso", 1, captures=caps)[0] is None
+    stale = {"scan_tc_kernel": ("mimo_r4_layer", 1, 123, "0" * 16)}
+    t, why = bench.captured_traffic("scan_tc_kernel", "mimo_r4_layer", 1, captures=stale)
+    assert t is None and "changed" in why
+    assert bench.captured_traffic("step_pipe_kernel", "decode", captures=caps)[0] is None
+    # every committed capture names a known kernel and a digest of its sources
+    for k, cap in bench.CAPTURES.items():
+        assert k in bench.KERNEL_SOURCES
+        assert cap is None or (len(cap) == 4 and len(cap[3]) == 16)
 
 
 def test_bench_defaults_are_one_gpu_and_minutes_of_work(monkeypatch):
@@ -131,4 +139,7 @@ def test_prefill_roofline_arithmetic():
     carry = b * H * (N * P * 4 + R * N * 2 + R * P * 2)
     got = bench.algorithmic_bytes(t, m(b, L, H, R, P, dtype=bf), fin)
     assert got == 3336 * token_heads + 4 * H + carry == 3_506_831_488
-    assert bench.algorithmic_flops(s) == 330_752 * token_heads
+    assert bench.algorithmic_flops(s, 64) == 330_752 * token_heads
+    # the tcgen05 path's chunk at R = 4 (one 128-row tile = 32 tokens):
+    # 33 * 16 * 192 + 4 * 4 * 128 * 64 = 232,448 FLOP per token-head
+    assert bench.algorithmic_flops(s, 32) == 232_448 * token_heads

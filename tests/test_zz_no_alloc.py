@@ -69,3 +69,10 @@ def test_static_scratch_rejects_sizes_beyond_its_limit():
     with pytest.raises(m3.M3Error) as e:
         m3.m3_scan_fwd_static(d, z, z, z, z, z, z, z, z)
     assert e.value.status == m3.M3_ERR_WORKSPACE
+
+
+def test_forgetting_the_cached_address_looks_it_up_again():
+    # what a caller does after a device reset; here the context is unchanged,
+    # so the looked-up address must simply serve the next call as before
+    m3.m3_static_forget_device()
+    _both(m3_synth.ScanShape(1, 900, 2, 2, 64, 128, 4, 64, "bf16", 0.0, 84), 84)
