@@ -60,8 +60,11 @@ constexpr int OFF_C = 32768;      // 32 KB: C~, later P
 constexpr int OFF_X = 65536;      // 16 KB: X
 constexpr int OFF_S = 81920;      // 16 KB: S_bf (rows n, 64 p)
 constexpr int OFF_MISC = 98304;
-constexpr int MISC_BYTES = 9216;
-constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;   // + alignment slack
+constexpr int MISC_BYTES = 10496;
+// dynamic shared memory of a launch (+ alignment slack); R >= 4 leaves the
+// second parity of the R < 4 tables out, which keeps more of the SM's L1
+template <int R>
+constexpr int smem_bytes() { return OFF_MISC + (R >= 4 ? 9216 : MISC_BYTES) + 1024; }
 
 struct Misc {
     uint64_t bar[8];              // load, ops, g, bw, p, y, free, spare
@@ -72,12 +75,24 @@ struct Misc {
     float2 qs[2][kNE][32];        // per token group: phase increments of pairs (2i, 2i+1), by tile parity
     union {
         float msk[32 * 36];       // R >= 4: decay mask per (token, token), rows padded
-        float cs[6][128];         // R < 4: c and gamma times e^{a_ref - a}, a_ref per block; a, gamma, c
+        float cs[2][6][128];      // R < 4, by tile parity (the next tile's are made one tile
+                                  // ahead): c and gamma times e^{a_ref - a}, a_ref per block; a, gamma, c
     } u;
 };
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region too small");
+static_assert(offsetof(Misc, u) + sizeof(float) * 32 * 36 <= 9216, "misc region of R >= 4 too small");
 
 enum { BAR_LOAD = 0, BAR_OPS, BAR_G, BAR_BW, BAR_P, BAR_Y, BAR_DRAIN };
+
+// per-tile scalars of a worker thread, made by the coefficient stage
+struct TileCoef {
+    float a2_last;      // log2 decay over the tile
+    float a2_tr;        // log2 decay up to the token of the thread's tile row
+    float cf_tr;        // pending weight c of that token (main pass); for
+                        // short tiles both hold the lane's own token's
+    float dsl;          // dt of token 32 gsl + lane (the warp's phase-pass source)
+    float a2sl, cfsl;   // summary pass: log2 decay and c of that token
+};
 
 // ------------------------------------------------------------ PTX wrappers --
 using namespace ptx;
@@ -213,8 +228,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     // 2l and 2l+1 (one 8-byte word of a B / C row).
     constexpr int NT = (T + 31) / 32;
     constexpr int TE = T / kNE;
+    constexpr bool kAhead = (R <= 2);        // coefficient stage one tile ahead
+    static_assert(kAhead || NT == 1, "short tiles fit one 32-token slice");
     constexpr bool kThReg = (TE <= 4);        // theta of the group held in registers for the tile
-    constexpr int kUnrollTE = kThReg ? TE : 4;
+    constexpr int kBatchTE = kThReg ? TE : 8;  // theta loads of the rotation pass issued together
     constexpr unsigned kFull = 0xffffffffu;
     constexpr float kLn2 = 0.69314718055994531f;
     const float A2 = Ah * kLog2e;             // decay per unit dt, log2 units
@@ -246,6 +263,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     auto theta_ld = [&](int t0n, int qcn, int kk) -> float2 {   // theta of pairs (2 lane, 2 lane + 1), raw
         const int t = min(g0 + kk, qcn - 1);
         return __ldg(reinterpret_cast<const float2*>(q.theta + (((size_t)b * L + t0n + t) * G + g) * (kN / 2)) + lane);
+    };
+    auto prefetch_tok = [&](int kn) {         // L2 prefetch of a tile's dt / lambda (and the token after it)
+        const int t0n = tok0 + kn * T;
+        const int qn = min(T + 1, L - t0n);
+        for (int t = wk; t < qn; t += kWorkers) {
+            const size_t o = ((size_t)b * L + t0n + t) * H + h;
+            prefetch_l2(q.dt + o);
+            prefetch_l2(q.lam + o);
+        }
     };
     auto prefetch_theta = [&](int kn) {       // L2 prefetch of a tile's theta rows (256 B per token)
         const int t0n = tok0 + kn * T;
@@ -282,10 +308,141 @@ __global__ void __launch_bounds__(kThreads, 2)
     float y_ea = 0.f;                         // e^{a_t} of this thread's row in that tile
     float2 carry = make_float2(0.f, 0.f);     // cumulative phase of pairs 2 lane, 2 lane + 1 (reduced)
     float seg_a = 0.f;                        // log decay of the segment so far
+    // ---- coefficient stage of tile kn (run one tile ahead, while the
+    // previous tile's MMAs are in flight): per-token coefficients from the
+    // raw dt / lambda loads of tile kn, the mask tables of parity kn & 1, and
+    // the scalars the tile's own passes need later
+    auto coef_stage = [&](int kn) -> TileCoef {
+        const int t0n = tok0 + kn * T;
+        const int qcn = min(T, tok1 - t0n);
+        const int pb = kn & 1;
+            // this tile's inputs; tokens past the end count as dt = 0, lambda = 1
+            float dtv[NT], lmv[NT];
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                const bool in = lane + 32 * j < qcn;
+                dtv[j] = in ? dt_n[j] : 0.f;
+                lmv[j] = in ? lam_n[j] : 1.f;
+            }
+            const bool nx_in = t0n + qcn < L;
+            const float dx = nx_in ? dx_n : 0.f, lx = nx_in ? lx_n : 1.f;
+            // coefficients of every token (log2 units): a2 = inclusive scan of
+            // dt A, gamma = lambda dt, c = gamma + (1 - lambda') dt' with ' the
+            // next token (past the tile: the token after it, zero past the end)
+            float a2v[NT], gmv[NT], cfv[NT];
+            float a2_last;
+            {
+                float run = 0.f;
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    float v = dtv[j] * A2;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const float u = __shfl_up_sync(kFull, v, o);
+                        if (lane >= o) v += u;
+                    }
+                    a2v[j] = v + run;
+                    run = __shfl_sync(kFull, a2v[j], 31);
+                }
+                a2_last = run;
+                float up[NT];
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    gmv[j] = lmv[j] * dtv[j];
+                    up[j] = (1.f - lmv[j]) * dtv[j];
+                }
+                const float ux = (1.f - lx) * dx;
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    float nx = __shfl_down_sync(kFull, up[j], 1);
+                    if (j + 1 < NT) {
+                        const float first = __shfl_sync(kFull, up[j + 1 < NT ? j + 1 : j], 0);
+                        if (lane == 31) nx = first;
+                    }
+                    if (lane + 32 * j + 1 == T) nx = ux;
+                    cfv[j] = gmv[j] + nx;
+                }
+            }
+            if (!SUMMARY && R >= 4) {
+                // decay mask per (token t, token u) of the tile, shared by the R x R
+                // rank block: e^{a_t - a_u} (gamma_u if u == t, c_u if u < t), 0 above
+                constexpr int LD = T + 4;
+#pragma unroll
+                for (int e = wk; e < T * T; e += kWorkers) {
+                    const int t = e / T, u = e % T;
+                    const float at = __shfl_sync(kFull, a2v[0], t), au = __shfl_sync(kFull, a2v[0], u);
+                    const float gu = __shfl_sync(kFull, gmv[0], u), cu = __shfl_sync(kFull, cfv[0], u);
+                    m->u.msk[t * LD + u] = (u <= t) ? exp2f(at - au) * (u == t ? gu : cu) : 0.f;
+                }
+            }
+            if (!SUMMARY && R < 4 && qe == 0) {
+                // long tiles: the mask of a 16-column block (GT tokens) factors as
+                // e^{a_t - a_ref} x e^{a_ref - a_u} (gamma_u or c_u), a_ref = a at the
+                // block's first token, whenever the block's own decay is small
+                // enough that the second factor cannot overflow; such blocks get
+                // a_ref, the others +inf (element-wise path)
+                constexpr int GT = 16 / R;
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    const int t = lane + 32 * j;
+                    const float aref = __shfl_sync(kFull, a2v[j], lane & ~(GT - 1));
+                    const float aend = __shfl_sync(kFull, a2v[j], lane | (GT - 1));
+                    const bool ok = aref - aend <= 60.f;
+                    const float colf = exp2f(aref - a2v[j]);
+                    m->u.cs[pb][0][t] = ok ? cfv[j] * colf : 0.f;
+                    m->u.cs[pb][1][t] = ok ? gmv[j] * colf : 0.f;
+                    if ((lane & (GT - 1)) == 0) m->u.cs[pb][2][t / GT] = ok ? aref : __int_as_float(0x7f800000);
+                    m->u.cs[pb][3][t] = a2v[j];
+                    m->u.cs[pb][4][t] = gmv[j];
+                    m->u.cs[pb][5][t] = cfv[j];
+                }
+            }
+        TileCoef c;
+        c.a2_last = a2_last;
+        // (short tiles, one slice: the lane's own a and c; the row's are
+        // fetched where they are used)
+        c.a2_tr = kAhead ? __shfl_sync(kFull, pick<NT>(a2v, rsl), rln) : a2v[0];
+        c.cf_tr = SUMMARY ? 0.f : (kAhead ? __shfl_sync(kFull, pick<NT>(cfv, rsl), rln) : cfv[0]);
+        c.dsl = pick<NT>(dtv, gsl);
+        c.a2sl = SUMMARY ? pick<NT>(a2v, gsl) : 0.f;
+        c.cfsl = SUMMARY ? pick<NT>(cfv, gsl) : 0.f;
+        return c;
+    };
+    // ---- phase pass 1 of tile kn: this group's increments of pairs
+    // (2 lane, 2 lane + 1), published in qs[kn & 1]; thf(kk) gives the theta
+    // of token g0 + kk (theta past the tile's end meets dt = 0)
+    auto pass1_stage = [&](int kn, float dsl, auto&& thf) {
+        // theta loads issued in batches of up to 8 tokens before their use
+        constexpr int KB = TE < 8 ? TE : 8;
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int k0 = 0; k0 < TE; k0 += KB) {
+            float2 thv[KB];
+#pragma unroll
+            for (int kk = 0; kk < KB; ++kk) thv[kk] = thf(k0 + kk);
+#pragma unroll
+            for (int kk = 0; kk < KB; ++kk) {
+                const float d = __shfl_sync(kFull, dsl, gln + k0 + kk);
+                acc.x = fmaf(d, thv[kk].x, acc.x);
+                acc.y = fmaf(d, thv[kk].y, acc.y);
+            }
+        }
+        m->qs[kn & 1][qe][lane] = acc;
+    };
+    auto pass1_ahead = [&](int kn, float dsl) {   // theta straight from memory (L2)
+        const int t0n = tok0 + kn * T;
+        const int qcn = min(T, tok1 - t0n);
+        pass1_stage(kn, dsl, [&](int kk) { return theta_ld(t0n, qcn, kk); });
+    };
+    TileCoef cur = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (warp > 0 && ntiles > 0) {
         load_tok(0);
         prefetch_theta(0);
         if (ntiles > 1) prefetch_theta(1);
+        if (kAhead) {
+            cur = coef_stage(0);
+            pass1_ahead(0, cur.dsl);
+        }
     }
 
     uint32_t pending_load = 0;   // control lane: a TMA load is in flight
@@ -381,16 +538,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
 
         // ---------------------------------------------------------- workers
-        // this tile's inputs; tokens past the end count as dt = 0, lambda = 1
-        float dtv[NT], lmv[NT];
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-            const bool in = lane + 32 * j < qc;
-            dtv[j] = in ? dt_n[j] : 0.f;
-            lmv[j] = in ? lam_n[j] : 1.f;
-        }
-        const bool nx_in = t0 + qc < L;
-        const float dx = nx_in ? dx_n : 0.f, lx = nx_in ? lx_n : 1.f;
+        // Long tiles (R <= 2): tile k's coefficients (cur), mask tables and
+        // phase increments were made one tile ahead, in the previous tile's
+        // MMA wait; the next tile's dt / lambda go to L2 now and are loaded
+        // once this tile's MMAs are issued.  Short tiles (R >= 4) make them
+        // here: their MMA waits are too short to hide the stage (measured).
+        if (kAhead && k + 1 < ntiles) prefetch_tok(k + 1);
         // theta of tokens g0 + kk (zero past the end): short groups load it
         // here, ahead of its first use (L2 hits, prefetched two tiles ahead);
         // long groups reload it where it is used
@@ -404,96 +557,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             const float2 v = kThReg ? th[kThReg ? kk : 0] : theta_ld(t0, qc, kk);
             return (g0 + kk < qc) ? v : make_float2(0.f, 0.f);
         };
-        // coefficients of every token (log2 units): a2 = inclusive scan of
-        // dt A, gamma = lambda dt, c = gamma + (1 - lambda') dt' with ' the
-        // next token (past the tile: the token after it, zero past the end)
-        float a2v[NT], gmv[NT], cfv[NT];
-        float a2_last;
-        {
-            float run = 0.f;
-#pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                float v = dtv[j] * A2;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float u = __shfl_up_sync(kFull, v, o);
-                    if (lane >= o) v += u;
-                }
-                a2v[j] = v + run;
-                run = __shfl_sync(kFull, a2v[j], 31);
-            }
-            a2_last = run;
-            float up[NT];
-#pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                gmv[j] = lmv[j] * dtv[j];
-                up[j] = (1.f - lmv[j]) * dtv[j];
-            }
-            const float ux = (1.f - lx) * dx;
-#pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                float nx = __shfl_down_sync(kFull, up[j], 1);
-                if (j + 1 < NT) {
-                    const float first = __shfl_sync(kFull, up[j + 1 < NT ? j + 1 : j], 0);
-                    if (lane == 31) nx = first;
-                }
-                if (lane + 32 * j + 1 == T) nx = ux;
-                cfv[j] = gmv[j] + nx;
-            }
-        }
-        if (!SUMMARY && R >= 4) {
-            // decay mask per (token t, token u) of the tile, shared by the R x R
-            // rank block: e^{a_t - a_u} (gamma_u if u == t, c_u if u < t), 0 above
-            constexpr int LD = T + 4;
-#pragma unroll
-            for (int e = wk; e < T * T; e += kWorkers) {
-                const int t = e / T, u = e % T;
-                const float at = __shfl_sync(kFull, a2v[0], t), au = __shfl_sync(kFull, a2v[0], u);
-                const float gu = __shfl_sync(kFull, gmv[0], u), cu = __shfl_sync(kFull, cfv[0], u);
-                m->u.msk[t * LD + u] = (u <= t) ? exp2f(at - au) * (u == t ? gu : cu) : 0.f;
-            }
-        }
-        if (!SUMMARY && R < 4 && qe == 0) {
-            // long tiles: the mask of a 16-column block (GT tokens) factors as
-            // e^{a_t - a_ref} x e^{a_ref - a_u} (gamma_u or c_u), a_ref = a at the
-            // block's first token, whenever the block's own decay is small
-            // enough that the second factor cannot overflow; such blocks get
-            // a_ref, the others +inf (element-wise path)
-            constexpr int GT = 16 / R;
-#pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                const int t = lane + 32 * j;
-                const float aref = __shfl_sync(kFull, a2v[j], lane & ~(GT - 1));
-                const float aend = __shfl_sync(kFull, a2v[j], lane | (GT - 1));
-                const bool ok = aref - aend <= 60.f;
-                const float colf = exp2f(aref - a2v[j]);
-                m->u.cs[0][t] = ok ? cfv[j] * colf : 0.f;
-                m->u.cs[1][t] = ok ? gmv[j] * colf : 0.f;
-                if ((lane & (GT - 1)) == 0) m->u.cs[2][t / GT] = ok ? aref : __int_as_float(0x7f800000);
-                m->u.cs[3][t] = a2v[j];
-                m->u.cs[4][t] = gmv[j];
-                m->u.cs[5][t] = cfv[j];
-            }
-        }
-        // phase pass 1: this group's increments of pairs (2 lane, 2 lane + 1)
-        const float dsl = pick<NT>(dtv, gsl);
-        {
-            // theta loads issued in batches of up to 8 tokens before their use
-            constexpr int KB = TE < 8 ? TE : 8;
-            float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int k0 = 0; k0 < TE; k0 += KB) {
-                float2 thv[KB];
-#pragma unroll
-                for (int kk = 0; kk < KB; ++kk) thv[kk] = th_at(k0 + kk);
-#pragma unroll
-                for (int kk = 0; kk < KB; ++kk) {
-                    const float d = __shfl_sync(kFull, dsl, gln + k0 + kk);
-                    acc.x = fmaf(d, thv[kk].x, acc.x);
-                    acc.y = fmaf(d, thv[kk].y, acc.y);
-                }
-            }
-            m->qs[par][qe][lane] = acc;
+        if (!kAhead) {
+            cur = coef_stage(k);
+            pass1_stage(k, cur.dsl, th_at);
         }
         // the previous tile's output, while this tile's TMA load lands
         if (!SUMMARY && y_tile >= 0) {
@@ -503,6 +569,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_wait(&m->bar[BAR_LOAD], par, m, status, 10);
         // one barrier per tile: publishes qs and msk; all workers agree to stop
         if (workers_any(*(volatile int*)&m->abort_flag)) break;
+        // the shared base as an opaque value produced after the barrier: the
+        // rotation's loads take their addresses from it, so they cannot be
+        // moved above the tile's arrival, while they may be hoisted above the
+        // pass's own stores (which never touch the same bytes)
+        uint32_t sb_ld = sbase;
+        asm volatile("" : "+r"(sb_ld));
         float2 ph = carry;
         {
             float2 tot = make_float2(0.f, 0.f);
@@ -525,47 +597,52 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int chunk = (lane & 15) >> 1;
             const uint32_t inb = (uint32_t)(lane & 1) * 8u;
             ph = make_float2(wrap_pi_f(ph.x), wrap_pi_f(ph.y));
-            const float a2sl = SUMMARY ? pick<NT>(a2v, gsl) : 0.f;
-            const float cfsl = SUMMARY ? pick<NT>(cfv, gsl) : 0.f;
-#pragma unroll(kUnrollTE)
-            for (int kk = 0; kk < TE; ++kk) {
-                const int t = g0 + kk;
-                const float d = __shfl_sync(kFull, dsl, gln + kk);
-                const float2 tk = th_at(kk);
-                ph.x = fmaf(d, tk.x, ph.x);
-                ph.y = fmaf(d, tk.y, ph.y);
-                float s0, k0, s1, k1;
-                __sincosf(ph.x, &s0, &k0);
-                __sincosf(ph.y, &s1, &k1);
-                if (SUMMARY) {
-                    // the summary pass needs only w_t B~_t: fold w into the rotation
-                    const float wt = exp2f(a2_last - __shfl_sync(kFull, a2sl, gln + kk)) *
-                                     __shfl_sync(kFull, cfsl, gln + kk);
-                    s0 *= wt; k0 *= wt; s1 *= wt; k1 *= wt;
-                }
-                const uint32_t cc0 = pack_bf16x2(k0, k0), sn0 = pack_bf16x2(s0, -s0);
-                const uint32_t cc1 = pack_bf16x2(k1, k1), sn1 = pack_bf16x2(s1, -s1);
-                // all loads of the token's rows first, then the stores: the
-                // compiler cannot tell that the swizzled rows do not overlap,
-                // so interleaving would serialise each row behind the last store
-                constexpr int NM = SUMMARY ? 1 : 2;      // B, and C in the main pass
-                uint2 vv[NM][R];
+            const float dsl = cur.dsl, a2sl = cur.a2sl, cfsl = cur.cfsl, a2_last = cur.a2_last;
+#pragma unroll 1
+            for (int kb = 0; kb < TE; kb += kBatchTE) {
+                float2 tb[kBatchTE];
 #pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    const uint32_t off = atom + sw128(t * R + r, chunk) + inb;
+                for (int kx = 0; kx < kBatchTE; ++kx) tb[kx] = th_at(kb + kx);
 #pragma unroll
-                    for (int mt = 0; mt < NM; ++mt)
-                        vv[mt][r] = *reinterpret_cast<const uint2*>(smem + (mt ? OFF_C : OFF_B) + off);
-                }
+                for (int kx = 0; kx < kBatchTE; ++kx) {
+                    const int kk = kb + kx;
+                    const int t = g0 + kk;
+                    const float d = __shfl_sync(kFull, dsl, gln + kk);
+                    const float2 tk = tb[kx];
+                    ph.x = fmaf(d, tk.x, ph.x);
+                    ph.y = fmaf(d, tk.y, ph.y);
+                    float s0, k0, s1, k1;
+                    __sincosf(ph.x, &s0, &k0);
+                    __sincosf(ph.y, &s1, &k1);
+                    if (SUMMARY) {
+                        // the summary pass needs only w_t B~_t: fold w into the rotation
+                        const float wt = exp2f(a2_last - __shfl_sync(kFull, a2sl, gln + kk)) *
+                                         __shfl_sync(kFull, cfsl, gln + kk);
+                        s0 *= wt; k0 *= wt; s1 *= wt; k1 *= wt;
+                    }
+                    const uint32_t cc0 = pack_bf16x2(k0, k0), sn0 = pack_bf16x2(s0, -s0);
+                    const uint32_t cc1 = pack_bf16x2(k1, k1), sn1 = pack_bf16x2(s1, -s1);
+                    // all loads of the token's rows first, then the stores (the
+                    // loads are free to move ahead of earlier tokens' stores)
+                    constexpr int NM = SUMMARY ? 1 : 2;      // B, and C in the main pass
+                    uint2 vv[NM][R];
 #pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    const uint32_t off = atom + sw128(t * R + r, chunk) + inb;
+                    for (int r = 0; r < R; ++r) {
+                        const uint32_t off = atom + sw128(t * R + r, chunk) + inb;
 #pragma unroll
-                    for (int mt = 0; mt < NM; ++mt) {
-                        uint2 v = vv[mt][r];
-                        v.x = rot_bf(v.x, cc0, sn0);
-                        v.y = rot_bf(v.y, cc1, sn1);
-                        *reinterpret_cast<uint2*>(smem + (mt ? OFF_C : OFF_B) + off) = v;
+                        for (int mt = 0; mt < NM; ++mt)
+                            vv[mt][r] = lds64_free(sb_ld + (mt ? OFF_C : OFF_B) + off);
+                    }
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        const uint32_t off = atom + sw128(t * R + r, chunk) + inb;
+#pragma unroll
+                        for (int mt = 0; mt < NM; ++mt) {
+                            uint2 v = vv[mt][r];
+                            v.x = rot_bf(v.x, cc0, sn0);
+                            v.y = rot_bf(v.y, cc1, sn1);
+                            *reinterpret_cast<uint2*>(smem + (mt ? OFF_C : OFF_B) + off) = v;
+                        }
                     }
                 }
             }
@@ -573,14 +650,21 @@ __global__ void __launch_bounds__(kThreads, 2)
         fence_async_smem();
         tc_fence_before();       // the deferred y's TMEM reads precede the next MMAs
         mbar_arrive(&m->bar[BAR_OPS]);
-        // the next tile's dt / lambda: for short tiles their loads are issued
-        // here, while the tile's MMAs run (measured faster than after them)
-        if (k + 1 < ntiles) load_tok(k + 1);
-
+        // the next tile's coefficients, mask tables and phase increments,
+        // while this tile's MMAs run
+        TileCoef nxt = cur;
+        if (k + 1 < ntiles) {
+            load_tok(k + 1);     // (short tiles: consumed at the next tile's top)
+            if (kAhead) {
+                nxt = coef_stage(k + 1);
+                pass1_ahead(k + 1, nxt.dsl);
+            }
+        }
         // this thread's tile row: its token's log2 decay and pending weight
-        const float a2_tr = __shfl_sync(kFull, pick<NT>(a2v, rsl), rln);
+        const float a2_tr = kAhead ? cur.a2_tr : __shfl_sync(kFull, cur.a2_tr, rln);
+        const float a2_last = cur.a2_last;
         if (!SUMMARY) {
-            const float cf_tr = __shfl_sync(kFull, pick<NT>(cfv, rsl), rln);
+            const float cf_tr = kAhead ? cur.cf_tr : __shfl_sync(kFull, cur.cf_tr, rln);
             mbar_wait(&m->bar[BAR_G], par, m, status, 11);
             tc_fence_after();
             // w_t X_t for the chunk-local state, into the S_bf region (free once
@@ -627,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 } else {
                     constexpr int GT = 16 / R;            // tokens per 16-column block
                     const int u0 = col0 / R;              // the block's first token (warp-uniform)
-                    const float aref = m->u.cs[2][u0 / GT];
+                    const float aref = m->u.cs[par][2][u0 / GT];
                     if (u0 > tr) {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) v[j] = 0.f;
@@ -635,8 +719,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                         const float rowf = exp2f(a2_tr - aref);
 #pragma unroll
                         for (int i4 = 0; i4 < GT / 4; ++i4) {
-                            const float4 fc = reinterpret_cast<const float4*>(m->u.cs[0] + u0)[i4];
-                            const float4 fg = reinterpret_cast<const float4*>(m->u.cs[1] + u0)[i4];
+                            const float4 fc = reinterpret_cast<const float4*>(m->u.cs[par][0] + u0)[i4];
+                            const float4 fg = reinterpret_cast<const float4*>(m->u.cs[par][1] + u0)[i4];
                             const float mc[4] = {fc.x, fc.y, fc.z, fc.w}, mg[4] = {fg.x, fg.y, fg.z, fg.w};
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
@@ -651,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
                         for (int j = 0; j < 16; j += R) {
                             const int uu = u0 + j / R;
-                            const float au = m->u.cs[3][uu], gu = m->u.cs[4][uu], cu = m->u.cs[5][uu];
+                            const float au = m->u.cs[par][3][uu], gu = m->u.cs[par][4][uu], cu = m->u.cs[par][5][uu];
                             const float mkv = (uu <= tr) ? exp2f(a2_tr - au) * (uu == tr ? gu : cu) : 0.f;
 #pragma unroll
                             for (int rr = 0; rr < R; ++rr) v[j + rr] *= mkv;
@@ -699,6 +783,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             y_tile = k;
             y_ea = exp2f(a2_tr);
         }
+        cur = nxt;
         // (the S_bf stores and S_loc reads above are ordered before the next
         // tile's MMAs by the fences ahead of that tile's OPS arrival)
     }
@@ -831,17 +916,17 @@ static cudaError_t launch_tc_R(const ScanParams& q, int* status, cudaStream_t st
         !make_tile_map(&mC, q.C, kN, R, q.ngroups, q.seqlen, q.batch, T) ||
         !make_tile_map(&mX, q.x, kP, R, q.nheads, q.seqlen, q.batch, T))
         return cudaErrorInvalidValue;
-    cudaFuncSetAttribute(scan_tc_kernel<R, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    cudaFuncSetAttribute(scan_tc_kernel<R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaFuncSetAttribute(scan_tc_kernel<R, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<R>());
+    cudaFuncSetAttribute(scan_tc_kernel<R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<R>());
     // two CTAs per SM need the largest shared-memory carveout
     cudaFuncSetAttribute(scan_tc_kernel<R, false>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     cudaFuncSetAttribute(scan_tc_kernel<R, true>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (q.nseg > 1) {
-        scan_tc_kernel<R, true><<<dim3(q.nseg - 1, q.nheads, q.batch), kThreads, SMEM_BYTES, st>>>(mB, mC, mX, q, status);
+        scan_tc_kernel<R, true><<<dim3(q.nseg - 1, q.nheads, q.batch), kThreads, smem_bytes<R>(), st>>>(mB, mC, mX, q, status);
         cudaError_t e = launch_scan_combine(q, st);
         if (e != cudaSuccess) return e;
     }
-    scan_tc_kernel<R, false><<<dim3(q.nseg, q.nheads, q.batch), kThreads, SMEM_BYTES, st>>>(mB, mC, mX, q, status);
+    scan_tc_kernel<R, false><<<dim3(q.nseg, q.nheads, q.batch), kThreads, smem_bytes<R>(), st>>>(mB, mC, mX, q, status);
     return cudaGetLastError();
 }
 
@@ -854,9 +939,9 @@ static cudaError_t launch_tc_summary_R(const ScanParams& q, int* status, cudaStr
         !make_tile_map(&mC, q.C, kN, R, q.ngroups, q.seqlen, q.batch, T) ||
         !make_tile_map(&mX, q.x, kP, R, q.nheads, q.seqlen, q.batch, T))
         return cudaErrorInvalidValue;
-    cudaFuncSetAttribute(scan_tc_kernel<R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaFuncSetAttribute(scan_tc_kernel<R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<R>());
     cudaFuncSetAttribute(scan_tc_kernel<R, true>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    scan_tc_kernel<R, true><<<dim3(q.nseg - 1, q.nheads, q.batch), kThreads, SMEM_BYTES, st>>>(mB, mC, mX, q, status);
+    scan_tc_kernel<R, true><<<dim3(q.nseg - 1, q.nheads, q.batch), kThreads, smem_bytes<R>(), st>>>(mB, mC, mX, q, status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_scan_combine(q, st);

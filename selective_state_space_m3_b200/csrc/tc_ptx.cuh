@@ -189,6 +189,14 @@ __device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 v) {
     memcpy(&u, &v, 4);
     return u;
 }
+// 8-byte shared-memory load with no memory side effects visible to the
+// compiler, so that it may be hoisted above unrelated shared stores (the
+// caller orders it after the data's arrival through the address operand)
+__device__ __forceinline__ uint2 lds64_free(uint32_t addr) {
+    uint2 v;
+    asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
 // one rotary pair in bf16x2: (x, y) -> (c x + s y, c y - s x), cc = (c, c),
 // sn = (s, -s); the product s*y is rounded to bf16 before the fused add
 __device__ __forceinline__ uint32_t rot_bf(uint32_t v, uint32_t cc, uint32_t sn) {
