@@ -91,7 +91,7 @@ struct TileCoef {
     float cf_tr;        // pending weight c of that token (main pass); for
                         // short tiles both hold the lane's own token's
     float dsl;          // dt of token 32 gsl + lane (the warp's phase-pass source)
-    float a2sl, cfsl;   // summary pass: log2 decay and c of that token
+    float wsl;          // summary pass: state weight e^{a_last - a} c of that token
 };
 
 // ------------------------------------------------------------ PTX wrappers --
@@ -404,8 +404,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         c.a2_tr = kAhead ? __shfl_sync(kFull, pick<NT>(a2v, rsl), rln) : a2v[0];
         c.cf_tr = SUMMARY ? 0.f : (kAhead ? __shfl_sync(kFull, pick<NT>(cfv, rsl), rln) : cfv[0]);
         c.dsl = pick<NT>(dtv, gsl);
-        c.a2sl = SUMMARY ? pick<NT>(a2v, gsl) : 0.f;
-        c.cfsl = SUMMARY ? pick<NT>(cfv, gsl) : 0.f;
+        c.wsl = SUMMARY ? exp2f(a2_last - pick<NT>(a2v, gsl)) * pick<NT>(cfv, gsl) : 0.f;
         return c;
     };
     // ---- phase pass 1 of tile kn: this group's increments of pairs
@@ -434,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int qcn = min(T, tok1 - t0n);
         pass1_stage(kn, dsl, [&](int kk) { return theta_ld(t0n, qcn, kk); });
     };
-    TileCoef cur = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    TileCoef cur = {0.f, 0.f, 0.f, 0.f, 0.f};
     if (warp > 0 && ntiles > 0) {
         load_tok(0);
         prefetch_theta(0);
@@ -597,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int chunk = (lane & 15) >> 1;
             const uint32_t inb = (uint32_t)(lane & 1) * 8u;
             ph = make_float2(wrap_pi_f(ph.x), wrap_pi_f(ph.y));
-            const float dsl = cur.dsl, a2sl = cur.a2sl, cfsl = cur.cfsl, a2_last = cur.a2_last;
+            const float dsl = cur.dsl, wsl = cur.wsl;
 #pragma unroll 1
             for (int kb = 0; kb < TE; kb += kBatchTE) {
                 float2 tb[kBatchTE];
@@ -616,8 +615,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     __sincosf(ph.y, &s1, &k1);
                     if (SUMMARY) {
                         // the summary pass needs only w_t B~_t: fold w into the rotation
-                        const float wt = exp2f(a2_last - __shfl_sync(kFull, a2sl, gln + kk)) *
-                                         __shfl_sync(kFull, cfsl, gln + kk);
+                        const float wt = __shfl_sync(kFull, wsl, gln + kk);
                         s0 *= wt; k0 *= wt; s1 *= wt; k1 *= wt;
                     }
                     const uint32_t cc0 = pack_bf16x2(k0, k0), sn0 = pack_bf16x2(s0, -s0);
