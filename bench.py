@@ -318,9 +318,12 @@ KERNEL_SOURCES = {
 }
 CAPTURES = {
     # kernel: (workload, plan segments or None, bytes per launch, source digest)
-    "scan_tc_kernel": None,
-    "step_pipe_kernel": None,
-    "rope_block_kernel": None,
+    "scan_tc_kernel": ("mimo_r4_layer_b8_h32_L4096_P64_N128_Q64_bf16", 1,
+                       2_982_587_136 + 525_263_360, "2ba555d9c21599f7"),
+    "step_pipe_kernel": ("decode_mimo_r4_b256_h32_P64_N128_x1000", None,
+                         304_192_768 + 224_838_400, "fb3967fb581615af"),
+    "rope_block_kernel": ("mimo_r4_layer_b8_h32_L4096_P64_N128_Q64_bf16", None,
+                          2_422_809_856 + 2_378_863_104, "1d5355e7ce240d9a"),
 }
 
 

@@ -171,8 +171,13 @@ __global__ void __launch_bounds__(256) step_kernel(StepParams q) {
 // copies of the next units are in flight while the current unit computes.
 // The updated state goes straight from registers to global memory with
 // coalesced float4 stores.  Same arithmetic and thread mapping as step_kernel.
+// Each thread makes the rotations of its own pairs (no barrier between a
+// unit's arrival and its state update); the y partials of the warps are
+// summed through the consumed state block.  (Adding them into a per-stage
+// accumulator with shared-memory atomics instead, which saves one more
+// barrier, measured 15 % slower.)
 struct PipeLayout {
-    int off_h, off_B, off_C, off_PB, off_X, off_PX, off_TH, off_S, off_CS, stage;
+    int off_h, off_B, off_C, off_PB, off_X, off_PX, off_TH, off_S, stage;
 };
 
 __host__ __device__ constexpr PipeLayout pipe_layout(int N, int P, int R, int es) {
@@ -185,8 +190,7 @@ __host__ __device__ constexpr PipeLayout pipe_layout(int N, int P, int R, int es
     l.off_PX = l.off_X + R * P * es;
     l.off_TH = l.off_PX + R * P * es;
     l.off_S = l.off_TH + (N / 2) * 4;          // dt, lambda, A
-    l.off_CS = l.off_S + 16;                   // cos, sin per rotary pair (computed in place)
-    l.stage = ((l.off_CS + (N / 2) * 8) + 127) & ~127;
+    l.stage = ((l.off_S + 16) + 127) & ~127;
     return l;
 }
 
@@ -281,15 +285,7 @@ __global__ void __launch_bounds__(256, 2) step_pipe_kernel(StepParams q, int uni
         const T* sPX = reinterpret_cast<const T*>(stg + lay.off_PX);
         const float* sTH = reinterpret_cast<const float*>(stg + lay.off_TH);
         const float* sc = reinterpret_cast<const float*>(stg + lay.off_S);
-        float2* sCS = reinterpret_cast<float2*>(psm + st * lay.stage + lay.off_CS);
         const float d = sc[0], lam = sc[1], a = sc[2];
-        // the rotation of each pair, once per unit
-        if (tid < NH) {
-            const int ip = tid;
-            float sv, cv;
-            sincosf((float)wrap_pi((double)d * (double)sTH[ip]), &sv, &cv);
-            sCS[ip] = make_float2(cv, sv);
-        }
         const float alpha = expf(d * a);
         const float beta = (1.0f - lam) * d * alpha;
         const float gamma = lam * d;
@@ -305,7 +301,6 @@ __global__ void __launch_bounds__(256, 2) step_pipe_kernel(StepParams q, int uni
                 px2[r][j] = make_float2(pv, pv);
                 xx2[r][j] = make_float2(xv, xv);
             }
-        __syncthreads();                 // cos/sin of every pair are in place
         // y partials per (rank, column), the two lanes holding the two rows of
         // each pair (summed at the end)
         float2 yacc2[R][4];
@@ -319,7 +314,10 @@ __global__ void __launch_bounds__(256, 2) step_pipe_kernel(StepParams q, int uni
             const int ip = ig + k * IG;
             if (ip >= NH) continue;
             const int n0 = 2 * ip, n1 = 2 * ip + 1;
-            const float2 cs = sCS[ip];
+            // the pair's rotation by dt theta (reduced to [-pi, pi]: the fast
+            // sine and cosine then err by ~1e-6)
+            float2 cs;
+            __sincosf(wrap_pi_f(d * sTH[ip]), &cs.y, &cs.x);
             const float4 h0 = reinterpret_cast<const float4*>(hs)[n0 * PC + pc];
             const float4 h1 = reinterpret_cast<const float4*>(hs)[n1 * PC + pc];
             // (row n0, row n1) of the previous B, of B_t and of C_t per rank

@@ -32,6 +32,16 @@ __device__ __forceinline__ double wrap_pi(double phi) {
     return phi - kTwoPi * rint(phi * (1.0 / kTwoPi));
 }
 
+// Reduce a float angle to [-pi, pi] (two-constant additive reduction:
+// 2*pi split into a float head and tail so k*2pi is formed exactly enough)
+__device__ __forceinline__ float wrap_pi_f(float x) {
+    constexpr float kInv2Pi = 0.15915494309189535f;
+    constexpr float k2PiHi = 6.28318548202514648f;      // float(2 pi)
+    constexpr float k2PiLo = -1.7484555314695172e-7f;   // 2 pi - float(2 pi)
+    const float k = rintf(x * kInv2Pi);
+    return fmaf(-k, k2PiLo, fmaf(-k, k2PiHi, x));
+}
+
 // Status word at the start of a scan workspace.
 struct WorkspaceHeader {
     int status;      // m3_status of the last device-side failure, 0 = none
