@@ -24,13 +24,16 @@
 // kernel runs the recurrence directly in float32.
 //
 // Mapping.  State columns p evolve independently (the transition acts on the
-// rows n).  A warp owns PC = 4 columns of one (batch, head) and every row:
-// lane l holds the rotary pairs i = l + 32 k (k < KP), i.e. rows 2i and 2i+1,
-// so a pair block never leaves its thread.  Readout and reflection sums over
-// n are warp shuffles; nothing crosses warps.  A CTA of 4 warps covers 16
-// columns and stages each token's B, C (and u), theta, dt, lambda and its 16
-// columns of x in shared memory with cp.async, a chunk of TK tokens ahead of
-// use (two buffers).
+// rows n).  A warp owns PCW (1, 2 or 4) columns of one (batch, head) and every
+// row: lane l holds the rotary pairs i = l + 32 k (k < KP), i.e. rows 2i and
+// 2i+1, so a pair block never leaves its thread.  Readout and reflection sums
+// over n are warp shuffles; nothing crosses warps.  A CTA of 4 warps covers
+// 4 PCW columns and stages each token's B, C (and u), theta, dt, lambda and
+// its columns of x in shared memory with cp.async, a chunk of TK tokens ahead
+// of use (two buffers); once a chunk has landed the CTA makes every token's
+// pair blocks and alpha, beta, gamma once, into the same slots, for all its
+// warps.  Few (batch, head) sequences get narrow warps (more warps in all,
+// to hide the per-token latency), many get wide ones (fewer shared loads).
 #include "m3_common.cuh"
 #include "m3_kernels.h"
 
@@ -38,13 +41,17 @@ namespace m3 {
 namespace seq {
 
 constexpr int kWarps = 4;
-constexpr int kPC = 4;                     // columns per warp
-constexpr int kCB = kWarps * kPC;          // columns per CTA
+constexpr int kMaxCB = kWarps * 4;         // columns per CTA at the widest warps
 constexpr int kThreads = 32 * kWarps;
 constexpr unsigned kFull = 0xffffffffu;
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+                 "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
                  "l"(gmem)
                  : "memory");
 }
@@ -56,19 +63,23 @@ __device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
-// Byte layout of one token's slot in shared memory (all offsets multiples of 16).
+// Byte layout of one token's slot in shared memory (all offsets multiples of
+// 16; x rows of the CTA's columns padded to 16 bytes).
 struct Slot {
-    int B, C, U, TH, X, DL, bytes;
+    int B, C, U, TH, X, XS, DL, CO, CS, bytes;
 };
-__host__ __device__ inline Slot slot_layout(int R, int N, int es, bool refl) {
+__host__ __device__ inline Slot slot_layout(int R, int N, int es, bool refl, int kcb) {
     Slot s;
     int o = 0;
     s.B = o;  o += R * N * es;
     s.C = o;  o += R * N * es;
     s.U = o;  o += refl ? N * es : 0;
     s.TH = o; o += (N / 2) * 4;
-    s.X = o;  o += R * kCB * es;
+    s.XS = kcb * es < 16 ? 16 : kcb * es;   // bytes per rank row of x
+    s.X = o;  o += R * s.XS;
     s.DL = o; o += 16;                      // dt, lambda
+    s.CO = o; o += 16;                      // alpha, beta, gamma (made after arrival)
+    s.CS = o; o += (N / 2) * 8;             // pair blocks (c, sn) (made after arrival)
     s.bytes = (o + 15) & ~15;
     return s;
 }
@@ -122,8 +133,10 @@ __device__ __forceinline__ void pair_block(int regime, float phi, float& c, floa
     }
 }
 
-template <typename T, int R, int KP, bool REFL>
+template <typename T, int R, int KP, bool REFL, int PCW>
 __global__ void __launch_bounds__(kThreads) seq_kernel(SeqParams q, int TK) {
+    constexpr int kPC = PCW;                   // columns per warp
+    constexpr int kCB = kWarps * kPC;          // columns per CTA
     extern __shared__ __align__(16) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c0 = blockIdx.x * kCB;            // first column of the CTA
@@ -140,7 +153,8 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(SeqParams q, int TK) {
     const T* Cg = static_cast<const T*>(q.C);
     const T* Ug = static_cast<const T*>(q.u);
     constexpr int es = sizeof(T);
-    const Slot sl = slot_layout(R, N, es, REFL);
+    const Slot sl = slot_layout(R, N, es, REFL, kCB);
+    const float sg = (REFL || q.regime == 0) ? 1.f : (q.regime == 1 ? 0.f : -1.f);
 
     // ---- staging of a chunk of tokens (cp.async, 16-byte pieces)
     auto stage = [&](int chunk, int buf) {
@@ -148,7 +162,8 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(SeqParams q, int TK) {
         const int nt = min(TK, L - t0);
         uint8_t* base = smem + (size_t)buf * TK * sl.bytes;
         const int pB = R * N * es / 16, pU = REFL ? N * es / 16 : 0, pT = NH * 4 / 16;
-        const int pX = kCB * es / 16;                    // per rank
+        constexpr int xb = kCB * es;                     // x bytes per rank row
+        const int pX = xb < 16 ? 1 : xb / 16;            // copies per rank row
         const int per = 2 * pB + pU + pT + R * pX;
         for (int e = tid; e < nt * per; e += kThreads) {
             const int tt = e / per;
@@ -176,9 +191,12 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(SeqParams q, int TK) {
             }
             k -= pT;
             const int r = k / pX, kk = k % pX;
-            if (c0 + kk * 16 / es < P)
-                cp_async16(s + sl.X + r * kCB * es + 16 * kk,
-                           reinterpret_cast<const uint8_t*>(xg + ((bt * H + h) * R + r) * P + c0) + 16 * kk);
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(xg + ((bt * H + h) * R + r) * P + c0) + 16 * kk;
+            if (xb < 16) {
+                if (c0 < P) cp_async8(s + sl.X + r * sl.XS, src);
+            } else if (c0 + kk * 16 / es < P) {
+                cp_async16(s + sl.X + r * sl.XS + 16 * kk, src);
+            }
         }
         for (int tt = tid; tt < nt; tt += kThreads) {
             const size_t o = ((size_t)b * L + t0 + tt) * H + h;
@@ -223,21 +241,39 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(SeqParams q, int TK) {
         __syncthreads();
         const int t0 = ch * TK;
         const int nt = min(TK, L - t0);
-        const uint8_t* base = smem + (size_t)(ch & 1) * TK * sl.bytes;
-        for (int tt = 0; tt < nt; ++tt) {
-            const uint8_t* s = base + (size_t)tt * sl.bytes;
+        uint8_t* base = smem + (size_t)(ch & 1) * TK * sl.bytes;
+        // every token's pair blocks and alpha, beta, gamma, once for all warps
+        for (int e = tid; e < nt * NH; e += kThreads) {
+            const int tt = e / NH, i = e - tt * NH;
+            uint8_t* s = base + (size_t)tt * sl.bytes;
+            const float d = reinterpret_cast<const float*>(s + sl.DL)[0];
+            float cc, sn, sgn;
+            pair_block(REFL ? 0 : q.regime, d * reinterpret_cast<const float*>(s + sl.TH)[i], cc, sn, sgn);
+            reinterpret_cast<float2*>(s + sl.CS)[i] = make_float2(cc, sn);
+        }
+        for (int tt = tid; tt < nt; tt += kThreads) {
+            uint8_t* s = base + (size_t)tt * sl.bytes;
             const float d = reinterpret_cast<const float*>(s + sl.DL)[0];
             const float lm = reinterpret_cast<const float*>(s + sl.DL)[1];
             const float al = expf(d * Ah);
-            const float be = (1.f - lm) * d * al;
-            const float ga = lm * d;
+            float* co = reinterpret_cast<float*>(s + sl.CO);
+            co[0] = al;
+            co[1] = (1.f - lm) * d * al;
+            co[2] = lm * d;
+        }
+        __syncthreads();
+        for (int tt = 0; tt < nt; ++tt) {
+            const uint8_t* s = base + (size_t)tt * sl.bytes;
+            const float al = reinterpret_cast<const float*>(s + sl.CO)[0];
+            const float be = reinterpret_cast<const float*>(s + sl.CO)[1];
+            const float ga = reinterpret_cast<const float*>(s + sl.CO)[2];
             // this token's x for the warp's columns (same for every lane)
             float xc[R][kPC];
 #pragma unroll
             for (int r = 0; r < R; ++r)
 #pragma unroll
                 for (int c = 0; c < kPC; ++c)
-                    xc[r][c] = ld_io(reinterpret_cast<const T*>(s + sl.X) + r * kCB + warp * kPC + c);
+                    xc[r][c] = ld_io(reinterpret_cast<const T*>(s + sl.X + r * sl.XS) + warp * kPC + c);
             // v = alpha h + beta B_{t-1} X_{t-1}^T
 #pragma unroll
             for (int k = 0; k < KP; ++k)
@@ -290,9 +326,8 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(SeqParams q, int TK) {
 #pragma unroll
             for (int k = 0; k < KP; ++k) {
                 const int i = lane + 32 * k;
-                const float th = i < NH ? reinterpret_cast<const float*>(s + sl.TH)[i] : 0.f;
-                float cc, sn, sg;
-                pair_block(REFL ? 0 : q.regime, d * th, cc, sn, sg);
+                const float2 cs = i < NH ? reinterpret_cast<const float2*>(s + sl.CS)[i] : make_float2(1.f, 0.f);
+                const float cc = cs.x, sn = cs.y;
 #pragma unroll
                 for (int c = 0; c < kPC; ++c) {
                     const float v0 = hs[k][0][c], v1 = hs[k][1][c];
@@ -372,35 +407,47 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(SeqParams q, int TK) {
             for (int c = 0; c < kPC; ++c) st_io(static_cast<T*>(q.fin_pX) + (bh * R + r) * P + cw + c, px[r][c]);
 }
 
-template <typename T, int R, int KP, bool REFL>
+template <typename T, int R, int KP, bool REFL, int PCW>
 static cudaError_t launch_t(const SeqParams& q, cudaStream_t st) {
-    const Slot sl = slot_layout(R, q.dstate, sizeof(T), REFL);
+    constexpr int kCB = kWarps * PCW;
+    const Slot sl = slot_layout(R, q.dstate, sizeof(T), REFL, kCB);
     // tokens per staged chunk: up to 16, two buffers within 96 KB
     int TK = (96 * 1024) / (2 * sl.bytes);
     if (TK > 16) TK = 16;
     if (TK < 1) return cudaErrorInvalidValue;
     const size_t smem = (size_t)2 * TK * sl.bytes;
-    cudaError_t e = cudaFuncSetAttribute(seq_kernel<T, R, KP, REFL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(seq_kernel<T, R, KP, REFL, PCW>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((q.headdim + kCB - 1) / kCB, q.nheads, q.batch);
-    seq_kernel<T, R, KP, REFL><<<grid, kThreads, smem, st>>>(q, TK);
+    seq_kernel<T, R, KP, REFL, PCW><<<grid, kThreads, smem, st>>>(q, TK);
     return cudaGetLastError();
+}
+
+// columns per warp: 4 (2 and 1 give more warps per SM but measured slower on
+// the SISO layer, 0.96 and 1.19 ms against 0.91 ms: the per-token work of a
+// warp is mostly fixed; M3_SEQ_COLS=1|2 selects them for comparison)
+template <typename T, int R, int KP, bool REFL>
+static cudaError_t launch_w(const SeqParams& q, cudaStream_t st) {
+    const char* ev = getenv("M3_SEQ_COLS");
+    if (ev && ev[0] == '1' && ev[1] == 0) return launch_t<T, R, KP, REFL, 1>(q, st);
+    if (ev && ev[0] == '2' && ev[1] == 0) return launch_t<T, R, KP, REFL, 2>(q, st);
+    return launch_t<T, R, KP, REFL, 4>(q, st);
 }
 
 template <typename T, bool REFL>
 static cudaError_t launch_rk(const SeqParams& q, cudaStream_t st) {
     const int KP = (q.dstate / 2 + 31) / 32;
     switch (q.rank * 8 + KP) {
-        case 1 * 8 + 1: return launch_t<T, 1, 1, REFL>(q, st);
-        case 1 * 8 + 2: return launch_t<T, 1, 2, REFL>(q, st);
-        case 1 * 8 + 4: return launch_t<T, 1, 4, REFL>(q, st);
-        case 2 * 8 + 1: return launch_t<T, 2, 1, REFL>(q, st);
-        case 2 * 8 + 2: return launch_t<T, 2, 2, REFL>(q, st);
-        case 2 * 8 + 4: return launch_t<T, 2, 4, REFL>(q, st);
-        case 4 * 8 + 1: return launch_t<T, 4, 1, REFL>(q, st);
-        case 4 * 8 + 2: return launch_t<T, 4, 2, REFL>(q, st);
-        case 4 * 8 + 4: return launch_t<T, 4, 4, REFL>(q, st);
+        case 1 * 8 + 1: return launch_w<T, 1, 1, REFL>(q, st);
+        case 1 * 8 + 2: return launch_w<T, 1, 2, REFL>(q, st);
+        case 1 * 8 + 4: return launch_w<T, 1, 4, REFL>(q, st);
+        case 2 * 8 + 1: return launch_w<T, 2, 1, REFL>(q, st);
+        case 2 * 8 + 2: return launch_w<T, 2, 2, REFL>(q, st);
+        case 2 * 8 + 4: return launch_w<T, 2, 4, REFL>(q, st);
+        case 4 * 8 + 1: return launch_w<T, 4, 1, REFL>(q, st);
+        case 4 * 8 + 2: return launch_w<T, 4, 2, REFL>(q, st);
+        case 4 * 8 + 4: return launch_w<T, 4, 4, REFL>(q, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -410,7 +457,7 @@ static cudaError_t launch_rk(const SeqParams& q, cudaStream_t st) {
 bool seq_supported(const m3_dims& d) {
     const int KP = (d.dstate / 2 + 31) / 32;
     return (d.rank == 1 || d.rank == 2 || d.rank == 4) && d.dstate % 8 == 0 && (KP == 1 || KP == 2 || KP == 4) &&
-           d.headdim % seq::kCB == 0;
+           d.headdim % seq::kMaxCB == 0;
 }
 
 cudaError_t launch_seq(const m3_dims& d, const SeqParams& q, cudaStream_t st) {
