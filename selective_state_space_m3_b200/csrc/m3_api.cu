@@ -9,6 +9,7 @@
 
 #include "m3_common.cuh"
 #include "m3_kernels.h"
+#include "m3_nvtx.h"
 
 namespace m3 {
 
@@ -240,6 +241,7 @@ m3_status m3_scan_plan(const m3_dims* d, int* launches, int* segments, int* chun
 m3_status m3_scan_fwd(const m3_dims* d, const void* x, const void* B, const void* C, const float* dt,
                       const float* A, const float* lambda, const float* theta, const m3_carry* init,
                       void* y, m3_carry* fin, void* workspace, size_t ws_bytes, void* stream) {
+    const NvtxRange range("m3_scan_fwd");
     m3_status s = check_dims(d, true);
     if (s != M3_OK) return s;
     const bool work = d->batch > 0 && d->seqlen > 0;
@@ -321,6 +323,7 @@ m3_status m3_scan_fwd(const m3_dims* d, const void* x, const void* B, const void
 m3_status m3_step(const m3_dims* d, m3_carry* state, const void* x, const void* B, const void* C,
                   const float* dt, const float* A, const float* lambda, const float* theta, void* y,
                   void* stream) {
+    const NvtxRange range("m3_step");
     m3_status s = check_dims(d, false);
     if (s != M3_OK) return s;
     if (!state) return M3_ERR_INVALID_ARG;
@@ -337,6 +340,7 @@ m3_status m3_step(const m3_dims* d, m3_carry* state, const void* x, const void* 
 
 m3_status m3_rope_bc(const m3_dims* d, const void* B, const void* C, const float* dt, const float* theta,
                      void* B_rot, void* C_rot, float* phase, void* stream) {
+    const NvtxRange range("m3_rope_bc");
     m3_status s = check_dims(d, false);
     if (s != M3_OK) return s;
     if (d->seqlen < 0) return M3_ERR_INVALID_ARG;
@@ -374,6 +378,7 @@ m3_status m3_scan_bwd(const m3_dims* d, const void* x, const void* B, const void
                       const void* dy, const m3_grad_carry* d_final, float* dx, float* dB, float* dC, float* ddt,
                       float* dA, float* dlambda, float* dtheta, m3_grad_carry* d_init, void* workspace,
                       size_t ws_bytes, void* stream) {
+    const NvtxRange range("m3_scan_bwd");
     m3_status s = check_dims(d, true);
     if (s != M3_OK) return s;
     if (!bwd_supported(*d)) return M3_ERR_UNSUPPORTED;
@@ -468,6 +473,7 @@ m3_status m3_scan_fwd_phase(const m3_dims* d, int mode, const int* perm, const f
                             const void* B, const void* C, const float* dt, const float* A, const float* lambda,
                             const float* theta, const m3_carry* init, void* y, m3_carry* final_state,
                             void* workspace, size_t ws_bytes, void* stream) {
+    const NvtxRange range("m3_scan_fwd_phase");
     m3_status s = check_dims(d, true);
     if (s != M3_OK) return s;
     PhaseLayout l;
@@ -583,12 +589,14 @@ static m3_status scan_variant(const m3_dims* d, int regime, const void* u, const
 m3_status m3_scan_fwd_damped(const m3_dims* d, int regime, const void* x, const void* B, const void* C,
                              const float* dt, const float* A, const float* lambda, const float* theta,
                              const m3_carry* init, void* y, m3_carry* final_state, void* stream) {
+    const NvtxRange range("m3_scan_fwd_damped");
     return scan_variant(d, regime, nullptr, x, B, C, dt, A, lambda, theta, init, y, final_state, stream);
 }
 
 m3_status m3_scan_fwd_reflect(const m3_dims* d, const void* u, const void* x, const void* B, const void* C,
                               const float* dt, const float* A, const float* lambda, const float* theta,
                               const m3_carry* init, void* y, m3_carry* final_state, void* stream) {
+    const NvtxRange range("m3_scan_fwd_reflect");
     // u is read only when there are tokens (like the other inputs)
     if (d && d->batch > 0 && d->seqlen > 0 && !ptrs_ok({u})) return M3_ERR_INVALID_ARG;
     return scan_variant(d, 0, u, x, B, C, dt, A, lambda, theta, init, y, final_state, stream);

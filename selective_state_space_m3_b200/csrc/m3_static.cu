@@ -17,6 +17,7 @@
 
 #include "m3_common.cuh"
 #include "m3_kernels.h"
+#include "m3_nvtx.h"
 
 namespace {
 
@@ -56,6 +57,7 @@ extern "C" m3_status m3_scan_fwd_static(const m3_dims* dims, const void* x, cons
                                         const float* dt, const float* A, const float* lambda,
                                         const float* theta, const m3_carry* init, void* y,
                                         m3_carry* final_state, void* stream) {
+    const m3::NvtxRange range("m3_scan_fwd_static");
     size_t need = 0;
     m3_status s = m3_scan_workspace_size(dims, &need);
     if (s != M3_OK) return s;
