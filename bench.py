@@ -232,7 +232,43 @@ def cpu_baseline_sample():
     out = {"value": val, "unit": "tokens/s", "cores": oracle.num_threads(), "host_cpus": os.cpu_count(),
            "kind": "oracle", "sample": oracle_sample_text(heads, calls), "seconds_per_call": dt}
     out["single_thread"] = oracle_single_thread()
+    out["decode"] = oracle_decode_sample()
     return out
+
+
+def oracle_decode_sample(budget_s: float = 5.0):
+    """The oracle's decode step on a fixed subset of the decode workload:
+    sequences j = 0 mod 16 of the 256 (all 32 heads), seeded carry and
+    tokens, as many steps as fit in about `budget_s` after one warm-up step;
+    tokens/s counts one token per sequence and step."""
+    import numpy as np
+    import torch
+    import m3_synth
+    import oracle
+    dec = m3_synth.DECODE
+    sub = list(range(0, dec.batch, 16))
+    c = m3_synth.make_carry(dec.batch, dec.nheads, dec.dstate, dec.headdim, dec.rank, dec.dtype, dec.seed,
+                            scale=0.5)
+    f64 = lambda t: t.to(torch.float64).numpy()
+    h, pB, pX = f64(c["h"])[sub], f64(c["prev_B"])[sub], f64(c["prev_x"])[sub]
+    A = -np.exp(np.linspace(-2, 1, dec.nheads))
+    toks = [{k: f64(v)[sub] for k, v in m3_synth.make_decode_token(dec, k).items()} for k in range(4)]
+
+    def one(k):
+        t = toks[k % len(toks)]
+        return oracle.step(h, pB, pX, t["x"], t["B"], t["C"], t["dt"], A, t["lam"], t["theta"])
+
+    t0 = time.perf_counter()
+    _, h, pB, pX = one(0)
+    first = max(time.perf_counter() - t0, 1e-6)
+    n = int(max(2, min(200, budget_s // first)))
+    t0 = time.perf_counter()
+    for k in range(n):
+        _, h, pB, pX = one(k + 1)
+    dt = (time.perf_counter() - t0) / n
+    return {"value": len(sub) / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"decode step on {len(sub)} of 256 sequences (j = 0 mod 16, all 32 heads), "
+                      f"{n} timed steps after a warm-up step"}
 
 
 def oracle_single_thread():

@@ -316,87 +316,87 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int t0n = tok0 + kn * T;
         const int qcn = min(T, tok1 - t0n);
         const int pb = kn & 1;
-            // this tile's inputs; tokens past the end count as dt = 0, lambda = 1
-            float dtv[NT], lmv[NT];
+        // this tile's inputs; tokens past the end count as dt = 0, lambda = 1
+        float dtv[NT], lmv[NT];
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+            const bool in = lane + 32 * j < qcn;
+            dtv[j] = in ? dt_n[j] : 0.f;
+            lmv[j] = in ? lam_n[j] : 1.f;
+        }
+        const bool nx_in = t0n + qcn < L;
+        const float dx = nx_in ? dx_n : 0.f, lx = nx_in ? lx_n : 1.f;
+        // coefficients of every token (log2 units): a2 = inclusive scan of
+        // dt A, gamma = lambda dt, c = gamma + (1 - lambda') dt' with ' the
+        // next token (past the tile: the token after it, zero past the end)
+        float a2v[NT], gmv[NT], cfv[NT];
+        float a2_last;
+        {
+            float run = 0.f;
 #pragma unroll
             for (int j = 0; j < NT; ++j) {
-                const bool in = lane + 32 * j < qcn;
-                dtv[j] = in ? dt_n[j] : 0.f;
-                lmv[j] = in ? lam_n[j] : 1.f;
+                float v = dtv[j] * A2;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float u = __shfl_up_sync(kFull, v, o);
+                    if (lane >= o) v += u;
+                }
+                a2v[j] = v + run;
+                run = __shfl_sync(kFull, a2v[j], 31);
             }
-            const bool nx_in = t0n + qcn < L;
-            const float dx = nx_in ? dx_n : 0.f, lx = nx_in ? lx_n : 1.f;
-            // coefficients of every token (log2 units): a2 = inclusive scan of
-            // dt A, gamma = lambda dt, c = gamma + (1 - lambda') dt' with ' the
-            // next token (past the tile: the token after it, zero past the end)
-            float a2v[NT], gmv[NT], cfv[NT];
-            float a2_last;
-            {
-                float run = 0.f;
+            a2_last = run;
+            float up[NT];
 #pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    float v = dtv[j] * A2;
-#pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const float u = __shfl_up_sync(kFull, v, o);
-                        if (lane >= o) v += u;
-                    }
-                    a2v[j] = v + run;
-                    run = __shfl_sync(kFull, a2v[j], 31);
-                }
-                a2_last = run;
-                float up[NT];
-#pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    gmv[j] = lmv[j] * dtv[j];
-                    up[j] = (1.f - lmv[j]) * dtv[j];
-                }
-                const float ux = (1.f - lx) * dx;
-#pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    float nx = __shfl_down_sync(kFull, up[j], 1);
-                    if (j + 1 < NT) {
-                        const float first = __shfl_sync(kFull, up[j + 1 < NT ? j + 1 : j], 0);
-                        if (lane == 31) nx = first;
-                    }
-                    if (lane + 32 * j + 1 == T) nx = ux;
-                    cfv[j] = gmv[j] + nx;
-                }
+            for (int j = 0; j < NT; ++j) {
+                gmv[j] = lmv[j] * dtv[j];
+                up[j] = (1.f - lmv[j]) * dtv[j];
             }
-            if (!SUMMARY && R >= 4) {
-                // decay mask per (token t, token u) of the tile, shared by the R x R
-                // rank block: e^{a_t - a_u} (gamma_u if u == t, c_u if u < t), 0 above
-                constexpr int LD = T + 4;
+            const float ux = (1.f - lx) * dx;
 #pragma unroll
-                for (int e = wk; e < T * T; e += kWorkers) {
-                    const int t = e / T, u = e % T;
-                    const float at = __shfl_sync(kFull, a2v[0], t), au = __shfl_sync(kFull, a2v[0], u);
-                    const float gu = __shfl_sync(kFull, gmv[0], u), cu = __shfl_sync(kFull, cfv[0], u);
-                    m->u.msk[t * LD + u] = (u <= t) ? exp2f(at - au) * (u == t ? gu : cu) : 0.f;
+            for (int j = 0; j < NT; ++j) {
+                float nx = __shfl_down_sync(kFull, up[j], 1);
+                if (j + 1 < NT) {
+                    const float first = __shfl_sync(kFull, up[j + 1 < NT ? j + 1 : j], 0);
+                    if (lane == 31) nx = first;
                 }
+                if (lane + 32 * j + 1 == T) nx = ux;
+                cfv[j] = gmv[j] + nx;
             }
-            if (!SUMMARY && R < 4 && qe == 0) {
-                // long tiles: the mask of a 16-column block (GT tokens) factors as
-                // e^{a_t - a_ref} x e^{a_ref - a_u} (gamma_u or c_u), a_ref = a at the
-                // block's first token, whenever the block's own decay is small
-                // enough that the second factor cannot overflow; such blocks get
-                // a_ref, the others +inf (element-wise path)
-                constexpr int GT = 16 / R;
+        }
+        if (!SUMMARY && R >= 4) {
+            // decay mask per (token t, token u) of the tile, shared by the R x R
+            // rank block: e^{a_t - a_u} (gamma_u if u == t, c_u if u < t), 0 above
+            constexpr int LD = T + 4;
 #pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    const int t = lane + 32 * j;
-                    const float aref = __shfl_sync(kFull, a2v[j], lane & ~(GT - 1));
-                    const float aend = __shfl_sync(kFull, a2v[j], lane | (GT - 1));
-                    const bool ok = aref - aend <= 60.f;
-                    const float colf = exp2f(aref - a2v[j]);
-                    m->u.cs[pb][0][t] = ok ? cfv[j] * colf : 0.f;
-                    m->u.cs[pb][1][t] = ok ? gmv[j] * colf : 0.f;
-                    if ((lane & (GT - 1)) == 0) m->u.cs[pb][2][t / GT] = ok ? aref : __int_as_float(0x7f800000);
-                    m->u.cs[pb][3][t] = a2v[j];
-                    m->u.cs[pb][4][t] = gmv[j];
-                    m->u.cs[pb][5][t] = cfv[j];
-                }
+            for (int e = wk; e < T * T; e += kWorkers) {
+                const int t = e / T, u = e % T;
+                const float at = __shfl_sync(kFull, a2v[0], t), au = __shfl_sync(kFull, a2v[0], u);
+                const float gu = __shfl_sync(kFull, gmv[0], u), cu = __shfl_sync(kFull, cfv[0], u);
+                m->u.msk[t * LD + u] = (u <= t) ? exp2f(at - au) * (u == t ? gu : cu) : 0.f;
             }
+        }
+        if (!SUMMARY && R < 4 && qe == 0) {
+            // long tiles: the mask of a 16-column block (GT tokens) factors as
+            // e^{a_t - a_ref} x e^{a_ref - a_u} (gamma_u or c_u), a_ref = a at the
+            // block's first token, whenever the block's own decay is small
+            // enough that the second factor cannot overflow; such blocks get
+            // a_ref, the others +inf (element-wise path)
+            constexpr int GT = 16 / R;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                const int t = lane + 32 * j;
+                const float aref = __shfl_sync(kFull, a2v[j], lane & ~(GT - 1));
+                const float aend = __shfl_sync(kFull, a2v[j], lane | (GT - 1));
+                const bool ok = aref - aend <= 60.f;
+                const float colf = exp2f(aref - a2v[j]);
+                m->u.cs[pb][0][t] = ok ? cfv[j] * colf : 0.f;
+                m->u.cs[pb][1][t] = ok ? gmv[j] * colf : 0.f;
+                if ((lane & (GT - 1)) == 0) m->u.cs[pb][2][t / GT] = ok ? aref : __int_as_float(0x7f800000);
+                m->u.cs[pb][3][t] = a2v[j];
+                m->u.cs[pb][4][t] = gmv[j];
+                m->u.cs[pb][5][t] = cfv[j];
+            }
+        }
         TileCoef c;
         c.a2_last = a2_last;
         // (short tiles, one slice: the lane's own a and c; the row's are
