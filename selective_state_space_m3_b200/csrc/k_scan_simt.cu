@@ -239,18 +239,37 @@ __global__ void __launch_bounds__(256) scan_combine_kernel(ScanParams q) {
     const float w0 = (1.f - q.lam[(size_t)b * L * H + h]) * q.dt[(size_t)b * L * H + h];
     float s0 = carry_in<T>(q, b, h, 2 * i, p, w0);
     float s1 = carry_in<T>(q, b, h, 2 * i + 1, p, w0);
-    for (int k = 0; k < q.nseg; ++k) {
-        const size_t bhs = bh * q.nseg + k;
-        q.ws_sin[(bhs * N + 2 * i) * P + p] = s0;
-        q.ws_sin[(bhs * N + 2 * i + 1) * P + p] = s1;
-        if (k + 1 == q.nseg) break;
-        const float dec = expf(q.ws_decay[bhs]);
-        const float v0 = fmaf(dec, s0, q.ws_sloc[(bhs * N + 2 * i) * P + p]);
-        const float v1 = fmaf(dec, s1, q.ws_sloc[(bhs * N + 2 * i + 1) * P + p]);
-        float sv, cv;
-        sincosf(q.ws_phase[bhs * NH + i], &sv, &cv);
-        s0 = cv * v0 - sv * v1;
-        s1 = sv * v0 + cv * v1;
+    // The summaries of a batch of segments are loaded before the chain runs
+    // through them (their loads would otherwise wait behind the previous
+    // segment's stores, one memory round trip per segment).
+    constexpr int KB = 8;
+    for (int k0 = 0; k0 < q.nseg; k0 += KB) {
+        float l0[KB], l1[KB], dl[KB], ph[KB];
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+            const int k = min(k0 + j, q.nseg - 1);
+            const size_t bhs = bh * q.nseg + k;
+            l0[j] = __ldg(q.ws_sloc + (bhs * N + 2 * i) * P + p);
+            l1[j] = __ldg(q.ws_sloc + (bhs * N + 2 * i + 1) * P + p);
+            dl[j] = __ldg(q.ws_decay + bhs);
+            ph[j] = __ldg(q.ws_phase + bhs * NH + i);
+        }
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+            const int k = k0 + j;
+            if (k >= q.nseg) break;
+            const size_t bhs = bh * q.nseg + k;
+            q.ws_sin[(bhs * N + 2 * i) * P + p] = s0;
+            q.ws_sin[(bhs * N + 2 * i + 1) * P + p] = s1;
+            if (k + 1 == q.nseg) break;
+            const float dec = expf(dl[j]);
+            const float v0 = fmaf(dec, s0, l0[j]);
+            const float v1 = fmaf(dec, s1, l1[j]);
+            float sv, cv;
+            sincosf(ph[j], &sv, &cv);
+            s0 = cv * v0 - sv * v1;
+            s1 = sv * v0 + cv * v1;
+        }
     }
 }
 
