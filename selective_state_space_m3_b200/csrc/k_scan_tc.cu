@@ -18,12 +18,15 @@
 // Per tile:
 //   TMA     B, C (bf16, SWIZZLE_128B, K-major: rows (t,r), 2 atoms of 64 n)
 //           and X (rows (t,r), 64 p) into shared memory; issued as soon as
-//           the previous tile's MMAs have read those buffers.
-//   workers dt/lambda -> a_t (warp scan, every warp keeps all tokens in
-//           registers), gamma, c, w = e^{a_last-a}c, e^{a}; cumulative phase
-//           per rotary pair (float, reduced to [-pi, pi] every token; the
-//           carry between tiles is reduced too); rotate B and C in place in
-//           bf16x2 arithmetic.  One worker barrier per tile.
+//           the previous tile's MMAs have read those buffers (with segments,
+//           the next tile is also prefetched into L2 at that point).
+//   workers coefficient stage: dt/lambda -> a_t (warp scan, every warp keeps
+//           all tokens in registers), gamma, c, w = e^{a_last-a}c, e^{a}, the
+//           mask tables and each warp's phase increments (for R <= 2 made one
+//           tile ahead, during the previous tile's MMA wait); cumulative phase
+//           per rotary pair (float, reduced to [-pi, pi] at the tile start and
+//           between tiles); rotate B and C in place in bf16x2 arithmetic.  One
+//           worker barrier per tile.
 //   MMA 1   G = C~ B~^T (128x128, K=128)      -> TMEM cols [0,128)
 //           Y_inter = C~ S_bf (128x64, K=128) -> TMEM cols [192,256)
 //   workers w X -> the S_bf region (free after MMA 1); P = mask o G ->
