@@ -573,6 +573,20 @@ def run_layer(cx, name):
         eager_ms = timed(lambda: call(stream))
         graph_ms = timed(g.replay)
         clk.active = False
+    unflushed_ms = None
+    if flush is not None:
+        # the graph replays back to back, inputs left in L2 (reported beside
+        # the flushed figure, never as it)
+        cx.barrier()
+        torch.cuda.synchronize()
+        u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        u0.record(stream)
+        for _ in range(n):
+            g.replay()
+        u1.record(stream)
+        torch.cuda.synchronize()
+        cx.barrier()
+        unflushed_ms = cx.max_over_ranks(u0.elapsed_time(u1)) / n
     assert m3.m3_device_status(ws) == m3.M3_OK
     del g
     gbs = abytes / (graph_ms / 1e3) / 1e9
@@ -589,7 +603,10 @@ def run_layer(cx, name):
                     "chunk_used": plan["chunk_used"]},
            "l2": ("inputs %.2f GB >> 126 MB L2; no flush" % (abytes / 1e9)) if flush is None
            else "L2 flushed (252 MB write) before every timed call",
-           "clocks": clk.summary(), "gpu_launches": 2 * n * plan["launches"], "calls_timed": n}
+           "clocks": clk.summary(), "gpu_launches": (3 if flush is not None else 2) * n * plan["launches"],
+           "calls_timed": n}
+    if unflushed_ms is not None:
+        out["unflushed_ms_per_call"] = unflushed_ms
     del flush, ws, dev
     return out
 
