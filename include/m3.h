@@ -53,15 +53,17 @@
  * wait on on-chip barriers bound every wait; on expiry they record
  * M3_ERR_DEVICE_TIMEOUT in the workspace's status word and return early,
  * which m3_device_status reports.  No C++ exception crosses this boundary.
- * Environment (testing and tuning only; unset in normal use).  Two variables
- * change the launch plan and are read on every plan, so a workspace-size query
- * and the call it serves must see the same values: M3_SCAN_PATH=simt sends
- * the prefill (m3_scan_fwd and the calls built on it) to the float32 SIMT
- * kernels even where the tensor-core path applies; M3_SCAN_NSEG=n (n >= 1)
- * cuts each sequence into n segments (at most one per chunk) instead of the
- * planner's choice; M3_TC_KERNEL=persistent runs the tensor-core prefill on
- * the persistent warp-specialised kernel (one CTA per SM, tiles pipelined
- * across roles) instead of the default tile kernel.
+ * Environment (testing and tuning only; unset in normal use).  Three
+ * variables change the prefill's launch plan and are read on every plan, so
+ * a workspace-size query and the call it serves must see the same values:
+ * M3_SCAN_PATH=simt sends the prefill (m3_scan_fwd and the calls built on it)
+ * to the float32 SIMT kernels even where the tensor-core path applies;
+ * M3_SCAN_NSEG=n (n >= 1) cuts each sequence into n segments (at most one per
+ * chunk) instead of the planner's choice; M3_TC_KERNEL=persistent runs the
+ * tensor-core prefill on the persistent warp-specialised kernel (one CTA per
+ * SM, tiles pipelined across roles) instead of the default tile kernel.
+ * M3_SEQ_COLS=1|2 runs the transition variants with 1 or 2 state columns per
+ * warp instead of 4 (for comparison; measured slower).
  * Buffer extents cannot be checked through plain pointers: every buffer must
  * hold at least the elements its layout gives for `dims` (nothing is read
  * from a buffer whose extent for `dims` is zero); a smaller buffer is read or
