@@ -228,3 +228,12 @@ def test_variants_reject_before_launching():
     for e in (dims(batch=0), dims(seqlen=0)):
         assert _variant_status(e, ptr=None) == m3.M3_OK
         assert _variant_status(e, ptr=None, reflect=True, u=None) == m3.M3_OK
+
+
+def test_static_forget_device_needs_a_current_device():
+    """m3_static_forget_device only clears a cached address: with a device it
+    returns M3_OK (twice in a row too), without one M3_ERR_CUDA; it never
+    launches anything."""
+    st = LIB.m3_static_forget_device()
+    assert st in (m3.M3_OK, m3.M3_ERR_CUDA)
+    assert LIB.m3_static_forget_device() == st
