@@ -359,7 +359,7 @@ CAPTURES = {
     "step_pipe_kernel": ("decode_mimo_r4_b256_h32_P64_N128_x1000", None,
                          304_192_768 + 224_838_400, "fb3967fb581615af"),
     "rope_block_kernel": ("mimo_r4_layer_b8_h32_L4096_P64_N128_Q64_bf16", None,
-                          2_422_809_856 + 2_378_863_104, "1d5355e7ce240d9a"),
+                          2_423_972_608 + 2_379_064_576, "e87a9f369ceb08c4"),
 }
 
 
