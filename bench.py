@@ -5,8 +5,12 @@ Default workload: the chunked prefill (m3_scan_fwd) of the 1.5B-scale MIMO
 layer -- batch 8, 32 heads, L = 4096, P = 64, N = 128, rank 4, chunk 64,
 bfloat16 x/B/C, float32 dt/A/lambda/theta -- on synthetic seeded inputs
 (m3_synth).  One step = one m3_scan_fwd over the whole batch, final carry
-included.  The decode step (m3_step, batch 256, 32 heads, rank 4, carry from
-the prefill) is measured in the same run and reported under "decode".
+included.  The same run reports, each in its own object: "e2e" (pinned host
+inputs in and y out inside the timed region), "rope" (m3_rope_bc), "bwd"
+(m3_scan_bwd), "phase" (two phase interventions), "layers" (the SISO layer and
+the long-context SISO layer), "decode" (m3_step, batch 256, 32 heads, rank 4,
+carry from the prefill), "variants" (damping regimes and reflection on the
+SISO layer) and "cpu_baseline" (the fp64 oracle on a bounded sample).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -49,8 +53,11 @@ def parse():
     ap.add_argument("--no-rope", action="store_true", help="skip the m3_rope_bc measurement")
     ap.add_argument("--no-layers", action="store_true",
                     help="skip the SISO and long-context SISO prefill objects")
-    ap.add_argument("--bwd", action="store_true", help="also time the backward pass m3_scan_bwd")
-    ap.add_argument("--phase", action="store_true", help="also time two phase interventions")
+    ap.add_argument("--no-bwd", action="store_true", help="skip the backward pass m3_scan_bwd")
+    ap.add_argument("--no-phase", action="store_true", help="skip the two phase interventions")
+    # accepted for older command lines: the two measurements now run by default
+    ap.add_argument("--bwd", action="store_true", help=argparse.SUPPRESS)
+    ap.add_argument("--phase", action="store_true", help=argparse.SUPPRESS)
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the damping-regime and reflection variants")
     ap.add_argument("--batch", type=int, default=0,
@@ -980,9 +987,9 @@ def main():
             run_e2e(cx, line, pf)
         if not args.no_rope:
             run_rope(cx, line, pf)
-        if args.bwd:
+        if not args.no_bwd:
             run_bwd(cx, line, pf)
-        if args.phase:
+        if not args.no_phase:
             run_phase(cx, line, pf)
         if args.layer == LAYER and not args.no_layers:
             # the other two prefill workloads, each in its own object

@@ -102,7 +102,7 @@ def test_bench_defaults_are_one_gpu_and_minutes_of_work(monkeypatch):
     a = bench.parse()
     assert a.gpus == 1 and a.warmup >= 3 and 1 <= a.steps <= 200
     assert a.impl == "ours" and a.layer == bench.LAYER and a.decode_steps == 1000
-    assert not a.bwd and not a.phase          # the optional measurements stay off by default
+    assert not a.no_bwd and not a.no_phase    # every measured part runs by default
 
 
 def test_reference_arm_prints_on_rank_0_only():
