@@ -362,7 +362,7 @@ KERNEL_SOURCES = {
 CAPTURES = {
     # kernel: (workload, plan segments or None, bytes per launch, source digest)
     "scan_tc_kernel": ("mimo_r4_layer_b8_h32_L4096_P64_N128_Q64_bf16", 1,
-                       2_984_268_544 + 524_173_568, "af1f9e9274c8c260"),
+                       2_982_520_064 + 523_729_152, "064aefd1c4555e7b"),
     "step_pipe_kernel": ("decode_mimo_r4_b256_h32_P64_N128_x1000", None,
                          304_192_768 + 224_838_400, "fb3967fb581615af"),
     "rope_block_kernel": ("mimo_r4_layer_b8_h32_L4096_P64_N128_Q64_bf16", None,

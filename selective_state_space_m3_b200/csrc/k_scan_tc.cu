@@ -415,7 +415,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     // of token g0 + kk (theta past the tile's end meets dt = 0)
     auto pass1_stage = [&](int kn, float dsl, auto&& thf) {
         // theta loads issued in batches of up to 8 tokens before their use
-        constexpr int KB = TE < 8 ? TE : 8;
+        // (long tiles, one tile ahead: all 16 at once)
+        constexpr int KB = kAhead ? TE : (TE < 8 ? TE : 8);
         float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
         for (int k0 = 0; k0 < TE; k0 += KB) {
