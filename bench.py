@@ -355,9 +355,9 @@ L2_BYTES = 126 * 1024 * 1024
 # workload and plan; otherwise "traffic" is null and the reason is given.
 # The ncu commands are in profiles/.
 KERNEL_SOURCES = {
-    "scan_tc_kernel": ("k_scan_tc.cu", "tc_ptx.cuh", "m3_common.cuh", "m3_kernels.h"),
-    "step_pipe_kernel": ("k_step.cu", "m3_common.cuh", "m3_kernels.h"),
-    "rope_block_kernel": ("k_rope.cu", "m3_common.cuh", "m3_kernels.h"),
+    "scan_tc_kernel": ("k_scan_tc.cu", "tc_ptx.cuh", "m3_common.cuh", "m3_kernels.h", "m3_bounds.cuh"),
+    "step_pipe_kernel": ("k_step.cu", "m3_common.cuh", "m3_kernels.h", "m3_bounds.cuh"),
+    "rope_block_kernel": ("k_rope.cu", "m3_common.cuh", "m3_kernels.h", "m3_bounds.cuh"),
 }
 CAPTURES = {
     # kernel: (workload, plan segments or None, bytes per launch, source digest)

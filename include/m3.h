@@ -318,6 +318,45 @@ m3_status m3_device_status(void* workspace, void* stream);
  * usable.  `workspace` needs at least 256 bytes. */
 m3_status m3_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void* stream);
 
+/* Index checks of the debug build.  The library compiled with
+ * -DM3_DEBUG_BOUNDS=1 (libm3_debug.so beside libm3.so) checks, in every
+ * kernel, each global-memory index against the element count that `dims`
+ * gives the buffer and each shared-memory index against the array or
+ * region it addresses, before the access.  A failed check skips the access
+ * (a load reads zero) and is counted in a device-side record; nothing traps
+ * and the context stays usable.  The release build (libm3.so) has no checks
+ * and its kernels are unchanged by them.
+ *
+ * m3_debug_bounds_report synchronises the device, then fills `out`:
+ * enabled = 1 in the debug build (0 otherwise, with everything else zero),
+ * failures = failed checks since the last clear, and site / index / limit of
+ * the first failure recorded by the lowest-numbered source file that has one
+ * (site = file * 1000 + check: 1 tile prefill, 2 SIMT prefill and segment
+ * combine, 3 decode step, 4 rope, 5 transition variants, 6 backward,
+ * 7 phase prologues, 8 persistent prefill, 9 this self-test; for a span the
+ * index is its last element).  `clear` != 0 resets the records after reading.
+ * M3_ERR_INVALID_ARG for a NULL `out`, M3_ERR_CUDA if the device cannot be
+ * read.  Host call; the release build touches no device. */
+typedef struct m3_bounds_report {
+    int enabled;
+    unsigned int failures;
+    int site;
+    long long index;
+    long long limit;
+} m3_bounds_report;
+m3_status m3_debug_bounds_report(m3_bounds_report* out, int clear);
+
+/* Diagnostic for the checks themselves (debug build only; the release build
+ * returns M3_ERR_UNSUPPORTED and launches nothing): one thread writes 1.0f to
+ * buffer[index] if the check index < limit passes.  The host requires
+ * 0 <= index < capacity and 0 <= limit <= capacity (M3_ERR_INVALID_ARG
+ * otherwise), so with index >= limit the check fails, the store is skipped
+ * and the failure is recorded as site 9001 -- and even a store that were not
+ * skipped would stay inside the caller's `capacity` floats.  `buffer` is a
+ * device pointer to `capacity` floats; enqueued on `stream`. */
+m3_status m3_selftest_bounds_check(float* buffer, long long capacity, long long index, long long limit,
+                                   void* stream);
+
 /* Prefill that allocates nothing and takes no workspace.
  * The paper has no counterpart to this call: it exists for callers that
  * cannot allocate device memory while they run -- for example a plugin

@@ -7,6 +7,12 @@ Every step of the scan runs in the library's CUDA kernels; there is no
 PyTorch or CPU implementation behind these calls, and importing the package
 fails if the library has not been built (``python -m
 selective_state_space_m3_b200.build``).
+
+With ``M3_DEBUG_BOUNDS=1`` in the environment at import, the package loads
+``libm3_debug.so`` instead: the same kernels with every global and
+shared-memory index checked (failed checks skip the access and are counted;
+read them with :func:`m3_debug_bounds_report`).  It is built beside the
+release library (``python -m selective_state_space_m3_b200.build --all``).
 """
 from __future__ import annotations
 
@@ -19,7 +25,8 @@ import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libm3.so")
+DEBUG_BOUNDS = os.environ.get("M3_DEBUG_BOUNDS", "") == "1"
+LIB_PATH = os.path.join(_PKG, "libm3_debug.so" if DEBUG_BOUNDS else "libm3.so")
 
 M3_OK, M3_ERR_INVALID_ARG, M3_ERR_UNSUPPORTED, M3_ERR_WORKSPACE, M3_ERR_CUDA, M3_ERR_DEVICE_TIMEOUT = range(6)
 M3_F32, M3_BF16 = 0, 1
@@ -41,10 +48,16 @@ class _Carry(ctypes.Structure):
     _fields_ = [("h", ctypes.c_void_p), ("prev_B", ctypes.c_void_p), ("prev_x", ctypes.c_void_p)]
 
 
+class _BoundsReport(ctypes.Structure):
+    _fields_ = [("enabled", ctypes.c_int), ("failures", ctypes.c_uint), ("site", ctypes.c_int),
+                ("index", ctypes.c_longlong), ("limit", ctypes.c_longlong)]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: the CUDA library must be built "
-                          "(python -m selective_state_space_m3_b200.build)")
+                          "(python -m selective_state_space_m3_b200.build"
+                          f"{' --debug' if DEBUG_BOUNDS else ''})")
     lib = ctypes.CDLL(LIB_PATH)
     V, S, I = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
     D, C = ctypes.POINTER(_Dims), ctypes.POINTER(_Carry)
@@ -62,6 +75,11 @@ def _load():
     lib.m3_static_forget_device.restype = I
     lib.m3_selftest_bounded_wait.argtypes = [V, S, V]
     lib.m3_selftest_bounded_wait.restype = I
+    lib.m3_debug_bounds_report.argtypes = [ctypes.POINTER(_BoundsReport), I]
+    lib.m3_debug_bounds_report.restype = I
+    LL = ctypes.c_longlong
+    lib.m3_selftest_bounds_check.argtypes = [V, LL, LL, LL, V]
+    lib.m3_selftest_bounds_check.restype = I
     lib.m3_scan_bwd_workspace_size.argtypes = [D, ctypes.POINTER(S)]
     lib.m3_scan_bwd_workspace_size.restype = I
     lib.m3_scan_bwd.argtypes = [D, V, V, V, V, V, V, V, C, V, C, V, V, V, V, V, V, V, C, V, S, V]
@@ -85,7 +103,8 @@ _lib = _load()
 
 # every symbol include/m3.h declares (checked by the CPU test suite)
 ABI_SYMBOLS = ("m3_scan_workspace_size", "m3_scan_fwd", "m3_step", "m3_rope_bc",
-               "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_scan_fwd_static",
+               "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_debug_bounds_report",
+               "m3_selftest_bounds_check", "m3_scan_fwd_static",
                "m3_static_forget_device", "m3_scan_bwd_workspace_size", "m3_scan_bwd", "m3_scan_phase_workspace_size",
                "m3_scan_fwd_phase", "m3_scan_fwd_damped", "m3_scan_fwd_reflect", "m3_status_string")
 
@@ -229,6 +248,24 @@ def m3_selftest_bounded_wait(workspace, stream=None) -> None:
                                          _stream(stream)), "m3_selftest_bounded_wait")
 
 
+def m3_debug_bounds_report(clear: bool = False) -> dict:
+    """The index checks' record (synchronises the device in the debug build):
+    enabled (1 in libm3_debug.so), failures, and site / index / limit of the
+    first failure."""
+    r = _BoundsReport()
+    _check(_lib.m3_debug_bounds_report(ctypes.byref(r), int(bool(clear))), "m3_debug_bounds_report")
+    return {"enabled": r.enabled, "failures": r.failures, "site": r.site, "index": r.index, "limit": r.limit}
+
+
+def m3_selftest_bounds_check(buffer, index: int, limit: int, stream=None) -> None:
+    """Debug build: one thread stores 1.0 to buffer[index] if index < limit
+    (float32 device buffer; index and limit within its size)."""
+    if buffer.dtype != torch.float32:
+        raise TypeError("the self-test buffer is float32")
+    _check(_lib.m3_selftest_bounds_check(_ptr(buffer), buffer.numel(), int(index), int(limit), _stream(stream)),
+           "m3_selftest_bounds_check")
+
+
 def m3_scan_bwd_workspace_size(dims: Dims) -> int:
     n = ctypes.c_size_t(0)
     d = dims.c()
@@ -325,7 +362,8 @@ def raw_lib():
 
 
 __all__ = ["Dims", "Carry", "M3Error", "m3_scan_workspace_size", "m3_scan_fwd", "m3_step",
-           "m3_rope_bc", "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_scan_fwd_static",
+           "m3_rope_bc", "m3_scan_plan", "m3_device_status", "m3_selftest_bounded_wait", "m3_debug_bounds_report",
+           "m3_selftest_bounds_check", "DEBUG_BOUNDS", "m3_scan_fwd_static",
            "m3_static_forget_device", "m3_scan_bwd_workspace_size", "m3_scan_bwd", "m3_status_string",
            "m3_scan_phase_workspace_size", "m3_scan_fwd_phase", "m3_scan_fwd_damped", "m3_scan_fwd_reflect",
            "M3_DAMP_UNDER", "M3_DAMP_CRITICAL", "M3_DAMP_OVER", "io_dtype_of", "ABI_SYMBOLS",

@@ -2,6 +2,10 @@
 
 nvcc cross-compiles for sm_100a without a GPU.  Each .cu file is compiled to
 an object in parallel, then linked into selective_state_space_m3_b200/libm3.so.
+With debug=True the same sources are compiled with -DM3_DEBUG_BOUNDS=1 into
+libm3_debug.so (every kernel index checked; include/m3.h,
+m3_debug_bounds_report), which the package loads instead of libm3.so when
+M3_DEBUG_BOUNDS=1 is set in the environment.
 """
 from __future__ import annotations
 
@@ -16,7 +20,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OUT = os.path.join(PKG, "libm3.so")
+OUT_DEBUG = os.path.join(PKG, "libm3_debug.so")
 OBJ = os.path.join(PKG, "_build")
+OBJ_DEBUG = os.path.join(PKG, "_build", "debug")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include")]
@@ -36,16 +42,20 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
+def build(force: bool = False, verbose: bool = False, extra_flags=(), debug: bool = False) -> str:
+    """Compile and link the release library (or, with debug, the index-checked one); returns its path."""
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdrs = sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) +
                   glob.glob(os.path.join(ROOT, "include", "*.h")))
-    os.makedirs(OBJ, exist_ok=True)
+    obj_dir, out = (OBJ_DEBUG, OUT_DEBUG) if debug else (OBJ, OUT)
+    if debug:
+        extra_flags = (*extra_flags, "-DM3_DEBUG_BOUNDS=1")
+    os.makedirs(obj_dir, exist_ok=True)
     nvcc = _nvcc()
     objs = []
 
     def compile_one(src):
-        obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(obj_dir, os.path.basename(src)[:-3] + ".o")
         if force or _stale(obj, [src] + hdrs):
             cmd = [nvcc, *ARCH, *FLAGS, *extra_flags, "-c", src, "-o", obj]
             if verbose:
@@ -59,15 +69,25 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
 
     with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
         objs = list(ex.map(compile_one, srcs))
-    if force or _stale(OUT, objs):
-        tmp = OUT + f".tmp{os.getpid()}"
+    if force or _stale(out, objs):
+        tmp = out + f".tmp{os.getpid()}"
         cmd = [nvcc, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, OUT)
-    return OUT
+        os.replace(tmp, out)
+    return out
+
+
+def build_all(force: bool = False, verbose: bool = False) -> tuple:
+    """Both libraries: libm3.so and libm3_debug.so."""
+    return build(force, verbose), build(force, verbose, debug=True)
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    if "--debug" in sys.argv:
+        print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug=True))
+    elif "--all" in sys.argv:
+        print(*build_all(force="--force" in sys.argv, verbose="-v" in sys.argv), sep="\n")
+    else:
+        print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))

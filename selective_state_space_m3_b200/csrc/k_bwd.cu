@@ -24,11 +24,25 @@
 // shuffles, reductions over rows shared memory.  Gradients of B, C and theta
 // (shared by the heads of a group) and of A are accumulated with atomics
 // into zeroed float32 buffers.
+#define M3_BOUNDS_FILE 6
+#include "m3_bounds.cuh"
 #include "m3_common.cuh"
 #include "m3_kernels.h"
 
 namespace m3 {
 namespace bwd {
+
+// element counts of the workspace parts (index checks of the debug build)
+__device__ __forceinline__ long long ext_ckpt(const BwdParams& q) {
+    return (long long)q.batch * q.nheads * ((q.seqlen + q.K - 1) / q.K) * q.dstate * q.headdim;
+}
+__device__ __forceinline__ long long ext_scr(const BwdParams& q) {
+    return (long long)q.batch * q.nheads * q.K * q.dstate * q.headdim;
+}
+// the rows (2i, 2i+1) x columns [p0, p0 + 16) of an N x P state block at
+// element offset `off` of a buffer: from row 2i, column p0 to row 2i+1,
+// column p0 + 15
+#define M3_STATE_SPAN(site, off, P, i, p0, ext) M3_SPAN(site, (off) + (size_t)(2 * (i)) * (P) + (p0), (P) + kPW, ext)
 
 constexpr int kPW = 16;            // state columns per thread
 constexpr int kMaxThreads = 256;
@@ -77,9 +91,11 @@ __device__ __forceinline__ void load_init_prev(const BwdParams& q, int b, int h,
     const size_t bh = (size_t)b * H + h;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-        if (q.init_pX) ld16<T>(static_cast<const T*>(q.init_pX) + (bh * R + r) * P + p0, k.x[r]);
+        if (q.init_pX && M3_SPAN(1, (bh * R + r) * P + p0, kPW, ext_pX(q)))
+            ld16<T>(static_cast<const T*>(q.init_pX) + (bh * R + r) * P + p0, k.x[r]);
         else for (int c = 0; c < kPW; ++c) k.x[r][c] = 0.f;
-        k.b[r] = q.init_pB ? ld2<T>(static_cast<const T*>(q.init_pB) + (bh * R + r) * N + 2 * i) : make_float2(0.f, 0.f);
+        k.b[r] = (q.init_pB && M3_SPAN(2, (bh * R + r) * N + 2 * i, 2, ext_pB(q)))
+                     ? ld2<T>(static_cast<const T*>(q.init_pB) + (bh * R + r) * N + 2 * i) : make_float2(0.f, 0.f);
     }
 }
 
@@ -139,22 +155,48 @@ __device__ void stage_block(const BwdParams& q, int b, int h, int g, int t0, int
         const size_t bt = (size_t)b * L + (t >= 0 ? t : 0);
         const uint4* src;
         uint4* dst;
+        long long soff = 0, sext = 0;      // source element offset and buffer extent (debug checks)
+        int doff;                          // destination byte offset in the slot
+        (void)soff; (void)sext;
         if (u < ux) {
             src = reinterpret_cast<const uint4*>(t >= 0 ? static_cast<const T*>(q.x) + ((bt * H + h) * R) * P
                   : (q.init_pX ? static_cast<const T*>(q.init_pX) + (((size_t)b * H + h) * R) * P : nullptr));
             dst = reinterpret_cast<uint4*>(slot + sl.ox);
+            doff = sl.ox;
+            if (M3_DEBUG_BOUNDS) {
+                soff = t >= 0 ? (long long)((bt * H + h) * R) * P : (long long)(((size_t)b * H + h) * R) * P;
+                sext = t >= 0 ? ext_x(q) : ext_pX(q);
+            }
         } else if ((u -= ux) < ub) {
             src = reinterpret_cast<const uint4*>(t >= 0 ? static_cast<const T*>(q.B) + ((bt * G + g) * R) * N
                   : (q.init_pB ? static_cast<const T*>(q.init_pB) + (((size_t)b * H + h) * R) * N : nullptr));
             dst = reinterpret_cast<uint4*>(slot + sl.ob);
+            doff = sl.ob;
+            if (M3_DEBUG_BOUNDS) {
+                soff = t >= 0 ? (long long)((bt * G + g) * R) * N : (long long)(((size_t)b * H + h) * R) * N;
+                sext = t >= 0 ? ext_bc(q) : ext_pB(q);
+            }
         } else if ((u -= ub) < ub) {
             src = t >= 0 ? reinterpret_cast<const uint4*>(static_cast<const T*>(q.C) + ((bt * G + g) * R) * N) : nullptr;
             dst = reinterpret_cast<uint4*>(slot + sl.oc);
+            doff = sl.oc;
+            if (M3_DEBUG_BOUNDS) {
+                soff = (long long)((bt * G + g) * R) * N;
+                sext = ext_bc(q);
+            }
         } else {
             u -= ub;
             src = t >= 0 ? reinterpret_cast<const uint4*>(static_cast<const T*>(q.dy) + ((bt * H + h) * R) * P) : nullptr;
             dst = reinterpret_cast<uint4*>(slot + sl.oy);
+            doff = sl.oy;
+            if (M3_DEBUG_BOUNDS) {
+                soff = (long long)((bt * H + h) * R) * P;
+                sext = ext_x(q);
+            }
         }
+        (void)doff;
+        if (!M3_SPAN(3, (slot - stg) + doff + 16 * u, 16, dyn_smem_bytes())) continue;
+        if (src && !M3_SPAN(4, soff * (long long)sizeof(T) + 16 * u, 16, sext * (long long)sizeof(T))) src = nullptr;
         dst[u] = src ? src[u] : make_uint4(0u, 0u, 0u, 0u);
     }
     {
@@ -165,8 +207,11 @@ __device__ void stage_block(const BwdParams& q, int b, int h, int g, int t0, int
             float v = 0.f;
             if (t >= 0) {
                 const size_t bt = (size_t)b * L + t;
-                v = u < N / 2 ? q.theta[(bt * G + g) * (N / 2) + u] : (u == N / 2 ? q.dt[bt * H + h] : q.lam[bt * H + h]);
+                if (u < N / 2 ? M3_IN(5, (bt * G + g) * (N / 2) + u, ext_theta(q)) : M3_IN(6, bt * H + h, ext_tok(q)))
+                    v = u < N / 2 ? q.theta[(bt * G + g) * (N / 2) + u] : (u == N / 2 ? q.dt[bt * H + h] : q.lam[bt * H + h]);
             }
+            if (!M3_SPAN(7, (slot - stg) + (u < N / 2 ? sl.oth + 4 * u : sl.osc + 4 * (u - N / 2)), 4, dyn_smem_bytes()))
+                continue;
             if (u < N / 2) reinterpret_cast<float*>(slot + sl.oth)[u] = v;
             else reinterpret_cast<float*>(slot + sl.osc)[u - N / 2] = v;
         }
@@ -222,15 +267,16 @@ __global__ void __launch_bounds__(kMaxThreads) ckpt_kernel(BwdParams q) {
     const int i = act ? tid / NPB : 0, p0 = act ? (tid % NPB) * kPW : 0;
     const int g = h / (q.nheads / q.ngroups);
     const size_t bh = (size_t)b * q.nheads + h;
-    const float A = q.A[h];
+    const float A = M3_IN(10, h, q.nheads) ? q.A[h] : 0.f;
     float h0[kPW], h1[kPW];
-    if (q.init_h) ld_state(q.init_h + bh * N * P, P, i, p0, h0, h1);
+    if (q.init_h && M3_STATE_SPAN(11, bh * N * P, P, i, p0, ext_h(q))) ld_state(q.init_h + bh * N * P, P, i, p0, h0, h1);
     else for (int c = 0; c < kPW; ++c) { h0[c] = 0.f; h1[c] = 0.f; }
     extern __shared__ __align__(16) uint8_t stg[];
     const StageLayout sl = stage_layout(R, N, P, (int)sizeof(T));
     for (int c = 0; c < nck; ++c) {
         const int t0 = c * K, t1 = min(L, t0 + K);
-        if (act) st_state(q.ws_ckpt + (bh * nck + c) * N * P, P, i, p0, h0, h1);
+        if (act && M3_STATE_SPAN(12, (bh * nck + c) * N * P, P, i, p0, ext_ckpt(q)))
+            st_state(q.ws_ckpt + (bh * nck + c) * N * P, P, i, p0, h0, h1);
         stage_block<T, R>(q, b, h, g, t0, t1, stg, sl, false);
         __syncthreads();
         if (act)
@@ -254,19 +300,23 @@ __global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
     const int i = act ? tid / NPB : 0, pb = act ? tid % NPB : 0, p0 = pb * kPW;
     const int g = h / (H / G);
     const size_t bh = (size_t)b * H + h;
-    const float A = q.A[h];
+    const float A = M3_IN(20, h, H) ? q.A[h] : 0.f;
     const int nwarps = (blockDim.x + 31) / 32;
     float* scr = q.ws_scratch + bh * (size_t)K * N * P;
+    const size_t scr_off = bh * (size_t)K * N * P;   // (debug checks)
+    (void)scr_off;
 
     float g0[kPW], g1[kPW], db0[kPW], db1[kPW];
-    if (q.d_fin_h && act) ld_state(q.d_fin_h + bh * N * P, P, i, p0, g0, g1);
+    if (q.d_fin_h && act && M3_STATE_SPAN(21, bh * N * P, P, i, p0, ext_h(q)))
+        ld_state(q.d_fin_h + bh * N * P, P, i, p0, g0, g1);
     else for (int c = 0; c < kPW; ++c) { g0[c] = 0.f; g1[c] = 0.f; }
     for (int c = 0; c < kPW; ++c) { db0[c] = 0.f; db1[c] = 0.f; }
     float dA_acc = 0.f;
     // gradients arriving at the final (B, x) copies: into dB_{L-1} (dx_{L-1} below)
     if (q.d_fin_pB && L > 0)
         for (int e = tid; e < R * N; e += blockDim.x)
-            atomicAdd(q.dB + (((size_t)b * L + L - 1) * G + g) * R * N + e, q.d_fin_pB[bh * R * N + e]);
+            if (M3_IN(22, (((size_t)b * L + L - 1) * G + g) * R * N + e, ext_bc(q)) && M3_IN(23, bh * R * N + e, ext_pB(q)))
+                atomicAdd(q.dB + (((size_t)b * L + L - 1) * G + g) * R * N + e, q.d_fin_pB[bh * R * N + e]);
 
     extern __shared__ __align__(16) uint8_t stg[];
     const StageLayout sl = stage_layout(R, N, P, (int)sizeof(T));
@@ -280,11 +330,14 @@ __global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
         {
             float h0[kPW], h1[kPW];
             if (act) {
-                ld_state(q.ws_ckpt + (bh * nck + c) * N * P, P, i, p0, h0, h1);
+                if (M3_STATE_SPAN(24, (bh * nck + c) * N * P, P, i, p0, ext_ckpt(q)))
+                    ld_state(q.ws_ckpt + (bh * nck + c) * N * P, P, i, p0, h0, h1);
+                else for (int e = 0; e < kPW; ++e) h0[e] = h1[e] = 0.f;
                 for (int t = t0; t < t1; ++t) {
                     fwd_token_stage<T, R>(h0, h1, stg + (size_t)(t - t0) * sl.bytes,
                                           stg + (size_t)(t - t0 + 1) * sl.bytes, sl, N, P, i, p0, A);
-                    st_state(scr + (size_t)(t - t0) * N * P, P, i, p0, h0, h1);
+                    if (M3_STATE_SPAN(25, scr_off + (size_t)(t - t0) * N * P, P, i, p0, ext_scr(q)))
+                        st_state(scr + (size_t)(t - t0) * N * P, P, i, p0, h0, h1);
                 }
             }
         }
@@ -308,7 +361,8 @@ __global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
             // phase 1 -- readout: g += C_t dy_t ; dC_t = h_t dy_t^T
             {
                 float ht0[kPW], ht1[kPW];
-                if (act) ld_state(scr + (size_t)(t - t0) * N * P, P, i, p0, ht0, ht1);
+                if (act && M3_STATE_SPAN(26, scr_off + (size_t)(t - t0) * N * P, P, i, p0, ext_scr(q)))
+                    ld_state(scr + (size_t)(t - t0) * N * P, P, i, p0, ht0, ht1);
                 else for (int e = 0; e < kPW; ++e) ht0[e] = ht1[e] = 0.f;
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
@@ -328,7 +382,7 @@ __global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
                         dc0 += __shfl_xor_sync(0xffffffffu, dc0, o);
                         dc1 += __shfl_xor_sync(0xffffffffu, dc1, o);
                     }
-                    if (act && pb == 0) {
+                    if (act && pb == 0 && M3_SPAN(27, ((bt * G + g) * R + r) * N + 2 * i, 2, ext_bc(q))) {
                         float* dCt = q.dC + ((bt * G + g) * R + r) * N + 2 * i;
                         atomicAdd(dCt, dc0);
                         atomicAdd(dCt + 1, dc1);
@@ -357,7 +411,7 @@ __global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
                     db_0 += __shfl_xor_sync(0xffffffffu, db_0, o);
                     db_1 += __shfl_xor_sync(0xffffffffu, db_1, o);
                 }
-                if (act && pb == 0) {
+                if (act && pb == 0 && M3_SPAN(28, ((bt * G + g) * R + r) * N + 2 * i, 2, ext_bc(q))) {
                     float* dBt = q.dB + ((bt * G + g) * R + r) * N + 2 * i;
                     atomicAdd(dBt, db_0);
                     atomicAdd(dBt + 1, db_1);
@@ -366,7 +420,7 @@ __global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
                 for (int o = NPB; o < 32; o <<= 1)
 #pragma unroll
                     for (int e = 0; e < kPW; ++e) dxr[e] += __shfl_xor_sync(0xffffffffu, dxr[e], o);
-                if (lane < NPB)
+                if (lane < NPB && M3_SPAN(29, (warp * NPB + lane) * kPW, kPW, kMaxThreads / 32 * 64))
 #pragma unroll
                     for (int e = 0; e < kPW; ++e) sDx[par][r][(warp * NPB + lane) * kPW + e] = dxr[e];
             }
@@ -382,7 +436,8 @@ __global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
             }
             {
                 float hp0[kPW], hp1[kPW];
-                if (act) {
+                if (act && (t > t0 ? M3_STATE_SPAN(30, scr_off + (size_t)(t - 1 - t0) * N * P, P, i, p0, ext_scr(q))
+                                   : M3_STATE_SPAN(31, (bh * nck + c) * N * P, P, i, p0, ext_ckpt(q)))) {
                     if (t > t0) ld_state(scr + (size_t)(t - 1 - t0) * N * P, P, i, p0, hp0, hp1);
                     else ld_state(q.ws_ckpt + (bh * nck + c) * N * P, P, i, p0, hp0, hp1);
                 } else {
@@ -426,7 +481,7 @@ __global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
             for (int o = 1; o < NPB; o <<= 1) dph += __shfl_xor_sync(0xffffffffu, dph, o);
             float s_ph = 0.f;
             if (act && pb == 0) {
-                atomicAdd(q.dtheta + (bt * G + g) * (N / 2) + i, dph * d);
+                if (M3_IN(32, (bt * G + g) * (N / 2) + i, ext_theta(q))) atomicAdd(q.dtheta + (bt * G + g) * (N / 2) + i, dph * d);
                 s_ph = dph * th;
             }
             // scalars: reduce over the warp, then over warps in shared memory
@@ -437,7 +492,7 @@ __global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
                 s_be += __shfl_xor_sync(0xffffffffu, s_be, o);
                 s_ph += __shfl_xor_sync(0xffffffffu, s_ph, o);
             }
-            if (lane == 0) {
+            if (lane == 0 && M3_IN(33, warp, 8)) {
                 sRed[par][warp][0] = s_ga;
                 sRed[par][warp][1] = s_al;
                 sRed[par][warp][2] = s_be;
@@ -449,29 +504,33 @@ __global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
                 const int r = e / P, p = e % P, pbk = p / kPW, col = p % kPW;
                 float acc = 0.f;
                 for (int w = 0; w < nwarps; ++w)
-                    if (w * 32 < nact) acc += sDx[par][r][(w * NPB + pbk) * kPW + col];
-                if (t == L - 1 && q.d_fin_pX) acc += q.d_fin_pX[bh * R * P + e];
-                q.dx[((bt * H + h) * R) * P + e] = acc;
+                    if (w * 32 < nact && M3_IN(34, (w * NPB + pbk) * kPW + col, kMaxThreads / 32 * 64))
+                        acc += sDx[par][r][(w * NPB + pbk) * kPW + col];
+                if (t == L - 1 && q.d_fin_pX && M3_IN(35, bh * R * P + e, ext_pX(q))) acc += q.d_fin_pX[bh * R * P + e];
+                if (M3_IN(36, ((bt * H + h) * R) * P + e, ext_x(q))) q.dx[((bt * H + h) * R) * P + e] = acc;
             }
             if (tid == 0) {
                 float dga = 0.f, dal = 0.f, dbe = 0.f, dphth = 0.f;
-                for (int w = 0; w < nwarps; ++w) {
+                for (int w = 0; w < nwarps && M3_IN(37, w, 8); ++w) {
                     dga += sRed[par][w][0];
                     dal += sRed[par][w][1];
                     dbe += sRed[par][w][2];
                     dphth += sRed[par][w][3];
                 }
-                q.ddt[bt * H + h] = dal * A * al + dbe * (1.f - lm) * (al + d * A * al) + dga * lm + dphth;
-                q.dlam[bt * H + h] = -dbe * d * al + dga * d;
+                if (M3_IN(38, bt * H + h, ext_tok(q))) {
+                    q.ddt[bt * H + h] = dal * A * al + dbe * (1.f - lm) * (al + d * A * al) + dga * lm + dphth;
+                    q.dlam[bt * H + h] = -dbe * d * al + dga * d;
+                }
                 dA_acc += dal * d * al + dbe * (1.f - lm) * d * d * al;
             }
             par ^= 1;
         }
         __syncthreads();      // scratch is rewritten by the next block's forward
     }
-    if (tid == 0) atomicAdd(q.dA + h, dA_acc);
+    if (tid == 0 && M3_IN(39, h, H)) atomicAdd(q.dA + h, dA_acc);
     // carry-in gradients: d h_{-1} = g ; d prev_B = D_{-1} prev_x ; d prev_x = D_{-1}^T prev_B
-    if (q.d_init_h && act) st_state(q.d_init_h + bh * N * P, P, i, p0, g0, g1);
+    if (q.d_init_h && act && M3_STATE_SPAN(40, bh * N * P, P, i, p0, ext_h(q)))
+        st_state(q.d_init_h + bh * N * P, P, i, p0, g0, g1);
     if (q.d_init_pB || q.d_init_pX) {
         Tok<R> pv;
         load_init_prev<T, R>(q, b, h, i, p0, pv);
@@ -496,6 +555,7 @@ __global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
         if (q.d_init_pB && act && pb == 0)
 #pragma unroll
             for (int r = 0; r < R; ++r) {
+                if (!M3_SPAN(41, (bh * R + r) * N + 2 * i, 2, ext_pB(q))) continue;
                 q.d_init_pB[(bh * R + r) * N + 2 * i] = dpb[r][0];
                 q.d_init_pB[(bh * R + r) * N + 2 * i + 1] = dpb[r][1];
             }
@@ -504,7 +564,7 @@ __global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
             for (int r = 0; r < R; ++r)
 #pragma unroll
                 for (int e = 0; e < kPW; ++e) dpx[r][e] += __shfl_xor_sync(0xffffffffu, dpx[r][e], o);
-        if (lane < NPB)
+        if (lane < NPB && M3_SPAN(42, (warp * NPB + lane) * kPW, kPW, kMaxThreads / 32 * 64))
 #pragma unroll
             for (int r = 0; r < R; ++r)
 #pragma unroll
@@ -515,8 +575,9 @@ __global__ void __launch_bounds__(kMaxThreads, 2) bwd_kernel(BwdParams q) {
                 const int r = e / P, p = e % P, pbk = p / kPW, col = p % kPW;
                 float acc = 0.f;
                 for (int w = 0; w < nwarps; ++w)
-                    if (w * 32 < nact) acc += sDx[0][r][(w * NPB + pbk) * kPW + col];
-                q.d_init_pX[(bh * R + r) * P + p] = acc;
+                    if (w * 32 < nact && M3_IN(43, (w * NPB + pbk) * kPW + col, kMaxThreads / 32 * 64))
+                        acc += sDx[0][r][(w * NPB + pbk) * kPW + col];
+                if (M3_IN(44, (bh * R + r) * P + p, ext_pX(q))) q.d_init_pX[(bh * R + r) * P + p] = acc;
             }
     }
 }
@@ -567,3 +628,5 @@ cudaError_t launch_bwd(const m3_dims& d, const BwdParams& q, cudaStream_t st) {
 }
 
 }  // namespace m3
+
+M3_BOUNDS_EXPORT(bwd)

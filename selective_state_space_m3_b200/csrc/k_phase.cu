@@ -12,6 +12,8 @@
 //     (m3_rope_bc, Proposition 3 of the "Mamba-3" summary, b-lab.team,
 //     section 2) with theta = 0, the unrotated side copied per head
 //     (expand_heads_kernel).
+#define M3_BOUNDS_FILE 7
+#include "m3_bounds.cuh"
 #include "m3_common.cuh"
 #include "m3_kernels.h"
 
@@ -26,11 +28,14 @@ __global__ void theta_transform_kernel(int mode, const float* __restrict__ in, c
     for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
         const size_t row = e / NH;
         const int i = (int)(e % NH);
-        float v;
+        float v = 0.f;
         switch (mode) {
             case M3_PHASE_ZERO: v = 0.f; break;
             case M3_PHASE_REVERSE: v = -in[e]; break;
-            case M3_PHASE_SHUFFLE: v = in[row * NH + perm[i]]; break;
+            case M3_PHASE_SHUFFLE:
+                // perm holds NH indices the host checked to be a permutation of [0, NH)
+                if (M3_IN(1, perm[i], NH)) v = in[row * NH + perm[i]];
+                break;
             case M3_PHASE_FIXED: v = freq[(row % G) * NH + i]; break;
             default: v = in[e]; break;
         }
@@ -48,7 +53,8 @@ __global__ void expand_heads_kernel(const uint4* __restrict__ src, uint4* __rest
         const int h = (int)(rest % H);
         const size_t bt = rest / H;
         const int g = h / (H / G);
-        dst[e] = src[(bt * G + g) * row_units + u];
+        if (M3_IN(2, (bt * G + g) * row_units + u, bt_count * (size_t)G * row_units))
+            dst[e] = src[(bt * G + g) * row_units + u];
     }
 }
 
@@ -76,3 +82,5 @@ cudaError_t launch_expand_heads(const void* src, void* dst, size_t bt_count, int
 }
 
 }  // namespace m3
+
+M3_BOUNDS_EXPORT(phase)

@@ -12,10 +12,21 @@
 // advances the running phase (double precision, reduced to [-pi, pi] every
 // token) and stores cos/sin per (token, pair), then all threads rotate the
 // block's B and C pairs with coalesced pair-wide loads and stores.
+#define M3_BOUNDS_FILE 4
+#include "m3_bounds.cuh"
 #include "m3_common.cuh"
 #include "m3_kernels.h"
 
 namespace m3 {
+
+// element counts of the per-head outputs (B~, C~; the phase), for the index
+// checks of the debug build
+__device__ __forceinline__ long long rx_rot(const RopeParams& q) {
+    return (long long)q.batch * q.seqlen * q.nheads * q.rank * q.dstate;
+}
+__device__ __forceinline__ long long rx_phase(const RopeParams& q) {
+    return (long long)q.batch * q.seqlen * q.nheads * (q.dstate / 2);
+}
 
 template <typename T> struct Pair;
 template <> struct Pair<float> {
@@ -52,15 +63,18 @@ __global__ void __launch_bounds__(256) rope_kernel(RopeParams q) {
     float* sSin = sCos + kRopeTB * NH;    // [TB][NH]
     float* sDt = sSin + kRopeTB * NH;     // [TB]
     const int tid = threadIdx.x;
+    if (!M3_SPAN(1, (sDt - smem) * 4, kRopeTB * 4, dyn_smem_bytes())) return;
 
     double phi[2] = {0.0, 0.0};           // pairs tid and tid + 256 (N <= 1024)
     for (int t0 = 0; t0 < L; t0 += kRopeTB) {
         const int tb = min(kRopeTB, L - t0);
         for (int e = tid; e < tb * NH; e += blockDim.x) {
             const int k = e / NH, i = e % NH;
-            sTh[e] = q.theta[(((size_t)b * L + t0 + k) * G + g) * NH + i];
+            sTh[e] = M3_IN(2, (((size_t)b * L + t0 + k) * G + g) * NH + i, ext_theta(q))
+                         ? q.theta[(((size_t)b * L + t0 + k) * G + g) * NH + i] : 0.f;
         }
-        for (int k = tid; k < tb; k += blockDim.x) sDt[k] = q.dt[((size_t)b * L + t0 + k) * H + h];
+        for (int k = tid; k < tb; k += blockDim.x)
+            sDt[k] = M3_IN(3, ((size_t)b * L + t0 + k) * H + h, ext_tok(q)) ? q.dt[((size_t)b * L + t0 + k) * H + h] : 0.f;
         __syncthreads();
         for (int s = 0; s < 2; ++s) {
             const int i = tid + s * blockDim.x;
@@ -72,7 +86,8 @@ __global__ void __launch_bounds__(256) rope_kernel(RopeParams q) {
                 sincosf((float)ph, &sv, &cv);
                 sCos[k * NH + i] = cv;
                 sSin[k * NH + i] = sv;
-                if (q.phase) q.phase[(((size_t)b * L + t0 + k) * H + h) * NH + i] = (float)ph;
+                if (q.phase && M3_IN(4, (((size_t)b * L + t0 + k) * H + h) * NH + i, rx_phase(q)))
+                    q.phase[(((size_t)b * L + t0 + k) * H + h) * NH + i] = (float)ph;
             }
             phi[s] = ph;
         }
@@ -86,6 +101,7 @@ __global__ void __launch_bounds__(256) rope_kernel(RopeParams q) {
             const size_t t = (size_t)b * L + t0 + k;
             const size_t src = ((t * G + g) * R + r) * N + 2 * i;
             const size_t dst = ((t * H + h) * R + r) * N + 2 * i;
+            if (!M3_SPAN(5, src, 2, ext_bc(q)) || !M3_SPAN(6, dst, 2, rx_rot(q))) continue;
             const float c = sCos[k * NH + i], s = sSin[k * NH + i];
             const auto bv = Pair<T>::ld(Bin + src);
             const auto cv = Pair<T>::ld(Cin + src);
@@ -173,9 +189,12 @@ __global__ void __launch_bounds__(256, 3) rope_block_kernel(RopeParams q) {
 #pragma unroll
         for (int j = 0; j < kThPer; ++j) {
             const int e = tid + 256 * j, k = min(e / kRpPairs, tbn - 1), i = e % kRpPairs;
-            thr[j] = __ldg(q.theta + (((size_t)b * L + tn + k) * G + g) * NH + i0 + i);
+            thr[j] = M3_IN(10, (((size_t)b * L + tn + k) * G + g) * NH + i0 + i, ext_theta(q))
+                         ? __ldg(q.theta + (((size_t)b * L + tn + k) * G + g) * NH + i0 + i) : 0.f;
         }
-        if (tid < kRpTok) dtr = __ldg(q.dt + ((size_t)b * L + tn + min(tid, tbn - 1)) * H + h);
+        if (tid < kRpTok)
+            dtr = M3_IN(11, ((size_t)b * L + tn + min(tid, tbn - 1)) * H + h, ext_tok(q))
+                      ? __ldg(q.dt + ((size_t)b * L + tn + min(tid, tbn - 1)) * H + h) : 0.f;
     };
     load_block(0);
     for (int t0 = 0; t0 < L; t0 += kRpTok) {
@@ -209,7 +228,8 @@ __global__ void __launch_bounds__(256, 3) rope_block_kernel(RopeParams q) {
             float sv, cv;
             sincosf((float)ph, &sv, &cv);
             sCS[kk][p] = make_float2(cv, sv);
-            if (q.phase && kk < tb) q.phase[(((size_t)b * L + t0 + kk) * H + h) * NH + i0 + p] = (float)ph;
+            if (q.phase && kk < tb && M3_IN(12, (((size_t)b * L + t0 + kk) * H + h) * NH + i0 + p, rx_phase(q)))
+                q.phase[(((size_t)b * L + t0 + kk) * H + h) * NH + i0 + p] = (float)ph;
         }
         __syncthreads();                                 // sCS ready; every thread has read sCarry
         if (qg == 0) sCarry[p] = wrap_pi(sCarry[p] + tot);
@@ -223,6 +243,10 @@ __global__ void __launch_bounds__(256, 3) rope_block_kernel(RopeParams q) {
                 const int e = min(e0 + tid + 256 * u, items - 1);
                 const int v = e % NV, kr = e / NV, r = kr % R, k = kr / R;
                 const size_t src = ((((size_t)b * L + t0 + k) * G + g) * R + r) * N + 2 * (i0 + v * VP);
+                if (!M3_SPAN(13, src, 2 * VP, ext_bc(q))) {
+                    vb[u] = vc[u] = make_uint4(0u, 0u, 0u, 0u);
+                    continue;
+                }
                 vb[u] = *reinterpret_cast<const uint4*>(Bin + src);
                 vc[u] = *reinterpret_cast<const uint4*>(Cin + src);
             }
@@ -244,6 +268,7 @@ __global__ void __launch_bounds__(256, 3) rope_block_kernel(RopeParams q) {
                     fc[2 * j] = cs.x * c0 + cs.y * c1;
                     fc[2 * j + 1] = cs.x * c1 - cs.y * c0;
                 }
+                if (!M3_SPAN(14, dst, 2 * VP, rx_rot(q))) continue;
                 *reinterpret_cast<uint4*>(Bo + dst) = Vec16<T>::pack(fb);
                 *reinterpret_cast<uint4*>(Co + dst) = Vec16<T>::pack(fc);
             }
@@ -277,3 +302,5 @@ m3_status launch_rope(const m3_dims& d, const RopeParams& q, cudaStream_t st) {
 }
 
 }  // namespace m3
+
+M3_BOUNDS_EXPORT(rope)

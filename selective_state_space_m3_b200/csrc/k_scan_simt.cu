@@ -27,6 +27,8 @@
 //      S_in(0) = h_{-1} + (1 - lambda_0) dt_0 B_{-1} x_{-1}^T;
 //   3. main kernel: each segment walks its chunks from S_in(k), writes y, and
 //      the last segment writes the final carry.
+#define M3_BOUNDS_FILE 2
+#include "m3_bounds.cuh"
 #include "m3_common.cuh"
 #include "m3_kernels.h"
 
@@ -44,12 +46,14 @@ template <typename T>
 __device__ __forceinline__ float carry_in(const ScanParams& q, int b, int h, int n, int p, float w0) {
     const int N = q.dstate, P = q.headdim, R = q.rank;
     const size_t bh = (size_t)b * q.nheads + h;
-    float v = q.init_h ? q.init_h[(bh * N + n) * P + p] : 0.f;
+    float v = (q.init_h && M3_IN(1, (bh * N + n) * P + p, ext_h(q))) ? q.init_h[(bh * N + n) * P + p] : 0.f;
     if (q.init_pB && q.init_pX) {
         const T* pB = static_cast<const T*>(q.init_pB) + bh * R * N;
         const T* pX = static_cast<const T*>(q.init_pX) + bh * R * P;
         float acc = 0.f;
-        for (int r = 0; r < R; ++r) acc = fmaf(ld_io(pB + r * N + n), ld_io(pX + r * P + p), acc);
+        for (int r = 0; r < R; ++r)
+            if (M3_IN(2, bh * R * N + r * N + n, ext_pB(q)) && M3_IN(3, bh * R * P + r * P + p, ext_pX(q)))
+                acc = fmaf(ld_io(pB + r * N + n), ld_io(pX + r * P + p), acc);
         v = fmaf(w0, acc, v);
     }
     return v;
@@ -66,7 +70,9 @@ __global__ void __launch_bounds__(256) scan_simt_kernel(ScanParams q) {
     const int tok1 = min(L, (seg + 1) * q.cps * qs);
     const size_t bh = (size_t)b * H + h;
     const size_t bhs = bh * q.nseg + seg;
-    const float Ah = q.A[h];
+    const float Ah = M3_IN(4, h, H) ? q.A[h] : 0.f;
+    const long long ext_ws = (long long)q.batch * H * q.nseg;   // segment summaries (debug checks)
+    (void)ext_ws;
 
     double* sPhi = smem_d;                                   // [NH]
     float* sf = reinterpret_cast<float*>(sPhi + NH);
@@ -85,15 +91,21 @@ __global__ void __launch_bounds__(256) scan_simt_kernel(ScanParams q) {
     float* sG = sf;                   if (!SUMMARY) sf += QRmax * QRmax;
     float* sS = sf;                   sf += N * P;
     float* sScal = sf;                // [0] = chunk decay e^{a_last}, [1] = segment log-decay
+    // the carved arrays end inside the launch's dynamic shared memory
+    if (!M3_SPAN(5, reinterpret_cast<const char*>(sScal) - reinterpret_cast<const char*>(smem_d), 8,
+                 dyn_smem_bytes()))
+        return;
 
     for (int i = tid; i < NH; i += nt) sPhi[i] = 0.0;
     if (tid == 0) sScal[1] = 0.f;
     if (SUMMARY) {
         for (int e = tid; e < N * P; e += nt) sS[e] = 0.f;
     } else if (q.nseg > 1) {
-        for (int e = tid; e < N * P; e += nt) sS[e] = q.ws_sin[bhs * N * P + e];
+        for (int e = tid; e < N * P; e += nt)
+            sS[e] = M3_IN(6, bhs * N * P + e, ext_ws * N * P) ? q.ws_sin[bhs * N * P + e] : 0.f;
     } else {
-        const float w0 = L > 0 ? (1.f - q.lam[(size_t)b * L * H + h]) * q.dt[(size_t)b * L * H + h] : 0.f;
+        const float w0 = (L > 0 && M3_IN(7, (size_t)b * L * H + h, ext_tok(q)))
+                             ? (1.f - q.lam[(size_t)b * L * H + h]) * q.dt[(size_t)b * L * H + h] : 0.f;
         for (int e = tid; e < N * P; e += nt) sS[e] = carry_in<T>(q, b, h, e / P, e % P, w0);
     }
     __syncthreads();
@@ -109,6 +121,7 @@ __global__ void __launch_bounds__(256) scan_simt_kernel(ScanParams q) {
         const int QR = qc * R;
         for (int k = tid; k < qc + has_next; k += nt) {
             const size_t o = ((size_t)b * L + c0 + k) * H + h;
+            if (!M3_IN(8, k, qs + 1) || !M3_IN(9, o, ext_tok(q))) continue;
             sDt[k] = q.dt[o];
             sLam[k] = q.lam[o];
         }
@@ -132,10 +145,12 @@ __global__ void __launch_bounds__(256) scan_simt_kernel(ScanParams q) {
         for (int i = tid; i < NH; i += nt) {
             double ph = sPhi[i];
             for (int k = 0; k < qc; ++k) {
-                const float th = q.theta[(((size_t)b * L + c0 + k) * G + g) * NH + i];
+                const float th = M3_IN(10, (((size_t)b * L + c0 + k) * G + g) * NH + i, ext_theta(q))
+                                     ? q.theta[(((size_t)b * L + c0 + k) * G + g) * NH + i] : 0.f;
                 ph = wrap_pi(ph + (double)sDt[k] * (double)th);
                 float sv, cv;
                 sincosf((float)ph, &sv, &cv);
+                if (!M3_IN(11, k * NH + i, qs * NH)) continue;
                 sCos[k * NH + i] = cv;
                 sSin[k * NH + i] = sv;
             }
@@ -146,6 +161,9 @@ __global__ void __launch_bounds__(256) scan_simt_kernel(ScanParams q) {
         for (int e = tid; e < qc * R * NH; e += nt) {
             const int i = e % NH, kr = e / NH, k = kr / R;
             const size_t src = ((((size_t)b * L + c0 + k) * G + g) * R + (kr % R)) * N + 2 * i;
+            if (!M3_IN(12, k * NH + i, qs * NH) || !M3_SPAN(13, kr * N + 2 * i, 2, QRmax * N) ||
+                !M3_SPAN(14, src, 2, ext_bc(q)))
+                continue;
             const float c = sCos[k * NH + i], s = sSin[k * NH + i];
             const float b0 = ld_io(Bg + src), b1 = ld_io(Bg + src + 1);
             sB[kr * N + 2 * i] = c * b0 + s * b1;
@@ -158,6 +176,8 @@ __global__ void __launch_bounds__(256) scan_simt_kernel(ScanParams q) {
         }
         for (int e = tid; e < QR * P; e += nt) {
             const int p = e % P, kr = e / P, k = kr / R;
+            if (!M3_IN(15, e, QRmax * P) || !M3_IN(16, ((((size_t)b * L + c0 + k) * H + h) * R + (kr % R)) * P + p, ext_x(q)))
+                continue;
             sX[e] = ld_io(xg + ((((size_t)b * L + c0 + k) * H + h) * R + (kr % R)) * P + p);
         }
         __syncthreads();
@@ -166,6 +186,9 @@ __global__ void __launch_bounds__(256) scan_simt_kernel(ScanParams q) {
             for (int e = tid; e < QR * QR; e += nt) {
                 const int i = e / QR, j = e % QR, ki = i / R, kj = j / R;
                 float v = 0.f;
+                if (!M3_IN(17, e, QRmax * QRmax) || !M3_SPAN(18, i * N, N, QRmax * N) ||
+                    !M3_SPAN(19, j * N, N, QRmax * N) || !M3_IN(20, ki, qs) || !M3_IN(21, kj, qs))
+                    continue;
                 if (kj <= ki) {
                     float dot = 0.f;
                     for (int n = 0; n < N; ++n) dot = fmaf(sC[i * N + n], sB[j * N + n], dot);
@@ -180,6 +203,10 @@ __global__ void __launch_bounds__(256) scan_simt_kernel(ScanParams q) {
                 const int i = e / P, p = e % P, ki = i / R;
                 float acc = 0.f, acc2 = 0.f;
                 const int jend = (ki + 1) * R;
+                if (!M3_SPAN(22, i * QR, jend, QRmax * QRmax) || !M3_IN(23, (jend - 1) * P + p, QRmax * P) ||
+                    !M3_SPAN(24, i * N, N, QRmax * N) || !M3_IN(25, ki, qs) ||
+                    !M3_IN(26, ((((size_t)b * L + c0 + ki) * H + h) * R + (i % R)) * P + p, ext_x(q)))
+                    continue;
                 for (int j = 0; j < jend; ++j) acc = fmaf(sG[i * QR + j], sX[j * P + p], acc);
                 for (int n = 0; n < N; ++n) acc2 = fmaf(sC[i * N + n], sS[n * P + p], acc2);
                 st_io(yg + ((((size_t)b * L + c0 + ki) * H + h) * R + (i % R)) * P + p,
@@ -192,6 +219,9 @@ __global__ void __launch_bounds__(256) scan_simt_kernel(ScanParams q) {
         for (int e = tid; e < N * P; e += nt) {
             const int n = e / P, p = e % P;
             float acc = 0.f;
+            if (!M3_IN(27, (QR - 1) * N + n, QRmax * N) || !M3_IN(28, (QR - 1) * P + p, QRmax * P) ||
+                !M3_IN(29, (QR - 1) / R, qs))
+                continue;
             for (int j = 0; j < QR; ++j) acc = fmaf(sB[j * N + n] * sW[j / R], sX[j * P + p], acc);
             sS[e] = fmaf(dec, sS[e], acc);
         }
@@ -199,9 +229,11 @@ __global__ void __launch_bounds__(256) scan_simt_kernel(ScanParams q) {
     }
 
     if (SUMMARY) {
-        for (int e = tid; e < N * P; e += nt) q.ws_sloc[bhs * N * P + e] = sS[e];
-        for (int i = tid; i < NH; i += nt) q.ws_phase[bhs * NH + i] = (float)sPhi[i];
-        if (tid == 0) q.ws_decay[bhs] = sScal[1];
+        for (int e = tid; e < N * P; e += nt)
+            if (M3_IN(30, bhs * N * P + e, ext_ws * N * P)) q.ws_sloc[bhs * N * P + e] = sS[e];
+        for (int i = tid; i < NH; i += nt)
+            if (M3_IN(31, bhs * NH + i, ext_ws * NH)) q.ws_phase[bhs * NH + i] = (float)sPhi[i];
+        if (tid == 0 && M3_IN(32, bhs, ext_ws)) q.ws_decay[bhs] = sScal[1];
     } else if (seg == q.nseg - 1) {
         // final carry in the original frame: h = R(Phi) h~
         if (q.fin_h) {
@@ -210,6 +242,7 @@ __global__ void __launch_bounds__(256) scan_simt_kernel(ScanParams q) {
                 float sv, cv;
                 sincosf((float)sPhi[i], &sv, &cv);
                 const float s0 = sS[(2 * i) * P + p], s1 = sS[(2 * i + 1) * P + p];
+                if (!M3_IN(33, (bh * N + 2 * i + 1) * P + p, ext_h(q))) continue;
                 q.fin_h[(bh * N + 2 * i) * P + p] = cv * s0 - sv * s1;
                 q.fin_h[(bh * N + 2 * i + 1) * P + p] = sv * s0 + cv * s1;
             }
@@ -217,12 +250,16 @@ __global__ void __launch_bounds__(256) scan_simt_kernel(ScanParams q) {
         if (q.fin_pB && L > 0) {
             T* o = static_cast<T*>(q.fin_pB) + bh * R * N;
             const T* s = Bg + (((size_t)b * L + L - 1) * G + g) * R * N;
-            for (int e = tid; e < R * N; e += nt) o[e] = s[e];
+            for (int e = tid; e < R * N; e += nt)
+                if (M3_IN(34, bh * R * N + e, ext_pB(q)) && M3_IN(35, (((size_t)b * L + L - 1) * G + g) * R * N + e, ext_bc(q)))
+                    o[e] = s[e];
         }
         if (q.fin_pX && L > 0) {
             T* o = static_cast<T*>(q.fin_pX) + bh * R * P;
             const T* s = xg + (((size_t)b * L + L - 1) * H + h) * R * P;
-            for (int e = tid; e < R * P; e += nt) o[e] = s[e];
+            for (int e = tid; e < R * P; e += nt)
+                if (M3_IN(36, bh * R * P + e, ext_pX(q)) && M3_IN(37, (((size_t)b * L + L - 1) * H + h) * R * P + e, ext_x(q)))
+                    o[e] = s[e];
         }
     }
 }
@@ -236,7 +273,10 @@ __global__ void __launch_bounds__(256) scan_combine_kernel(ScanParams q) {
     if (e >= NH * P) return;
     const int i = e / P, p = e % P;
     const size_t bh = (size_t)b * H + h;
-    const float w0 = (1.f - q.lam[(size_t)b * L * H + h]) * q.dt[(size_t)b * L * H + h];
+    const long long ext_ws = (long long)q.batch * H * q.nseg;   // segment summaries (debug checks)
+    (void)ext_ws;
+    const float w0 = M3_IN(40, (size_t)b * L * H + h, ext_tok(q))
+                         ? (1.f - q.lam[(size_t)b * L * H + h]) * q.dt[(size_t)b * L * H + h] : 0.f;
     float s0 = carry_in<T>(q, b, h, 2 * i, p, w0);
     float s1 = carry_in<T>(q, b, h, 2 * i + 1, p, w0);
     // The summaries of a batch of segments are loaded before the chain runs
@@ -249,18 +289,21 @@ __global__ void __launch_bounds__(256) scan_combine_kernel(ScanParams q) {
         for (int j = 0; j < KB; ++j) {
             const int k = min(k0 + j, q.nseg - 1);
             const size_t bhs = bh * q.nseg + k;
-            l0[j] = __ldg(q.ws_sloc + (bhs * N + 2 * i) * P + p);
-            l1[j] = __ldg(q.ws_sloc + (bhs * N + 2 * i + 1) * P + p);
-            dl[j] = __ldg(q.ws_decay + bhs);
-            ph[j] = __ldg(q.ws_phase + bhs * NH + i);
+            const bool ok = M3_IN(41, (bhs * N + 2 * i + 1) * P + p, ext_ws * N * P) && M3_IN(42, bhs * NH + i, ext_ws * NH);
+            l0[j] = ok ? __ldg(q.ws_sloc + (bhs * N + 2 * i) * P + p) : 0.f;
+            l1[j] = ok ? __ldg(q.ws_sloc + (bhs * N + 2 * i + 1) * P + p) : 0.f;
+            dl[j] = ok ? __ldg(q.ws_decay + bhs) : 0.f;
+            ph[j] = ok ? __ldg(q.ws_phase + bhs * NH + i) : 0.f;
         }
 #pragma unroll
         for (int j = 0; j < KB; ++j) {
             const int k = k0 + j;
             if (k >= q.nseg) break;
             const size_t bhs = bh * q.nseg + k;
-            q.ws_sin[(bhs * N + 2 * i) * P + p] = s0;
-            q.ws_sin[(bhs * N + 2 * i + 1) * P + p] = s1;
+            if (M3_IN(43, (bhs * N + 2 * i + 1) * P + p, ext_ws * N * P)) {
+                q.ws_sin[(bhs * N + 2 * i) * P + p] = s0;
+                q.ws_sin[(bhs * N + 2 * i + 1) * P + p] = s1;
+            }
             if (k + 1 == q.nseg) break;
             const float dec = expf(dl[j]);
             const float v0 = fmaf(dec, s0, l0[j]);
@@ -300,3 +343,5 @@ cudaError_t launch_scan_simt(const m3_dims& d, const ScanParams& q, cudaStream_t
 }
 
 }  // namespace m3
+
+M3_BOUNDS_EXPORT(scan_simt)

@@ -42,6 +42,8 @@
 // Every wait on an mbarrier is bounded (1 s); on expiry the kernel records
 // M3_ERR_DEVICE_TIMEOUT in the workspace status word, finishes the tile with
 // no further waiting and returns after freeing its TMEM.
+#define M3_BOUNDS_FILE 1
+#include "m3_bounds.cuh"
 #include "m3_kernels.h"
 #include "tc_ptx.cuh"
 
@@ -84,6 +86,9 @@ struct Misc {
 };
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region too small");
 static_assert(offsetof(Misc, u) + sizeof(float) * 32 * 36 <= 9216, "misc region of R >= 4 too small");
+// bytes of the misc region a launch of rank R uses
+template <int R>
+constexpr int misc_used() { return R >= 4 ? (int)(offsetof(Misc, u) + sizeof(float) * 32 * 36) : (int)sizeof(Misc); }
 
 enum { BAR_LOAD = 0, BAR_OPS, BAR_G, BAR_BW, BAR_P, BAR_Y, BAR_DRAIN };
 
@@ -138,6 +143,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint8_t* smem = smem_raw + ((1024u - (su32(smem_raw) & 1023u)) & 1023u);
     Misc* m = reinterpret_cast<Misc*>(smem + OFF_MISC);
     const uint32_t sbase = su32(smem);
+    // the whole shared-memory map (tiles and misc region) inside the launch's
+    // dynamic shared memory (uniform over the CTA, before any barrier)
+    if (!M3_SPAN(1, smem - smem_raw, OFF_MISC + misc_used<R>(), dyn_smem_bytes())) return;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -148,7 +156,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int ntiles = (tok1 - tok0 + T - 1) / T;
     const size_t bh = (size_t)b * H + h;
     const size_t bhs = bh * q.nseg + seg;
-    const float Ah = q.A[h];
+    const float Ah = M3_IN(2, h, H) ? q.A[h] : 0.f;
+    const long long ext_ws = (long long)q.batch * H * q.nseg;   // segment summaries (debug checks)
+    (void)ext_ws;
 
     // ---- setup
     if (tid == 0) {
@@ -182,19 +192,25 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int p = 0; p < kSC; ++p) S[p] = 0.f;
         } else if (q.nseg > 1) {
             const float4* src = reinterpret_cast<const float4*>(q.ws_sin + (bhs * kN + n) * kP + c0);
+            const bool ok = M3_SPAN(3, (bhs * kN + n) * kP + c0, kSC, ext_ws * kN * kP);
 #pragma unroll
             for (int c = 0; c < kSC / 4; ++c) {
-                const float4 v = src[c];
+                const float4 v = ok ? src[c] : make_float4(0.f, 0.f, 0.f, 0.f);
                 S[4 * c] = v.x; S[4 * c + 1] = v.y; S[4 * c + 2] = v.z; S[4 * c + 3] = v.w;
             }
         } else {
+            const bool ok = !q.init_h || M3_SPAN(4, (bh * kN + n) * kP + c0, kSC, ext_h(q));
 #pragma unroll
-            for (int p = 0; p < kSC; ++p) S[p] = q.init_h ? q.init_h[(bh * kN + n) * kP + c0 + p] : 0.f;
+            for (int p = 0; p < kSC; ++p) S[p] = (q.init_h && ok) ? q.init_h[(bh * kN + n) * kP + c0 + p] : 0.f;
             if (q.init_pB && q.init_pX) {
-                const float w0 = (1.f - q.lam[(size_t)b * L * H + h]) * q.dt[(size_t)b * L * H + h];
+                const bool ok0 = M3_IN(5, (size_t)b * L * H + h, ext_tok(q));
+                const float w0 = ok0 ? (1.f - q.lam[(size_t)b * L * H + h]) * q.dt[(size_t)b * L * H + h] : 0.f;
                 const __nv_bfloat16* pB = static_cast<const __nv_bfloat16*>(q.init_pB) + bh * R * kN;
                 const __nv_bfloat16* pX = static_cast<const __nv_bfloat16*>(q.init_pX) + bh * R * kP;
                 for (int r = 0; r < R; ++r) {
+                    if (!M3_IN(6, bh * R * kN + r * kN + n, ext_pB(q)) ||
+                        !M3_SPAN(7, bh * R * kP + r * kP + c0, kSC, ext_pX(q)))
+                        continue;
                     const float bv = w0 * __bfloat162float(pB[r * kN + n]);
 #pragma unroll
                     for (int p = 0; p < kSC; ++p) S[p] = fmaf(bv, __bfloat162float(pX[r * kP + c0 + p]), S[p]);
@@ -209,7 +225,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 v.y = pack_bf16x2(S[8 * c + 2], S[8 * c + 3]);
                 v.z = pack_bf16x2(S[8 * c + 4], S[8 * c + 5]);
                 v.w = pack_bf16x2(S[8 * c + 6], S[8 * c + 7]);
-                *reinterpret_cast<uint4*>(smem + OFF_S + sw128(n, c0 / 8 + c)) = v;
+                if (M3_SPAN(8, sw128(n, c0 / 8 + c), 16, 16384))
+                    *reinterpret_cast<uint4*>(smem + OFF_S + sw128(n, c0 / 8 + c)) = v;
             }
             fence_async_smem();
         }
@@ -255,23 +272,28 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int j = 0; j < NT; ++j) {
             const int t = min(lane + 32 * j, qcn - 1);
             const size_t o = ((size_t)b * L + t0n + t) * H + h;
-            dt_n[j] = __ldg(q.dt + o);
-            lam_n[j] = __ldg(q.lam + o);
+            const bool ok = M3_IN(9, o, ext_tok(q));
+            dt_n[j] = ok ? __ldg(q.dt + o) : 0.f;
+            lam_n[j] = ok ? __ldg(q.lam + o) : 1.f;
         }
         const int tn = min(t0n + qcn, L - 1);
         const size_t o = ((size_t)b * L + tn) * H + h;
-        dx_n = __ldg(q.dt + o);
-        lx_n = __ldg(q.lam + o);
+        const bool ok = M3_IN(10, o, ext_tok(q));
+        dx_n = ok ? __ldg(q.dt + o) : 0.f;
+        lx_n = ok ? __ldg(q.lam + o) : 1.f;
     };
     auto theta_ld = [&](int t0n, int qcn, int kk) -> float2 {   // theta of pairs (2 lane, 2 lane + 1), raw
         const int t = min(g0 + kk, qcn - 1);
-        return __ldg(reinterpret_cast<const float2*>(q.theta + (((size_t)b * L + t0n + t) * G + g) * (kN / 2)) + lane);
+        return M3_SPAN(11, (((size_t)b * L + t0n + t) * G + g) * (kN / 2) + 2 * lane, 2, ext_theta(q))
+                   ? __ldg(reinterpret_cast<const float2*>(q.theta + (((size_t)b * L + t0n + t) * G + g) * (kN / 2)) + lane)
+                   : make_float2(0.f, 0.f);
     };
     auto prefetch_tok = [&](int kn) {         // L2 prefetch of a tile's dt / lambda (and the token after it)
         const int t0n = tok0 + kn * T;
         const int qn = min(T + 1, L - t0n);
         for (int t = wk; t < qn; t += kWorkers) {
             const size_t o = ((size_t)b * L + t0n + t) * H + h;
+            if (!M3_IN(12, o, ext_tok(q))) continue;
             prefetch_l2(q.dt + o);
             prefetch_l2(q.lam + o);
         }
@@ -281,7 +303,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int qn = min(T, tok1 - t0n);
         for (int j = wk; j < 2 * T; j += kWorkers) {
             const int t = j >> 1;
-            if (t < qn) prefetch_l2(q.theta + (((size_t)b * L + t0n + t) * G + g) * (kN / 2) + (j & 1) * 32);
+            if (t < qn && M3_IN(13, (((size_t)b * L + t0n + t) * G + g) * (kN / 2) + (j & 1) * 32, ext_theta(q)))
+                prefetch_l2(q.theta + (((size_t)b * L + t0n + t) * G + g) * (kN / 2) + (j & 1) * 32);
         }
     };
     // y = Y_intra + e^{a_t} Y_inter of a finished tile (thread = tile row (t, r),
@@ -299,7 +322,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 yi[j] = o2.x;
                 yi[j + 1] = o2.y;
             }
-            if (tr < qcy) {
+            if (tr < qcy &&
+                M3_SPAN(14, ((((size_t)b * L + t0y + tr) * H + h) * R + (row % R)) * kP + c0 + 16 * hh, 16, ext_x(q))) {
                 uint4* dst = reinterpret_cast<uint4*>(
                     yg + ((((size_t)b * L + t0y + tr) * H + h) * R + (row % R)) * kP + c0 + 16 * hh);
                 dst[0] = pack_chunk(yi);
@@ -375,7 +399,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const int t = e / T, u = e % T;
                 const float at = __shfl_sync(kFull, a2v[0], t), au = __shfl_sync(kFull, a2v[0], u);
                 const float gu = __shfl_sync(kFull, gmv[0], u), cu = __shfl_sync(kFull, cfv[0], u);
-                m->u.msk[t * LD + u] = (u <= t) ? exp2f(at - au) * (u == t ? gu : cu) : 0.f;
+                if (M3_IN(15, t * LD + u, 32 * 36))
+                    m->u.msk[t * LD + u] = (u <= t) ? exp2f(at - au) * (u == t ? gu : cu) : 0.f;
             }
         }
         if (!SUMMARY && R < 4 && qe == 0) {
@@ -392,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const float aend = __shfl_sync(kFull, a2v[j], lane | (GT - 1));
                 const bool ok = aref - aend <= 60.f;
                 const float colf = exp2f(aref - a2v[j]);
+                if (!M3_IN(16, t, 128)) continue;
                 m->u.cs[pb][0][t] = ok ? cfv[j] * colf : 0.f;
                 m->u.cs[pb][1][t] = ok ? gmv[j] * colf : 0.f;
                 if ((lane & (GT - 1)) == 0) m->u.cs[pb][2][t / GT] = ok ? aref : __int_as_float(0x7f800000);
@@ -430,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 acc.y = fmaf(d, thv[kk].y, acc.y);
             }
         }
-        m->qs[kn & 1][qe][lane] = acc;
+        if (M3_IN(17, qe, kNE)) m->qs[kn & 1][qe][lane] = acc;
     };
     auto pass1_ahead = [&](int kn, float dsl) {   // theta straight from memory (L2)
         const int t0n = tok0 + kn * T;
@@ -466,6 +492,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                 // workers still run that tile's epilogue.
                 if (k > 0) mbar_wait(&m->bar[BAR_Y], (k - 1) & 1, m, status, 1);
                 const uint32_t bytes = SUMMARY ? (32768u + 16384u) : (65536u + 16384u);
+                // tensor coordinates (the copy engine bounds them itself: only noted)
+                M3_NOTE(18, t0, L);
+                M3_NOTE(19, g, G);
+                M3_NOTE(20, b, q.batch);
                 mbar_expect_tx(&m->bar[BAR_LOAD], bytes);
                 tma_load_5d(sbase + OFF_B, &tmB, &m->bar[BAR_LOAD], 0, 0, g, t0, b);
                 tma_load_5d(sbase + OFF_B + 16384, &tmB, &m->bar[BAR_LOAD], 64, 0, g, t0, b);
@@ -633,7 +663,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                         const uint32_t off = atom + sw128(t * R + r, chunk) + inb;
 #pragma unroll
                         for (int mt = 0; mt < NM; ++mt)
-                            vv[mt][r] = lds64_free(sb_ld + (mt ? OFF_C : OFF_B) + off);
+                            vv[mt][r] = M3_SPAN(21, off, 8, 32768) ? lds64_free(sb_ld + (mt ? OFF_C : OFF_B) + off)
+                                                                  : make_uint2(0u, 0u);
                     }
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
@@ -643,7 +674,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                             uint2 v = vv[mt][r];
                             v.x = rot_bf(v.x, cc0, sn0);
                             v.y = rot_bf(v.y, cc1, sn1);
-                            *reinterpret_cast<uint2*>(smem + (mt ? OFF_C : OFF_B) + off) = v;
+                            if (M3_SPAN(22, off, 8, 32768))
+                                *reinterpret_cast<uint2*>(smem + (mt ? OFF_C : OFF_B) + off) = v;
                         }
                     }
                 }
@@ -677,10 +709,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                 uint4 xv[8 / kWG];
 #pragma unroll
                 for (int c = 0; c < 8 / kWG; ++c)      // 16-byte chunks of the 128-byte row
-                    xv[c] = *reinterpret_cast<const uint4*>(smem + OFF_X + sw128(row, wg * (8 / kWG) + c));
+                    xv[c] = M3_SPAN(23, sw128(row, wg * (8 / kWG) + c), 16, 16384)
+                                ? *reinterpret_cast<const uint4*>(smem + OFF_X + sw128(row, wg * (8 / kWG) + c))
+                                : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
                 for (int c = 0; c < 8 / kWG; ++c)
-                    *reinterpret_cast<uint4*>(smem + OFF_S + sw128(row, wg * (8 / kWG) + c)) = scale_chunk(xv[c], w2);
+                    if (M3_SPAN(24, sw128(row, wg * (8 / kWG) + c), 16, 16384))
+                        *reinterpret_cast<uint4*>(smem + OFF_S + sw128(row, wg * (8 / kWG) + c)) = scale_chunk(xv[c], w2);
             }
             fence_async_smem();
             mbar_arrive(&m->bar[BAR_BW]);
@@ -696,7 +731,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                     constexpr int LD = T + 4;
                     const float* mrow = m->u.msk + tr * LD + col0 / R;
                     float mk[16 / R];
-                    if (R == 4) {
+                    if (!M3_SPAN(25, tr * LD + col0 / R, 16 / R, 32 * 36)) {
+#pragma unroll
+                        for (int i = 0; i < 16 / R; ++i) mk[i] = 0.f;
+                    } else if (R == 4) {
                         const float4 f = *reinterpret_cast<const float4*>(mrow);
                         mk[0] = f.x; mk[1] = f.y; mk[2 % (16 / R)] = f.z; mk[3 % (16 / R)] = f.w;
                     } else {
@@ -713,8 +751,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                 } else {
                     constexpr int GT = 16 / R;            // tokens per 16-column block
                     const int u0 = col0 / R;              // the block's first token (warp-uniform)
-                    const float aref = m->u.cs[par][2][u0 / GT];
-                    if (u0 > tr) {
+                    // (u0 + 16 / R <= T <= 128 keeps the cs rows below inside their 128 floats)
+                    const bool okc = M3_SPAN(26, u0, GT, 128);
+                    const float aref = okc ? m->u.cs[par][2][u0 / GT] : 0.f;
+                    if (u0 > tr || !okc) {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) v[j] = 0.f;
                     } else if (aref != __int_as_float(0x7f800000)) {
@@ -747,8 +787,9 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     const int cc = (col0 >> 3) + c;      // 16-byte chunk over 128 columns
-                    *reinterpret_cast<uint4*>(smem + OFF_C + (cc >> 3) * 16384 + sw128(row, cc & 7)) =
-                        pack_chunk(v + 8 * c);
+                    if (M3_SPAN(27, (cc >> 3) * 16384 + sw128(row, cc & 7), 16, 32768))
+                        *reinterpret_cast<uint4*>(smem + OFF_C + (cc >> 3) * 16384 + sw128(row, cc & 7)) =
+                            pack_chunk(v + 8 * c);
                 }
             }
             fence_async_smem();
@@ -777,7 +818,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (!SUMMARY) {
 #pragma unroll
                 for (int c = 0; c < kSC / 8; ++c)
-                    *reinterpret_cast<uint4*>(smem + OFF_S + sw128(row, c0 / 8 + c)) = pack_chunk(S + 8 * c);
+                    if (M3_SPAN(28, sw128(row, c0 / 8 + c), 16, 16384))
+                        *reinterpret_cast<uint4*>(smem + OFF_S + sw128(row, c0 / 8 + c)) = pack_chunk(S + 8 * c);
             }
         }
         seg_a += a2_last * kLn2;
@@ -806,13 +848,15 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int n = row;
         if (SUMMARY) {
             float4* dst = reinterpret_cast<float4*>(q.ws_sloc + (bhs * kN + n) * kP + c0);
+            if (M3_SPAN(29, (bhs * kN + n) * kP + c0, kSC, ext_ws * kN * kP)) {
 #pragma unroll
-            for (int c = 0; c < kSC / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
-            if (qe == 0) {
+                for (int c = 0; c < kSC / 4; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
+            }
+            if (qe == 0 && M3_SPAN(30, bhs * (kN / 2) + 2 * lane, 2, ext_ws * (kN / 2))) {
                 q.ws_phase[bhs * (kN / 2) + 2 * lane] = carry.x;
                 q.ws_phase[bhs * (kN / 2) + 2 * lane + 1] = carry.y;
             }
-            if (wk == 0) q.ws_decay[bhs] = seg_a;
+            if (wk == 0 && M3_IN(31, bhs, ext_ws)) q.ws_decay[bhs] = seg_a;
         } else if (seg == q.nseg - 1) {
             if (q.fin_h) {
                 // phase of pair n/2 is held by lane n/4 of every worker warp
@@ -821,21 +865,26 @@ __global__ void __launch_bounds__(kThreads, 2)
                 float sv, cv;
                 sincosf(phn, &sv, &cv);
                 float* dst = q.fin_h + (bh * kN + n) * kP + c0;
+                const bool ok = M3_SPAN(32, (bh * kN + n) * kP + c0, kSC, ext_h(q));
 #pragma unroll
                 for (int p = 0; p < kSC; ++p) {
                     const float other = __shfl_xor_sync(kFull, S[p], 1);
-                    dst[p] = (n & 1) ? (sv * other + cv * S[p]) : (cv * S[p] - sv * other);
+                    if (ok) dst[p] = (n & 1) ? (sv * other + cv * S[p]) : (cv * S[p] - sv * other);
                 }
             }
             if (q.fin_pB && L > 0) {
-                const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(q.B) + (((size_t)b * L + L - 1) * G + g) * R * kN;
-                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(q.fin_pB) + bh * R * kN;
-                for (int e = wk; e < R * kN; e += kWorkers) o[e] = s[e];
+                const size_t os = (((size_t)b * L + L - 1) * G + g) * R * kN, oo = bh * R * kN;
+                const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(q.B) + os;
+                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(q.fin_pB) + oo;
+                for (int e = wk; e < R * kN; e += kWorkers)
+                    if (M3_IN(33, os + e, ext_bc(q)) && M3_IN(34, oo + e, ext_pB(q))) o[e] = s[e];
             }
             if (q.fin_pX && L > 0) {
-                const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(q.x) + (((size_t)b * L + L - 1) * H + h) * R * kP;
-                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(q.fin_pX) + bh * R * kP;
-                for (int e = wk; e < R * kP; e += kWorkers) o[e] = s[e];
+                const size_t os = (((size_t)b * L + L - 1) * H + h) * R * kP, oo = bh * R * kP;
+                const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(q.x) + os;
+                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(q.fin_pX) + oo;
+                for (int e = wk; e < R * kP; e += kWorkers)
+                    if (M3_IN(35, os + e, ext_x(q)) && M3_IN(36, oo + e, ext_pX(q))) o[e] = s[e];
             }
         }
     }
@@ -970,3 +1019,5 @@ cudaError_t launch_scan_tc(const m3_dims& d, const ScanParams& q, int* status, c
 }
 
 }  // namespace m3
+
+M3_BOUNDS_EXPORT(scan_tc)

@@ -46,6 +46,8 @@
 // kernel records M3_ERR_DEVICE_TIMEOUT in the workspace status word, every
 // role leaves its loop, in-flight copies and MMAs are drained (bounded) and
 // the TMEM is freed.
+#define M3_BOUNDS_FILE 8
+#include "m3_bounds.cuh"
 #include "m3_kernels.h"
 #include "tc_ptx.cuh"
 
@@ -241,6 +243,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sbase = su32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int L = q.seqlen, H = q.nheads, G = q.ngroups;
+    // the shared-memory map inside the launch's dynamic shared memory
+    // (uniform over the CTA, before any barrier)
+    if (!M3_SPAN(1, smem - smem_raw, OFF_MISC + (int)sizeof(Misc), dyn_smem_bytes())) return;
+    const long long ext_ho = (long long)gridDim.x;                // hand-off slots (debug checks)
+    const long long ext_ws = (long long)q.batch * H * q.nseg;     // segment inputs (debug checks)
+    (void)ext_ho; (void)ext_ws;
 
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
@@ -291,6 +299,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t st = sbase + s * ST_BYTES;
                 if (k >= 2 && !bwait(bc ? &m->empty_bc[s] : &m->empty_x[s], ((k - 2) >> 1) & 1, m, status, bc ? 1 : 5))
                     break;
+                // tensor coordinates (the copy engine bounds them itself: only noted)
+                M3_NOTE(2, t0, L);
+                M3_NOTE(3, cu.b, q.batch);
+                M3_NOTE(4, bc ? cu.g : cu.h, bc ? G : H);
                 if (bc) {
                     uint64_t* fb = &m->full_bc[s];
                     mbar_expect_tx(fb, 65536u);
@@ -419,7 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     yi[j] = o2.x;
                     yi[j + 1] = o2.y;
                 }
-                if (tr < pend_qc) {
+                if (tr < pend_qc &&
+                    M3_SPAN(10, ((((size_t)pend_b * L + pend_t0 + tr) * H + pend_h) * R + rr) * kP + 16 * hh, 16, ext_x(q))) {
                     uint4* dst = reinterpret_cast<uint4*>(yrow + 16 * hh);
                     dst[0] = pack_chunk(yi);
                     dst[1] = pack_chunk(yi + 8);
@@ -449,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         while (true) {
                             int seen = 0, stop = 0;
                             if (lane == 0) {
-                                seen = ld_acquire_gpu(wa.ho_flag + pc.slot_in) == wa.call_id;
+                                seen = M3_IN(11, pc.slot_in, ext_ho) && ld_acquire_gpu(wa.ho_flag + pc.slot_in) == wa.call_id;
                                 stop = !seen && (*(volatile int*)&m->abort_flag || globaltimer_ns() - t0w > kWaitNs);
                             }
                             seen = __shfl_sync(kFull, seen, 0);
@@ -474,27 +487,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (__any_sync(kFull, !got || !*(volatile int*)&m->ho_ok)) break;
                     }
                     const float4* src = reinterpret_cast<const float4*>(wa.ho_state + ((size_t)pc.slot_in * kN + n) * kP);
+                    const bool okh = M3_SPAN(12, ((size_t)pc.slot_in * kN + n) * kP, kP, ext_ho * kN * kP);
 #pragma unroll
                     for (int c = 0; c < kP / 4; ++c) {
-                        const float4 v = __ldcg(src + c);
+                        const float4 v = okh ? __ldcg(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
                         S[4 * c] = v.x; S[4 * c + 1] = v.y; S[4 * c + 2] = v.z; S[4 * c + 3] = v.w;
                     }
                 } else if (pc.init == 2) {
                     const size_t bhs = bh * q.nseg + pc.seg;
                     const float4* src = reinterpret_cast<const float4*>(q.ws_sin + (bhs * kN + n) * kP);
+                    const bool oks = M3_SPAN(13, (bhs * kN + n) * kP, kP, ext_ws * kN * kP);
 #pragma unroll
                     for (int c = 0; c < kP / 4; ++c) {
-                        const float4 v = src[c];
+                        const float4 v = oks ? src[c] : make_float4(0.f, 0.f, 0.f, 0.f);
                         S[4 * c] = v.x; S[4 * c + 1] = v.y; S[4 * c + 2] = v.z; S[4 * c + 3] = v.w;
                     }
                 } else {
+                    const bool oki = !q.init_h || M3_SPAN(14, (bh * kN + n) * kP, kP, ext_h(q));
 #pragma unroll
-                    for (int p = 0; p < kP; ++p) S[p] = q.init_h ? q.init_h[(bh * kN + n) * kP + p] : 0.f;
+                    for (int p = 0; p < kP; ++p) S[p] = (q.init_h && oki) ? q.init_h[(bh * kN + n) * kP + p] : 0.f;
                     if (q.init_pB && q.init_pX) {
-                        const float w0 = (1.f - q.lam[(size_t)b * L * H + h]) * q.dt[(size_t)b * L * H + h];
+                        const bool ok0 = M3_IN(15, (size_t)b * L * H + h, ext_tok(q));
+                        const float w0 = ok0 ? (1.f - q.lam[(size_t)b * L * H + h]) * q.dt[(size_t)b * L * H + h] : 0.f;
                         const __nv_bfloat16* pB = static_cast<const __nv_bfloat16*>(q.init_pB) + bh * R * kN;
                         const __nv_bfloat16* pX = static_cast<const __nv_bfloat16*>(q.init_pX) + bh * R * kP;
                         for (int r = 0; r < R; ++r) {
+                            if (!M3_IN(16, bh * R * kN + r * kN + n, ext_pB(q)) ||
+                                !M3_SPAN(17, bh * R * kP + r * kP, kP, ext_pX(q)))
+                                continue;
                             const float bv = w0 * __bfloat162float(pB[r * kN + n]);
 #pragma unroll
                             for (int p = 0; p < kP; ++p) S[p] = fmaf(bv, __bfloat162float(pX[r * kP + p]), S[p]);
@@ -503,7 +523,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
 #pragma unroll
                 for (int c = 0; c < kP / 8; ++c)
-                    *reinterpret_cast<uint4*>(smem + OFF_SBF + sw128(n, c)) = pack_chunk(S + 8 * c);
+                    if (M3_SPAN(18, sw128(n, c), 16, 16384))
+                        *reinterpret_cast<uint4*>(smem + OFF_SBF + sw128(n, c)) = pack_chunk(S + 8 * c);
                 fence_async_smem();
                 tc_fence_before();
                 mbar_arrive(&m->sbf);
@@ -539,7 +560,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!last_of_piece) {
 #pragma unroll
                 for (int c = 0; c < kP / 8; ++c)
-                    *reinterpret_cast<uint4*>(smem + OFF_SBF + sw128(row, c)) = pack_chunk(S + 8 * c);
+                    if (M3_SPAN(19, sw128(row, c), 16, 16384))
+                        *reinterpret_cast<uint4*>(smem + OFF_SBF + sw128(row, c)) = pack_chunk(S + 8 * c);
             } else if (pc.fin != 0) {
                 // ---- the piece's outgoing state: h = R(Phi) S (original frame)
                 const int n = row;
@@ -549,6 +571,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __sincosf(phn, &sv, &cv);         // phn is reduced to [-pi, pi]: error ~4e-7
                 float* dst = pc.fin == 2 ? wa.ho_state + ((size_t)pc.slot_out * kN + n) * kP
                                          : (q.fin_h ? q.fin_h + (bh * kN + n) * kP : nullptr);
+                // (the partner exchange below is warp-wide: a failed check
+                // only drops this thread's stores)
+                const bool okd = pc.fin == 2 ? M3_SPAN(20, ((size_t)pc.slot_out * kN + n) * kP, kP, ext_ho * kN * kP)
+                                             : M3_SPAN(21, (bh * kN + n) * kP, kP, ext_h(q));
+                (void)okd;
                 if (dst) {
                     // rows n and n ^ 1 (one rotary pair) sit in adjacent lanes;
                     // four columns at a time go through a shared-memory slot
@@ -564,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int z = 0; z < 4; ++z)
                             o[z] = (n & 1) ? (sv * o4[z] + cv * S[p + z]) : (cv * S[p + z] - sv * o4[z]);
-                        *reinterpret_cast<float4*>(dst + p) = make_float4(o[0], o[1], o[2], o[3]);
+                        if (okd) *reinterpret_cast<float4*>(dst + p) = make_float4(o[0], o[1], o[2], o[3]);
                     }
                 }
                 if (pc.fin == 2) {
@@ -576,7 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (e < 32) {
                         const bool all = bwait(&m->ho_w, 0, m, status, 23);
                         __syncwarp();
-                        if (all && lane == 0) st_release_gpu(wa.ho_flag + pc.slot_out, wa.call_id);
+                        if (all && lane == 0 && M3_IN(22, pc.slot_out, ext_ho))
+                            st_release_gpu(wa.ho_flag + pc.slot_out, wa.call_id);
                         __syncwarp();
                     }
                 } else if (L > 0) {
@@ -584,12 +612,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (q.fin_pB) {
                         const __nv_bfloat16* sB = static_cast<const __nv_bfloat16*>(q.B) + (((size_t)b * L + L - 1) * G + g) * R * kN;
                         __nv_bfloat16* o = static_cast<__nv_bfloat16*>(q.fin_pB) + bh * R * kN;
-                        for (int z = e; z < R * kN; z += kEWT) o[z] = sB[z];
+                        for (int z = e; z < R * kN; z += kEWT)
+                            if (M3_IN(23, (((size_t)b * L + L - 1) * G + g) * R * kN + z, ext_bc(q)) &&
+                                M3_IN(24, bh * R * kN + z, ext_pB(q)))
+                                o[z] = sB[z];
                     }
                     if (q.fin_pX) {
                         const __nv_bfloat16* sX = static_cast<const __nv_bfloat16*>(q.x) + (((size_t)b * L + L - 1) * H + h) * R * kP;
                         __nv_bfloat16* o = static_cast<__nv_bfloat16*>(q.fin_pX) + bh * R * kP;
-                        for (int z = e; z < R * kP; z += kEWT) o[z] = sX[z];
+                        for (int z = e; z < R * kP; z += kEWT)
+                            if (M3_IN(25, (((size_t)b * L + L - 1) * H + h) * R * kP + z, ext_x(q)) &&
+                                M3_IN(26, bh * R * kP + z, ext_pX(q)))
+                                o[z] = sX[z];
                     }
                 }
             }
@@ -618,7 +652,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         constexpr int LD = T + 4;
                         const float* mrow = U.msk + tr * LD + col0 / R;
                         float mk[16 / R];
-                        if (R == 4) {
+                        if (!M3_SPAN(27, tr * LD + col0 / R, 16 / R, 32 * 36)) {
+#pragma unroll
+                            for (int i = 0; i < 16 / R; ++i) mk[i] = 0.f;
+                        } else if (R == 4) {
                             const float4 f = *reinterpret_cast<const float4*>(mrow);
                             mk[0] = f.x; mk[1] = f.y; mk[2 % (16 / R)] = f.z; mk[3 % (16 / R)] = f.w;
                         } else {
@@ -634,8 +671,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
                         constexpr int GT = 16 / R;            // tokens per 16-column block
                         const int u0 = col0 / R;
-                        const float aref = U.cs[2][u0 / GT];
-                        if (u0 > tr) {
+                        // (u0 + 16 / R <= T <= 128 keeps the cs rows below inside their 128 floats)
+                        const bool okc = M3_SPAN(28, u0, GT, 128);
+                        const float aref = okc ? U.cs[2][u0 / GT] : 0.f;
+                        if (u0 > tr || !okc) {
 #pragma unroll
                             for (int j = 0; j < 16; ++j) v[j] = 0.f;
                         } else if (aref != __int_as_float(0x7f800000)) {
@@ -706,14 +745,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < NT; ++j) {
                 const int t = min(lane + 32 * j, qcn - 1);
                 const size_t o = ((size_t)b * L + t0n + t) * H + h;
-                dt_n[j] = __ldg(q.dt + o);
-                lam_n[j] = __ldg(q.lam + o);
+                const bool ok = M3_IN(30, o, ext_tok(q));
+                dt_n[j] = ok ? __ldg(q.dt + o) : 0.f;
+                lam_n[j] = ok ? __ldg(q.lam + o) : 1.f;
             }
             const int tn = min(t0n + qcn, L - 1);
             const size_t o = ((size_t)b * L + tn) * H + h;
-            dx_n = __ldg(q.dt + o);
-            lx_n = __ldg(q.lam + o);
-            a_n = __ldg(q.A + h);
+            const bool ok = M3_IN(31, o, ext_tok(q));
+            dx_n = ok ? __ldg(q.dt + o) : 0.f;
+            lx_n = ok ? __ldg(q.lam + o) : 1.f;
+            a_n = M3_IN(32, h, H) ? __ldg(q.A + h) : 0.f;
         };
         // theta row of token kk of this warp's group in tile c (pairs 2 lane, 2 lane + 1)
         auto theta_row = [&](const Cursor& c, int& qcn) -> const float2* {
@@ -728,14 +769,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int b = c.b, g = c.g;
             const int t0n = c.j * T, qcn = min(T, L - t0n);
             for (int z = r; z < 2 * qcn; z += kRWT)
-                prefetch_l2(q.theta + (((size_t)b * L + t0n + (z >> 1)) * G + g) * (kN / 2) + (z & 1) * 32);
+                if (M3_IN(33, (((size_t)b * L + t0n + (z >> 1)) * G + g) * (kN / 2) + (z & 1) * 32, ext_theta(q)))
+                    prefetch_l2(q.theta + (((size_t)b * L + t0n + (z >> 1)) * G + g) * (kN / 2) + (z & 1) * 32);
         };
         if (cu.ok) {
             load_tok(cu);
             int qc0;
             const float2* tp = theta_row(cu, qc0);
 #pragma unroll
-            for (int kk = 0; kk < TE; ++kk) th_n[kk] = __ldg(tp + (size_t)min(g0 + kk, qc0 - 1) * th_tok);
+            for (int kk = 0; kk < TE; ++kk)
+                th_n[kk] = M3_SPAN(34, (((size_t)cu.b * L + cu.j * T) * G + cu.g) * (kN / 2) + 2 * lane +
+                                           (size_t)min(g0 + kk, qc0 - 1) * 2 * th_tok, 2, ext_theta(q))
+                               ? __ldg(tp + (size_t)min(g0 + kk, qc0 - 1) * th_tok) : make_float2(0.f, 0.f);
             Cursor c1 = cu;
             c1.next(wa, q);
             if (c1.ok) prefetch_theta(c1);
@@ -842,6 +887,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float aend = __shfl_sync(kFull, a2v[j], lane | (GT - 1));
                     const bool okb = aref - aend <= 60.f;
                     const float colf = exp2f(aref - a2v[j]);
+                    if (!M3_IN(36, t, 128)) continue;
                     m->u[tb].cs[0][t] = okb ? cfv[j] * colf : 0.f;
                     m->u[tb].cs[1][t] = okb ? gmv[j] * colf : 0.f;
                     if ((lane & (GT - 1)) == 0) m->u[tb].cs[2][t / GT] = okb ? aref : __int_as_float(0x7f800000);
@@ -876,7 +922,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int z = 0; z < PER; ++z) {
                     const int u = u0 + z;
                     const float mv = exp2f(at - m->ts[tb][u]) * (u == t ? m->cg[s][0][u] : m->cg[s][1][u]);
-                    m->u[tb].msk[t * LD + u] = (u <= t) ? mv : 0.f;
+                    if (M3_IN(35, t * LD + u, 32 * 36)) m->u[tb].msk[t * LD + u] = (u <= t) ? mv : 0.f;
                 }
             }
             float2 ph = carry;
@@ -921,8 +967,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int rk = 0; rk < R; ++rk) {
                             const uint32_t off = atom + sw128((g0 + k0 + kb) * R + rk, chunk) + inb;
-                            vv[kb][0][rk] = *reinterpret_cast<const uint2*>(st + ST_B + off);
-                            vv[kb][1][rk] = *reinterpret_cast<const uint2*>(st + ST_C + off);
+                            const bool okr = M3_SPAN(37, off, 8, 32768);
+                            vv[kb][0][rk] = okr ? *reinterpret_cast<const uint2*>(st + ST_B + off) : make_uint2(0u, 0u);
+                            vv[kb][1][rk] = okr ? *reinterpret_cast<const uint2*>(st + ST_C + off) : make_uint2(0u, 0u);
                         }
                     float cs[KB][4];
 #pragma unroll
@@ -932,7 +979,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ph.x = fmaf(d, th_n[kk].x, ph.x);
                         ph.y = fmaf(d, th_n[kk].y, ph.y);
                         ph = make_float2(wrap_pi_f(ph.x), wrap_pi_f(ph.y));
-                        if (tpn) th_n[kk] = __ldg(tpn + (size_t)min(g0 + kk, qcn - 1) * th_tok);
+                        if (tpn && M3_SPAN(38, (((size_t)cn.b * L + cn.j * T) * G + cn.g) * (kN / 2) + 2 * lane +
+                                                   (size_t)min(g0 + kk, qcn - 1) * 2 * th_tok, 2, ext_theta(q)))
+                            th_n[kk] = __ldg(tpn + (size_t)min(g0 + kk, qcn - 1) * th_tok);
                         __sincosf(ph.x, &cs[kb][0], &cs[kb][1]);
                         __sincosf(ph.y, &cs[kb][2], &cs[kb][3]);
                     }
@@ -946,7 +995,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 uint2 v = vv[kb][mt][rk];
                                 v.x = rot_f32(v.x, cs[kb][1], cs[kb][0]);
                                 v.y = rot_f32(v.y, cs[kb][3], cs[kb][2]);
-                                *reinterpret_cast<uint2*>(st + (mt ? ST_C : ST_B) + off) = v;
+                                if (M3_SPAN(39, off, 8, 32768))
+                                    *reinterpret_cast<uint2*>(st + (mt ? ST_C : ST_B) + off) = v;
                             }
                         }
                 }
@@ -962,10 +1012,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint8_t* xs = smem + s * ST_BYTES + ST_X;
                 uint4 xv[4];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) xv[c] = *reinterpret_cast<const uint4*>(xs + sw128(xr, xc0 + c));
+                for (int c = 0; c < 4; ++c)
+                    xv[c] = M3_SPAN(40, sw128(xr, xc0 + c), 16, 16384) ? *reinterpret_cast<const uint4*>(xs + sw128(xr, xc0 + c))
+                                                                      : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
-                    *reinterpret_cast<uint4*>(smem + OFF_WX + sw128(xr, xc0 + c)) = scale_chunk_f32(xv[c], wt);
+                    if (M3_SPAN(41, sw128(xr, xc0 + c), 16, 16384))
+                        *reinterpret_cast<uint4*>(smem + OFF_WX + sw128(xr, xc0 + c)) = scale_chunk_f32(xv[c], wt);
             }
             fence_async_smem();
             mbar_arrive(&m->rot[s]);
@@ -1028,3 +1081,5 @@ cudaError_t launch_scan_ws(const m3_dims& d, const ScanParams& q, const WsPlanAr
 }
 
 }  // namespace m3
+
+M3_BOUNDS_EXPORT(scan_ws)

@@ -34,11 +34,18 @@
 // pair blocks and alpha, beta, gamma once, into the same slots, for all its
 // warps.  Few (batch, head) sequences get narrow warps (more warps in all,
 // to hide the per-token latency), many get wide ones (fewer shared loads).
+#define M3_BOUNDS_FILE 5
+#include "m3_bounds.cuh"
 #include "m3_common.cuh"
 #include "m3_kernels.h"
 
 namespace m3 {
 namespace seq {
+
+// element count of the reflection vectors u (index checks of the debug build)
+__device__ __forceinline__ long long ext_u(const SeqParams& q) {
+    return (long long)q.batch * q.seqlen * q.ngroups * q.dstate;
+}
 
 constexpr int kWarps = 4;
 constexpr int kMaxCB = kWarps * 4;         // columns per CTA at the widest warps
@@ -147,7 +154,7 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(SeqParams q, int TK) {
     const size_t bh = (size_t)b * H + h;
     const int cw = c0 + warp * kPC;             // first column of this warp
     const bool wact = cw < P;                   // warp has columns (P is a multiple of 16)
-    const float Ah = q.A[h];
+    const float Ah = M3_IN(1, h, H) ? q.A[h] : 0.f;
     const T* xg = static_cast<const T*>(q.x);
     const T* Bg = static_cast<const T*>(q.B);
     const T* Cg = static_cast<const T*>(q.C);
@@ -170,37 +177,45 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(SeqParams q, int TK) {
             int k = e % per;
             const size_t bt = (size_t)b * L + t0 + tt;
             uint8_t* s = base + (size_t)tt * sl.bytes;
+            // the token's slot inside the launch's dynamic shared memory
+            if (!M3_SPAN(2, s - smem, sl.bytes, dyn_smem_bytes())) continue;
             if (k < pB) {
-                cp_async16(s + sl.B + 16 * k, reinterpret_cast<const uint8_t*>(Bg + (bt * G + g) * R * N) + 16 * k);
+                if (M3_SPAN(3, (bt * G + g) * R * N * es + 16 * k, 16, ext_bc(q) * es))
+                    cp_async16(s + sl.B + 16 * k, reinterpret_cast<const uint8_t*>(Bg + (bt * G + g) * R * N) + 16 * k);
                 continue;
             }
             k -= pB;
             if (k < pB) {
-                cp_async16(s + sl.C + 16 * k, reinterpret_cast<const uint8_t*>(Cg + (bt * G + g) * R * N) + 16 * k);
+                if (M3_SPAN(4, (bt * G + g) * R * N * es + 16 * k, 16, ext_bc(q) * es))
+                    cp_async16(s + sl.C + 16 * k, reinterpret_cast<const uint8_t*>(Cg + (bt * G + g) * R * N) + 16 * k);
                 continue;
             }
             k -= pB;
             if (k < pU) {
-                cp_async16(s + sl.U + 16 * k, reinterpret_cast<const uint8_t*>(Ug + (bt * G + g) * N) + 16 * k);
+                if (M3_SPAN(5, (bt * G + g) * N * es + 16 * k, 16, ext_u(q) * es))
+                    cp_async16(s + sl.U + 16 * k, reinterpret_cast<const uint8_t*>(Ug + (bt * G + g) * N) + 16 * k);
                 continue;
             }
             k -= pU;
             if (k < pT) {
-                cp_async16(s + sl.TH + 16 * k, reinterpret_cast<const uint8_t*>(q.theta + (bt * G + g) * NH) + 16 * k);
+                if (M3_SPAN(6, (bt * G + g) * NH * 4 + 16 * k, 16, ext_theta(q) * 4))
+                    cp_async16(s + sl.TH + 16 * k, reinterpret_cast<const uint8_t*>(q.theta + (bt * G + g) * NH) + 16 * k);
                 continue;
             }
             k -= pT;
             const int r = k / pX, kk = k % pX;
             const uint8_t* src = reinterpret_cast<const uint8_t*>(xg + ((bt * H + h) * R + r) * P + c0) + 16 * kk;
             if (xb < 16) {
-                if (c0 < P) cp_async8(s + sl.X + r * sl.XS, src);
-            } else if (c0 + kk * 16 / es < P) {
+                if (c0 < P && M3_SPAN(7, (((bt * H + h) * R + r) * P + c0) * es, 8, ext_x(q) * es))
+                    cp_async8(s + sl.X + r * sl.XS, src);
+            } else if (c0 + kk * 16 / es < P && M3_SPAN(8, (((bt * H + h) * R + r) * P + c0) * es + 16 * kk, 16, ext_x(q) * es)) {
                 cp_async16(s + sl.X + r * sl.XS + 16 * kk, src);
             }
         }
         for (int tt = tid; tt < nt; tt += kThreads) {
             const size_t o = ((size_t)b * L + t0 + tt) * H + h;
             uint8_t* s = base + (size_t)tt * sl.bytes + sl.DL;
+            if (!M3_IN(9, o, ext_tok(q)) || !M3_SPAN(10, s - smem, 8, dyn_smem_bytes())) continue;
             cp_async4(s, q.dt + o);
             cp_async4(s + 4, q.lam + o);
         }
@@ -217,18 +232,21 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(SeqParams q, int TK) {
         for (int e = 0; e < 2; ++e) {
 #pragma unroll
             for (int c = 0; c < kPC; ++c)
-                hs[k][e][c] = (q.init_h && i < NH && wact) ? q.init_h[(bh * N + 2 * i + e) * P + cw + c] : 0.f;
+                hs[k][e][c] = (q.init_h && i < NH && wact && M3_IN(11, (bh * N + 2 * i + e) * P + cw + c, ext_h(q)))
+                                  ? q.init_h[(bh * N + 2 * i + e) * P + cw + c] : 0.f;
 #pragma unroll
             for (int r = 0; r < R; ++r)
-                pb[k][e][r] = (q.init_pB && i < NH) ? ld_io(static_cast<const T*>(q.init_pB) + (bh * R + r) * N + 2 * i + e)
-                                                    : 0.f;
+                pb[k][e][r] = (q.init_pB && i < NH && M3_IN(12, (bh * R + r) * N + 2 * i + e, ext_pB(q)))
+                                  ? ld_io(static_cast<const T*>(q.init_pB) + (bh * R + r) * N + 2 * i + e)
+                                  : 0.f;
         }
     }
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int c = 0; c < kPC; ++c)
-            px[r][c] = (q.init_pX && wact) ? ld_io(static_cast<const T*>(q.init_pX) + (bh * R + r) * P + cw + c) : 0.f;
+            px[r][c] = (q.init_pX && wact && M3_IN(13, (bh * R + r) * P + cw + c, ext_pX(q)))
+                           ? ld_io(static_cast<const T*>(q.init_pX) + (bh * R + r) * P + cw + c) : 0.f;
 
     const int nchunks = (L + TK - 1) / TK;
     stage(0, 0);
@@ -242,6 +260,8 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(SeqParams q, int TK) {
         const int t0 = ch * TK;
         const int nt = min(TK, L - t0);
         uint8_t* base = smem + (size_t)(ch & 1) * TK * sl.bytes;
+        // the chunk's slots inside the launch's dynamic shared memory (uniform)
+        if (!M3_SPAN(14, base - smem, (size_t)nt * sl.bytes, dyn_smem_bytes())) break;
         // every token's pair blocks and alpha, beta, gamma, once for all warps
         for (int e = tid; e < nt * NH; e += kThreads) {
             const int tt = e / NH, i = e - tt * NH;
@@ -369,7 +389,8 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(SeqParams q, int TK) {
             constexpr int SPAN = 32 / NV;          // lanes holding one value's total
             if (wact && (lane % SPAN) == 0) {
                 const int idx = lane / SPAN, r = idx / kPC, c = idx % kPC;
-                st_io(static_cast<T*>(q.y) + ((((size_t)b * L + t0 + tt) * H + h) * R + r) * P + cw + c, yv[0]);
+                if (M3_IN(15, ((((size_t)b * L + t0 + tt) * H + h) * R + r) * P + cw + c, ext_x(q)))
+                    st_io(static_cast<T*>(q.y) + ((((size_t)b * L + t0 + tt) * H + h) * R + r) * P + cw + c, yv[0]);
             }
 #pragma unroll
             for (int k = 0; k < KP; ++k)
@@ -394,17 +415,23 @@ __global__ void __launch_bounds__(kThreads) seq_kernel(SeqParams q, int TK) {
         for (int e = 0; e < 2; ++e) {
             if (q.fin_h && wact)
 #pragma unroll
-                for (int c = 0; c < kPC; ++c) q.fin_h[(bh * N + 2 * i + e) * P + cw + c] = hs[k][e][c];
+                for (int c = 0; c < kPC; ++c)
+                    if (M3_IN(16, (bh * N + 2 * i + e) * P + cw + c, ext_h(q)))
+                        q.fin_h[(bh * N + 2 * i + e) * P + cw + c] = hs[k][e][c];
             if (q.fin_pB && blockIdx.x == 0 && warp == 0)
 #pragma unroll
-                for (int r = 0; r < R; ++r) st_io(static_cast<T*>(q.fin_pB) + (bh * R + r) * N + 2 * i + e, pb[k][e][r]);
+                for (int r = 0; r < R; ++r)
+                    if (M3_IN(17, (bh * R + r) * N + 2 * i + e, ext_pB(q)))
+                        st_io(static_cast<T*>(q.fin_pB) + (bh * R + r) * N + 2 * i + e, pb[k][e][r]);
         }
     }
     if (q.fin_pX && wact && lane == 0)
 #pragma unroll
         for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int c = 0; c < kPC; ++c) st_io(static_cast<T*>(q.fin_pX) + (bh * R + r) * P + cw + c, px[r][c]);
+            for (int c = 0; c < kPC; ++c)
+                if (M3_IN(18, (bh * R + r) * P + cw + c, ext_pX(q)))
+                    st_io(static_cast<T*>(q.fin_pX) + (bh * R + r) * P + cw + c, px[r][c]);
 }
 
 template <typename T, int R, int KP, bool REFL, int PCW>
@@ -468,3 +495,5 @@ cudaError_t launch_seq(const m3_dims& d, const SeqParams& q, cudaStream_t st) {
 }
 
 }  // namespace m3
+
+M3_BOUNDS_EXPORT(seq)

@@ -13,10 +13,22 @@
 // through registers with 128-bit coalesced loads/stores issued before any
 // other work; the small per-token operands (B_t, C_t, x_t, the previous B and
 // x, and the pair rotations) are staged in shared memory as float32.
+#define M3_BOUNDS_FILE 3
+#include "m3_bounds.cuh"
 #include "m3_common.cuh"
 #include "m3_kernels.h"
 
 namespace m3 {
+
+// element counts of the step's buffers, for the index checks of the debug build
+__device__ __forceinline__ long long sx_h(const StepParams& q) {
+    return (long long)q.batch * q.nheads * q.dstate * q.headdim;
+}
+__device__ __forceinline__ long long sx_bc(const StepParams& q, int R) { return (long long)q.batch * q.ngroups * R * q.dstate; }
+__device__ __forceinline__ long long sx_pb(const StepParams& q, int R) { return (long long)q.batch * q.nheads * R * q.dstate; }
+__device__ __forceinline__ long long sx_x(const StepParams& q, int R) { return (long long)q.batch * q.nheads * R * q.headdim; }
+__device__ __forceinline__ long long sx_tok(const StepParams& q) { return (long long)q.batch * q.nheads; }
+__device__ __forceinline__ long long sx_th(const StepParams& q) { return (long long)q.batch * q.ngroups * (q.dstate / 2); }
 
 // T: io element type; R: rank; NPT: rotary pairs per thread.
 template <typename T, int R, int NPT>
@@ -37,7 +49,7 @@ __global__ void __launch_bounds__(256) step_kernel(StepParams q) {
 #pragma unroll
     for (int k = 0; k < NPT; ++k) {
         const int i = ig + k * IG;
-        if (i < NH) {
+        if (i < NH && M3_SPAN(1, (size_t)bh * N * P + (size_t)(2 * i + 1) * P + 4 * pc, 4, sx_h(q))) {
             s0[k] = hs[(size_t)(2 * i) * PC + pc];
             s1[k] = hs[(size_t)(2 * i + 1) * PC + pc];
         }
@@ -52,25 +64,31 @@ __global__ void __launch_bounds__(256) step_kernel(StepParams q) {
     float* sX = sPB + R * N;          // [R][P]
     float* sPX = sX + R * P;          // [R][P]
     float* sY = sPX + R * P;          // [warps][R][P]
+    if (!M3_SPAN(13, (sY - smem) * 4, (blockDim.x >> 5) * R * P * 4, dyn_smem_bytes())) return;
     const T* Bg = static_cast<const T*>(q.B) + ((size_t)b * q.ngroups + g) * R * N;
     const T* Cg = static_cast<const T*>(q.C) + ((size_t)b * q.ngroups + g) * R * N;
     T* PBh = static_cast<T*>(q.prev_B) + (size_t)bh * R * N;
     T* PXh = static_cast<T*>(q.prev_x) + (size_t)bh * R * P;
     const T* Xh = static_cast<const T*>(q.x) + (size_t)bh * R * P;
     for (int e = tid; e < R * N; e += blockDim.x) {
+        if (!M3_IN(2, ((size_t)b * q.ngroups + g) * R * N + e, sx_bc(q, R)) || !M3_IN(3, (size_t)bh * R * N + e, sx_pb(q, R)))
+            continue;
         sB[e] = ld_io(Bg + e);
         sC[e] = ld_io(Cg + e);
         sPB[e] = ld_io(PBh + e);
     }
     for (int e = tid; e < R * P; e += blockDim.x) {
+        if (!M3_IN(4, (size_t)bh * R * P + e, sx_x(q, R))) continue;
         sX[e] = ld_io(Xh + e);
         sPX[e] = ld_io(PXh + e);
     }
-    const float d = q.dt[bh];
-    const float lam = q.lam[bh];
-    const float a = q.A[h];
+    const bool okt = M3_IN(5, bh, sx_tok(q)) && M3_IN(6, h, q.nheads);
+    const float d = okt ? q.dt[bh] : 0.f;
+    const float lam = okt ? q.lam[bh] : 0.f;
+    const float a = okt ? q.A[h] : 0.f;
     const float* th = q.theta + ((size_t)b * q.ngroups + g) * NH;
     for (int i = tid; i < NH; i += blockDim.x) {
+        if (!M3_IN(7, ((size_t)b * q.ngroups + g) * NH + i, sx_th(q))) continue;
         const double phi = wrap_pi((double)d * (double)th[i]);
         float sv, cv;
         sincosf((float)phi, &sv, &cv);
@@ -130,6 +148,7 @@ __global__ void __launch_bounds__(256) step_kernel(StepParams q) {
 #pragma unroll
             for (int r = 0; r < R; ++r) yacc[r][j] = fmaf(c0[r], w0, fmaf(c1[r], w1, yacc[r][j]));
         }
+        if (!M3_SPAN(8, (size_t)bh * N * P + (size_t)n1 * P + 4 * pc, 4, sx_h(q))) continue;
         hs[(size_t)n0 * PC + pc] = make_float4(u0[0], u0[1], u0[2], u0[3]);
         hs[(size_t)n1 * PC + pc] = make_float4(u1[0], u1[1], u1[2], u1[3]);
     }
@@ -146,7 +165,9 @@ __global__ void __launch_bounds__(256) step_kernel(StepParams q) {
 #pragma unroll
         for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) sY[(warp * R + r) * P + 4 * lane + j] = yacc[r][j];
+            for (int j = 0; j < 4; ++j)
+                if (M3_IN(9, (warp * R + r) * P + 4 * lane + j, nwarps * R * P))
+                    sY[(warp * R + r) * P + 4 * lane + j] = yacc[r][j];
     }
     __syncthreads();
     T* Yh = static_cast<T*>(q.y) + (size_t)bh * R * P;
@@ -154,12 +175,14 @@ __global__ void __launch_bounds__(256) step_kernel(StepParams q) {
         const int r = e / P, p = e % P;
         float acc = 0.f;
         for (int w = 0; w < nwarps; ++w) acc += sY[(w * R + r) * P + p];
-        st_io(Yh + e, acc);
+        if (M3_IN(10, (size_t)bh * R * P + e, sx_x(q, R))) st_io(Yh + e, acc);
     }
 
     // 5. this token's (B, x) become the carry's previous (B, x)
-    for (int e = tid; e < R * N; e += blockDim.x) st_io(PBh + e, sB[e]);
-    for (int e = tid; e < R * P; e += blockDim.x) st_io(PXh + e, sX[e]);
+    for (int e = tid; e < R * N; e += blockDim.x)
+        if (M3_IN(11, (size_t)bh * R * N + e, sx_pb(q, R))) st_io(PBh + e, sB[e]);
+    for (int e = tid; e < R * P; e += blockDim.x)
+        if (M3_IN(12, (size_t)bh * R * P + e, sx_x(q, R))) st_io(PXh + e, sX[e]);
 }
 
 // ---------------------------------------------------------------------------
@@ -233,7 +256,10 @@ __global__ void __launch_bounds__(256, 2) step_pipe_kernel(StepParams q, int uni
             const char* src_h = reinterpret_cast<const char*>(q.h + (size_t)u * N * P);
             constexpr int nh = N * P / 4, nb = R * N * (int)sizeof(T) / 16, nx = R * P * (int)sizeof(T) / 16;
 #pragma unroll
-            for (int c0 = 0; c0 < nh; c0 += 256) cp16(d0 + lay.off_h + 16 * (c0 + tid), src_h + 16 * (c0 + tid));
+            for (int c0 = 0; c0 < nh; c0 += 256)
+                if (M3_SPAN(20, (size_t)u * N * P + 4 * (c0 + tid), 4, sx_h(q)) &&
+                    M3_SPAN(21, st * lay.stage + lay.off_h + 16 * (c0 + tid), 16, dyn_smem_bytes()))
+                    cp16(d0 + lay.off_h + 16 * (c0 + tid), src_h + 16 * (c0 + tid));
             const char* sB = reinterpret_cast<const char*>(static_cast<const T*>(q.B) + bg * R * N);
             const char* sC = reinterpret_cast<const char*>(static_cast<const T*>(q.C) + bg * R * N);
             const char* sPB = reinterpret_cast<const char*>(static_cast<const T*>(q.prev_B) + (size_t)u * R * N);
@@ -243,7 +269,10 @@ __global__ void __launch_bounds__(256, 2) step_pipe_kernel(StepParams q, int uni
 #pragma unroll
             for (int c0 = 0; c0 < nb; c0 += 256) {
                 const int c = c0 + tid;
-                if (nb % 256 == 0 || c < nb) {
+                if ((nb % 256 == 0 || c < nb) &&
+                    M3_SPAN(22, (bg * R * N) * sizeof(T) + 16 * c, 16, sx_bc(q, R) * (long long)sizeof(T)) &&
+                    M3_SPAN(23, ((size_t)u * R * N) * sizeof(T) + 16 * c, 16, sx_pb(q, R) * (long long)sizeof(T)) &&
+                    M3_SPAN(24, st * lay.stage + lay.off_PB + 16 * c, 16, dyn_smem_bytes())) {
                     cp16(d0 + lay.off_B + 16 * c, sB + 16 * c);
                     cp16(d0 + lay.off_C + 16 * c, sC + 16 * c);
                     cp16(d0 + lay.off_PB + 16 * c, sPB + 16 * c);
@@ -252,13 +281,18 @@ __global__ void __launch_bounds__(256, 2) step_pipe_kernel(StepParams q, int uni
 #pragma unroll
             for (int c0 = 0; c0 < nx; c0 += 256) {
                 const int c = c0 + tid;
-                if (nx % 256 == 0 || c < nx) {
+                if ((nx % 256 == 0 || c < nx) &&
+                    M3_SPAN(25, ((size_t)u * R * P) * sizeof(T) + 16 * c, 16, sx_x(q, R) * (long long)sizeof(T)) &&
+                    M3_SPAN(26, st * lay.stage + lay.off_PX + 16 * c, 16, dyn_smem_bytes())) {
                     cp16(d0 + lay.off_X + 16 * c, sX + 16 * c);
                     cp16(d0 + lay.off_PX + 16 * c, sPX + 16 * c);
                 }
             }
-            if (tid < NH / 4) cp16(d0 + lay.off_TH + 16 * tid, sTH + 16 * tid);
-            if (tid == 0) {
+            if (tid < NH / 4 && M3_SPAN(27, bg * NH + 4 * tid, 4, sx_th(q)) &&
+                M3_SPAN(28, st * lay.stage + lay.off_TH + 16 * tid, 16, dyn_smem_bytes()))
+                cp16(d0 + lay.off_TH + 16 * tid, sTH + 16 * tid);
+            if (tid == 0 && M3_IN(29, u, sx_tok(q)) && M3_IN(30, h, H) &&
+                M3_SPAN(31, st * lay.stage + lay.off_S, 12, dyn_smem_bytes())) {
                 cp4(d0 + lay.off_S, q.dt + u);
                 cp4(d0 + lay.off_S + 4, q.lam + u);
                 cp4(d0 + lay.off_S + 8, q.A + h);
@@ -349,6 +383,7 @@ __global__ void __launch_bounds__(256, 2) step_pipe_kernel(StepParams q, int uni
 #pragma unroll
                 for (int r = 0; r < R; ++r) yacc2[r][j] = __ffma2_rn(cc[r], w, yacc2[r][j]);
             }
+            if (!M3_SPAN(32, (size_t)u * N * P + (size_t)n1 * P + 4 * pc, 4, sx_h(q))) continue;
             hg[(size_t)n0 * PC + pc] = make_float4(o0[0], o0[1], o0[2], o0[3]);
             hg[(size_t)n1 * PC + pc] = make_float4(o1[0], o1[1], o1[2], o1[3]);
         }
@@ -384,7 +419,7 @@ __global__ void __launch_bounds__(256, 2) step_pipe_kernel(StepParams q, int uni
                 float acc = 0.f;
 #pragma unroll
                 for (int w = 0; w < 8; ++w) acc += sY[w * R * P + e];
-                st_io(Yh + e, acc);
+                if (M3_IN(33, (size_t)u * R * P + e, sx_x(q, R))) st_io(Yh + e, acc);
             }
         }
         // this token's (B, x) become the carry's previous (B, x): 16-byte copies
@@ -396,10 +431,14 @@ __global__ void __launch_bounds__(256, 2) step_pipe_kernel(StepParams q, int uni
             const uint4* iX = reinterpret_cast<const uint4*>(sX);
 #pragma unroll
             for (int c0 = 0; c0 < nb; c0 += 256)
-                if (nb % 256 == 0 || c0 + tid < nb) oB[c0 + tid] = iB[c0 + tid];
+                if ((nb % 256 == 0 || c0 + tid < nb) &&
+                    M3_SPAN(34, ((size_t)u * R * N) * sizeof(T) + 16 * (c0 + tid), 16, sx_pb(q, R) * (long long)sizeof(T)))
+                    oB[c0 + tid] = iB[c0 + tid];
 #pragma unroll
             for (int c0 = 0; c0 < nx; c0 += 256)
-                if (nx % 256 == 0 || c0 + tid < nx) oX[c0 + tid] = iX[c0 + tid];
+                if ((nx % 256 == 0 || c0 + tid < nx) &&
+                    M3_SPAN(35, ((size_t)u * R * P) * sizeof(T) + 16 * (c0 + tid), 16, sx_x(q, R) * (long long)sizeof(T)))
+                    oX[c0 + tid] = iX[c0 + tid];
         }
     }
     cp_wait<0>();
@@ -500,3 +539,5 @@ m3_status launch_step(const m3_dims& d, const StepParams& q, cudaStream_t st) {
 }
 
 }  // namespace m3
+
+M3_BOUNDS_EXPORT(step)

@@ -7,11 +7,31 @@
 #include <atomic>
 #include <vector>
 
+#define M3_BOUNDS_FILE 9
+#include "m3_bounds.cuh"
 #include "m3_common.cuh"
 #include "m3_kernels.h"
 #include "m3_nvtx.h"
 
 namespace m3 {
+
+#if M3_DEBUG_BOUNDS
+// readers of the per-file check records (each kernel file defines its own)
+cudaError_t bounds_take_scan_tc(BoundsRecord* out, bool clear);
+cudaError_t bounds_take_scan_simt(BoundsRecord* out, bool clear);
+cudaError_t bounds_take_step(BoundsRecord* out, bool clear);
+cudaError_t bounds_take_rope(BoundsRecord* out, bool clear);
+cudaError_t bounds_take_seq(BoundsRecord* out, bool clear);
+cudaError_t bounds_take_bwd(BoundsRecord* out, bool clear);
+cudaError_t bounds_take_phase(BoundsRecord* out, bool clear);
+cudaError_t bounds_take_scan_ws(BoundsRecord* out, bool clear);
+cudaError_t bounds_take_api(BoundsRecord* out, bool clear);
+
+// the check itself, on one index the caller chose (m3_selftest_bounds_check)
+__global__ void bounds_selftest_kernel(float* buf, long long index, long long limit) {
+    if (M3_IN(1, index, limit)) buf[index] = 1.f;
+}
+#endif
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -609,6 +629,46 @@ m3_status m3_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void
                : M3_ERR_CUDA;
 }
 
+m3_status m3_debug_bounds_report(m3_bounds_report* out, int clear) {
+    if (!out) return M3_ERR_INVALID_ARG;
+    memset(out, 0, sizeof(*out));
+#if M3_DEBUG_BOUNDS
+    using Take = cudaError_t (*)(BoundsRecord*, bool);
+    // in file order (site = file * 1000 + check)
+    const Take takes[] = {bounds_take_scan_tc, bounds_take_scan_simt, bounds_take_step,
+                          bounds_take_rope,    bounds_take_seq,       bounds_take_bwd,
+                          bounds_take_phase,   bounds_take_scan_ws,   bounds_take_api};
+    out->enabled = 1;
+    if (cudaDeviceSynchronize() != cudaSuccess) return M3_ERR_CUDA;
+    for (Take take : takes) {
+        BoundsRecord r;
+        if (take(&r, clear != 0) != cudaSuccess) return M3_ERR_CUDA;
+        if (r.failures != 0u && out->failures == 0u) {
+            out->site = r.site;
+            out->index = r.index;
+            out->limit = r.limit;
+        }
+        out->failures += r.failures;
+    }
+#else
+    (void)clear;
+#endif
+    return M3_OK;
+}
+
+m3_status m3_selftest_bounds_check(float* buffer, long long capacity, long long index, long long limit,
+                                   void* stream) {
+    if (!buffer || capacity < 1 || index < 0 || index >= capacity || limit < 0 || limit > capacity)
+        return M3_ERR_INVALID_ARG;
+#if M3_DEBUG_BOUNDS
+    bounds_selftest_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(buffer, index, limit);
+    return cudaGetLastError() == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+#else
+    (void)stream;
+    return M3_ERR_UNSUPPORTED;
+#endif
+}
+
 m3_status m3_device_status(void* workspace, void* stream) {
     if (!workspace) return M3_ERR_INVALID_ARG;
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return M3_ERR_CUDA;
@@ -622,3 +682,5 @@ m3_status m3_device_status(void* workspace, void* stream) {
 }
 
 }  // extern "C"
+
+M3_BOUNDS_EXPORT(api)

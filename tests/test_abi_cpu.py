@@ -237,3 +237,46 @@ def test_static_forget_device_needs_a_current_device():
     st = LIB.m3_static_forget_device()
     assert st in (m3.M3_OK, m3.M3_ERR_CUDA)
     assert LIB.m3_static_forget_device() == st
+
+
+def test_release_build_has_no_index_checks():
+    """libm3.so: the bounds report says 'disabled' without touching a device,
+    and the checks' self-test validates its arguments, then refuses
+    (M3_ERR_UNSUPPORTED) without launching."""
+    if m3.DEBUG_BOUNDS:
+        pytest.skip("the package was imported with the index-checked library")
+    assert m3.m3_debug_bounds_report() == {"enabled": 0, "failures": 0, "site": 0, "index": 0, "limit": 0}
+    assert LIB.m3_debug_bounds_report(None, 0) == m3.M3_ERR_INVALID_ARG
+    st = LIB.m3_selftest_bounds_check
+    assert st(GOOD, 64, 40, 32, None) == m3.M3_ERR_UNSUPPORTED
+    assert st(None, 64, 40, 32, None) == m3.M3_ERR_INVALID_ARG      # no buffer
+    assert st(GOOD, 64, 64, 32, None) == m3.M3_ERR_INVALID_ARG      # index past the buffer
+    assert st(GOOD, 64, -1, 32, None) == m3.M3_ERR_INVALID_ARG
+    assert st(GOOD, 64, 3, 65, None) == m3.M3_ERR_INVALID_ARG       # limit past the buffer
+    assert st(GOOD, 0, 0, 0, None) == m3.M3_ERR_INVALID_ARG
+
+
+def test_debug_library_is_built_and_exports_every_symbol():
+    """libm3_debug.so (the index-checked build) sits beside libm3.so, exports
+    the same ABI, and is what the package loads under M3_DEBUG_BOUNDS=1; its
+    report needs a device (M3_ERR_CUDA without one)."""
+    dbg = os.path.join(os.path.dirname(m3.LIB_PATH), "libm3_debug.so")
+    assert os.path.exists(dbg)
+    out = subprocess.run(["nm", "-D", "--defined-only", dbg], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(m3_[a-z0-9_]+)$", out, flags=re.M))
+    assert set(declared_functions()) <= exported
+    code = (
+        "import torch, selective_state_space_m3_b200 as m3\n"
+        "assert m3.DEBUG_BOUNDS and m3.LIB_PATH.endswith('libm3_debug.so'), m3.LIB_PATH\n"
+        "lib = m3.raw_lib()\n"
+        "assert lib.m3_selftest_bounds_check(0x10000, 64, 64, 32, None) == m3.M3_ERR_INVALID_ARG\n"
+        "if not torch.cuda.is_available():\n"
+        "    try:\n"
+        "        m3.m3_debug_bounds_report()\n"
+        "        raise SystemExit('report without a device')\n"
+        "    except m3.M3Error as e:\n"
+        "        assert e.status == m3.M3_ERR_CUDA, e\n"
+        "print('debug ok')\n")
+    env = dict(os.environ, M3_DEBUG_BOUNDS="1", PYTHONPATH=ROOT)
+    r = subprocess.run([os.sys.executable, "-c", code], capture_output=True, text=True, env=env, cwd=ROOT, timeout=300)
+    assert r.returncode == 0 and "debug ok" in r.stdout, r.stdout + r.stderr
