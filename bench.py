@@ -362,11 +362,11 @@ KERNEL_SOURCES = {
 CAPTURES = {
     # kernel: (workload, plan segments or None, bytes per launch, source digest)
     "scan_tc_kernel": ("mimo_r4_layer_b8_h32_L4096_P64_N128_Q64_bf16", 1,
-                       2_982_520_064 + 523_729_152, "064aefd1c4555e7b"),
+                       2_982_388_224 + 523_830_528, "f41c574135517d21"),
     "step_pipe_kernel": ("decode_mimo_r4_b256_h32_P64_N128_x1000", None,
-                         304_192_768 + 224_838_400, "fb3967fb581615af"),
+                         304_190_208 + 224_724_480, "87cab08d84241421"),
     "rope_block_kernel": ("mimo_r4_layer_b8_h32_L4096_P64_N128_Q64_bf16", None,
-                          2_423_972_608 + 2_379_064_576, "e87a9f369ceb08c4"),
+                          2_423_474_432 + 2_379_173_888, "722d31272b55c86c"),
 }
 
 
