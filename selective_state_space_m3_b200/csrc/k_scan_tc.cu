@@ -65,7 +65,7 @@ constexpr int OFF_C = 32768;      // 32 KB: C~, later P
 constexpr int OFF_X = 65536;      // 16 KB: X
 constexpr int OFF_S = 81920;      // 16 KB: S_bf (rows n, 64 p)
 constexpr int OFF_MISC = 98304;
-constexpr int MISC_BYTES = 10496;
+constexpr int MISC_BYTES = 12544;
 // dynamic shared memory of a launch (+ alignment slack); R >= 4 leaves the
 // second parity of the R < 4 tables out, which keeps more of the SM's L1
 template <int R>
@@ -80,8 +80,12 @@ struct Misc {
     float2 qs[2][kNE][32];        // per token group: phase increments of pairs (2i, 2i+1), by tile parity
     union {
         float msk[32 * 36];       // R >= 4: decay mask per (token, token), rows padded
-        float cs[2][6][128];      // R < 4, by tile parity (the next tile's are made one tile
+        struct {
+            float cs[2][6][128];  // R < 4, by tile parity (the next tile's are made one tile
                                   // ahead): c and gamma times e^{a_ref - a}, a_ref per block; a, gamma, c
+            float tk[2][2][132];  // R < 4, by tile parity: dt and lambda of the next tile's
+                                  // tokens (clamped to its last) and of the token after it
+        };
     } u;
 };
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region too small");
@@ -108,6 +112,13 @@ using namespace ptx;
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Misc* m, int* status, int where) {
     return mbar_wait_flag(b, parity, &m->abort_flag, status, where);
 }
+
+// 4-byte global -> shared copies of the long tiles' dt / lambda staging
+__device__ __forceinline__ void cp_async4(float* dst, const float* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(su32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void workers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kWorkers) : "memory"); }
 // all workers get the OR of `cond` (named barrier 1 with a reduction), so
@@ -288,15 +299,32 @@ __global__ void __launch_bounds__(kThreads, 2)
                    ? __ldg(reinterpret_cast<const float2*>(q.theta + (((size_t)b * L + t0n + t) * G + g) * (kN / 2)) + lane)
                    : make_float2(0.f, 0.f);
     };
-    auto prefetch_tok = [&](int kn) {         // L2 prefetch of a tile's dt / lambda (and the token after it)
+    // long tiles: tile kn's dt / lambda copied into shared memory (parity kn & 1)
+    // by cp.async, a tile ahead of their use: slot s < 128 holds token
+    // min(s, last of the tile), slot 128 the token after the tile (or the last
+    // token); the copies land before the worker barrier of the tile that
+    // issues them and are read after it, so no register waits on them
+    auto stage_tok = [&](int kn) {
         const int t0n = tok0 + kn * T;
-        const int qn = min(T + 1, L - t0n);
-        for (int t = wk; t < qn; t += kWorkers) {
-            const size_t o = ((size_t)b * L + t0n + t) * H + h;
-            if (!M3_IN(12, o, ext_tok(q))) continue;
-            prefetch_l2(q.dt + o);
-            prefetch_l2(q.lam + o);
+        const int qcn = min(T, tok1 - t0n);
+        if (wk <= T) {
+            const int t = wk < T ? t0n + min(wk, qcn - 1) : min(t0n + qcn, L - 1);
+            const size_t o = ((size_t)b * L + t) * H + h;
+            if (M3_IN(12, o, ext_tok(q))) {
+                cp_async4(&m->u.tk[kn & 1][0][wk], q.dt + o);
+                cp_async4(&m->u.tk[kn & 1][1][wk], q.lam + o);
+            }
         }
+        cp_async_commit();
+    };
+    auto take_tok = [&](int kn) {             // the staged values of tile kn into the load registers
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+            dt_n[j] = m->u.tk[kn & 1][0][lane + 32 * j];
+            lam_n[j] = m->u.tk[kn & 1][1][lane + 32 * j];
+        }
+        dx_n = m->u.tk[kn & 1][0][T];
+        lx_n = m->u.tk[kn & 1][1][T];
     };
     auto prefetch_theta = [&](int kn) {       // L2 prefetch of a tile's theta rows (256 B per token)
         const int t0n = tok0 + kn * T;
@@ -576,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         // MMA wait; the next tile's dt / lambda go to L2 now and are loaded
         // once this tile's MMAs are issued.  Short tiles (R >= 4) make them
         // here: their MMA waits are too short to hide the stage (measured).
-        if (kAhead && k + 1 < ntiles) prefetch_tok(k + 1);
+        if (kAhead && k + 1 < ntiles) stage_tok(k + 1);
         // theta of tokens g0 + kk (zero past the end): short groups load it
         // here, ahead of its first use (L2 hits, prefetched two tiles ahead);
         // long groups reload it where it is used
@@ -600,7 +628,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             y_tile = -1;
         }
         mbar_wait(&m->bar[BAR_LOAD], par, m, status, 10);
-        // one barrier per tile: publishes qs and msk; all workers agree to stop
+        if (kAhead) cp_async_wait_all();          // this thread's staged dt / lambda have landed
+        // one barrier per tile: publishes qs, msk and the staged dt / lambda;
+        // all workers agree to stop
         if (workers_any(*(volatile int*)&m->abort_flag)) break;
         // the shared base as an opaque value produced after the barrier: the
         // rotation's loads take their addresses from it, so they cannot be
@@ -688,7 +718,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         // while this tile's MMAs run
         TileCoef nxt = cur;
         if (k + 1 < ntiles) {
-            load_tok(k + 1);     // (short tiles: consumed at the next tile's top)
+            // short tiles: consumed at the next tile's top; long tiles: staged
+            if (kAhead) take_tok(k + 1);
+            else load_tok(k + 1);
             if (kAhead) {
                 nxt = coef_stage(k + 1);
                 pass1_ahead(k + 1, nxt.dsl);
