@@ -23,7 +23,8 @@
 //   workers coefficient stage: dt/lambda -> a_t (warp scan, every warp keeps
 //           all tokens in registers), gamma, c, w = e^{a_last-a}c, e^{a}, the
 //           mask tables and each warp's phase increments (for R <= 2 made one
-//           tile ahead, during the previous tile's MMA wait); cumulative phase
+//           tile ahead, during the previous tile's MMA wait, from dt/lambda
+//           that cp.async copied into shared memory a tile earlier); cumulative phase
 //           per rotary pair (float, reduced to [-pi, pi] at the tile start and
 //           between tiles); rotate B and C in place in bf16x2 arithmetic.  One
 //           worker barrier per tile.
@@ -35,9 +36,9 @@
 //           Y_intra = P X (128x64, K=128)      -> TMEM cols [0,64)
 //   workers S = e^{a_last} S + S_loc (float32, registers, thread = state row);
 //           S_bf = bf16(S) for the next tile; y = Y_intra + e^{a_t} Y_inter.
-// Two CTAs share an SM (about 105 KB of shared memory, 256 TMEM columns and
-// at most 96 registers per thread each), so one CTA's loads and MMAs overlap
-// the other's SIMT work.
+// Two CTAs share an SM (108.5 KB of shared memory for R >= 4, 111.9 KB for
+// R < 4, 256 TMEM columns and at most 96 registers per thread each), so one
+// CTA's loads and MMAs overlap the other's SIMT work.
 //
 // Every wait on an mbarrier is bounded (1 s); on expiry the kernel records
 // M3_ERR_DEVICE_TIMEOUT in the workspace status word, finishes the tile with
