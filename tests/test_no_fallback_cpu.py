@@ -1,6 +1,7 @@
 """The product path has no CPU fallback (no GPU needed).
 
-* Without libm3.so the package does not import: it raises ImportError.
+* Without libm3.so the package does not import: it raises ImportError (and
+  likewise without libm3_debug.so when M3_DEBUG_BOUNDS=1 asks for it).
 * Every entry point refuses host tensors before anything reaches the
   library, so no computation can silently run on the host.
 * Neither the package's Python nor its CUDA sources reach the oracle, and
@@ -32,6 +33,22 @@ def test_missing_library_fails_the_import(tmp_path):
                        timeout=300)
     assert r.returncode != 0
     assert "ImportError" in r.stderr and "libm3.so is missing" in r.stderr
+
+
+def test_missing_debug_library_fails_the_import_under_the_debug_switch(tmp_path):
+    """M3_DEBUG_BOUNDS=1 asks for the index-checked library: with only the
+    release library present the import fails too (no quiet fallback to it)."""
+    dst = tmp_path / "selective_state_space_m3_b200"
+    dst.mkdir()
+    for f in glob.glob(os.path.join(PKG, "*.py")):
+        shutil.copy(f, dst)
+    shutil.copy(os.path.join(PKG, "libm3.so"), dst)
+    assert not (dst / "libm3_debug.so").exists()
+    r = subprocess.run([sys.executable, "-c", "import selective_state_space_m3_b200"], cwd=tmp_path,
+                       env={**os.environ, "PYTHONPATH": str(tmp_path), "M3_DEBUG_BOUNDS": "1"},
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "libm3_debug.so is missing" in r.stderr
 
 
 def _host_case():
