@@ -362,7 +362,7 @@ KERNEL_SOURCES = {
 CAPTURES = {
     # kernel: (workload, plan segments or None, bytes per launch, source digest)
     "scan_tc_kernel": ("mimo_r4_layer_b8_h32_L4096_P64_N128_Q64_bf16", 1,
-                       2_983_532_288 + 525_264_128, "60eddef2f96a207d"),
+                       2_982_624_000 + 525_852_416, "09d664a50f617954"),
     "step_pipe_kernel": ("decode_mimo_r4_b256_h32_P64_N128_x1000", None,
                          304_190_208 + 224_724_480, "87cab08d84241421"),
     "rope_block_kernel": ("mimo_r4_layer_b8_h32_L4096_P64_N128_Q64_bf16", None,

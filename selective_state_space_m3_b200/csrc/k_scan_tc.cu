@@ -301,8 +301,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                    : make_float2(0.f, 0.f);
     };
     // long tiles: tile kn's dt / lambda copied into shared memory (parity kn & 1)
-    // by cp.async, a tile ahead of their use: slot s < 128 holds token
-    // min(s, last of the tile), slot 128 the token after the tile (or the last
+    // by cp.async, a tile ahead of their use: slot s < T holds token
+    // min(s, last of the tile), slot T the token after the tile (or the last
     // token); the copies land before the worker barrier of the tile that
     // issues them and are read after it, so no register waits on them
     auto stage_tok = [&](int kn) {
@@ -602,9 +602,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         // ---------------------------------------------------------- workers
         // Long tiles (R <= 2): tile k's coefficients (cur), mask tables and
         // phase increments were made one tile ahead, in the previous tile's
-        // MMA wait; the next tile's dt / lambda go to L2 now and are loaded
-        // once this tile's MMAs are issued.  Short tiles (R >= 4) make them
-        // here: their MMA waits are too short to hide the stage (measured).
+        // MMA wait; the next tile's dt / lambda are copied into shared memory
+        // now and read once this tile's MMAs are issued.  Short tiles (R >= 4)
+        // make them here: their MMA waits are too short to hide the stage
+        // (measured).
         if (kAhead && k + 1 < ntiles) stage_tok(k + 1);
         // theta of tokens g0 + kk (zero past the end): short groups load it
         // here, ahead of its first use (L2 hits, prefetched two tiles ahead);
