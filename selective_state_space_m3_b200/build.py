@@ -80,8 +80,11 @@ def build(force: bool = False, verbose: bool = False, extra_flags=(), debug: boo
 
 
 def build_all(force: bool = False, verbose: bool = False) -> tuple:
-    """Both libraries: libm3.so and libm3_debug.so."""
-    return build(force, verbose), build(force, verbose, debug=True)
+    """Both libraries, compiled side by side: libm3.so and libm3_debug.so."""
+    with concurrent.futures.ThreadPoolExecutor(max_workers=2) as ex:
+        rel = ex.submit(build, force, verbose)
+        dbg = ex.submit(build, force, verbose, (), True)
+        return rel.result(), dbg.result()
 
 
 if __name__ == "__main__":
